@@ -1,0 +1,278 @@
+"""CPU oracle for int8 per-window recurrent-state decode (LeapQuant).
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` import this
+package.  It shares no code with the CUDA library and the library never calls
+it.
+
+The arithmetic lives in ``lq_oracle.c`` (plain C, FP64, OpenMP over heads);
+this module only marshals numpy arrays and holds the mapping from a model's
+gate parameters to the (D_t, k~_t, b_t) of equation 1, which is the
+arithmetic of one Table 4 row each:
+
+* "LeapQuant: Efficient Linear Attention with Accurate Recurrent State
+  Quantization", Appendix, Table 4: Gated DeltaNet is D_t = alpha_t I,
+  k~_t = beta_t k_t, b_t = alpha_t k_t.
+* Kimi Delta Attention (named in the same page's Abstract, no Table 4 row in
+  the text): D_t = Diag(alpha_t), k~_t = beta_t k_t, b_t = alpha_t * k_t, the
+  diagonal-gate analogue, whose record size 2 d_k + d_v matches the GLA row.
+
+Layouts are head-major: a state is ``[nh, d_v, d_k]``, a token tensor is
+``[nh, n, d]``.  Every function accepts any array-like and returns float64
+(or the stored formats int8 / float32 / int32 for snapshots).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "lq_oracle.c")
+_LIB = os.path.join(_HERE, "liblq_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def compile_oracle(force: bool = False) -> str:
+    """Compiles ``lq_oracle.c`` into ``liblq_oracle.so`` (gcc, -O2, strict IEEE)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".{os.getpid()}.tmp"
+        cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
+               "-Wall", "-Wextra", "-shared", "-fPIC", "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            # LQ_ORACLE_LIB lets the mutation meta-test load a deliberately
+            # broken build of this oracle to show that the pins catch it.
+            path = os.environ.get("LQ_ORACLE_LIB") or compile_oracle()
+            lib = ctypes.CDLL(path)
+            P = ctypes.c_void_p
+            I = ctypes.c_int
+            lib.lqo_eq1_steps.argtypes = [I, I, I, I, P, P, P, P, P, P, P]
+            lib.lqo_quantize.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P]
+            lib.lqo_dequantize.argtypes = [I, I, I, I, P, P, P, P, P, P]
+            lib.lqo_window.argtypes = [I] * 9 + [P] * 14
+            lib.lqo_rebuild.argtypes = [I] * 7 + [P] * 9
+            for f in (lib.lqo_eq1_steps, lib.lqo_quantize, lib.lqo_dequantize,
+                      lib.lqo_window, lib.lqo_rebuild):
+                f.restype = None
+            _lib = lib
+    return _lib
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+# --------------------------------------------------------------------------
+# Table 4 instances (the gate parameters of a model -> D_t, k~_t, b_t).
+# --------------------------------------------------------------------------
+
+def gdn_instance(alpha, beta, k):
+    """Gated DeltaNet row of Table 4: D = alpha I, k~ = beta k, b = alpha k.
+
+    alpha, beta: [nh, n]; k: [nh, n, d_k].  Returns d [nh, n, 1], k~, b."""
+    alpha = np.asarray(alpha, np.float64)
+    beta = np.asarray(beta, np.float64)
+    k = np.asarray(k, np.float64)
+    return alpha[..., None], beta[..., None] * k, alpha[..., None] * k
+
+
+def kda_instance(alpha, beta, k):
+    """Diagonal (per key channel) gate: D = Diag(alpha), k~ = beta k, b = alpha * k.
+
+    alpha: [nh, n, d_k]; beta: [nh, n]; k: [nh, n, d_k]."""
+    alpha = np.asarray(alpha, np.float64)
+    beta = np.asarray(beta, np.float64)
+    k = np.asarray(k, np.float64)
+    return alpha, beta[..., None] * k, alpha * k
+
+
+# --------------------------------------------------------------------------
+# Equation 1, explicit stepping.
+# --------------------------------------------------------------------------
+
+def eq1_steps(S0, d, kt, b, v, q=None):
+    """n steps of S_t = S_{t-1} Diag(d_t) + (v_t - S_{t-1} b_t) k~_t^T, o_t = S_t q_t.
+
+    S0 [nh, dv, dk]; d [nh, n, 1 or dk]; kt, b, q [nh, n, dk]; v [nh, n, dv].
+    Returns (o [nh, n, dv] or None, S_n [nh, dv, dk]) in FP64."""
+    S = _c(S0, np.float64).copy()
+    nh, dv, dk = S.shape
+    kt = _c(kt, np.float64)
+    n = kt.shape[1]
+    d = _c(np.broadcast_to(np.asarray(d, np.float64), (nh, n, dk)), np.float64)
+    b = _c(b, np.float64)
+    v = _c(v, np.float64)
+    qq = None if q is None else _c(q, np.float64)
+    o = None if q is None else np.zeros((nh, n, dv), np.float64)
+    _load().lqo_eq1_steps(nh, dv, dk, n, _p(S), _p(d), _p(kt), _p(b), _p(v), _p(qq), _p(o))
+    return o, S
+
+
+# --------------------------------------------------------------------------
+# Snapshot: quantize / dequantize.
+# --------------------------------------------------------------------------
+
+class Snapshot(dict):
+    """codes int8 [nh,dv,dk], row_scale f32 [nh,dv], col_smooth f32 [nh,dk],
+    comp_row i32 [nh,r], comp_val f32 [nh,r,dk] (+ row_norm f64 [nh,dv] when
+    produced by quantize)."""
+
+    @property
+    def n_comp(self):
+        return self["comp_row"].shape[1]
+
+
+def quantize(S, n_comp: int, smoothing: bool = True) -> Snapshot:
+    """Compensator selection, residual smoothing and per-row int8 codes of an
+    FP32 state ``S`` [nh, dv, dk] (rounded to FP32 first if it is not)."""
+    S = _c(S, np.float32)
+    nh, dv, dk = S.shape
+    assert 0 <= n_comp <= dv
+    out = Snapshot(
+        codes=np.zeros((nh, dv, dk), np.int8),
+        row_scale=np.zeros((nh, dv), np.float32),
+        col_smooth=np.zeros((nh, dk), np.float32),
+        comp_row=np.zeros((nh, n_comp), np.int32),
+        comp_val=np.zeros((nh, n_comp, dk), np.float32),
+        row_norm=np.zeros((nh, dv), np.float64),
+    )
+    _load().lqo_quantize(nh, dv, dk, n_comp, int(bool(smoothing)), _p(S), _p(out["codes"]),
+                         _p(out["row_scale"]), _p(out["col_smooth"]), _p(out["comp_row"]),
+                         _p(out["comp_val"]), _p(out["row_norm"]))
+    return out
+
+
+def _snap_arrays(snap):
+    codes = _c(snap["codes"], np.int8)
+    nh, dv, dk = codes.shape
+    comp_row = _c(snap["comp_row"], np.int32).reshape(nh, -1)
+    r = comp_row.shape[1]
+    return (codes, _c(snap["row_scale"], np.float32), _c(snap["col_smooth"], np.float32),
+            comp_row, _c(snap["comp_val"], np.float32).reshape(nh, r, dk), nh, dv, dk, r)
+
+
+def dequantize(snap) -> np.ndarray:
+    """S^_0 = Diag(sigma) Q Diag(c) + compensator rows, FP64 [nh, dv, dk]."""
+    codes, rs, cs, cr, cv, nh, dv, dk, r = _snap_arrays(snap)
+    out = np.zeros((nh, dv, dk), np.float64)
+    _load().lqo_dequantize(nh, dv, dk, r, _p(codes), _p(rs), _p(cs), _p(cr), _p(cv), _p(out))
+    return out
+
+
+# --------------------------------------------------------------------------
+# Per-window decode (buffered form), rebuild and commit.
+# --------------------------------------------------------------------------
+
+class Records(dict):
+    """Window buffer: L [nh, W, gdim] (cumulative log gate), k [nh, W, dk]
+    (k~), u [nh, W, dv]; positions 1..pos are filled.  FP64 arrays holding
+    FP32 values (unless produced with exact=True)."""
+
+
+def empty_records(nh: int, W: int, dk: int, dv: int, gdim: int) -> Records:
+    return Records(L=np.zeros((nh, W, gdim)), k=np.zeros((nh, W, dk)), u=np.zeros((nh, W, dv)))
+
+
+def window(snap, records: Records, pos: int, d, kt, b, v, q, exact: bool = False):
+    """Decode n tokens at window positions pos+1..pos+n from the fixed
+    boundary snapshot and the buffered records (updated in place).
+
+    d [nh, n, gdim] (gdim 1 = scalar gate, d_k = diagonal gate); kt, b, q
+    [nh, n, dk]; v [nh, n, dv].  Returns o [nh, n, dv] (FP64)."""
+    codes, rs, cs, cr, cv, nh, dv, dk, r = _snap_arrays(snap)
+    W = records["k"].shape[1]
+    gdim = records["L"].shape[2]
+    d = _c(d, np.float64)
+    n = d.shape[1]
+    assert d.shape == (nh, n, gdim)
+    assert 0 <= pos and pos + n <= W
+    for key in ("L", "k", "u"):
+        records[key] = _c(records[key], np.float64)
+    kt, b, v, q = (_c(a, np.float64) for a in (kt, b, v, q))
+    o = np.zeros((nh, n, dv), np.float64)
+    _load().lqo_window(nh, dv, dk, r, gdim, W, pos, n, int(bool(exact)), _p(codes), _p(rs), _p(cs),
+                       _p(cr), _p(cv), _p(records["L"]), _p(records["k"]), _p(records["u"]),
+                       _p(d), _p(kt), _p(b), _p(v), _p(q), _p(o))
+    return o
+
+
+def rebuild(snap, records: Records, n: int) -> np.ndarray:
+    """S_n = S^_0 D_{1..n} + sum_{m<=n} u_m (D_{m+1..n} k~_m)^T, FP64 [nh, dv, dk]."""
+    codes, rs, cs, cr, cv, nh, dv, dk, r = _snap_arrays(snap)
+    W = records["k"].shape[1]
+    gdim = records["L"].shape[2]
+    assert 0 <= n <= W
+    L, K, U = (_c(records[key], np.float64) for key in ("L", "k", "u"))
+    out = np.zeros((nh, dv, dk), np.float64)
+    _load().lqo_rebuild(nh, dv, dk, r, gdim, W, n, _p(codes), _p(rs), _p(cs), _p(cr), _p(cv),
+                        _p(L), _p(K), _p(U), _p(out))
+    return out
+
+
+def commit(snap, records: Records, n: int, n_comp: int, smoothing: bool = True):
+    """Window commit: rebuild S_n (kept as an FP32 state), then quantize.
+
+    Returns (new snapshot, S_n as float32)."""
+    S = rebuild(snap, records, n).astype(np.float32)
+    return quantize(S, n_comp, smoothing), S
+
+
+def decode_run(snap, d, kt, b, v, q, W: int, n_comp: int, smoothing: bool = True,
+               on_commit=None):
+    """Free-running per-window decode of T tokens: windows of W tokens, each
+    committed at its end (the last, possibly short, window too).
+
+    ``on_commit(window_index, snapshot)`` is called after each commit.
+    Returns (o [nh, T, dv], final snapshot)."""
+    nh, T = np.asarray(kt).shape[:2]
+    dv = np.asarray(v).shape[2]
+    dk = np.asarray(kt).shape[2]
+    gdim = np.asarray(d).shape[2]
+    o = np.zeros((nh, T, dv))
+    widx = 0
+    for t0 in range(0, T, W):
+        t1 = min(T, t0 + W)
+        rec = empty_records(nh, W, dk, dv, gdim)
+        sl = slice(t0, t1)
+        o[:, sl] = window(snap, rec, 0, d[:, sl], kt[:, sl], b[:, sl], v[:, sl], q[:, sl])
+        snap, _ = commit(snap, rec, t1 - t0, n_comp, smoothing)
+        if on_commit is not None:
+            on_commit(widx, snap)
+        widx += 1
+    return o, snap
+
+
+def prefill(S0, d, kt, b, v, q, snapshot_every: int, n_comp: int, smoothing: bool = True):
+    """Prefill by the token recurrence (equation 1, FP64 state) with a
+    quantized snapshot of the state, rounded to FP32, after every
+    ``snapshot_every`` tokens (one state per that many cached tokens).
+
+    Returns (o [nh, T, dv], list of snapshots, final FP64 state)."""
+    S = _c(S0, np.float64)
+    nh, T = np.asarray(kt).shape[:2]
+    dv = S.shape[1]
+    o = np.zeros((nh, T, dv))
+    snaps = []
+    for t0 in range(0, T, snapshot_every):
+        t1 = min(T, t0 + snapshot_every)
+        sl = slice(t0, t1)
+        o[:, sl], S = eq1_steps(S, d[:, sl], kt[:, sl], b[:, sl], v[:, sl], q[:, sl])
+        if t1 - t0 == snapshot_every:
+            snaps.append(quantize(S.astype(np.float32), n_comp, smoothing))
+    return o, snaps, S

@@ -1,0 +1,66 @@
+"""The oracle's pins catch plausible mistakes.
+
+Each case plants one mistake in a copy of the oracle's C source (on the CPU,
+never in the CUDA path), builds it, and runs the pin suite against that build
+in a subprocess: the suite must fail.  The unmodified source must pass.
+"""
+import os
+import subprocess
+import sys
+import tempfile
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "lq_oracle.c")
+
+MUTATIONS = {
+    "drop_compensator_rows": (
+        "Sh[(size_t)row * dk + j] += (double)comp_val[(size_t)c * dk + j];", ";"),
+    "wrong_sign_update": ("u[i] = vt[i] - acc;", "u[i] = vt[i] + acc;"),
+    "decay_off_by_one": (
+        "for (int j = 0; j < dk; ++j) x[j] = decay(L, gdim, t - 1, 0, j) * bt[j];",
+        "for (int j = 0; j < dk; ++j) x[j] = decay(L, gdim, t, 0, j) * bt[j];"),
+    "output_drops_own_token": ("for (int m = 1; m <= t; ++m) {", "for (int m = 1; m < t; ++m) {"),
+    "rebuild_drops_last_record": ("for (int m = 1; m <= n; ++m)", "for (int m = 1; m < n; ++m)"),
+    "gate_index_transposed": (
+        "Sh[(size_t)i * dk + j] = Sh[(size_t)i * dk + j] * dt[j] + u[i] * kk[j];",
+        "Sh[(size_t)i * dk + j] = Sh[(size_t)i * dk + j] * dt[i % dk] + u[i] * kk[j];"),
+    "ties_to_larger_row": ("norm[i] > norm[best]", "norm[i] >= norm[best]"),
+    "smoothing_without_sqrt": ("(float)sqrt(m) : 1.0f", "(float)m : 1.0f"),
+    "round_half_away": ("qv = rint(f32(", "qv = round(f32("),
+    "scale_255": ("double sigma = f32(mx / 127.0);", "double sigma = f32(mx / 255.0);"),
+}
+
+
+def _build(src_text, out_dir):
+    c = os.path.join(out_dir, "lq_oracle.c")
+    so = os.path.join(out_dir, "liblq_oracle.so")
+    with open(c, "w") as f:
+        f.write(src_text)
+    subprocess.run(["gcc", "-O2", "-std=c11", "-fopenmp", "-ffp-contract=off", "-shared", "-fPIC",
+                    "-o", so, c, "-lm"], check=True)
+    return so
+
+
+def _run_pins(so):
+    env = dict(os.environ, LQ_ORACLE_LIB=so)
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    return r.returncode
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pins_catch_mutation(name):
+    old, new = MUTATIONS[name]
+    src = open(SRC).read()
+    assert src.count(old) >= 1, f"mutation anchor not found: {old}"
+    with tempfile.TemporaryDirectory() as d:
+        so = _build(src.replace(old, new), d)
+        assert _run_pins(so) != 0, f"pins did not catch mutation {name}"
+
+
+def test_unmutated_oracle_passes_pins():
+    with tempfile.TemporaryDirectory() as d:
+        assert _run_pins(_build(open(SRC).read(), d)) == 0
