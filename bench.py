@@ -1,0 +1,523 @@
+#!/usr/bin/env python
+"""Decode throughput of the int8 per-window recurrent state on B200.
+
+Workload (default): Gated DeltaNet decode, batch 256 x 32 heads, d_k = d_v =
+128, bf16 q/k/v/o, int8 state with per-row scales, window W = 16, r = 4
+Compensator Tokens, smoothing on.  One STEP is one window: W decode launches
+through the C ABI (the commit fused into the last), i.e. batch * W tokens.
+
+Timing: W_warm untimed steps, then exactly K steps bracketed by a barrier and
+torch.cuda.synchronize() on both sides, timed with CUDA events on the
+launching stream, max over ranks.  Each step replays a CUDA graph of the
+window's launches; event-record nodes inside the graph time every launch for
+the roofline.  Each decode launch reads about 250 MB (int8 state, records,
+inputs), twice the 126 MB L2, so every launch streams from HBM.
+
+Multi-GPU (torchrun): every rank decodes its own shard of sequences (batch
+per rank fixed: weak scaling); no collective on the data path; the host
+gathers the max elapsed time at the end.
+
+--impl reference times the CPU oracle (plain C, FP64) on the host cores on a
+bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import math
+import os
+import re
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "decode tokens/s (state-update+output) and HBM GB/s as % of B200 peak"
+FALLBACK_HBM_GBS = 6650.0
+
+
+# --------------------------------------------------------------------------
+# Algorithmic bytes (per (sequence, head) and launch)
+# --------------------------------------------------------------------------
+
+def snapshot_bytes(dk, dv, r):
+    return dv * dk + 4 * dv + 4 * dk + r * (4 + 4 * dk)
+
+
+def record_bytes(dk, dv, gate):
+    return 4 * ((dk if gate == "diag" else 1) + dk + dv)
+
+
+def decode_launch_bytes(dk, dv, r, gate, e, t, commit):
+    """Bytes one decode launch at window position t must move per head:
+    read the snapshot and the t-1 buffered records, read q, k, v, alpha,
+    beta, write o and record t; a fused commit also writes the new snapshot."""
+    G = dk if gate == "diag" else 1
+    rec = record_bytes(dk, dv, gate)
+    b = snapshot_bytes(dk, dv, r) + (t - 1) * rec + e * (2 * dk + dv) + 4 * G + 4 + e * dv + rec
+    if commit:
+        b += snapshot_bytes(dk, dv, r)
+    return b
+
+
+# --------------------------------------------------------------------------
+# Helpers
+# --------------------------------------------------------------------------
+
+def _dist():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def aggregate(elapsed_ms: float, tokens_per_rank: int, world: int, group=None):
+    """Max elapsed time over ranks and the whole-job token rate (host-side
+    reduction of two scalars; no data-path collective)."""
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        dev = "cuda" if dist.get_backend(group) == "nccl" else "cpu"
+        t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
+        elapsed_ms = float(t.item())
+    return elapsed_ms, tokens_per_rank * world / (elapsed_ms / 1e3)
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_digest():
+    h = hashlib.sha1()
+    for f in sorted(glob.glob(os.path.join(ROOT, "linear_attention_recurrent_int8_b200", "csrc", "*"))):
+        with open(f, "rb") as fh:
+            h.update(os.path.basename(f).encode())
+            h.update(fh.read())
+    return h.hexdigest()[:12]
+
+
+def profiled_traffic(kernel_key: str):
+    """dram bytes per launch recorded by an ncu capture summary under
+    profiles/, if it was taken on the current kernel sources."""
+    digest = source_digest()
+    for f in glob.glob(os.path.join(ROOT, "profiles", "*.md")):
+        text = open(f).read()
+        m_key = re.search(r"^traffic_key:\s*(\S+)", text, re.M)
+        m_src = re.search(r"^source_sha1:\s*(\S+)", text, re.M)
+        m_val = re.search(r"^traffic_bytes_per_launch:\s*([0-9.eE+]+)", text, re.M)
+        if m_key and m_src and m_val and m_key.group(1) == kernel_key and m_src.group(1) == digest:
+            return float(m_val.group(1))
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 50 ms."""
+
+    FIELDS = ["clocks.sm", "clocks.max.sm", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, device_index: int):
+        self.rows = []
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(device_index), "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append((time.monotonic(), [x.strip() for x in line.split(",")]))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0, t1, t_warm0):
+        def pick(a, b):
+            return [r for (t, r) in self.rows if a <= t <= b and len(r) == len(self.FIELDS)]
+        rows = pick(t0, t1)
+        window = "timed region"
+        if len(rows) < 3:
+            rows = pick(t_warm0, t1)
+            window = "warm-up and timed region (timed region shorter than 3 samples)"
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm = sorted(float(r[0]) for r in rows if r[0].replace(".", "").isdigit())
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[3 + i].lower() == "active"})
+        mx = rows[0][1]
+        return {"sm_mhz": sm[len(sm) // 2] if sm else None,
+                "sm_max_mhz": float(mx) if mx.replace(".", "").isdigit() else None,
+                "reasons": reasons, "samples": len(rows), "window": window}
+
+
+# --------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline and the reference arm)
+# --------------------------------------------------------------------------
+
+def oracle_window_rate(wl, n_seq: int, w_index: int = 0):
+    """Times the CPU oracle on n_seq sequences x all heads for one window of
+    decode plus its commit.  Returns (tokens/s, seconds, threads)."""
+    import numpy as np
+    cores = len(os.sched_getaffinity(0))
+    os.environ.setdefault("OMP_NUM_THREADS", str(cores))
+    import oracle
+    from linear_attention_recurrent_int8_b200 import synth
+    bs = np.arange(n_seq)
+    hs = np.arange(wl.heads)
+    S0 = synth.initial_state(wl.seed, bs, hs, wl.d_k, wl.d_v, wl.outlier_rows, wl.outlier_cols,
+                             wl.outlier_scale).reshape(n_seq * wl.heads, wl.d_v, wl.d_k)
+    tok = synth.tokens(wl.seed, bs, hs, w_index * wl.window, (w_index + 1) * wl.window, wl.d_k,
+                       wl.d_v, wl.gate, wl.io)
+
+    def hm(x):
+        x = np.asarray(x)
+        B, T, H = x.shape[:3]
+        return np.ascontiguousarray(np.swapaxes(x, 1, 2).reshape((B * H, T) + x.shape[3:]))
+
+    inst = oracle.kda_instance if wl.gate == "diag" else oracle.gdn_instance
+    d, kt, b = inst(hm(tok["alpha"]), hm(tok["beta"]), hm(tok["k"]))
+    v, q = hm(tok["v"]), hm(tok["q"])
+    snap = oracle.quantize(S0, wl.n_comp, wl.smoothing)
+    gdim = wl.d_k if wl.gate == "diag" else 1
+    t0 = time.perf_counter()
+    rec = oracle.empty_records(n_seq * wl.heads, wl.window, wl.d_k, wl.d_v, gdim)
+    oracle.window(snap, rec, 0, d, kt, b, v, q)
+    oracle.commit(snap, rec, wl.window, wl.n_comp, wl.smoothing)
+    dt = time.perf_counter() - t0
+    return n_seq * wl.window / dt, dt, int(os.environ["OMP_NUM_THREADS"])
+
+
+def calibrated_sample(wl, target_s: float):
+    _, dt1, _ = oracle_window_rate(wl, 1)
+    n = int(max(1, min(wl.batch, math.floor(target_s / max(dt1, 1e-6)))))
+    return n
+
+
+# --------------------------------------------------------------------------
+# Arms
+# --------------------------------------------------------------------------
+
+def run_reference(args, wl):
+    rank, world, _ = _dist()
+    if rank != 0:
+        return None
+    n_seq = calibrated_sample(wl, args.ref_seconds)
+    for i in range(args.warmup):
+        oracle_window_rate(wl, n_seq, i)
+    total_tok, total_s = 0, 0.0
+    for i in range(args.steps):
+        rate, dt, cores = oracle_window_rate(wl, n_seq, args.warmup + i)
+        total_tok += n_seq * wl.window
+        total_s += dt
+    value = total_tok / total_s
+    sample = (f"{n_seq} of {wl.batch} sequences x {wl.heads} heads, one window of {wl.window} "
+              f"decode tokens plus its commit per step")
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total_s / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(wl, args),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def workload_config(wl, args):
+    return {
+        "workload": (f"{wl.name}: {'KDA per-channel' if wl.gate == 'diag' else 'GDN scalar'}-gate "
+                     f"decode, batch {wl.batch} x {wl.heads} heads, d_k={wl.d_k}, d_v={wl.d_v}, "
+                     f"window W={wl.window}, r={wl.n_comp} compensators, {wl.io} q/k/v/o, "
+                     f"int8 state with per-row scales"),
+        "batch_per_gpu": wl.batch, "heads": wl.heads, "d_k": wl.d_k, "d_v": wl.d_v,
+        "window": wl.window, "n_comp": wl.n_comp, "gate": wl.gate, "io": wl.io,
+        "smoothing": bool(wl.smoothing), "state": "int8 codes + fp32 row scales",
+        "step": f"one window: {wl.window} decode launches (commit fused into the last)",
+        "tokens_per_step_per_gpu": wl.batch * wl.window,
+        "l2": "inputs larger than L2: each decode launch reads ~%.0f MB vs 126 MB L2" % (
+            wl.batch * wl.heads * decode_launch_bytes(wl.d_k, wl.d_v, wl.n_comp, wl.gate,
+                                                      2 if wl.io == "bf16" else 4, 1, False) / 1e6),
+        "graph": not args.no_graph,
+    }
+
+
+def run_lq(args, wl):
+    import numpy as np
+    import torch
+
+    import linear_attention_recurrent_int8_b200 as lq
+    from linear_attention_recurrent_int8_b200 import synth
+
+    rank, world, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    group = None
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    lq.load_library()
+    cfg = lq.Config(batch=wl.batch, heads=wl.heads, d_k=wl.d_k, d_v=wl.d_v, window=wl.window,
+                    n_comp=wl.n_comp, gate=lq.LQ_GATE_DIAG if wl.gate == "diag" else lq.LQ_GATE_SCALAR,
+                    io_dtype=lq.LQ_BF16 if wl.io == "bf16" else lq.LQ_F32,
+                    smoothing=int(wl.smoothing), auto_commit=1)
+    W = wl.window
+    e = 2 if wl.io == "bf16" else 4
+    st = lq.State(cfg, dev)
+    # this rank's shard of sequences: global sequence index offset
+    b0 = rank * wl.batch
+    bs, hs = np.arange(b0, b0 + wl.batch), np.arange(wl.heads)
+    S0 = synth.torch_initial_state(wl.seed, bs, hs, wl.d_k, wl.d_v, wl.outlier_rows, wl.outlier_cols,
+                                   wl.outlier_scale, dev)
+    lq.lq_state_init(st, S0.reshape(wl.nh, wl.d_v, wl.d_k))
+    del S0
+
+    n_slots = max(1, min(args.slots, args.steps + args.warmup))
+    slots = []
+    for sidx in range(n_slots):
+        tok = synth.torch_tokens(wl.seed + rank, wl.batch, wl.heads, sidx * W, (sidx + 1) * W,
+                                 wl.d_k, wl.d_v, wl.gate, wl.io, dev)
+        per_t = []
+        for t in range(W):
+            per_t.append([tok[k][:, t:t + 1].contiguous() for k in ("q", "k", "v", "alpha", "beta")])
+        o = torch.empty((wl.batch, 1, wl.heads, wl.d_v), dtype=cfg.io_torch_dtype, device=dev)
+        slots.append((per_t, o))
+    torch.cuda.synchronize()
+
+    def run_window(slot, events=None):
+        per_t, o = slot
+        if events:
+            events[0].record()
+        for t in range(W):
+            lq.lq_decode_window(st, *per_t[t], 1, o)
+            if events:
+                events[t + 1].record()
+
+    # one eager window (also sets kernel attributes before any capture)
+    run_window(slots[0])
+    torch.cuda.synchronize()
+
+    graphs = []
+    if not args.no_graph:
+        s = torch.cuda.Stream(device=dev)
+        for slot in slots:
+            evs = [torch.cuda.Event(enable_timing=True) for _ in range(W + 1)]
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s):
+                run_window(slot, evs)
+            graphs.append((g, evs))
+        assert st.pos == 0
+    else:
+        for slot in slots:
+            graphs.append((None, [torch.cuda.Event(enable_timing=True) for _ in range(W + 1)]))
+
+    def step(i):
+        g, evs = graphs[i % len(graphs)]
+        if g is not None:
+            g.replay()
+        else:
+            run_window(slots[i % len(slots)], evs)
+
+    sampler = ClockSampler(local) if not args.no_clocks else None
+    t_warm0 = time.monotonic()
+    for i in range(args.warmup):
+        step(i)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    cur = torch.cuda.current_stream(dev)
+    t0 = time.monotonic()
+    start.record(cur)
+    for i in range(args.steps):
+        step(args.warmup + i)
+    end.record(cur)
+    torch.cuda.synchronize()
+    t1 = time.monotonic()
+    if world > 1:
+        dist.barrier()
+    if sampler:
+        sampler.stop()
+    elapsed = start.elapsed_time(end)
+    elapsed_max, value = aggregate(elapsed, wl.batch * W * args.steps, world, group)
+
+    # per-launch times from the event nodes of the last replay of each graph
+    dec_ms, com_ms, dec_bytes, com_bytes = [], [], 0.0, 0.0
+    nh = wl.nh
+    used = range(min(len(graphs), args.steps + args.warmup))
+    for gi in used:
+        evs = graphs[gi][1]
+        for t in range(W):
+            ms = evs[t].elapsed_time(evs[t + 1])
+            commit = t == W - 1
+            nbytes = nh * decode_launch_bytes(wl.d_k, wl.d_v, wl.n_comp, wl.gate, e, t + 1, commit)
+            if commit:
+                com_ms.append(ms)
+                com_bytes += nbytes
+            else:
+                dec_ms.append(ms)
+                dec_bytes += nbytes
+    peak, peak_kind = measured_peaks()
+    if dec_ms:
+        dec_avg_ms = sum(dec_ms) / len(dec_ms)
+        achieved = dec_bytes / len(dec_ms) / (dec_avg_ms / 1e3) / 1e9
+        traffic = profiled_traffic(f"decode:{wl.name}")
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": traffic,
+                "kernel": "decode_kernel (non-commit launches, window positions 1..W-1)",
+                "bytes_per_launch": dec_bytes / len(dec_ms), "avg_launch_us": dec_avg_ms * 1e3,
+                "peak_source": f"{peak_kind} hbm_gbs (copy)"}
+    else:
+        roof = None
+    extra = {}
+    if com_ms:
+        c_avg = sum(com_ms) / len(com_ms)
+        extra["commit_launch_us"] = c_avg * 1e3
+        extra["commit_launch_gbs"] = com_bytes / len(com_ms) / (c_avg / 1e3) / 1e9
+    step_bytes = nh * sum(decode_launch_bytes(wl.d_k, wl.d_v, wl.n_comp, wl.gate, e, t + 1,
+                                              t == W - 1) for t in range(W))
+    extra["step_gbs"] = step_bytes / (elapsed / args.steps / 1e3) / 1e9
+
+    # end to end through the C ABI from pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, wl, st, cfg, dev, world, group)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed_max / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic", "config": workload_config(wl, args),
+        "roofline": roof, "gpu_launches": W * args.steps,
+        "detail": extra,
+    }
+    line["config"]["parallelism"] = f"dp{world} (independent sequence shards, no collective)"
+    if e2e:
+        line["e2e"] = e2e
+    if sampler:
+        line["clocks"] = sampler.summary(t0, t1, t_warm0)
+    if rank == 0 and world == 1 and not args.no_cpu:
+        n_seq = calibrated_sample(wl, args.cpu_seconds)
+        rate, dt, cores = oracle_window_rate(wl, n_seq)
+        line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                "sample": f"{n_seq} of {wl.batch} sequences x {wl.heads} heads, one "
+                                          f"window of {W} decode tokens plus its commit ({dt:.1f} s)"}
+    if lq.lq_device_errors() != 0:
+        line["device_errors"] = True
+    if world > 1:
+        import torch.distributed as dist
+        del graphs
+        dist.destroy_process_group()
+    return line if rank == 0 else None
+
+
+def run_e2e(args, wl, st, cfg, dev, world, group):
+    import torch
+
+    import linear_attention_recurrent_int8_b200 as lq
+    from linear_attention_recurrent_int8_b200 import synth
+    W = wl.window
+    rank, _, _ = _dist()
+    tok = synth.torch_tokens(wl.seed + rank, wl.batch, wl.heads, 0, W, wl.d_k, wl.d_v, wl.gate, wl.io,
+                             dev)
+    # host layout [W][B, 1, H, ...]: each token's inputs are contiguous
+    keys = ("q", "k", "v", "alpha", "beta")
+    host = {k: tok[k].transpose(0, 1).unsqueeze(2).contiguous().cpu().pin_memory() for k in keys}
+    dbuf = {k: torch.empty_like(host[k], device=dev) for k in keys}
+    o_dev = torch.empty((W, wl.batch, 1, wl.heads, wl.d_v), dtype=cfg.io_torch_dtype, device=dev)
+    o_host = torch.empty(o_dev.shape, dtype=o_dev.dtype, pin_memory=True)
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = o_host.numel() * o_host.element_size()
+
+    def one():
+        for k in keys:
+            dbuf[k].copy_(host[k], non_blocking=True)
+        for t in range(W):
+            lq.lq_decode_window(st, *[dbuf[k][t] for k in keys], 1, o_dev[t])
+        o_host.copy_(o_dev, non_blocking=True)
+
+    for _ in range(3):
+        one()
+    torch.cuda.synchronize()
+    n = max(1, min(args.steps, args.e2e_steps))
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(n):
+        one()
+    b.record()
+    torch.cuda.synchronize()
+    ms, rate = aggregate(a.elapsed_time(b), wl.batch * W * n, world, group)
+    return {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "steps": n}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["lq", "reference"], default="lq")
+    ap.add_argument("--workload", default="gdn_256x32_d128_bf16")
+    ap.add_argument("--window", type=int, default=None, help="override W (comparators / sweep)")
+    ap.add_argument("--n-comp", type=int, default=None, help="override r")
+    ap.add_argument("--no-smoothing", action="store_true")
+    ap.add_argument("--slots", type=int, default=8, help="distinct input windows (graphs)")
+    ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--ref-seconds", type=float, default=5.0)
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)
+
+    import dataclasses
+    from linear_attention_recurrent_int8_b200 import synth
+    wl = synth.WORKLOADS[args.workload]
+    over = {}
+    if args.window is not None:
+        over["window"] = args.window
+    if args.n_comp is not None:
+        over["n_comp"] = args.n_comp
+    if args.no_smoothing:
+        over["smoothing"] = False
+    if over:
+        wl = dataclasses.replace(wl, **over)
+
+    line = run_reference(args, wl) if args.impl == "reference" else run_lq(args, wl)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,200 @@
+/*
+ * lq.h -- C ABI of liblq: int8 per-window recurrent-state decode for
+ * delta-rule linear attention (Gated DeltaNet scalar gate, Kimi-Delta-
+ * Attention per-channel gate) on NVIDIA B200 (sm_100a).
+ *
+ * The method is LeapQuant ("LeapQuant: Efficient Linear Attention with
+ * Accurate Recurrent State Quantization", Abstract and Figure 2): the int8
+ * boundary state S^_0 stays fixed for a window of W tokens, the window's
+ * updates are buffered in FP32, every output o_t = S_t q_t is computed from
+ * S^_0 plus the buffer, and at the window end the state is rebuilt, its
+ * largest rows are kept as FP32 Compensator Tokens (Figure 4), the residual is
+ * smoothed across key channels and re-quantized once to int8.
+ *
+ * Recurrence (equation 1 of the paper, whose instances are its Appendix
+ * Table 4):  S_t = S_{t-1} D_t + (v_t - S_{t-1} b_t) k~_t^T,  o_t = S_t q_t,
+ * with S in R^{d_v x d_k} (row = value channel), k~_t = beta_t k_t and
+ *   scalar gate (Gated DeltaNet, Table 4):   D_t = alpha_t I,       b_t = alpha_t k_t
+ *   diagonal gate (Kimi Delta Attention):    D_t = Diag(alpha_t),   b_t = alpha_t * k_t.
+ *
+ * Conventions of every call:
+ *  - Every pointer argument named as device memory is caller-owned CUDA
+ *    device memory (for example a torch tensor's data_ptr()).  The library
+ *    allocates no device memory and keeps no pointer after a call returns,
+ *    except the ones the caller stores in lq_state.
+ *  - Calls are asynchronous on `stream` (NULL = the legacy default stream).
+ *    They never synchronize, except lq_device_errors.
+ *  - Arguments are validated before anything is launched.  A call that
+ *    returns an error status has launched nothing and changed nothing.
+ *  - A launch failure reported by the CUDA runtime returns LQ_ERR_CUDA.
+ *  - No C++ exception crosses this boundary.
+ *  - One lq_state is used by one stream at a time.
+ *  - Layouts are row-major.  B = batch, H = heads, n = tokens of the call.
+ *      activations  q, k: [B, n, H, d_k]   v, o: [B, n, H, d_v]
+ *                   alpha: [B, n, H] (scalar gate) or [B, n, H, d_k] (diagonal)
+ *                   beta:  [B, n, H]                       (all FP32)
+ *      q, k, v, o are FP32 or BF16 (lq_config.io_dtype).
+ *  - Pointers marked (16B) must be 16-byte aligned (LQ_ERR_MISALIGNED).
+ */
+#ifndef LQ_H
+#define LQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define LQ_API __attribute__((visibility("default")))
+#else
+#define LQ_API
+#endif
+
+/* Same type as cudaStream_t, so the header needs no CUDA include. */
+typedef struct CUstream_st *lq_stream_t;
+
+typedef enum {
+    LQ_OK = 0,
+    LQ_ERR_INVALID_ARGUMENT = 1, /* null pointer, bad size or enum value    */
+    LQ_ERR_UNSUPPORTED = 2,      /* valid but not built: d_k, d_v not in {64,128} */
+    LQ_ERR_WINDOW_FULL = 3,      /* pos + n_steps > W                       */
+    LQ_ERR_WINDOW_OPEN = 4,      /* the call needs pos == 0                  */
+    LQ_ERR_MISALIGNED = 5,       /* a (16B) pointer is not 16-byte aligned   */
+    LQ_ERR_CUDA = 6              /* the CUDA runtime reported an error       */
+} lq_status;
+
+typedef enum { LQ_GATE_SCALAR = 0, LQ_GATE_DIAG = 1 } lq_gate;
+typedef enum { LQ_F32 = 0, LQ_BF16 = 1 } lq_dtype;
+
+typedef struct {
+    int32_t batch;       /* B >= 1                                          */
+    int32_t heads;       /* H >= 1                                          */
+    int32_t d_k;         /* 64 or 128                                       */
+    int32_t d_v;         /* 64 or 128                                       */
+    int32_t window;      /* W in [1, 32]: tokens per quantization window    */
+    int32_t n_comp;      /* r in [0, 16], r <= d_v: Compensator Tokens      */
+    int32_t gate;        /* lq_gate                                         */
+    int32_t io_dtype;    /* lq_dtype of q, k, v, o                          */
+    int32_t smoothing;   /* 1: residual smoothing on; 0: c == 1             */
+    int32_t auto_commit; /* 1: the decode call that fills the window also
+                            commits it, inside the same launch              */
+} lq_config;
+
+/* The quantized boundary state of every (b, h), all device memory:
+ *   codes      int8    [B*H][d_v][d_k]  (16B)  Q, residual codes in [-127,127]
+ *   row_scale  float   [B*H][d_v]       (16B)  sigma_i (0 for a zero row)
+ *   col_smooth float   [B*H][d_k]       (16B)  c_j (1 when smoothing is off)
+ *   comp_row   int32   [B*H][r]                row index of each compensator,
+ *                                              largest l2 norm first
+ *   comp_val   float   [B*H][r][d_k]    (16B)  the compensator rows (FP32)
+ * S^_0 = Diag(row_scale) codes Diag(col_smooth) + sum_c e_{comp_row[c]} comp_val[c]^T.
+ * comp_row and comp_val may be NULL when r == 0. */
+typedef struct {
+    int8_t *codes;
+    float *row_scale;
+    float *col_smooth;
+    int32_t *comp_row;
+    float *comp_val;
+} lq_snapshot;
+
+/* A decode state.  The caller fills `snap` and the three window buffers with
+ * device pointers before lq_state_init; the library fills `cfg` and `pos`.
+ *   buf_gate float [B*H][W][1 or d_k] (16B) running log gate L_t = sum log alpha
+ *   buf_k    float [B*H][W][d_k]      (16B) k~_t = beta_t k_t
+ *   buf_u    float [B*H][W][d_v]      (16B) u_t = v_t - S_{t-1} b_t
+ * `pos` counts the tokens buffered in the open window (the same for every
+ * sequence of the batch).  `impl` is reserved (NULL). */
+typedef struct {
+    lq_config cfg;
+    lq_snapshot snap;
+    float *buf_gate;
+    float *buf_k;
+    float *buf_u;
+    int32_t pos;
+    void *impl;
+} lq_state;
+
+/* Number of elements of one buffer of a state with configuration `cfg`
+ * (for sizing allocations); -1 for an invalid configuration.
+ * which: 0 codes, 1 row_scale, 2 col_smooth, 3 comp_row, 4 comp_val,
+ *        5 buf_gate, 6 buf_k, 7 buf_u. */
+LQ_API int64_t lq_buffer_elems(const lq_config *cfg, int32_t which);
+
+/* Initialises `st` with configuration `cfg` and quantizes the FP32 state
+ * S_init [B*H][d_v][d_k] (device, (16B)) into st->snap: compensator
+ * selection, residual smoothing, per-row int8 codes (the commit quantizer).
+ * S_init == NULL means the zero state.  Sets pos = 0. */
+LQ_API lq_status lq_state_init(lq_state *st, const lq_config *cfg, const float *S_init,
+                        lq_stream_t stream);
+
+/* Decodes n_steps tokens (window positions pos+1 .. pos+n_steps) for every
+ * sequence and head: for each token, u_t = v_t - S_{t-1} b_t and
+ * o_t = S_t q_t computed from the fixed int8 boundary state plus the buffered
+ * FP32 records ("LeapQuant: ...", Figure 2), and the record (L_t, k~_t, u_t)
+ * is appended.  All n_steps tokens run inside one launch.
+ * Requires 0 <= n_steps and pos + n_steps <= W (else LQ_ERR_WINDOW_FULL);
+ * n_steps == 0 is a no-op.  When cfg.auto_commit is set and the window
+ * becomes full, the same launch commits it (see lq_window_commit) and pos
+ * returns to 0; otherwise pos += n_steps. */
+LQ_API lq_status lq_decode_window(lq_state *st, const void *q, const void *k, const void *v,
+                           const float *alpha, const float *beta, int32_t n_steps,
+                           void *o, lq_stream_t stream);
+
+/* Window commit ("LeapQuant: ...", Figures 2 and 4): rebuilds the FP32
+ * state S_pos = S^_0 D_{1..pos} + sum_m u_m (D_{m+1..pos} k~_m)^T, keeps its
+ * r largest-norm rows as Compensator Tokens, smooths the residual across key
+ * channels and re-quantizes it to int8 into st->snap; pos returns to 0.
+ * A no-op when pos == 0. */
+LQ_API lq_status lq_window_commit(lq_state *st, lq_stream_t stream);
+
+/* Prefill of T tokens from the FP32 state S_fp32 [B*H][d_v][d_k] (device,
+ * (16B), in/out: the caller passes zeros for a fresh prompt; on return it
+ * holds the state after the T tokens).  Outputs o [B, T, H, d_v].  After
+ * every `snapshot_every` tokens the FP32 state is quantized (commit
+ * quantizer) into snaps[i] (host array of T / snapshot_every snapshots
+ * holding device pointers; may be NULL), one state per that many cached
+ * tokens ("LeapQuant: ...", Figure 1(b)).  On return st->snap holds the
+ * quantized state after T tokens, ready for decode.  The FP32 state is
+ * carried across snapshots unquantized.
+ * Requires pos == 0 (else LQ_ERR_WINDOW_OPEN), T >= 0, snapshot_every >= 1
+ * and, when snaps != NULL, T % snapshot_every == 0.  T == 0 is a no-op. */
+LQ_API lq_status lq_prefill_chunk(lq_state *st, float *S_fp32, const void *q, const void *k,
+                           const void *v, const float *alpha, const float *beta,
+                           int32_t T, int32_t snapshot_every, const lq_snapshot *snaps,
+                           void *o, lq_stream_t stream);
+
+/* Copies the committed boundary state into `dst` (device buffers of the same
+ * sizes): a prefix-cache snapshot.  Requires pos == 0 (LQ_ERR_WINDOW_OPEN). */
+LQ_API lq_status lq_state_snapshot(const lq_state *st, const lq_snapshot *dst, lq_stream_t stream);
+
+/* Copies a snapshot back into st->snap and sets pos = 0 (resume from a
+ * prefix-cache snapshot).  Requires pos == 0 (LQ_ERR_WINDOW_OPEN). */
+LQ_API lq_status lq_state_restore(lq_state *st, const lq_snapshot *src, lq_stream_t stream);
+
+/* Comparator (not LeapQuant): n_steps of the recurrence on an FP32 state
+ * S [B*H][d_v][d_k] (device, (16B), in/out) that is read and written every
+ * step -- the FP32 per-step baseline of the paper's Table 2.  Uses cfg's
+ * batch, heads, d_k, d_v, gate and io_dtype; inputs as lq_decode_window. */
+LQ_API lq_status lq_fp32_step(const lq_config *cfg, float *S, const void *q, const void *k,
+                       const void *v, const float *alpha, const float *beta,
+                       int32_t n_steps, void *o, lq_stream_t stream);
+
+/* Releases host resources of `st` (none today); device buffers stay the
+ * caller's. */
+LQ_API void lq_state_destroy(lq_state *st);
+
+/* Static string naming a status. */
+LQ_API const char *lq_status_string(lq_status s);
+
+/* Reads and clears the library's device error word (synchronizes the
+ * device).  Bit 0: a kernel gave up waiting for its own asynchronous copies
+ * (bounded wait expired); the affected outputs are not valid. */
+LQ_API lq_status lq_device_errors(uint32_t *flags);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LQ_H */

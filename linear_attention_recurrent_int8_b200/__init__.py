@@ -1,0 +1,270 @@
+"""Python binding of liblq (include/lq.h): int8 per-window recurrent-state
+decode for delta-rule linear attention on NVIDIA B200.
+
+This module only marshals arguments: torch tensors become device pointers,
+torch streams become ``cudaStream_t``.  Every step of the computation runs in
+the CUDA kernels of ``liblq.so``; there is no CPU or PyTorch fallback, and a
+missing or unloadable library raises.
+
+The functions carry the C names (``lq_state_init``, ``lq_decode_window``,
+``lq_window_commit``, ``lq_prefill_chunk``, ``lq_state_snapshot``,
+``lq_state_restore``, ``lq_fp32_step``, ...).  ``State`` and ``Snapshot`` own
+the torch tensors whose pointers the C structs hold.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from dataclasses import dataclass
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "liblq.so")
+
+LQ_OK, LQ_ERR_INVALID_ARGUMENT, LQ_ERR_UNSUPPORTED, LQ_ERR_WINDOW_FULL, \
+    LQ_ERR_WINDOW_OPEN, LQ_ERR_MISALIGNED, LQ_ERR_CUDA = range(7)
+LQ_GATE_SCALAR, LQ_GATE_DIAG = 0, 1
+LQ_F32, LQ_BF16 = 0, 1
+
+# Every symbol include/lq.h declares.
+ABI_SYMBOLS = ("lq_buffer_elems", "lq_state_init", "lq_decode_window", "lq_window_commit",
+               "lq_prefill_chunk", "lq_state_snapshot", "lq_state_restore", "lq_fp32_step",
+               "lq_state_destroy", "lq_status_string", "lq_device_errors")
+
+
+class LQError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {status_name(status)}")
+        self.status = status
+
+
+class LqConfig(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("batch", "heads", "d_k", "d_v", "window", "n_comp",
+                                              "gate", "io_dtype", "smoothing", "auto_commit")]
+
+
+class LqSnapshot(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("row_scale", ctypes.c_void_p),
+                ("col_smooth", ctypes.c_void_p), ("comp_row", ctypes.c_void_p),
+                ("comp_val", ctypes.c_void_p)]
+
+
+class LqState(ctypes.Structure):
+    _fields_ = [("cfg", LqConfig), ("snap", LqSnapshot), ("buf_gate", ctypes.c_void_p),
+                ("buf_k", ctypes.c_void_p), ("buf_u", ctypes.c_void_p), ("pos", ctypes.c_int32),
+                ("impl", ctypes.c_void_p)]
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def load_library(build: bool = True):
+    """Loads liblq.so, compiling it first when it is missing or stale."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if build:
+                from .build import build_library
+                build_library()
+            if not os.path.exists(LIB_PATH):
+                raise ImportError(f"liblq.so not found at {LIB_PATH}")
+            lib = ctypes.CDLL(LIB_PATH)
+            P, I32 = ctypes.c_void_p, ctypes.c_int32
+            sig = {
+                "lq_buffer_elems": (ctypes.c_int64, [ctypes.POINTER(LqConfig), I32]),
+                "lq_state_init": (I32, [ctypes.POINTER(LqState), ctypes.POINTER(LqConfig), P, P]),
+                "lq_decode_window": (I32, [ctypes.POINTER(LqState), P, P, P, P, P, I32, P, P]),
+                "lq_window_commit": (I32, [ctypes.POINTER(LqState), P]),
+                "lq_prefill_chunk": (I32, [ctypes.POINTER(LqState), P, P, P, P, P, P, I32, I32,
+                                           ctypes.POINTER(LqSnapshot), P, P]),
+                "lq_state_snapshot": (I32, [ctypes.POINTER(LqState), ctypes.POINTER(LqSnapshot), P]),
+                "lq_state_restore": (I32, [ctypes.POINTER(LqState), ctypes.POINTER(LqSnapshot), P]),
+                "lq_fp32_step": (I32, [ctypes.POINTER(LqConfig), P, P, P, P, P, P, I32, P, P]),
+                "lq_state_destroy": (None, [ctypes.POINTER(LqState)]),
+                "lq_status_string": (ctypes.c_char_p, [I32]),
+                "lq_device_errors": (I32, [ctypes.POINTER(ctypes.c_uint32)]),
+            }
+            for name, (res, args) in sig.items():
+                f = getattr(lib, name)
+                f.restype = res
+                f.argtypes = args
+            _lib = lib
+    return _lib
+
+
+def status_name(status: int) -> str:
+    return lq_status_string(status)
+
+
+def _check(status: int, where: str):
+    if status != LQ_OK:
+        raise LQError(status, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+# --------------------------------------------------------------------------
+# Configuration, snapshot and state holders
+# --------------------------------------------------------------------------
+
+@dataclass
+class Config:
+    batch: int
+    heads: int
+    d_k: int = 128
+    d_v: int = 128
+    window: int = 16
+    n_comp: int = 4
+    gate: int = LQ_GATE_SCALAR
+    io_dtype: int = LQ_BF16
+    smoothing: int = 1
+    auto_commit: int = 1
+
+    def c(self) -> LqConfig:
+        return LqConfig(self.batch, self.heads, self.d_k, self.d_v, self.window, self.n_comp,
+                        self.gate, self.io_dtype, self.smoothing, self.auto_commit)
+
+    @property
+    def gdim(self) -> int:
+        return self.d_k if self.gate == LQ_GATE_DIAG else 1
+
+    @property
+    def io_torch_dtype(self):
+        import torch
+        return torch.bfloat16 if self.io_dtype == LQ_BF16 else torch.float32
+
+
+class Snapshot:
+    """Device tensors of one quantized boundary state (layouts of lq_snapshot)."""
+
+    def __init__(self, cfg: Config, device, tensors: dict | None = None):
+        import torch
+        bh = cfg.batch * cfg.heads
+        if tensors is None:
+            tensors = dict(
+                codes=torch.zeros((bh, cfg.d_v, cfg.d_k), dtype=torch.int8, device=device),
+                row_scale=torch.zeros((bh, cfg.d_v), dtype=torch.float32, device=device),
+                col_smooth=torch.ones((bh, cfg.d_k), dtype=torch.float32, device=device),
+                comp_row=torch.zeros((bh, cfg.n_comp), dtype=torch.int32, device=device),
+                comp_val=torch.zeros((bh, cfg.n_comp, cfg.d_k), dtype=torch.float32, device=device),
+            )
+        self.t = tensors
+
+    def __getitem__(self, key):
+        return self.t[key]
+
+    def c(self) -> LqSnapshot:
+        t = self.t
+        has = t["comp_row"].numel() > 0
+        return LqSnapshot(t["codes"].data_ptr(), t["row_scale"].data_ptr(),
+                          t["col_smooth"].data_ptr(),
+                          t["comp_row"].data_ptr() if has else None,
+                          t["comp_val"].data_ptr() if has else None)
+
+    def cpu(self) -> dict:
+        return {k: v.cpu().numpy() for k, v in self.t.items()}
+
+
+class State:
+    """A decode state: the boundary snapshot plus the window buffers, all
+    device memory allocated here by torch, and the C struct pointing at them."""
+
+    def __init__(self, cfg: Config, device="cuda"):
+        import torch
+        self.cfg = cfg
+        self.device = torch.device(device)
+        bh = cfg.batch * cfg.heads
+        self.snap = Snapshot(cfg, self.device)
+        self.buf_gate = torch.zeros((bh, cfg.window, cfg.gdim), dtype=torch.float32, device=device)
+        self.buf_k = torch.zeros((bh, cfg.window, cfg.d_k), dtype=torch.float32, device=device)
+        self.buf_u = torch.zeros((bh, cfg.window, cfg.d_v), dtype=torch.float32, device=device)
+        self.c = LqState()
+        self.c.cfg = cfg.c()
+        self.c.snap = self.snap.c()
+        self.c.buf_gate = self.buf_gate.data_ptr()
+        self.c.buf_k = self.buf_k.data_ptr()
+        self.c.buf_u = self.buf_u.data_ptr()
+        self.c.pos = 0
+        self.c.impl = None
+
+    @property
+    def pos(self) -> int:
+        return self.c.pos
+
+
+# --------------------------------------------------------------------------
+# The C entry points, same names
+# --------------------------------------------------------------------------
+
+def lq_status_string(status: int) -> str:
+    return load_library().lq_status_string(int(status)).decode()
+
+
+def lq_buffer_elems(cfg: Config, which: int) -> int:
+    c = cfg.c()
+    return load_library().lq_buffer_elems(ctypes.byref(c), which)
+
+
+def lq_state_init(st: State, S_init=None, stream=None) -> None:
+    c = st.cfg.c()
+    _check(load_library().lq_state_init(ctypes.byref(st.c), ctypes.byref(c), _ptr(S_init),
+                                        _stream(stream)), "lq_state_init")
+
+
+def lq_decode_window(st: State, q, k, v, alpha, beta, n_steps: int, o, stream=None) -> None:
+    _check(load_library().lq_decode_window(ctypes.byref(st.c), _ptr(q), _ptr(k), _ptr(v),
+                                           _ptr(alpha), _ptr(beta), int(n_steps), _ptr(o),
+                                           _stream(stream)), "lq_decode_window")
+
+
+def lq_window_commit(st: State, stream=None) -> None:
+    _check(load_library().lq_window_commit(ctypes.byref(st.c), _stream(stream)), "lq_window_commit")
+
+
+def lq_prefill_chunk(st: State, S_fp32, q, k, v, alpha, beta, T: int, snapshot_every: int,
+                     snaps, o, stream=None) -> None:
+    arr = None
+    if snaps is not None:
+        arr = (LqSnapshot * len(snaps))(*[s.c() for s in snaps])
+    _check(load_library().lq_prefill_chunk(ctypes.byref(st.c), _ptr(S_fp32), _ptr(q), _ptr(k),
+                                           _ptr(v), _ptr(alpha), _ptr(beta), int(T),
+                                           int(snapshot_every), arr, _ptr(o), _stream(stream)),
+           "lq_prefill_chunk")
+
+
+def lq_state_snapshot(st: State, dst: Snapshot, stream=None) -> None:
+    c = dst.c()
+    _check(load_library().lq_state_snapshot(ctypes.byref(st.c), ctypes.byref(c), _stream(stream)),
+           "lq_state_snapshot")
+
+
+def lq_state_restore(st: State, src: Snapshot, stream=None) -> None:
+    c = src.c()
+    _check(load_library().lq_state_restore(ctypes.byref(st.c), ctypes.byref(c), _stream(stream)),
+           "lq_state_restore")
+
+
+def lq_fp32_step(cfg: Config, S, q, k, v, alpha, beta, n_steps: int, o, stream=None) -> None:
+    c = cfg.c()
+    _check(load_library().lq_fp32_step(ctypes.byref(c), _ptr(S), _ptr(q), _ptr(k), _ptr(v),
+                                       _ptr(alpha), _ptr(beta), int(n_steps), _ptr(o),
+                                       _stream(stream)), "lq_fp32_step")
+
+
+def lq_state_destroy(st: State) -> None:
+    load_library().lq_state_destroy(ctypes.byref(st.c))
+
+
+def lq_device_errors() -> int:
+    flags = ctypes.c_uint32(0)
+    _check(load_library().lq_device_errors(ctypes.byref(flags)), "lq_device_errors")
+    return flags.value

@@ -1,0 +1,319 @@
+// lq_api.cu -- the C ABI of liblq (declared in include/lq.h): argument
+// validation, status codes and kernel dispatch.  Every entry point validates
+// all of its arguments before it launches anything, so a call that returns an
+// error has no side effect.  No exception crosses the ABI.
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/lq.h"
+#include "lq_kernels.h"
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool aligned_to(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+lq_status check_config(const lq_config *c) {
+    if (!c) return LQ_ERR_INVALID_ARGUMENT;
+    if (c->batch < 1 || c->heads < 1) return LQ_ERR_INVALID_ARGUMENT;
+    if ((int64_t)c->batch * c->heads > 0x7fffffffLL) return LQ_ERR_INVALID_ARGUMENT;
+    if (c->d_k < 1 || c->d_v < 1) return LQ_ERR_INVALID_ARGUMENT;
+    if ((c->d_k != 64 && c->d_k != 128) || (c->d_v != 64 && c->d_v != 128))
+        return LQ_ERR_UNSUPPORTED;
+    if (c->window < 1 || c->window > 32) return LQ_ERR_INVALID_ARGUMENT;
+    if (c->n_comp < 0 || c->n_comp > 16 || c->n_comp > c->d_v) return LQ_ERR_INVALID_ARGUMENT;
+    if (c->gate != LQ_GATE_SCALAR && c->gate != LQ_GATE_DIAG) return LQ_ERR_INVALID_ARGUMENT;
+    if (c->io_dtype != LQ_F32 && c->io_dtype != LQ_BF16) return LQ_ERR_INVALID_ARGUMENT;
+    if ((c->smoothing != 0 && c->smoothing != 1) || (c->auto_commit != 0 && c->auto_commit != 1))
+        return LQ_ERR_INVALID_ARGUMENT;
+    return LQ_OK;
+}
+
+lq_status check_snapshot(const lq_config *c, const lq_snapshot *s) {
+    if (!s || !s->codes || !s->row_scale || !s->col_smooth) return LQ_ERR_INVALID_ARGUMENT;
+    if (c->n_comp > 0 && (!s->comp_row || !s->comp_val)) return LQ_ERR_INVALID_ARGUMENT;
+    if (!aligned16(s->codes) || !aligned16(s->row_scale) || !aligned16(s->col_smooth))
+        return LQ_ERR_MISALIGNED;
+    if (c->n_comp > 0 && (!aligned16(s->comp_val) || !aligned_to(s->comp_row, 4)))
+        return LQ_ERR_MISALIGNED;
+    return LQ_OK;
+}
+
+lq_status check_state(const lq_state *st) {
+    if (!st) return LQ_ERR_INVALID_ARGUMENT;
+    lq_status e = check_config(&st->cfg);
+    if (e != LQ_OK) return e;
+    e = check_snapshot(&st->cfg, &st->snap);
+    if (e != LQ_OK) return e;
+    if (!st->buf_gate || !st->buf_k || !st->buf_u) return LQ_ERR_INVALID_ARGUMENT;
+    if (!aligned16(st->buf_gate) || !aligned16(st->buf_k) || !aligned16(st->buf_u))
+        return LQ_ERR_MISALIGNED;
+    if (st->pos < 0 || st->pos > st->cfg.window) return LQ_ERR_INVALID_ARGUMENT;
+    return LQ_OK;
+}
+
+lq_status check_tokens(const lq_config *c, const void *q, const void *k, const void *v,
+                       const float *alpha, const float *beta, const void *o) {
+    if (!q || !k || !v || !alpha || !beta || !o) return LQ_ERR_INVALID_ARGUMENT;
+    const size_t es = c->io_dtype == LQ_BF16 ? 2 : 4;
+    if (!aligned_to(q, es) || !aligned_to(k, es) || !aligned_to(v, es) || !aligned_to(o, es) ||
+        !aligned_to(alpha, 4) || !aligned_to(beta, 4))
+        return LQ_ERR_MISALIGNED;
+    return LQ_OK;
+}
+
+lq::DecodeArgs decode_args(const lq_state *st) {
+    lq::DecodeArgs a{};
+    a.codes = st->snap.codes;
+    a.row_scale = st->snap.row_scale;
+    a.col_smooth = st->snap.col_smooth;
+    a.comp_row = st->cfg.n_comp > 0 ? st->snap.comp_row : nullptr;
+    a.comp_val = st->cfg.n_comp > 0 ? st->snap.comp_val : nullptr;
+    a.buf_gate = st->buf_gate;
+    a.buf_k = st->buf_k;
+    a.buf_u = st->buf_u;
+    a.B = st->cfg.batch;
+    a.H = st->cfg.heads;
+    a.W = st->cfg.window;
+    a.R = st->cfg.n_comp;
+    a.pos = st->pos;
+    a.smoothing = st->cfg.smoothing;
+    return a;
+}
+
+lq::QuantArgs quant_args(const lq_config *c, const float *S, const lq_snapshot *s) {
+    lq::QuantArgs a{};
+    a.S = S;
+    a.codes = s->codes;
+    a.row_scale = s->row_scale;
+    a.col_smooth = s->col_smooth;
+    a.comp_row = c->n_comp > 0 ? s->comp_row : nullptr;
+    a.comp_val = c->n_comp > 0 ? s->comp_val : nullptr;
+    a.BH = c->batch * c->heads;
+    a.R = c->n_comp;
+    a.smoothing = c->smoothing;
+    return a;
+}
+
+lq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? LQ_OK : LQ_ERR_CUDA; }
+
+lq_status copy_snapshot(const lq_config *c, const lq_snapshot *dst, const lq_snapshot *src,
+                        cudaStream_t stream) {
+    const size_t bh = (size_t)c->batch * c->heads;
+    const cudaMemcpyKind kind = cudaMemcpyDeviceToDevice;
+    cudaError_t e = cudaMemcpyAsync(dst->codes, src->codes, bh * c->d_v * c->d_k, kind, stream);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(dst->row_scale, src->row_scale, bh * c->d_v * 4, kind, stream);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(dst->col_smooth, src->col_smooth, bh * c->d_k * 4, kind, stream);
+    if (e == cudaSuccess && c->n_comp > 0)
+        e = cudaMemcpyAsync(dst->comp_row, src->comp_row, bh * c->n_comp * 4, kind, stream);
+    if (e == cudaSuccess && c->n_comp > 0)
+        e = cudaMemcpyAsync(dst->comp_val, src->comp_val, bh * c->n_comp * c->d_k * 4, kind,
+                            stream);
+    return cuda_status(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+int64_t lq_buffer_elems(const lq_config *cfg, int32_t which) {
+    if (check_config(cfg) != LQ_OK) return -1;
+    const int64_t bh = (int64_t)cfg->batch * cfg->heads;
+    const int64_t G = cfg->gate == LQ_GATE_DIAG ? cfg->d_k : 1;
+    switch (which) {
+        case 0: return bh * cfg->d_v * cfg->d_k;
+        case 1: return bh * cfg->d_v;
+        case 2: return bh * cfg->d_k;
+        case 3: return bh * cfg->n_comp;
+        case 4: return bh * cfg->n_comp * cfg->d_k;
+        case 5: return bh * cfg->window * G;
+        case 6: return bh * cfg->window * cfg->d_k;
+        case 7: return bh * cfg->window * cfg->d_v;
+        default: return -1;
+    }
+}
+
+lq_status lq_state_init(lq_state *st, const lq_config *cfg, const float *S_init,
+                        lq_stream_t stream) {
+    if (!st) return LQ_ERR_INVALID_ARGUMENT;
+    lq_status e = check_config(cfg);
+    if (e != LQ_OK) return e;
+    lq_state tmp = *st;
+    tmp.cfg = *cfg;
+    tmp.pos = 0;
+    e = check_state(&tmp);
+    if (e != LQ_OK) return e;
+    if (S_init && !aligned16(S_init)) return LQ_ERR_MISALIGNED;
+    e = cuda_status(lq::launch_quantize(quant_args(cfg, S_init, &tmp.snap), cfg->d_k, cfg->d_v,
+                                        (cudaStream_t)stream));
+    if (e != LQ_OK) return e;
+    st->cfg = *cfg;
+    st->pos = 0;
+    st->impl = nullptr;
+    return LQ_OK;
+}
+
+lq_status lq_decode_window(lq_state *st, const void *q, const void *k, const void *v,
+                           const float *alpha, const float *beta, int32_t n_steps, void *o,
+                           lq_stream_t stream) {
+    lq_status e = check_state(st);
+    if (e != LQ_OK) return e;
+    if (n_steps < 0) return LQ_ERR_INVALID_ARGUMENT;
+    if (n_steps == 0) return LQ_OK;
+    if (st->pos + n_steps > st->cfg.window) return LQ_ERR_WINDOW_FULL;
+    e = check_tokens(&st->cfg, q, k, v, alpha, beta, o);
+    if (e != LQ_OK) return e;
+    lq::DecodeArgs a = decode_args(st);
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.alpha = alpha;
+    a.beta = beta;
+    a.o = o;
+    a.n_steps = n_steps;
+    const bool commit = st->cfg.auto_commit && st->pos + n_steps == st->cfg.window;
+    e = cuda_status(lq::launch_decode(a, st->cfg.d_k, st->cfg.d_v, st->cfg.gate,
+                                      st->cfg.io_dtype == LQ_BF16, commit, (cudaStream_t)stream));
+    if (e != LQ_OK) return e;
+    st->pos = commit ? 0 : st->pos + n_steps;
+    return LQ_OK;
+}
+
+lq_status lq_window_commit(lq_state *st, lq_stream_t stream) {
+    lq_status e = check_state(st);
+    if (e != LQ_OK) return e;
+    if (st->pos == 0) return LQ_OK;
+    lq::DecodeArgs a = decode_args(st);
+    a.n_steps = 0;
+    e = cuda_status(lq::launch_decode(a, st->cfg.d_k, st->cfg.d_v, st->cfg.gate,
+                                      st->cfg.io_dtype == LQ_BF16, true, (cudaStream_t)stream));
+    if (e != LQ_OK) return e;
+    st->pos = 0;
+    return LQ_OK;
+}
+
+lq_status lq_prefill_chunk(lq_state *st, float *S_fp32, const void *q, const void *k,
+                           const void *v, const float *alpha, const float *beta, int32_t T,
+                           int32_t snapshot_every, const lq_snapshot *snaps, void *o,
+                           lq_stream_t stream) {
+    lq_status e = check_state(st);
+    if (e != LQ_OK) return e;
+    if (st->pos != 0) return LQ_ERR_WINDOW_OPEN;
+    if (T < 0 || snapshot_every < 1) return LQ_ERR_INVALID_ARGUMENT;
+    if (T == 0) return LQ_OK;
+    if (snaps && T % snapshot_every != 0) return LQ_ERR_INVALID_ARGUMENT;
+    if (!S_fp32) return LQ_ERR_INVALID_ARGUMENT;
+    if (!aligned16(S_fp32)) return LQ_ERR_MISALIGNED;
+    e = check_tokens(&st->cfg, q, k, v, alpha, beta, o);
+    if (e != LQ_OK) return e;
+    if (snaps) {
+        const int n = T / snapshot_every;
+        for (int i = 0; i < n; ++i) {
+            e = check_snapshot(&st->cfg, &snaps[i]);
+            if (e != LQ_OK) return e;
+        }
+    }
+    const lq_config *c = &st->cfg;
+    cudaStream_t s = (cudaStream_t)stream;
+    lq::RecurArgs r{};
+    r.S = S_fp32;
+    r.q = q;
+    r.k = k;
+    r.v = v;
+    r.alpha = alpha;
+    r.beta = beta;
+    r.o = o;
+    r.B = c->batch;
+    r.H = c->heads;
+    r.T_total = T;
+    for (int t0 = 0, i = 0; t0 < T; t0 += snapshot_every, ++i) {
+        r.t0 = t0;
+        r.nt = T - t0 < snapshot_every ? T - t0 : snapshot_every;
+        e = cuda_status(lq::launch_recurrence(r, c->d_k, c->d_v, c->gate, c->io_dtype == LQ_BF16,
+                                              true, s));
+        if (e != LQ_OK) return e;
+        if (snaps) {
+            e = cuda_status(lq::launch_quantize(quant_args(c, S_fp32, &snaps[i]), c->d_k, c->d_v, s));
+            if (e != LQ_OK) return e;
+        }
+    }
+    return cuda_status(lq::launch_quantize(quant_args(c, S_fp32, &st->snap), c->d_k, c->d_v, s));
+}
+
+lq_status lq_state_snapshot(const lq_state *st, const lq_snapshot *dst, lq_stream_t stream) {
+    lq_status e = check_state(st);
+    if (e != LQ_OK) return e;
+    if (st->pos != 0) return LQ_ERR_WINDOW_OPEN;
+    e = check_snapshot(&st->cfg, dst);
+    if (e != LQ_OK) return e;
+    return copy_snapshot(&st->cfg, dst, &st->snap, (cudaStream_t)stream);
+}
+
+lq_status lq_state_restore(lq_state *st, const lq_snapshot *src, lq_stream_t stream) {
+    lq_status e = check_state(st);
+    if (e != LQ_OK) return e;
+    if (st->pos != 0) return LQ_ERR_WINDOW_OPEN;
+    e = check_snapshot(&st->cfg, src);
+    if (e != LQ_OK) return e;
+    e = copy_snapshot(&st->cfg, &st->snap, src, (cudaStream_t)stream);
+    if (e == LQ_OK) st->pos = 0;
+    return e;
+}
+
+lq_status lq_fp32_step(const lq_config *cfg, float *S, const void *q, const void *k,
+                       const void *v, const float *alpha, const float *beta, int32_t n_steps,
+                       void *o, lq_stream_t stream) {
+    lq_status e = check_config(cfg);
+    if (e != LQ_OK) return e;
+    if (n_steps < 0) return LQ_ERR_INVALID_ARGUMENT;
+    if (n_steps == 0) return LQ_OK;
+    if (!S) return LQ_ERR_INVALID_ARGUMENT;
+    if (!aligned16(S)) return LQ_ERR_MISALIGNED;
+    e = check_tokens(cfg, q, k, v, alpha, beta, o);
+    if (e != LQ_OK) return e;
+    lq::RecurArgs r{};
+    r.S = S;
+    r.q = q;
+    r.k = k;
+    r.v = v;
+    r.alpha = alpha;
+    r.beta = beta;
+    r.o = o;
+    r.B = cfg->batch;
+    r.H = cfg->heads;
+    r.T_total = n_steps;
+    r.t0 = 0;
+    r.nt = n_steps;
+    return cuda_status(lq::launch_recurrence(r, cfg->d_k, cfg->d_v, cfg->gate,
+                                             cfg->io_dtype == LQ_BF16, false, (cudaStream_t)stream));
+}
+
+void lq_state_destroy(lq_state *st) {
+    if (st) st->impl = nullptr;
+}
+
+const char *lq_status_string(lq_status s) {
+    switch (s) {
+        case LQ_OK: return "LQ_OK";
+        case LQ_ERR_INVALID_ARGUMENT: return "LQ_ERR_INVALID_ARGUMENT";
+        case LQ_ERR_UNSUPPORTED: return "LQ_ERR_UNSUPPORTED";
+        case LQ_ERR_WINDOW_FULL: return "LQ_ERR_WINDOW_FULL";
+        case LQ_ERR_WINDOW_OPEN: return "LQ_ERR_WINDOW_OPEN";
+        case LQ_ERR_MISALIGNED: return "LQ_ERR_MISALIGNED";
+        case LQ_ERR_CUDA: return "LQ_ERR_CUDA";
+    }
+    return "LQ_UNKNOWN_STATUS";
+}
+
+lq_status lq_device_errors(uint32_t *flags) {
+    if (!flags) return LQ_ERR_INVALID_ARGUMENT;
+    unsigned int v = 0;
+    const cudaError_t e = lq::read_and_clear_dev_error(&v);
+    *flags = v;
+    return cuda_status(e);
+}
+
+}  // extern "C"

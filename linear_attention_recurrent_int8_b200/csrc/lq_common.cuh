@@ -1,0 +1,176 @@
+// lq_common.cuh -- device helpers shared by the liblq kernels (sm_100a).
+//
+// * 1-D bulk copies global -> shared (cp.async.bulk, the TMA's untiled form,
+//   no multicast) completing on an mbarrier, and a bounded wait on it.
+// * Warp reductions (butterfly and transposing), io conversions.
+// * The library's device error word.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace lq {
+
+// Device error word, read and cleared by lq_device_errors().
+extern __device__ unsigned int g_dev_error;
+constexpr unsigned int kErrWaitTimeout = 1u;
+
+// A bounded wait gives up after this many nanoseconds of global time.
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ unsigned long long global_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+                 : "memory");
+    // make the initialised barrier visible to the async (TMA) proxy
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile(
+        "{ .reg .b64 st; mbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1; }" ::"r"(
+            smem_u32(bar)),
+        "r"(bytes)
+        : "memory");
+}
+
+// Bulk copy of `bytes` (multiple of 16; both addresses 16-byte aligned) from
+// global to this CTA's shared memory, completing `bytes` transactions on bar.
+__device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src_gmem, uint32_t bytes,
+                                         uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, "
+        "[%3];" ::"r"(smem_u32(dst_smem)),
+        "l"(src_gmem), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, "
+        "p; }"
+        : "=r"(done)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// Waits for phase `parity` of `bar` to complete, for at most kWaitLimitNs.
+// On expiry it records kErrWaitTimeout in the device error word and returns
+// false; the caller then skips its work (its outputs are not valid).
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = global_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_ns() - t0 > kWaitLimitNs) {
+            atomicOr(&g_dev_error, kErrWaitTimeout);
+            return false;
+        }
+    }
+    return true;
+}
+
+// ---------------------------------------------------------------------------
+// Warp reductions
+// ---------------------------------------------------------------------------
+
+// Sum over aligned groups of WIDTH lanes (butterfly; every lane gets the sum).
+template <int WIDTH>
+__device__ __forceinline__ float group_sum(float x) {
+#pragma unroll
+    for (int s = WIDTH / 2; s > 0; s >>= 1) x += __shfl_xor_sync(0xffffffffu, x, s);
+    return x;
+}
+
+template <int WIDTH>
+__device__ __forceinline__ float group_max(float x) {
+#pragma unroll
+    for (int s = WIDTH / 2; s > 0; s >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, s));
+    return x;
+}
+
+// Transposing reduction: each lane holds N partial values; the N sums are
+// taken over aligned groups of WIDTH lanes.  Each halving step exchanges half
+// of the remaining values with the partner lane, so N values cost about N
+// shuffles instead of N*log2(WIDTH).  On return v[0] holds the sum of value
+// index transposed_index<N, WIDTH>(lane).
+template <int N, int S>
+__device__ __forceinline__ void transposed_sum_step(float *v, int lane) {
+    if constexpr (S > 0) {
+        if constexpr (N > 1) {
+            const bool upper = (lane & S) != 0;
+#pragma unroll
+            for (int i = 0; i < N / 2; ++i) {
+                float send = upper ? v[i] : v[i + N / 2];
+                float keep = upper ? v[i + N / 2] : v[i];
+                v[i] = keep + __shfl_xor_sync(0xffffffffu, send, S);
+            }
+            transposed_sum_step<N / 2, S / 2>(v, lane);
+        } else {
+            v[0] += __shfl_xor_sync(0xffffffffu, v[0], S);
+            transposed_sum_step<1, S / 2>(v, lane);
+        }
+    }
+}
+
+template <int N, int WIDTH>
+__device__ __forceinline__ void transposed_sum(float (&v)[N], int lane) {
+    transposed_sum_step<N, WIDTH / 2>(v, lane);
+}
+
+template <int N, int S>
+__device__ __forceinline__ int transposed_index_step(int lane) {
+    if constexpr (S > 0 && N > 1)
+        return ((lane & S) ? N / 2 : 0) + transposed_index_step<N / 2, S / 2>(lane);
+    else
+        return 0;
+}
+
+template <int N, int WIDTH>
+__device__ __forceinline__ int transposed_index(int lane) {
+    return transposed_index_step<N, WIDTH / 2>(lane);
+}
+
+// ---------------------------------------------------------------------------
+// int8 codes -> FP32, io conversions
+// ---------------------------------------------------------------------------
+
+// Four int8 codes packed in a 32-bit word -> four exact FP32 values.  Each
+// biased byte (Q + 128) is placed in the low mantissa bits of 2^23, giving
+// 2^23 + Q + 128 exactly; one subtraction recovers Q.
+__device__ __forceinline__ void codes4_to_f32(uint32_t w, float (&f)[4]) {
+    const uint32_t u = w ^ 0x80808080u;
+    f[0] = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7650)) - 8388736.0f;
+    f[1] = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7651)) - 8388736.0f;
+    f[2] = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7652)) - 8388736.0f;
+    f[3] = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7653)) - 8388736.0f;
+}
+
+template <bool BF16>
+__device__ __forceinline__ float load_io(const void *p, size_t i) {
+    if constexpr (BF16)
+        return __bfloat162float(static_cast<const __nv_bfloat16 *>(p)[i]);
+    else
+        return static_cast<const float *>(p)[i];
+}
+
+template <bool BF16>
+__device__ __forceinline__ void store_io(void *p, size_t i, float x) {
+    if constexpr (BF16)
+        static_cast<__nv_bfloat16 *>(p)[i] = __float2bfloat16_rn(x);
+    else
+        static_cast<float *>(p)[i] = x;
+}
+
+}  // namespace lq

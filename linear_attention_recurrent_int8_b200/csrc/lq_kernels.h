@@ -1,0 +1,71 @@
+// lq_kernels.h -- internal interface between the C-ABI layer (lq_api.cu) and
+// the kernel launchers.  Not installed; not part of the ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace lq {
+
+// Arguments of the decode / commit kernel (one CTA per (b, h)).
+struct DecodeArgs {
+    int8_t *codes;
+    float *row_scale;
+    float *col_smooth;
+    int32_t *comp_row;
+    float *comp_val;
+    float *buf_gate;
+    float *buf_k;
+    float *buf_u;
+    const void *q;
+    const void *k;
+    const void *v;
+    const float *alpha;
+    const float *beta;
+    void *o;
+    int B, H, W, R;
+    int pos;      // records already buffered
+    int n_steps;  // tokens decoded by this launch (0: commit only)
+    int smoothing;
+};
+
+// Arguments of the quantize-from-FP32 kernel (init, prefill snapshots).
+struct QuantArgs {
+    const float *S;  // [BH][DV][DK], nullptr = zeros
+    int8_t *codes;
+    float *row_scale;
+    float *col_smooth;
+    int32_t *comp_row;
+    float *comp_val;
+    int BH, R, smoothing;
+};
+
+// Arguments of the FP32-state recurrence kernel (prefill, FP32 per-step).
+struct RecurArgs {
+    float *S;  // [BH][DV][DK] in/out
+    const void *q;
+    const void *k;
+    const void *v;
+    const float *alpha;
+    const float *beta;
+    void *o;
+    int B, H;
+    int T_total;  // tokens in the activation tensors (time stride)
+    int t0, nt;   // tokens [t0, t0+nt) processed by this launch
+};
+
+cudaError_t launch_decode(const DecodeArgs &a, int d_k, int d_v, int gate, bool bf16, bool commit,
+                          cudaStream_t stream);
+int decode_smem_bytes(int d_k, int d_v, int gate, int R, int W);
+
+// Reads the device error word and clears it (synchronizes the device).
+cudaError_t read_and_clear_dev_error(unsigned int *out);
+
+cudaError_t launch_quantize(const QuantArgs &a, int d_k, int d_v, cudaStream_t stream);
+
+// rows_per_cta selects the parallelisation: the full head (one CTA per head,
+// for a few tokens) or a slice of rows (many CTAs per head, for long runs).
+cudaError_t launch_recurrence(const RecurArgs &a, int d_k, int d_v, int gate, bool bf16,
+                              bool long_run, cudaStream_t stream);
+
+}  // namespace lq

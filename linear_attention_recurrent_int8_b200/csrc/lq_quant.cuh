@@ -1,0 +1,183 @@
+// lq_quant.cuh -- the register tile of one head's state and the commit
+// quantizer on it: Compensator Tokens, residual smoothing, per-row int8.
+//
+// "LeapQuant: Efficient Linear Attention with Accurate Recurrent State
+// Quantization", Abstract and Figure 4: the state's largest outliers are kept
+// as a few high-precision Compensator Tokens (flattening the residual's row
+// l2 norms), the residual is smoothed across channels and quantized once to
+// 8 bits.  The pages fix neither rule; this library's rule is:
+//   C2  the r rows of largest l2 norm become compensators (largest first, an
+//       exact tie to the smaller row), stored exactly in FP32, and are zeroed
+//       in the residual R;
+//   C3  c_j = sqrt(max_i |R_ij|) (1 for a zero column or with smoothing off),
+//       R' = R / c_j;
+//   C4  sigma_i = max_j |R'_ij| / 127, Q_ij = rne(R'_ij / sigma_i) in
+//       [-127, 127], Q = 0 where sigma_i = 0.
+// Every division and square root in C3-C4 is one IEEE round-to-nearest FP32
+// operation (__fdiv_rn, __fsqrt_rn), so the codes of a given FP32 state are
+// exactly determined.
+#pragma once
+
+#include "lq_common.cuh"
+
+namespace lq {
+
+constexpr int kMaxComp = 16;
+
+// Ownership of a d_v x d_k state by a CTA of NWARPS warps.  Each lane owns 4
+// consecutive key channels (columns) of NR rows: LPR lanes cover one row, a
+// warp instruction covers RPI rows, warp w owns rows [w*RPW, (w+1)*RPW).
+template <int DK, int DV, int NWARPS>
+struct Tile {
+    static constexpr int LPR = DK / 4;
+    static constexpr int RPI = 32 / LPR;
+    static constexpr int RPW = DV / NWARPS;
+    static constexpr int NR = RPW / RPI;
+    static constexpr int NTHREADS = NWARPS * 32;
+    static_assert(DK == 64 || DK == 128, "d_k must be 64 or 128");
+    static_assert(RPW % RPI == 0 && NR >= 1, "tile does not divide the state");
+    __device__ static int col0(int lane) { return 4 * (lane % LPR); }
+    __device__ static int row(int warp, int lane, int n) {
+        return warp * RPW + n * RPI + lane / LPR;
+    }
+};
+
+// Device pointers of one head's snapshot.
+struct SnapPtr {
+    int8_t *codes;      // [DV][DK]
+    float *row_scale;   // [DV]
+    float *col_smooth;  // [DK]
+    int32_t *comp_row;  // [R]
+    float *comp_val;    // [R][DK]
+};
+
+// Shared scratch of the quantizer.
+template <int DK, int DV, int NWARPS>
+struct QuantSmem {
+    float rowss[DV];
+    int comp_idx[DV];
+    float colpart[NWARPS * Tile<DK, DV, NWARPS>::RPI][DK];
+    float cs[DK];
+    int sel[kMaxComp];
+};
+
+// C2-C4 on the register tile S (the FP32 state of one head, owned as Tile
+// describes), writing the snapshot to `out`.  All threads of the CTA call it.
+template <int DK, int DV, int NWARPS>
+__device__ __forceinline__ void quantize_tile(float (&S)[Tile<DK, DV, NWARPS>::NR][4], int R,
+                                              bool smoothing, QuantSmem<DK, DV, NWARPS> &sm,
+                                              const SnapPtr &out) {
+    using T = Tile<DK, DV, NWARPS>;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int c0 = T::col0(lane);
+    const bool lead = (lane % T::LPR) == 0;
+
+    // C2 (1/2): squared row norms (order-preserving for the selection)
+#pragma unroll
+    for (int n = 0; n < T::NR; ++n) {
+        float ss = S[n][0] * S[n][0];
+        ss = fmaf(S[n][1], S[n][1], ss);
+        ss = fmaf(S[n][2], S[n][2], ss);
+        ss = fmaf(S[n][3], S[n][3], ss);
+        ss = group_sum<T::LPR>(ss);
+        if (lead) sm.rowss[T::row(warp, lane, n)] = ss;
+    }
+    for (int i = tid; i < DV; i += T::NTHREADS) sm.comp_idx[i] = -1;
+    __syncthreads();
+
+    // C2 (2/2): warp 0 selects the R largest, ties to the smaller row
+    if (warp == 0 && R > 0) {
+        constexpr int PER = DV / 32;
+        float val[PER];
+#pragma unroll
+        for (int p = 0; p < PER; ++p) val[p] = sm.rowss[lane + 32 * p];
+        for (int c = 0; c < R; ++c) {
+            float bv = -1.0f;
+            int bi = DV;
+#pragma unroll
+            for (int p = 0; p < PER; ++p)
+                if (val[p] > bv) {
+                    bv = val[p];
+                    bi = lane + 32 * p;
+                }
+#pragma unroll
+            for (int s = 16; s > 0; s >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, bv, s);
+                const int oi = __shfl_xor_sync(0xffffffffu, bi, s);
+                if (ov > bv || (ov == bv && oi < bi)) {
+                    bv = ov;
+                    bi = oi;
+                }
+            }
+#pragma unroll
+            for (int p = 0; p < PER; ++p)
+                if (lane + 32 * p == bi) val[p] = -1.0f;
+            if (lane == 0) {
+                sm.sel[c] = bi;
+                sm.comp_idx[bi] = c;
+            }
+        }
+    }
+    __syncthreads();
+
+    // Compensator rows leave the residual, exactly
+#pragma unroll
+    for (int n = 0; n < T::NR; ++n) {
+        const int c = sm.comp_idx[T::row(warp, lane, n)];
+        if (c >= 0) {
+            *reinterpret_cast<float4 *>(out.comp_val + (size_t)c * DK + c0) =
+                make_float4(S[n][0], S[n][1], S[n][2], S[n][3]);
+            S[n][0] = S[n][1] = S[n][2] = S[n][3] = 0.0f;
+        }
+    }
+    if (tid < R) out.comp_row[tid] = sm.sel[tid];
+
+    // C3: smoothing factor per key channel
+    {
+        float cm[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int n = 0; n < T::NR; ++n)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) cm[e] = fmaxf(cm[e], fabsf(S[n][e]));
+        *reinterpret_cast<float4 *>(&sm.colpart[warp * T::RPI + lane / T::LPR][c0]) =
+            make_float4(cm[0], cm[1], cm[2], cm[3]);
+    }
+    __syncthreads();
+    for (int j = tid; j < DK; j += T::NTHREADS) {
+        float m = 0.0f;
+#pragma unroll 4
+        for (int p = 0; p < NWARPS * T::RPI; ++p) m = fmaxf(m, sm.colpart[p][j]);
+        const float c = (smoothing && m > 0.0f) ? __fsqrt_rn(m) : 1.0f;
+        sm.cs[j] = c;
+        out.col_smooth[j] = c;
+    }
+    __syncthreads();
+    float cj[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) cj[e] = sm.cs[c0 + e];
+
+    // C4: per-row scale and codes of R' = R / c
+#pragma unroll
+    for (int n = 0; n < T::NR; ++n) {
+        float mx = 0.0f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            S[n][e] = __fdiv_rn(S[n][e], cj[e]);
+            mx = fmaxf(mx, fabsf(S[n][e]));
+        }
+        mx = group_max<T::LPR>(mx);
+        const float sigma = __fdiv_rn(mx, 127.0f);
+        const int row = T::row(warp, lane, n);
+        if (lead) out.row_scale[row] = sigma;
+        uint32_t packed = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            float qv = 0.0f;
+            if (sigma > 0.0f) qv = fminf(fmaxf(rintf(__fdiv_rn(S[n][e], sigma)), -127.0f), 127.0f);
+            packed |= (static_cast<uint32_t>(static_cast<int>(qv)) & 0xFFu) << (8 * e);
+        }
+        *reinterpret_cast<uint32_t *>(out.codes + (size_t)row * DK + c0) = packed;
+    }
+}
+
+}  // namespace lq

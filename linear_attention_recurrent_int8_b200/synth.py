@@ -303,3 +303,25 @@ def torch_tokens(seed: int, batch: int, heads: int, t0: int, t1: int, d_k: int, 
     alpha = torch.sigmoid(-xa).float()
     return dict(q=q.contiguous(), k=k.contiguous(), v=v.contiguous(), alpha=alpha.contiguous(),
                 beta=beta.contiguous())
+
+
+def torch_initial_state(seed: int, batch_idx, head_idx, d_k: int, d_v: int, outlier_rows: int,
+                        outlier_cols: int, outlier_scale: float, device):
+    """Device-side counterpart of :func:`initial_state`: [nb, nh, d_v, d_k] float32."""
+    import torch
+    bs = np.asarray(batch_idx)
+    hs = np.asarray(head_idx)
+    S = torch_grid(seed, TID_S0, bs, hs, np.arange(d_v), np.arange(d_k), device)
+    S = S.permute(0, 2, 1, 3).contiguous().float()  # [nb, nh, dv, dk]
+    if outlier_rows or outlier_cols:
+        scale_r = np.ones((len(bs), len(hs), d_v), np.float32)
+        scale_c = np.ones((len(bs), len(hs), d_k), np.float32)
+        for ib, b in enumerate(bs):
+            for ih, h in enumerate(hs):
+                if outlier_rows:
+                    scale_r[ib, ih, _pick(seed, TID_OUT_ROWS, int(b), int(h), d_v, outlier_rows)] = outlier_scale
+                if outlier_cols:
+                    scale_c[ib, ih, _pick(seed, TID_OUT_COLS, int(b), int(h), d_k, outlier_cols)] = outlier_scale
+        S *= torch.from_numpy(scale_r).to(device)[..., :, None]
+        S *= torch.from_numpy(scale_c).to(device)[..., None, :]
+    return S

@@ -1,0 +1,226 @@
+"""Helpers for the GPU parity tests: inputs, oracle runs and comparisons.
+
+Parity is checked window by window and anchored on the ORACLE: for each
+window both sides start from the oracle's snapshot (uploaded to the device
+with lq_state_restore), decode the window's tokens from the same seeded
+inputs, and commit.  Outputs, buffered records and the next snapshot are then
+compared.  Anchoring keeps two free-running chains from drifting apart after a
+legitimate +-1 LSB code flip; no value produced by the CUDA path is ever fed
+to the oracle.
+
+Tolerances (ours, from the arithmetic):
+  outputs   l2-relative per output vector <= 1e-3 (FP32 io), 2e-2 (BF16 io)
+  codes     within +-1 LSB
+  scales, smoothing, compensators   within 1e-5 relative (compensators
+            relative to the largest magnitude of their row)
+  compensator rows  equal, except near-ties (norms within 1e-5 relative of
+            the r-th largest), where the reconstructions are compared instead.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+import linear_attention_recurrent_int8_b200 as lq
+from linear_attention_recurrent_int8_b200 import synth
+
+OUT_TOL = {"fp32": 1e-3, "bf16": 2e-2}
+SCALE_RTOL = 1e-5
+NEAR_TIE = 1e-5
+
+
+def io_dtype(io):
+    return torch.bfloat16 if io == "bf16" else torch.float32
+
+
+def make_config(wl: synth.DecodeWorkload, **over) -> lq.Config:
+    c = lq.Config(batch=wl.batch, heads=wl.heads, d_k=wl.d_k, d_v=wl.d_v, window=wl.window,
+                  n_comp=wl.n_comp, gate=lq.LQ_GATE_DIAG if wl.gate == "diag" else lq.LQ_GATE_SCALAR,
+                  io_dtype=lq.LQ_BF16 if wl.io == "bf16" else lq.LQ_F32,
+                  smoothing=int(wl.smoothing), auto_commit=1)
+    for k, v in over.items():
+        setattr(c, k, v)
+    return c
+
+
+def heads_major(x):
+    """[B, T, H, ...] -> [B*H, T, ...]"""
+    x = np.asarray(x)
+    B, T, H = x.shape[:3]
+    return np.ascontiguousarray(np.swapaxes(x, 1, 2).reshape((B * H, T) + x.shape[3:]))
+
+
+def oracle_tokens(tok: dict, gate: str):
+    """Oracle-side (d, k~, b, v, q) [nh, n, ...] from synth.tokens output."""
+    q, k, v = heads_major(tok["q"]), heads_major(tok["k"]), heads_major(tok["v"])
+    alpha, beta = heads_major(tok["alpha"]), heads_major(tok["beta"])
+    if gate == "diag":
+        d, kt, b = oracle.kda_instance(alpha, beta, k)
+    else:
+        d, kt, b = oracle.gdn_instance(alpha, beta, k)
+    return d, kt, b, v, q
+
+
+def to_device_tokens(tok: dict, io: str, device="cuda"):
+    dt = io_dtype(io)
+    out = {}
+    for key in ("q", "k", "v"):
+        out[key] = torch.from_numpy(np.ascontiguousarray(tok[key])).to(device=device, dtype=dt)
+    for key in ("alpha", "beta"):
+        out[key] = torch.from_numpy(np.ascontiguousarray(tok[key])).to(device=device,
+                                                                       dtype=torch.float32)
+    return out
+
+
+def upload_snapshot(cfg: lq.Config, snap: dict, device="cuda") -> lq.Snapshot:
+    t = dict(codes=torch.from_numpy(np.ascontiguousarray(snap["codes"])).to(device),
+             row_scale=torch.from_numpy(np.ascontiguousarray(snap["row_scale"])).to(device),
+             col_smooth=torch.from_numpy(np.ascontiguousarray(snap["col_smooth"])).to(device),
+             comp_row=torch.from_numpy(np.ascontiguousarray(snap["comp_row"], np.int32)).to(device),
+             comp_val=torch.from_numpy(np.ascontiguousarray(snap["comp_val"])).to(device))
+    return lq.Snapshot(cfg, device, t)
+
+
+def download_snapshot(st: lq.State) -> dict:
+    return {k: v.detach().cpu().numpy() for k, v in st.snap.t.items()}
+
+
+def rel_l2(a, b, axis=-1):
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    num = np.linalg.norm(a - b, axis=axis)
+    den = np.maximum(np.linalg.norm(b, axis=axis), 1e-30)
+    return num / den
+
+
+def compare_outputs(o_gpu, o_ref, io, what="outputs"):
+    r = rel_l2(o_gpu, o_ref)
+    worst = float(r.max()) if r.size else 0.0
+    assert worst <= OUT_TOL[io], f"{what}: worst l2-relative error {worst:.3e} > {OUT_TOL[io]}"
+    return worst
+
+
+def compare_snapshots(gpu: dict, ref: dict, ref_norms=None, heads=None, exact_codes=False):
+    """Compares a device snapshot with the oracle's, head by head.
+
+    Returns a dict of statistics.  ``ref_norms`` [nh, dv] (oracle row norms
+    of the state that was quantized) enables the near-tie rule."""
+    nh = ref["codes"].shape[0]
+    heads = range(nh) if heads is None else heads
+    stats = dict(code_flips=0, near_ties=0, heads=0)
+    for h in heads:
+        stats["heads"] += 1
+        rc_g = [int(x) for x in gpu["comp_row"][h]]
+        rc_r = [int(x) for x in ref["comp_row"][h]]
+        if rc_g != rc_r:
+            # several results correct: rows whose norms tie (within 1e-5) with the r-th largest
+            assert ref_norms is not None, f"head {h}: compensator rows {rc_g} != {rc_r}"
+            norms = ref_norms[h]
+            r = len(rc_r)
+            kth = np.sort(norms)[::-1][r - 1]
+            for row in set(rc_g) ^ set(rc_r):
+                assert abs(norms[row] - kth) <= NEAR_TIE * kth, \
+                    f"head {h}: compensator rows {rc_g} != {rc_r} and row {row} is not a near-tie"
+            stats["near_ties"] += 1
+            sg = oracle.dequantize({k: v[h:h + 1] for k, v in gpu.items()})[0]
+            sr = oracle.dequantize({k: v[h:h + 1] for k, v in ref.items()})[0]
+            step = (ref["row_scale"][h][:, None].astype(np.float64) * ref["col_smooth"][h][None, :]
+                    + gpu["row_scale"][h][:, None] * gpu["col_smooth"][h][None, :])
+            assert np.all(np.abs(sg - sr) <= 1.5 * step + 1e-6 * np.abs(sr).max()), \
+                f"head {h}: reconstructions differ beyond one code step"
+            continue
+        np.testing.assert_allclose(gpu["row_scale"][h], ref["row_scale"][h], rtol=SCALE_RTOL,
+                                   atol=0, err_msg=f"row_scale head {h}")
+        np.testing.assert_allclose(gpu["col_smooth"][h], ref["col_smooth"][h], rtol=SCALE_RTOL,
+                                   atol=0, err_msg=f"col_smooth head {h}")
+        if len(rc_r):
+            cv_g = gpu["comp_val"][h].astype(np.float64)
+            cv_r = ref["comp_val"][h].astype(np.float64)
+            scale = np.abs(cv_r).max(axis=1, keepdims=True)
+            assert np.all(np.abs(cv_g - cv_r) <= SCALE_RTOL * scale), f"comp_val head {h}"
+        d = np.abs(gpu["codes"][h].astype(np.int32) - ref["codes"][h].astype(np.int32))
+        if exact_codes:
+            assert d.max() == 0, f"codes differ in head {h}"
+        assert d.max() <= 1, f"codes differ by {d.max()} LSB in head {h}"
+        stats["code_flips"] += int((d > 0).sum())
+    return stats
+
+
+class AnchoredRun:
+    """Runs a workload on the device window by window, anchored on the
+    oracle, and checks every window."""
+
+    def __init__(self, wl: synth.DecodeWorkload, cfg: lq.Config | None = None,
+                 steps_per_call: int = 1, commit_mode: str = "auto", device="cuda"):
+        self.wl = wl
+        self.cfg = cfg or make_config(wl)
+        if commit_mode != "auto":
+            self.cfg.auto_commit = 0
+        self.steps_per_call = steps_per_call
+        self.commit_mode = commit_mode  # "auto" | "explicit"
+        self.device = device
+        self.st = lq.State(self.cfg, device)
+        self.bs = np.arange(wl.batch)
+        self.hs = np.arange(wl.heads)
+        self.stats = dict(windows=0, worst_out=0.0, code_flips=0, near_ties=0)
+
+    def init(self):
+        wl, cfg = self.wl, self.cfg
+        S0 = synth.initial_state(wl.seed, self.bs, self.hs, wl.d_k, wl.d_v, wl.outlier_rows,
+                                 wl.outlier_cols, wl.outlier_scale)
+        S0 = S0.reshape(wl.nh, wl.d_v, wl.d_k)
+        lq.lq_state_init(self.st, torch.from_numpy(S0).to(self.device))
+        torch.cuda.synchronize()
+        ref = oracle.quantize(S0, cfg.n_comp, bool(cfg.smoothing))
+        st = compare_snapshots(download_snapshot(self.st), ref, ref["row_norm"], exact_codes=True)
+        self.stats["near_ties"] += st["near_ties"]
+        self.snap = ref
+        return ref
+
+    def window(self, w: int, ntok: int | None = None):
+        """Runs window w (tokens w*W .. w*W+ntok-1) from the oracle's snapshot."""
+        wl, cfg = self.wl, self.cfg
+        W = cfg.window
+        ntok = W if ntok is None else ntok
+        t0 = w * W
+        lq.lq_state_restore(self.st, upload_snapshot(cfg, self.snap, self.device))
+        tok = synth.tokens(wl.seed, self.bs, self.hs, t0, t0 + ntok, wl.d_k, wl.d_v, wl.gate, wl.io)
+        dev = to_device_tokens(tok, wl.io, self.device)
+        o = torch.empty((wl.batch, ntok, wl.heads, wl.d_v), dtype=io_dtype(wl.io), device=self.device)
+        s = 0
+        while s < ntok:
+            n = min(self.steps_per_call, ntok - s)
+            sl = slice(s, s + n)
+            args = [dev[key][:, sl].contiguous() for key in ("q", "k", "v", "alpha", "beta")]
+            out = torch.empty((wl.batch, n, wl.heads, wl.d_v), dtype=io_dtype(wl.io),
+                              device=self.device)
+            lq.lq_decode_window(self.st, *args, n, out)
+            o[:, sl] = out
+            s += n
+        if self.commit_mode == "explicit" or ntok < W:
+            lq.lq_window_commit(self.st)
+        torch.cuda.synchronize()
+        assert self.st.pos == 0
+
+        d, kt, b, v, q = oracle_tokens(tok, wl.gate)
+        rec = oracle.empty_records(wl.nh, W, wl.d_k, wl.d_v, cfg.gdim)
+        o_ref = oracle.window(self.snap, rec, 0, d, kt, b, v, q)
+        new_snap, S_n = oracle.commit(self.snap, rec, ntok, cfg.n_comp, bool(cfg.smoothing))
+
+        o_gpu = heads_major(o.float().cpu().numpy())
+        worst = compare_outputs(o_gpu, o_ref, wl.io, f"outputs window {w}")
+        # buffered records (FP32) against the oracle's
+        bk = self.st.buf_k.cpu().numpy()[:, :ntok]
+        bu = self.st.buf_u.cpu().numpy()[:, :ntok]
+        bL = self.st.buf_gate.cpu().numpy()[:, :ntok]
+        assert rel_l2(bk, rec["k"][:, :ntok]).max() < 1e-6, "buffered k~ differ"
+        assert rel_l2(bu, rec["u"][:, :ntok]).max() < 1e-3, "buffered u differ"
+        np.testing.assert_allclose(bL, rec["L"][:, :ntok], rtol=1e-5, atol=1e-5)
+        st = compare_snapshots(download_snapshot(self.st), new_snap, new_snap["row_norm"])
+        self.stats["windows"] += 1
+        self.stats["worst_out"] = max(self.stats["worst_out"], worst)
+        self.stats["code_flips"] += st["code_flips"]
+        self.stats["near_ties"] += st["near_ties"]
+        self.snap = new_snap
+        return o_gpu, o_ref

@@ -1,0 +1,162 @@
+"""The C-ABI library builds, loads and exports every symbol include/lq.h
+declares; its host-side validation rejects bad arguments before any launch.
+No GPU: nothing here reaches a kernel launch."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import linear_attention_recurrent_int8_b200 as lq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lq.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"LQ_API\s+[\w\s\*]+?\b(lq_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = lq.load_library()
+    declared = _declared()
+    assert declared == sorted(lq.ABI_SYMBOLS)
+    out = subprocess.run(["nm", "-D", "--defined-only", lq.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = sorted(set(re.findall(r"\bT (lq_\w+)$", out, re.M)))
+    assert exported == declared
+    for name in declared:
+        assert getattr(lib, name) is not None
+
+
+def test_status_strings():
+    names = ["LQ_OK", "LQ_ERR_INVALID_ARGUMENT", "LQ_ERR_UNSUPPORTED", "LQ_ERR_WINDOW_FULL",
+             "LQ_ERR_WINDOW_OPEN", "LQ_ERR_MISALIGNED", "LQ_ERR_CUDA"]
+    for i, n in enumerate(names):
+        assert lq.lq_status_string(i) == n
+    assert lq.lq_status_string(99) == "LQ_UNKNOWN_STATUS"
+
+
+def test_buffer_elems():
+    cfg = lq.Config(batch=3, heads=5, d_k=128, d_v=64, window=16, n_comp=4,
+                    gate=lq.LQ_GATE_DIAG)
+    bh = 15
+    want = [bh * 64 * 128, bh * 64, bh * 128, bh * 4, bh * 4 * 128, bh * 16 * 128,
+            bh * 16 * 128, bh * 16 * 64]
+    assert [lq.lq_buffer_elems(cfg, w) for w in range(8)] == want
+    assert lq.lq_buffer_elems(cfg, 8) == -1
+    cfg.gate = lq.LQ_GATE_SCALAR
+    assert lq.lq_buffer_elems(cfg, 5) == bh * 16
+    cfg.d_k = 96
+    assert lq.lq_buffer_elems(cfg, 0) == -1
+
+
+class _Buf:
+    """A fake aligned 'device' address; validation never dereferences it."""
+
+    def __init__(self, addr):
+        self.addr = addr
+
+    def data_ptr(self):
+        return self.addr
+
+
+def _fake_state(cfg, pos=0, base=0x10000000):
+    st = lq.LqState()
+    st.cfg = cfg.c()
+    a = [base + 0x100000 * i for i in range(8)]
+    st.snap = lq.LqSnapshot(a[0], a[1], a[2], a[3], a[4])
+    st.buf_gate, st.buf_k, st.buf_u = a[5], a[6], a[7]
+    st.pos = pos
+    st.impl = None
+    return st
+
+
+def _decode(st, n, q=0x20000000, o=0x21000000, stream=None):
+    lib = lq.load_library()
+    return lib.lq_decode_window(ctypes.byref(st), q, q + 0x100000, q + 0x200000, q + 0x300000,
+                                q + 0x400000, n, o, stream)
+
+
+def test_decode_validation_without_launch():
+    lib = lq.load_library()
+    cfg = lq.Config(batch=2, heads=3, window=4, n_comp=2)
+    assert lib.lq_decode_window(None, None, None, None, None, None, 1, None, None) == \
+        lq.LQ_ERR_INVALID_ARGUMENT
+    # window full: pos + n > W
+    assert _decode(_fake_state(cfg, pos=3), 2) == lq.LQ_ERR_WINDOW_FULL
+    # n_steps == 0 is a no-op, n_steps < 0 invalid
+    assert _decode(_fake_state(cfg, pos=4), 0) == lq.LQ_OK
+    assert _decode(_fake_state(cfg), -1) == lq.LQ_ERR_INVALID_ARGUMENT
+    # null inputs
+    st = _fake_state(cfg)
+    assert lib.lq_decode_window(ctypes.byref(st), None, 1, 1, 1, 1, 1, 1, None) == \
+        lq.LQ_ERR_INVALID_ARGUMENT
+    # misaligned state buffer
+    st = _fake_state(cfg)
+    st.buf_k = st.buf_k + 4
+    assert _decode(st, 1) == lq.LQ_ERR_MISALIGNED
+    # misaligned bf16 activation (odd address)
+    assert _decode(_fake_state(cfg), 1, q=0x20000001) == lq.LQ_ERR_MISALIGNED
+    # unsupported head size, bad window, too many compensators
+    for field, val, want in (("d_k", 96, lq.LQ_ERR_UNSUPPORTED), ("window", 33, lq.LQ_ERR_INVALID_ARGUMENT),
+                             ("window", 0, lq.LQ_ERR_INVALID_ARGUMENT),
+                             ("n_comp", 17, lq.LQ_ERR_INVALID_ARGUMENT),
+                             ("gate", 2, lq.LQ_ERR_INVALID_ARGUMENT),
+                             ("batch", 0, lq.LQ_ERR_INVALID_ARGUMENT)):
+        c2 = lq.Config(batch=2, heads=3, window=4, n_comp=2)
+        setattr(c2, field, val)
+        assert _decode(_fake_state(c2), 1) == want, field
+    # compensator pointers may be null only when n_comp == 0
+    st = _fake_state(cfg)
+    st.snap.comp_val = None
+    assert _decode(st, 1) == lq.LQ_ERR_INVALID_ARGUMENT
+
+
+def test_commit_snapshot_prefill_validation_without_launch():
+    lib = lq.load_library()
+    cfg = lq.Config(batch=1, heads=2, window=8, n_comp=1)
+    # commit at pos == 0 is a no-op
+    assert lib.lq_window_commit(ctypes.byref(_fake_state(cfg, pos=0)), None) == lq.LQ_OK
+    # snapshot / restore / prefill need a closed window
+    dst = lq.LqSnapshot(0x30000000, 0x30100000, 0x30200000, 0x30300000, 0x30400000)
+    assert lib.lq_state_snapshot(ctypes.byref(_fake_state(cfg, pos=3)), ctypes.byref(dst), None) == \
+        lq.LQ_ERR_WINDOW_OPEN
+    assert lib.lq_state_restore(ctypes.byref(_fake_state(cfg, pos=3)), ctypes.byref(dst), None) == \
+        lq.LQ_ERR_WINDOW_OPEN
+    p = 0x40000000
+    args = [p, p + 0x100000, p + 0x200000, p + 0x300000, p + 0x400000, p + 0x500000]
+    st = _fake_state(cfg, pos=2)
+    assert lib.lq_prefill_chunk(ctypes.byref(st), *args, 128, 64, None, p + 0x600000, None) == \
+        lq.LQ_ERR_WINDOW_OPEN
+    st = _fake_state(cfg)
+    assert lib.lq_prefill_chunk(ctypes.byref(st), *args, 0, 64, None, p + 0x600000, None) == lq.LQ_OK
+    assert lib.lq_prefill_chunk(ctypes.byref(st), *args, 128, 0, None, p + 0x600000, None) == \
+        lq.LQ_ERR_INVALID_ARGUMENT
+    snaps = (lq.LqSnapshot * 2)(dst, dst)
+    assert lib.lq_prefill_chunk(ctypes.byref(st), *args, 100, 64, snaps, p + 0x600000, None) == \
+        lq.LQ_ERR_INVALID_ARGUMENT
+    bad = list(args)
+    bad[0] += 4
+    assert lib.lq_prefill_chunk(ctypes.byref(st), *bad, 128, 64, None, p + 0x600000, None) == \
+        lq.LQ_ERR_MISALIGNED
+    # fp32 comparator: negative steps, null state
+    c = cfg.c()
+    assert lib.lq_fp32_step(ctypes.byref(c), None, *args[1:], 1, p, None) == lq.LQ_ERR_INVALID_ARGUMENT
+    assert lib.lq_fp32_step(ctypes.byref(c), p, *args[1:], -1, p, None) == lq.LQ_ERR_INVALID_ARGUMENT
+    assert lib.lq_fp32_step(ctypes.byref(c), p, *args[1:], 0, p, None) == lq.LQ_OK
+
+
+def test_state_init_validation_without_launch():
+    lib = lq.load_library()
+    cfg = lq.Config(batch=1, heads=1, d_v=64, d_k=64, n_comp=65)
+    st = _fake_state(lq.Config(batch=1, heads=1))
+    c = cfg.c()
+    assert lib.lq_state_init(ctypes.byref(st), ctypes.byref(c), None, None) == \
+        lq.LQ_ERR_INVALID_ARGUMENT
+    cfg.n_comp = 4
+    c = cfg.c()
+    assert lib.lq_state_init(ctypes.byref(st), ctypes.byref(c), 0x1234, None) == lq.LQ_ERR_MISALIGNED
+    assert lib.lq_state_init(None, ctypes.byref(c), None, None) == lq.LQ_ERR_INVALID_ARGUMENT
