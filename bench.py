@@ -326,7 +326,8 @@ def run_lq(args, wl):
     if not args.no_graph:
         s = torch.cuda.Stream(device=dev)
         for slot in slots:
-            evs = [torch.cuda.Event(enable_timing=True) for _ in range(W + 1)]
+            # external events become event-record nodes of the graph
+            evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(W + 1)]
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=s):
                 run_window(slot, evs)

@@ -348,10 +348,10 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeArgs a) {
 }
 
 // Opts a kernel into its largest possible dynamic shared memory (W = 32,
-// r = 16) once per device; launches then pass their actual size.
+// r = 16) once per device; launches then pass their actual size.  `done`
+// is the caller's per-kernel record of the devices already set up.
 template <typename K>
-cudaError_t opt_in_smem(K kern, int max_bytes) {
-    static std::atomic<uint64_t> done{0};
+cudaError_t opt_in_smem(K kern, int max_bytes, std::atomic<uint64_t> &done) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -368,7 +368,8 @@ cudaError_t launch_decode_t(const DecodeArgs &a, cudaStream_t stream) {
     constexpr int QB = sizeof(QuantSmem<DK, DV, kWarps>);
     const DecodeLayout L = decode_layout(DK, DV, G, a.R, a.W, QB);
     auto kern = decode_kernel<DK, DV, GATE, BF16, COMMIT>;
-    cudaError_t e = opt_in_smem(kern, decode_layout(DK, DV, G, kMaxComp, 32, QB).total);
+    static std::atomic<uint64_t> done{0};  // one per kernel instantiation
+    cudaError_t e = opt_in_smem(kern, decode_layout(DK, DV, G, kMaxComp, 32, QB).total, done);
     if (e != cudaSuccess) return e;
     kern<<<a.B * a.H, kThreads, L.total, stream>>>(a);
     return cudaGetLastError();
