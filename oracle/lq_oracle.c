@@ -124,16 +124,19 @@ void lqo_eq1_steps(int nh, int dv, int dk, int n, double *S, const double *d,
  *      R = S with those rows set to zero.
  *  C3  m_j = max_i |R_ij|;  c_j = fp32(sqrt(m_j)), or 1 when m_j = 0 or when
  *      smoothing is off (SmoothQuant-style migration with strength 1/2 along
- *      the key channels).  R'_ij = fp32(R_ij / c_j).
- *  C4  sigma_i = fp32(max_j |R'_ij| / 127);
- *      Q_ij = clamp(rne(fp32(R'_ij / sigma_i)), -127, 127), Q_i. = 0 when
- *      sigma_i = 0.  Round half to even; no zero point; -128 unused.
+ *      the key channels).  Each factor is inverted once, ic_j = fp32(1 / c_j),
+ *      and R'_ij = fp32(R_ij * ic_j).
+ *  C4  mx_i = max_j |R'_ij|;  sigma_i = fp32(mx_i / 127) (the stored scale);
+ *      is_i = fp32(127 / mx_i);  Q_ij = clamp(rne(fp32(R'_ij * is_i)), -127,
+ *      127), Q_i. = 0 when mx_i = 0.  Round half to even; no zero point;
+ *      -128 unused.
  *
- * Every division and square root above is one IEEE FP32 operation on FP32
- * operands (an FP64 operation rounded once to FP32 gives the same result), so
- * the quantization decision is taken in FP32, the precision of the stored
- * format.  The row norms (an argmax decision) are computed in FP64; when two
- * norms are within rounding of each other either selection is correct.
+ * Every division, square root and product above is one IEEE FP32 operation
+ * on FP32 operands (an FP64 operation rounded once to FP32 gives the same
+ * result), so the quantization decision is taken in FP32, the precision of
+ * the stored format.  The row norms (an argmax decision) are computed in
+ * FP64; when two norms are within rounding of each other either selection is
+ * correct.
  *
  * row_norm [nh][dv] (optional) receives n_i.                               */
 void lqo_quantize(int nh, int dv, int dk, int r, int smoothing, const float *S,
@@ -178,9 +181,11 @@ void lqo_quantize(int nh, int dv, int dk, int r, int smoothing, const float *S,
             }
             c[j] = (smoothing && m > 0.0) ? (float)sqrt(m) : 1.0f;
         }
-        for (int i = 0; i < dv; ++i)
-            for (int j = 0; j < dk; ++j)
-                R[(size_t)i * dk + j] = f32(R[(size_t)i * dk + j] / (double)c[j]);
+        for (int j = 0; j < dk; ++j) {
+            double ic = f32(1.0 / (double)c[j]);
+            for (int i = 0; i < dv; ++i)
+                R[(size_t)i * dk + j] = f32(R[(size_t)i * dk + j] * ic);
+        }
         /* C4: per-row symmetric int8. */
         for (int i = 0; i < dv; ++i) {
             double mx = 0.0;
@@ -189,11 +194,12 @@ void lqo_quantize(int nh, int dv, int dk, int r, int smoothing, const float *S,
                 if (a > mx) mx = a;
             }
             double sigma = f32(mx / 127.0);
+            double is = mx > 0.0 ? f32(127.0 / mx) : 0.0;
             row_scale[(size_t)h * dv + i] = (float)sigma;
             for (int j = 0; j < dk; ++j) {
                 double qv = 0.0;
-                if (sigma > 0.0) {
-                    qv = rint(f32(R[(size_t)i * dk + j] / sigma)); /* ties to even */
+                if (mx > 0.0) {
+                    qv = rint(f32(R[(size_t)i * dk + j] * is)); /* ties to even */
                     if (qv > 127.0) qv = 127.0;
                     if (qv < -127.0) qv = -127.0;
                 }

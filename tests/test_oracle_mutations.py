@@ -29,6 +29,8 @@ MUTATIONS = {
     "ties_to_larger_row": ("norm[i] > norm[best]", "norm[i] >= norm[best]"),
     "smoothing_without_sqrt": ("(float)sqrt(m) : 1.0f", "(float)m : 1.0f"),
     "round_half_away": ("qv = rint(f32(", "qv = round(f32("),
+    "no_inverse_scale_rounding": ("double is = mx > 0.0 ? f32(127.0 / mx) : 0.0;",
+                                  "double is = mx > 0.0 ? 127.0 / mx : 0.0;"),
     "scale_255": ("double sigma = f32(mx / 127.0);", "double sigma = f32(mx / 255.0);"),
 }
 

@@ -465,19 +465,24 @@ def test_quantizer_golden_hand_case():
 
 
 def test_quantizer_decision_is_fp32():
-    """Codes are rne of the FP32 quotient of FP32 operands: recompute the
-    decision with numpy float32 arithmetic (IEEE single) from the oracle's
-    own scales and compare bit for bit."""
-    S = _outlier_state(seed=10)
+    """Codes are rne of FP32 products of FP32 operands (inverse smoothing
+    factor and inverse scale each rounded once): recompute the decision with
+    numpy float32 arithmetic (IEEE single) and compare bit for bit."""
+    # large enough (5e5 codes) that rounding the inverse scale differently
+    # moves some quotient across a .5 boundary
+    S = _outlier_state(nh=32, dv=128, dk=128, seed=10)
     snap = oracle.quantize(S, 2)
+    one, q127 = np.float32(1), np.float32(127)
     for h in range(S.shape[0]):
         R = S[h].copy()
         R[snap["comp_row"][h]] = 0
-        Rp = R / snap["col_smooth"][h][None, :]          # float32 / float32
-        sig = (np.abs(Rp).max(axis=1) / np.float32(127)).astype(np.float32)
-        np.testing.assert_array_equal(sig, snap["row_scale"][h])
+        ic = (one / snap["col_smooth"][h]).astype(np.float32)
+        Rp = (R * ic[None, :]).astype(np.float32)
+        mx = np.abs(Rp).max(axis=1).astype(np.float32)
+        np.testing.assert_array_equal((mx / q127).astype(np.float32), snap["row_scale"][h])
         with np.errstate(divide="ignore", invalid="ignore"):
-            Q = np.where(sig[:, None] > 0, np.rint(Rp / sig[:, None]), 0)
+            inv = np.where(mx > 0, q127 / mx, np.float32(0)).astype(np.float32)
+        Q = np.where(mx[:, None] > 0, np.rint((Rp * inv[:, None]).astype(np.float32)), 0)
         np.testing.assert_array_equal(np.clip(Q, -127, 127).astype(np.int8), snap["codes"][h])
 
 
