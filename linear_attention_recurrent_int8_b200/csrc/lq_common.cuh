@@ -81,6 +81,37 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
     return true;
 }
 
+// Named barrier 1 over the first NT threads of the CTA (the consumer warps of
+// a warp-specialised kernel; barrier 0 is __syncthreads).
+template <int NT>
+__device__ __forceinline__ void consumer_sync() {
+    asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory");
+}
+
+// Same barrier, returning whether `pred` was true in any participating thread.
+template <int NT>
+__device__ __forceinline__ bool consumer_sync_or(bool pred) {
+    uint32_t out;
+    asm volatile(
+        "{ .reg .pred p, q; setp.ne.u32 p, %1, 0; bar.red.or.pred q, 1, %2, p; selp.u32 %0, 1, 0, "
+        "q; }"
+        : "=r"(out)
+        : "r"((uint32_t)pred), "n"(NT)
+        : "memory");
+    return out != 0;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("{ .reg .b64 st; mbarrier.arrive.shared::cta.b64 st, [%0]; }" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+// Orders this thread's generic-proxy shared-memory accesses before later
+// asynchronous-proxy (bulk copy) writes to the same memory.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // ---------------------------------------------------------------------------
 // Warp reductions
 // ---------------------------------------------------------------------------
@@ -127,6 +158,46 @@ __device__ __forceinline__ void transposed_sum_step(float *v, int lane) {
 template <int N, int WIDTH>
 __device__ __forceinline__ void transposed_sum(float (&v)[N], int lane) {
     transposed_sum_step<N, WIDTH / 2>(v, lane);
+}
+
+// Same as transposed_sum with max instead of sum.
+template <int N, int S>
+__device__ __forceinline__ void transposed_max_step(float *v, int lane) {
+    if constexpr (S > 0) {
+        if constexpr (N > 1) {
+            const bool upper = (lane & S) != 0;
+#pragma unroll
+            for (int i = 0; i < N / 2; ++i) {
+                float send = upper ? v[i] : v[i + N / 2];
+                float keep = upper ? v[i + N / 2] : v[i];
+                v[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, S));
+            }
+            transposed_max_step<N / 2, S / 2>(v, lane);
+        } else {
+            v[0] = fmaxf(v[0], __shfl_xor_sync(0xffffffffu, v[0], S));
+            transposed_max_step<1, S / 2>(v, lane);
+        }
+    }
+}
+
+template <int N, int WIDTH>
+__device__ __forceinline__ void transposed_max(float (&v)[N], int lane) {
+    transposed_max_step<N, WIDTH / 2>(v, lane);
+}
+
+// A lane offset (within its WIDTH-lane group) that holds value index n after
+// a transposed reduction of N values.
+template <int N, int S>
+__host__ __device__ constexpr int transposed_owner_step(int n) {
+    if constexpr (S > 0 && N > 1)
+        return (n >= N / 2 ? S : 0) + transposed_owner_step<N / 2, S / 2>(n >= N / 2 ? n - N / 2 : n);
+    else
+        return 0;
+}
+
+template <int N, int WIDTH>
+__host__ __device__ constexpr int transposed_owner(int n) {
+    return transposed_owner_step<N, WIDTH / 2>(n);
 }
 
 template <int N, int S>

@@ -10,12 +10,13 @@
 //       exact tie to the smaller row), stored exactly in FP32, and are zeroed
 //       in the residual R;
 //   C3  c_j = sqrt(max_i |R_ij|) (1 for a zero column or with smoothing off),
-//       R' = R / c_j;
-//   C4  sigma_i = max_j |R'_ij| / 127, Q_ij = rne(R'_ij / sigma_i) in
-//       [-127, 127], Q = 0 where sigma_i = 0.
-// Every division and square root in C3-C4 is one IEEE round-to-nearest FP32
-// operation (__fdiv_rn, __fsqrt_rn), so the codes of a given FP32 state are
-// exactly determined.
+//       R'_ij = R_ij * (1 / c_j);
+//   C4  mx_i = max_j |R'_ij|, sigma_i = mx_i / 127 (stored),
+//       Q_ij = rne(R'_ij * (127 / mx_i)) in [-127, 127], Q = 0 where mx_i = 0.
+// Each smoothing factor and each row is inverted once; every element then
+// costs one FP32 product per step.  Every division, square root and product
+// is one IEEE round-to-nearest FP32 operation (__fdiv_rn, __fsqrt_rn, __fmul_rn),
+// so the codes of a given FP32 state are exactly determined.
 #pragma once
 
 #include "lq_common.cuh"
@@ -51,18 +52,21 @@ struct SnapPtr {
     float *comp_val;    // [R][DK]
 };
 
-// Shared scratch of the quantizer.
+// Shared scratch of the quantizer.  colpart rows are written with 16-byte
+// vector stores, so the struct and that member are 16-byte aligned.
 template <int DK, int DV, int NWARPS>
-struct QuantSmem {
+struct alignas(16) QuantSmem {
     float rowss[DV];
     int comp_idx[DV];
-    float colpart[NWARPS * Tile<DK, DV, NWARPS>::RPI][DK];
+    alignas(16) float colpart[NWARPS * Tile<DK, DV, NWARPS>::RPI][DK];
     float cs[DK];
     int sel[kMaxComp];
 };
 
 // C2-C4 on the register tile S (the FP32 state of one head, owned as Tile
-// describes), writing the snapshot to `out`.  All threads of the CTA call it.
+// describes), writing the snapshot to `out`.  The NWARPS*32 threads that own
+// the tile (threads 0 .. NWARPS*32-1) call it; it synchronises them on named
+// barrier 1.
 template <int DK, int DV, int NWARPS>
 __device__ __forceinline__ void quantize_tile(float (&S)[Tile<DK, DV, NWARPS>::NR][4], int R,
                                               bool smoothing, QuantSmem<DK, DV, NWARPS> &sm,
@@ -70,20 +74,26 @@ __device__ __forceinline__ void quantize_tile(float (&S)[Tile<DK, DV, NWARPS>::N
     using T = Tile<DK, DV, NWARPS>;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int c0 = T::col0(lane);
-    const bool lead = (lane % T::LPR) == 0;
 
-    // C2 (1/2): squared row norms (order-preserving for the selection)
+    const int gbase = lane & ~(T::LPR - 1);  // first lane of this lane's row group
+    // C2 (1/2): squared row norms (order-preserving for the selection),
+    // reduced across the row's lanes with a transposing reduction
+    {
+        float ss[T::NR];
 #pragma unroll
-    for (int n = 0; n < T::NR; ++n) {
-        float ss = S[n][0] * S[n][0];
-        ss = fmaf(S[n][1], S[n][1], ss);
-        ss = fmaf(S[n][2], S[n][2], ss);
-        ss = fmaf(S[n][3], S[n][3], ss);
-        ss = group_sum<T::LPR>(ss);
-        if (lead) sm.rowss[T::row(warp, lane, n)] = ss;
+        for (int n = 0; n < T::NR; ++n) {
+            ss[n] = S[n][0] * S[n][0];
+            ss[n] = fmaf(S[n][1], S[n][1], ss[n]);
+            ss[n] = fmaf(S[n][2], S[n][2], ss[n]);
+            ss[n] = fmaf(S[n][3], S[n][3], ss[n]);
+        }
+        transposed_sum<T::NR, T::LPR>(ss, lane);
+        const int n = transposed_index<T::NR, T::LPR>(lane);
+        if ((lane & (T::LPR - 1)) == transposed_owner<T::NR, T::LPR>(n))
+            sm.rowss[T::row(warp, lane, n)] = ss[0];
     }
     for (int i = tid; i < DV; i += T::NTHREADS) sm.comp_idx[i] = -1;
-    __syncthreads();
+    consumer_sync<T::NTHREADS>();
 
     // C2 (2/2): warp 0 selects the R largest, ties to the smaller row
     if (warp == 0 && R > 0) {
@@ -118,7 +128,7 @@ __device__ __forceinline__ void quantize_tile(float (&S)[Tile<DK, DV, NWARPS>::N
             }
         }
     }
-    __syncthreads();
+    consumer_sync<T::NTHREADS>();
 
     // Compensator rows leave the residual, exactly
 #pragma unroll
@@ -142,38 +152,50 @@ __device__ __forceinline__ void quantize_tile(float (&S)[Tile<DK, DV, NWARPS>::N
         *reinterpret_cast<float4 *>(&sm.colpart[warp * T::RPI + lane / T::LPR][c0]) =
             make_float4(cm[0], cm[1], cm[2], cm[3]);
     }
-    __syncthreads();
+    consumer_sync<T::NTHREADS>();
     for (int j = tid; j < DK; j += T::NTHREADS) {
         float m = 0.0f;
 #pragma unroll 4
         for (int p = 0; p < NWARPS * T::RPI; ++p) m = fmaxf(m, sm.colpart[p][j]);
         const float c = (smoothing && m > 0.0f) ? __fsqrt_rn(m) : 1.0f;
-        sm.cs[j] = c;
         out.col_smooth[j] = c;
+        sm.cs[j] = __fdiv_rn(1.0f, c);  // the inverse, used below
     }
-    __syncthreads();
-    float cj[4];
+    consumer_sync<T::NTHREADS>();
+    float ic[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) cj[e] = sm.cs[c0 + e];
+    for (int e = 0; e < 4; ++e) ic[e] = sm.cs[c0 + e];
 
-    // C4: per-row scale and codes of R' = R / c
+    // C4: per-row scale and codes of R' = R * (1/c).  Row maxima are reduced
+    // with a transposing reduction; each row's scale and inverse scale are
+    // computed once, by the lane that holds the row's maximum, and broadcast.
+    float inv_own;
+    {
+        float mx[T::NR];
+#pragma unroll
+        for (int n = 0; n < T::NR; ++n) {
+            mx[n] = 0.0f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                S[n][e] = __fmul_rn(S[n][e], ic[e]);
+                mx[n] = fmaxf(mx[n], fabsf(S[n][e]));
+            }
+        }
+        transposed_max<T::NR, T::LPR>(mx, lane);
+        const int n = transposed_index<T::NR, T::LPR>(lane);
+        inv_own = mx[0] > 0.0f ? __fdiv_rn(127.0f, mx[0]) : 0.0f;
+        if ((lane & (T::LPR - 1)) == transposed_owner<T::NR, T::LPR>(n))
+            out.row_scale[T::row(warp, lane, n)] = __fdiv_rn(mx[0], 127.0f);
+    }
 #pragma unroll
     for (int n = 0; n < T::NR; ++n) {
-        float mx = 0.0f;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            S[n][e] = __fdiv_rn(S[n][e], cj[e]);
-            mx = fmaxf(mx, fabsf(S[n][e]));
-        }
-        mx = group_max<T::LPR>(mx);
-        const float sigma = __fdiv_rn(mx, 127.0f);
+        const float inv =
+            __shfl_sync(0xffffffffu, inv_own, gbase + transposed_owner<T::NR, T::LPR>(n));
         const int row = T::row(warp, lane, n);
-        if (lead) out.row_scale[row] = sigma;
         uint32_t packed = 0;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            float qv = 0.0f;
-            if (sigma > 0.0f) qv = fminf(fmaxf(rintf(__fdiv_rn(S[n][e], sigma)), -127.0f), 127.0f);
+            const float qv = fminf(fmaxf(rintf(__fmul_rn(S[n][e], inv)), -127.0f), 127.0f);
             packed |= (static_cast<uint32_t>(static_cast<int>(qv)) & 0xFFu) << (8 * e);
         }
         *reinterpret_cast<uint32_t *>(out.codes + (size_t)row * DK + c0) = packed;
