@@ -397,6 +397,12 @@ def run_lq(args, wl):
     else:
         roof = None
     extra = {}
+    # average duration of the launch at each window position (us)
+    pos_us = []
+    for t in range(W):
+        vals = [graphs[gi][1][t].elapsed_time(graphs[gi][1][t + 1]) for gi in used]
+        pos_us.append(round(1e3 * sum(vals) / len(vals), 1))
+    extra["launch_us_by_position"] = pos_us
     if com_ms:
         c_avg = sum(com_ms) / len(com_ms)
         extra["commit_launch_us"] = c_avg * 1e3

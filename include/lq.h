@@ -30,8 +30,9 @@
  *  - No C++ exception crosses this boundary.
  *  - One lq_state is used by one stream at a time.
  *  - Layouts are row-major.  B = batch, H = heads, n = tokens of the call.
- *      activations  q, k: [B, n, H, d_k]   v, o: [B, n, H, d_v]
- *                   alpha: [B, n, H] (scalar gate) or [B, n, H, d_k] (diagonal)
+ *      activations  q, k: [B, n, H, d_k] (16B)   v: [B, n, H, d_v] (16B)
+ *                   o: [B, n, H, d_v] (aligned to its element)
+ *                   alpha: [B, n, H] (scalar gate) or [B, n, H, d_k] (diagonal, (16B))
  *                   beta:  [B, n, H]                       (all FP32)
  *      q, k, v, o are FP32 or BF16 (lq_config.io_dtype).
  *  - Pointers marked (16B) must be 16-byte aligned (LQ_ERR_MISALIGNED).

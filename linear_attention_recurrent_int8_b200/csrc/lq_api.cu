@@ -56,9 +56,11 @@ lq_status check_state(const lq_state *st) {
 lq_status check_tokens(const lq_config *c, const void *q, const void *k, const void *v,
                        const float *alpha, const float *beta, const void *o) {
     if (!q || !k || !v || !alpha || !beta || !o) return LQ_ERR_INVALID_ARGUMENT;
+    // q, k, v rows (and a diagonal gate's alpha rows) are moved with 16-byte
+    // bulk copies and vector loads; o is written element by element
     const size_t es = c->io_dtype == LQ_BF16 ? 2 : 4;
-    if (!aligned_to(q, es) || !aligned_to(k, es) || !aligned_to(v, es) || !aligned_to(o, es) ||
-        !aligned_to(alpha, 4) || !aligned_to(beta, 4))
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned_to(o, es) ||
+        !aligned_to(alpha, c->gate == LQ_GATE_DIAG ? 16 : 4) || !aligned_to(beta, 4))
         return LQ_ERR_MISALIGNED;
     return LQ_OK;
 }

@@ -55,13 +55,30 @@ __device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src_gmem, u
         : "memory");
 }
 
+// 4-byte asynchronous copy global -> shared (both 4-byte aligned).
+__device__ __forceinline__ void cp_async4(void *dst_smem, const void *src_gmem) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst_smem)), "l"(src_gmem)
+                 : "memory");
+}
+
+// Makes `bar` track completion of this thread's earlier cp.async copies: its
+// pending arrival count is raised by one now and lowered when they complete.
+__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t *bar) {
+    asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Tests phase `parity` of `bar`; while it is incomplete the thread may be
+// suspended (not spinning) for up to kSuspendHintNs, and resumes as soon as
+// the phase completes.
+constexpr uint32_t kSuspendHintNs = 100000;
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     uint32_t done;
     asm volatile(
-        "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, "
-        "p; }"
+        "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3; selp.u32 %0, 1, "
+        "0, p; }"
         : "=r"(done)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "n"(kSuspendHintNs)
         : "memory");
     return done != 0;
 }
@@ -217,6 +234,12 @@ __device__ __forceinline__ int transposed_index(int lane) {
 // int8 codes -> FP32, io conversions
 // ---------------------------------------------------------------------------
 
+// Exact int -> FP32 for |a| < 2^22 on the integer/FP32 pipes: the bits of
+// 1.5 * 2^23 + a, minus 1.5 * 2^23.
+__device__ __forceinline__ float small_int_to_f32(int a) {
+    return __int_as_float(0x4B400000 + a) - 12582912.0f;
+}
+
 // Four int8 codes packed in a 32-bit word -> four exact FP32 values.  Each
 // biased byte (Q + 128) is placed in the low mantissa bits of 2^23, giving
 // 2^23 + Q + 128 exactly; one subtraction recovers Q.
@@ -228,12 +251,52 @@ __device__ __forceinline__ void codes4_to_f32(uint32_t w, float (&f)[4]) {
     f[3] = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7653)) - 8388736.0f;
 }
 
+// N consecutive floats (N = 2 or 4, address 8- or 16-byte aligned).
+template <int N>
+__device__ __forceinline__ void load_vec(float (&v)[N], const float *p) {
+    if constexpr (N == 4) {
+        const float4 x = *reinterpret_cast<const float4 *>(p);
+        v[0] = x.x, v[1] = x.y, v[2] = x.z, v[3] = x.w;
+    } else {
+        static_assert(N == 2, "vector width");
+        const float2 x = *reinterpret_cast<const float2 *>(p);
+        v[0] = x.x, v[1] = x.y;
+    }
+}
+
+template <int N>
+__device__ __forceinline__ void store_vec(float *p, const float (&v)[N]) {
+    if constexpr (N == 4) {
+        *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
+    } else {
+        static_assert(N == 2, "vector width");
+        *reinterpret_cast<float2 *>(p) = make_float2(v[0], v[1]);
+    }
+}
+
 template <bool BF16>
 __device__ __forceinline__ float load_io(const void *p, size_t i) {
     if constexpr (BF16)
         return __bfloat162float(static_cast<const __nv_bfloat16 *>(p)[i]);
     else
         return static_cast<const float *>(p)[i];
+}
+
+// N consecutive io elements starting at element i (N = 2 or 4; element
+// address aligned to N elements).
+template <bool BF16, int N>
+__device__ __forceinline__ void load_io_vec(float (&v)[N], const void *p, size_t i) {
+    if constexpr (BF16) {
+        const __nv_bfloat162 *q = reinterpret_cast<const __nv_bfloat162 *>(
+            static_cast<const __nv_bfloat16 *>(p) + i);
+#pragma unroll
+        for (int e = 0; e < N / 2; ++e) {
+            const float2 f = __bfloat1622float2(q[e]);
+            v[2 * e] = f.x, v[2 * e + 1] = f.y;
+        }
+    } else {
+        load_vec<N>(v, static_cast<const float *>(p) + i);
+    }
 }
 
 template <bool BF16>

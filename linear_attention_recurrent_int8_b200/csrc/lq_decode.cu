@@ -16,24 +16,28 @@
 // pseudo-records at window position 0 (Figure 4; they share the update path
 // of real tokens), so they enter with decay e^{L_t}.
 //
-// Kernel structure (persistent, warp-specialised):
-//  * a grid of at most (SMs x CTAs per SM) CTAs walks the (sequence, head)
-//    pairs with a grid stride;
-//  * warp 8 of each CTA is the producer: one lane streams every head's int8
-//    codes, scales, smoothing factors, compensators, buffered records and the
-//    token's q/k/v into a ring of shared-memory stages with 1-D bulk copies
-//    (no multicast), one "full" mbarrier per stage;
-//  * warps 0-7 consume: the codes are dequantized in registers and multiplied
-//    against two vectors at once (FP32 FMA), the two dot products of each row
-//    are reduced with a transposing warp reduction, then each value channel
-//    forms u_t and o_t.  The next head's scalar inputs are prefetched into
-//    registers while the current head is computed.  Consumers synchronise on
-//    named barrier 1 and release a stage through its "empty" mbarrier;
+// Kernel structure (persistent, warp-specialised, 11 warps per CTA):
+//  * the grid walks the (sequence, head) pairs with a grid stride; each head
+//    goes through a ring of shared-memory stages;
+//  * producer (warp 8, one lane): streams the head's int8 codes, scales,
+//    smoothing factors, compensators, buffered records and the first token's
+//    q/k/v into a stage with 1-D bulk copies (no multicast) -> "full";
+//  * prep A (warp 9): for every token of the call, the vectors
+//    x_k = c e^L k and x_q = c e^L q split into three int8 limbs per
+//    16-channel chunk, and k~_t . q_t -> "prepared";
+//  * prep B (warp 10): the records (L_t, k~_t) of the new tokens and every
+//    coefficient (k~_m e^{L_t-L_m}) . k_t, . q_t of the buffered records and
+//    compensators -> "prepared";
+//  * consumers (warps 0-7): warp w owns value rows [w*d_v/8, (w+1)*d_v/8).  It
+//    forms S^_0 x for its rows (dp4a of the codes with the limbs, FP32
+//    combine, transposing warp reduction), then u_t and o_t for the same rows
+//    from the coefficients and its own buffered u.  No CTA barrier is needed
+//    per head; the consumers release the stage through "empty";
 //  * when the window fills (or for a standalone commit, launched with no
 //    tokens) the consumers rebuild the FP32 state of the head in registers and
 //    re-quantize it in place (lq_quant.cuh).
 // Every wait is bounded (lq_common.cuh); a wait that expires sets the device
-// error word and the CTA stops consuming.
+// error word and the waiting warp stops.
 #include <atomic>
 #include <cstddef>
 
@@ -48,18 +52,39 @@ namespace {
 
 constexpr int kConsumerWarps = 8;
 constexpr int kConsumers = kConsumerWarps * 32;
-constexpr int kThreads = kConsumers + 32;
+constexpr int kProducerWarp = 8, kPrepAWarp = 9, kPrepBWarp = 10, kPrepBWarps = 2;
+constexpr int kPrepWarps = 1 + kPrepBWarps;
+constexpr int kThreads = (kConsumerWarps + 1 + kPrepWarps) * 32;
 constexpr int kMaxStages = 8;
 constexpr int kCoef = 32 + kMaxComp + 1;
 
 __host__ __device__ constexpr int align16(int x) { return (x + 15) & ~15; }
 
-// Byte offsets inside one stage (one head's operands).
-struct StageLayout {
-    int codes, sig, cs, compv, compr, recK, recU, recL, q, k, v, al, bytes;
+// Per-token results of the prep warps inside a stage.
+struct PrepLayout {
+    int limb, lscale, coefA, coefG, bytes;
 };
 
-__host__ __device__ inline StageLayout stage_layout(int DK, int DV, int gate, int R, int W, int e) {
+__host__ __device__ inline PrepLayout prep_layout(int DK) {
+    PrepLayout P{};
+    int o = 0;
+    P.limb = o;   o += 6 * DK;            // int8 [6][DK]: x_k limbs 0..2, x_q limbs 0..2
+    P.lscale = o; o += 16;                 // float [2]: scales of x_k, x_q
+    P.coefA = o;  o += 4 * kCoef;          // records, compensators
+    P.coefG = o;  o += 4 * kCoef;          // records, compensators, own token (k~.q)
+    P.bytes = align16(o);
+    return P;
+}
+
+// Byte offsets inside one stage (one head's operands).  `nrec` is the number
+// of record slots the stage holds (records read plus records written), `n`
+// the number of tokens of the call.
+struct StageLayout {
+    int codes, sig, cs, compv, compr, recK, recU, recL, q, k, v, al, scal, prep, bytes;
+};
+
+__host__ __device__ inline StageLayout stage_layout(int DK, int DV, int gate, int R, int nrec,
+                                                   int n, int e) {
     StageLayout L{};
     int o = 0;
     L.codes = o; o += align16(DV * DK);
@@ -67,95 +92,101 @@ __host__ __device__ inline StageLayout stage_layout(int DK, int DV, int gate, in
     L.cs = o;    o += align16(4 * DK);
     L.compv = o; o += align16(4 * R * DK);
     L.compr = o; o += align16(4 * kMaxComp);
-    L.recK = o;  o += align16(4 * W * DK);
-    L.recU = o;  o += align16(4 * W * DV);
-    L.recL = o;  o += align16(4 * W * (gate == 1 ? DK : 1));
+    L.recK = o;  o += align16(4 * nrec * DK);
+    L.recU = o;  o += align16(4 * nrec * DV);
+    L.recL = o;  o += align16(4 * nrec * (gate == 1 ? DK : 1));
     L.q = o;     o += align16(e * DK);
     L.k = o;     o += align16(e * DK);
     L.v = o;     o += align16(e * DV);
     L.al = o;    o += gate == 1 ? align16(4 * DK) : 0;
+    L.scal = o;  o += 16;                  // float: alpha (scalar gate), beta of token 0
+    L.prep = o;  o += n * prep_layout(DK).bytes;
     L.bytes = align16(o);
     return L;
 }
 
-// Per-CTA scratch shared by the consumer warps.  Members read with 16-byte
-// vector loads (xk, xq, and the quantizer's colpart) are 16-byte aligned; the
-// scratch itself starts on a 16-byte boundary after the stages.
+// Scratch of the commit (consumer warps only).
 template <int DK, int DV>
-struct alignas(16) Scratch {
-    alignas(16) float qf[DK];
-    alignas(16) float kf[DK];
-    alignas(16) float gk[DK];
-    alignas(16) float gq[DK];
-    alignas(16) float xk[DK];
-    alignas(16) float xq[DK];
-    alignas(16) float kt[DK];
-    // x_k and x_q split into three int8 limbs per 16-column chunk:
-    // x ~= s_chunk * (X0 + X1 / 2^7 + X2 / 2^14)
-    alignas(16) int8_t limb[6][DK];
-    float lscale[2][DK / 16];
-    float coefA[kCoef], coefG[kCoef];
-    float y[2 * DV];
-    float misc[4];
+struct alignas(16) CommitScratch {
+    alignas(16) float gW[DK];
+    alignas(16) float cgW[DK];
     QuantSmem<DK, DV, kConsumerWarps> quant;
 };
-using ScratchA = Scratch<128, 128>;
-using ScratchB = Scratch<64, 64>;
-using ScratchC = Scratch<64, 128>;
-using QuantA = QuantSmem<128, 128, kConsumerWarps>;
-using QuantB = QuantSmem<64, 64, kConsumerWarps>;
-static_assert(offsetof(ScratchA, xk) % 16 == 0 && offsetof(ScratchB, xq) % 16 == 0 &&
-                  offsetof(ScratchA, quant) % 16 == 0 && offsetof(ScratchC, quant) % 16 == 0 &&
-                  offsetof(QuantA, colpart) % 16 == 0 && offsetof(QuantB, colpart) % 16 == 0,
-              "vector-accessed scratch must be 16-byte aligned");
+using CommitA = CommitScratch<128, 128>;
+static_assert(offsetof(CommitA, cgW) % 16 == 0 && offsetof(CommitA, quant) % 16 == 0,
+              "vector-accessed commit scratch must be 16-byte aligned");
 
-__host__ __device__ constexpr int header_bytes() { return 2 * kMaxStages * 8; }
+__host__ __device__ constexpr int header_bytes() { return 3 * kMaxStages * 8; }
 
-// Splits x_j (held by thread j of a 16-thread chunk) into three int8 limbs
-// with a per-chunk scale s = max|x| / 127:  x ~= s (X0 + X1/2^7 + X2/2^14),
-// |error| <= s / 2^15.  Writes limb[0..2][j] and lscale[j / 16].
-template <int DKL>
-__device__ __forceinline__ void split_limbs_t(float x, int8_t (*limb)[DKL], float *lscale, int j) {
-    float m = fabsf(x);
+template <int DK, int DV, bool COMMIT>
+__host__ __device__ constexpr int scratch_bytes() {
+    return COMMIT ? (int)sizeof(CommitScratch<DK, DV>) : 0;
+}
+
+// Splits the d_k-vector x (lane l holds x_j for the CPL channels
+// j = j0 .. j0+CPL-1) into three int8 limbs with one scale
+// s = max_j |x_j| / 127:  x ~= s (X0 + X1/2^7 + X2/2^14), |error| <= s / 2^15
+// (plus FP32 rounding).  Writes limb[0..2][j] and *lscale.
+template <int CPL>
+__device__ __forceinline__ void split_limbs(const float (&x)[CPL], int8_t *limb, int DK,
+                                            float *lscale, int j0) {
+    float m = 0.0f;
 #pragma unroll
-    for (int s = 8; s > 0; s >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, s));
+    for (int e = 0; e < CPL; ++e) m = fmaxf(m, fabsf(x[e]));
+    m = group_max<32>(m);
     const float inv = m > 0.0f ? __fdiv_rn(127.0f, m) : 0.0f;
-    const float t = x * inv;
-    const float x0 = rintf(t);
-    const float r1 = (t - x0) * 128.0f;
-    const float x1 = rintf(r1);
-    const float x2 = rintf((r1 - x1) * 128.0f);
-    limb[0][j] = (int8_t)(int)x0;
-    limb[1][j] = (int8_t)(int)x1;
-    limb[2][j] = (int8_t)(int)x2;
-    if ((j & 15) == 0) lscale[j >> 4] = m * (1.0f / 127.0f);
+    uint32_t w0 = 0, w1 = 0, w2 = 0;
+#pragma unroll
+    for (int e = 0; e < CPL; ++e) {
+        const float t = x[e] * inv;
+        const float x0 = rintf(t);
+        const float r1 = (t - x0) * 128.0f;
+        const float x1 = rintf(r1);
+        const float x2 = rintf((r1 - x1) * 128.0f);
+        w0 |= (static_cast<uint32_t>(static_cast<int>(x0)) & 0xFFu) << (8 * e);
+        w1 |= (static_cast<uint32_t>(static_cast<int>(x1)) & 0xFFu) << (8 * e);
+        w2 |= (static_cast<uint32_t>(static_cast<int>(x2)) & 0xFFu) << (8 * e);
+    }
+    if constexpr (CPL == 4) {
+        *reinterpret_cast<uint32_t *>(limb + j0) = w0;
+        *reinterpret_cast<uint32_t *>(limb + DK + j0) = w1;
+        *reinterpret_cast<uint32_t *>(limb + 2 * DK + j0) = w2;
+    } else {
+        *reinterpret_cast<uint16_t *>(limb + j0) = (uint16_t)w0;
+        *reinterpret_cast<uint16_t *>(limb + DK + j0) = (uint16_t)w1;
+        *reinterpret_cast<uint16_t *>(limb + 2 * DK + j0) = (uint16_t)w2;
+    }
+    if (threadIdx.x % 32 == 0) *lscale = m * (1.0f / 127.0f);
 }
 
 template <int DK, int DV, int GATE, bool BF16, bool COMMIT>
 __global__ void __launch_bounds__(kThreads, COMMIT ? 1 : 2) decode_kernel(const DecodeArgs a, const int S) {
-    using T = Tile<DK, DV, kConsumerWarps>;
     constexpr int E = BF16 ? 2 : 4;
+    constexpr int RPW = DV / kConsumerWarps;  // value rows per consumer warp
     extern __shared__ __align__(128) unsigned char smem[];
     uint64_t *full = reinterpret_cast<uint64_t *>(smem);
-    uint64_t *empty = full + kMaxStages;
-    const StageLayout SL = stage_layout(DK, DV, GATE, a.R, a.W, E);
+    uint64_t *prepared = full + kMaxStages;
+    uint64_t *empty = prepared + kMaxStages;
+    const int nsteps = a.n_steps, pos = a.pos;
+    const StageLayout SL = stage_layout(DK, DV, GATE, a.R, pos + nsteps, nsteps, E);
+    const PrepLayout PL = prep_layout(DK);
     unsigned char *stages = smem + header_bytes();
-    auto &sc = *reinterpret_cast<Scratch<DK, DV> *>(stages + (size_t)S * SL.bytes);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int BH = a.B * a.H;
-    const int R = a.R, W = a.W, pos = a.pos, nsteps = a.n_steps;
+    const int R = a.R, W = a.W;
 
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kConsumerWarps);
+            mbar_init(&prepared[s], kPrepWarps);
+            mbar_init(&empty[s], kConsumerWarps + kPrepWarps);
         }
     }
     __syncthreads();
 
     // ------------------------------------------------------------ producer
-    if (warp == kConsumerWarps) {
+    if (warp == kProducerWarp) {
         if (lane != 0) return;
         int i = 0;
         bool ok = true;
@@ -172,6 +203,20 @@ __global__ void __launch_bounds__(kThreads, COMMIT ? 1 : 2) decode_kernel(const 
                 nsteps > 0 ? (uint32_t)(E * (2 * DK + DV) + (GATE == 1 ? 4 * DK : 0)) : 0u;
             const uint32_t bytes = DV * DK + 4 * DV + 4 * DK + 4 * R * DK + 4 * pos * (DK + DV) +
                                    (GATE == 1 ? 4 * pos * DK : 0) + in_bytes;
+            // small operands by 4-byte copies, tracked by the same barrier:
+            // alpha and beta of token 0, the scalar-gate records, the
+            // compensator rows
+            float *scal = reinterpret_cast<float *>(st + SL.scal);
+            if (nsteps > 0) {
+                if (GATE == 0) cp_async4(scal, a.alpha + tok);
+                cp_async4(scal + 1, a.beta + tok);
+            }
+            if (GATE == 0)
+                for (int m = 0; m < pos; ++m)
+                    cp_async4(st + SL.recL + 4 * m, a.buf_gate + (size_t)bh * W + m);
+            for (int c = 0; c < R; ++c)
+                cp_async4(st + SL.compr + 4 * c, a.comp_row + (size_t)bh * R + c);
+            cp_async_mbar_arrive(&full[s]);
             mbar_arrive_expect_tx(&full[s], bytes);
             bulk_g2s(st + SL.codes, a.codes + (size_t)bh * DV * DK, DV * DK, &full[s]);
             bulk_g2s(st + SL.sig, a.row_scale + (size_t)bh * DV, 4 * DV, &full[s]);
@@ -202,190 +247,205 @@ __global__ void __launch_bounds__(kThreads, COMMIT ? 1 : 2) decode_kernel(const 
         return;
     }
 
-    // ------------------------------------------------------------ consumers
-    const int c0 = T::col0(lane);
-    // registers prefetched one head ahead: scalar gate and beta of token 0,
-    // the last scalar-gate record L_pos (every thread), the scalar-gate
-    // records (thread m holds L_{m+1}) and the compensator rows
-    float pf_alpha = 0.f, pf_beta = 0.f, pf_L = 0.f, pf_Lprev = 0.f;
-    int pf_comp = 0;
-    auto prefetch = [&](int bh) {
-        if (bh >= BH) return;
-        const int b = bh / a.H, h = bh % a.H;
-        const size_t tok = (size_t)b * nsteps * a.H + h;
-        if (nsteps > 0) {
-            if (GATE == 0) pf_alpha = a.alpha[tok];
-            pf_beta = a.beta[tok];
+    // ------------------------------------------------------------ prep warps
+    if (warp >= kPrepAWarp) {
+        const bool isA = warp == kPrepAWarp;
+        const int bpart = warp - kPrepBWarp;  // prep B: this warp's share of coefficient passes
+        constexpr int CPL = DK / 32;          // contiguous key channels per lane
+        const int j0 = CPL * lane;
+        int i = 0;
+        for (int bh = blockIdx.x; bh < BH; bh += gridDim.x, ++i) {
+            const int s = i % S;
+            if (!mbar_wait_bounded(&full[s], (i / S) & 1)) break;
+            unsigned char *st = stages + (size_t)s * SL.bytes;
+            const float *cs_s = reinterpret_cast<const float *>(st + SL.cs);
+            const float *compv_s = reinterpret_cast<const float *>(st + SL.compv);
+            const float *scal = reinterpret_cast<const float *>(st + SL.scal);
+            float *recK_s = reinterpret_cast<float *>(st + SL.recK);
+            float *recL_s = reinterpret_cast<float *>(st + SL.recL);
+            const int b = bh / a.H, h = bh % a.H;
+            float Ls = (GATE == 0 && pos > 0) ? recL_s[pos - 1] : 0.0f;  // scalar gate chain
+            float Lc[CPL];                                             // diagonal, own channels
+            if (GATE == 1 && pos > 0) {
+                load_vec<CPL>(Lc, recL_s + (pos - 1) * DK + j0);
+            } else {
+#pragma unroll
+                for (int e = 0; e < CPL; ++e) Lc[e] = 0.0f;
+            }
+            for (int sidx = 0; sidx < nsteps; ++sidx) {
+                const int t = pos + sidx + 1, nrec = t - 1;
+                const size_t tok = ((size_t)b * nsteps + sidx) * a.H + h;
+                const float beta = sidx == 0 ? scal[1] : a.beta[tok];
+                unsigned char *slot = st + SL.prep + sidx * PL.bytes;
+                float *coefA = reinterpret_cast<float *>(slot + PL.coefA);
+                float *coefG = reinterpret_cast<float *>(slot + PL.coefG);
+                float g_s = 0.0f;
+                if (GATE == 0) {
+                    Ls = Ls + logf(sidx == 0 ? scal[0] : a.alpha[tok]);
+                    g_s = expf(Ls);
+                }
+                float kj[CPL], qj[CPL], gj[CPL];
+                if (sidx == 0) {
+                    load_io_vec<BF16, CPL>(qj, st + SL.q, j0);
+                    load_io_vec<BF16, CPL>(kj, st + SL.k, j0);
+                } else {
+                    load_io_vec<BF16, CPL>(qj, a.q, tok * DK + j0);
+                    load_io_vec<BF16, CPL>(kj, a.k, tok * DK + j0);
+                }
+                if (GATE == 1) {
+                    float al[CPL];
+                    if (sidx == 0) load_vec<CPL>(al, reinterpret_cast<const float *>(st + SL.al) + j0);
+                    else load_vec<CPL>(al, a.alpha + tok * DK + j0);
+#pragma unroll
+                    for (int e = 0; e < CPL; ++e) {
+                        Lc[e] = Lc[e] + logf(al[e]);
+                        gj[e] = expf(Lc[e]);
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < CPL; ++e) gj[e] = g_s;
+                }
+                if (isA) {
+                    // limbs of x_k = c e^L k and x_q = c e^L q; own-token k~ . q
+                    int8_t *limb = reinterpret_cast<int8_t *>(slot + PL.limb);
+                    float *lscale = reinterpret_cast<float *>(slot + PL.lscale);
+                    float cj[CPL], xk[CPL], xq[CPL], kq = 0.0f;
+                    load_vec<CPL>(cj, cs_s + j0);
+#pragma unroll
+                    for (int e = 0; e < CPL; ++e) {
+                        xk[e] = cj[e] * (gj[e] * kj[e]);
+                        xq[e] = cj[e] * (gj[e] * qj[e]);
+                        kq = fmaf(beta * kj[e], qj[e], kq);
+                    }
+                    split_limbs<CPL>(xk, limb, DK, lscale, j0);
+                    split_limbs<CPL>(xq, limb + 3 * DK, DK, lscale + 1, j0);
+                    kq = group_sum<32>(kq);
+                    if (lane == 0) coefG[nrec + R] = kq;
+                } else {
+                    // records of this token: L_t and k~_t.  Every prep-B warp
+                    // writes the same values to shared memory (it reads them
+                    // back for later tokens of the call); warp 0 of them also
+                    // writes global memory.
+                    float ktj[CPL];
+#pragma unroll
+                    for (int e = 0; e < CPL; ++e) ktj[e] = beta * kj[e];
+                    store_vec<CPL>(recK_s + nrec * DK + j0, ktj);
+                    if (GATE == 1) store_vec<CPL>(recL_s + nrec * DK + j0, Lc);
+                    if (GATE == 0 && lane == 0) recL_s[nrec] = Ls;
+                    if (bpart == 0) {
+                        store_vec<CPL>(a.buf_k + ((size_t)bh * W + nrec) * DK + j0, ktj);
+                        if (GATE == 1)
+                            store_vec<CPL>(a.buf_gate + ((size_t)bh * W + nrec) * DK + j0, Lc);
+                        if (GATE == 0 && lane == 0) a.buf_gate[(size_t)bh * W + nrec] = Ls;
+                    }
+                    __syncwarp();
+                    // coefficients of records 0..nrec-1 and compensators,
+                    // eight items per pass, passes shared round-robin by the
+                    // prep-B warps; the 16 partial dot products of a pass are
+                    // reduced together with a transposing reduction
+                    const int nitems = nrec + R;
+                    for (int base = 8 * bpart; base < nitems; base += 8 * kPrepBWarps) {
+                        float part[16];
+#pragma unroll
+                        for (int q8 = 0; q8 < 8; ++q8) {
+                            const int it = base + q8;
+                            float da = 0.0f, dq = 0.0f;
+                            if (it < nitems) {
+                                float w[CPL];
+                                if (it < nrec) {
+                                    load_vec<CPL>(w, recK_s + it * DK + j0);
+                                    if (GATE == 1) {
+                                        float Lm[CPL];
+                                        load_vec<CPL>(Lm, recL_s + it * DK + j0);
+#pragma unroll
+                                        for (int e = 0; e < CPL; ++e) w[e] *= expf(Lc[e] - Lm[e]);
+                                    }
+#pragma unroll
+                                    for (int e = 0; e < CPL; ++e) {
+                                        da = fmaf(w[e], kj[e], da);
+                                        dq = fmaf(w[e], qj[e], dq);
+                                    }
+                                } else {
+                                    load_vec<CPL>(w, compv_s + (it - nrec) * DK + j0);
+#pragma unroll
+                                    for (int e = 0; e < CPL; ++e) {
+                                        da = fmaf(w[e], gj[e] * kj[e], da);
+                                        dq = fmaf(w[e], gj[e] * qj[e], dq);
+                                    }
+                                }
+                            }
+                            part[q8] = da;
+                            part[8 + q8] = dq;
+                        }
+                        transposed_sum<16, 32>(part, lane);
+                        const int idx = transposed_index<16, 32>(lane);
+                        const int it = base + (idx & 7);
+                        if (it < nitems && lane == transposed_owner<16, 32>(idx)) {
+                            float v = part[0];
+                            if (GATE == 0 && it < nrec) v *= expf(Ls - recL_s[it]);
+                            if (idx < 8) coefA[it] = v;
+                            else coefG[it] = v;
+                        }
+                    }
+                }
+                __syncwarp();
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&prepared[s]);
+                mbar_arrive(&empty[s]);
+            }
         }
-        if (GATE == 0 && pos > 0) pf_Lprev = a.buf_gate[(size_t)bh * W + pos - 1];
-        if (GATE == 0 && tid < pos) pf_L = a.buf_gate[(size_t)bh * W + tid];
-        if (tid < R) pf_comp = a.comp_row[(size_t)bh * R + tid];
-    };
-    prefetch(blockIdx.x);
+        return;
+    }
+
+    // ------------------------------------------------------------ consumers
+    constexpr int LPR16 = DK / 16, RPI16 = 32 / LPR16, NRM = RPW / RPI16;
+    constexpr int LPRD = 32 / RPW;  // lanes per value row in the combine
+    static_assert(NRM >= 1 && RPW % RPI16 == 0 && LPRD >= 1 && 32 % RPW == 0, "tiling");
+    const int cc = lane % LPR16, sub = lane / LPR16;
+    const int rloc = lane / LPRD, part = lane % LPRD;  // combine: local row, record share
+    // lanes holding y_k / y_q of local row rloc after the matvec reduction
+    const int src_k = (rloc % RPI16) * LPR16 + transposed_owner<2 * NRM, LPR16>(rloc / RPI16);
+    const int src_q = (rloc % RPI16) * LPR16 + transposed_owner<2 * NRM, LPR16>(NRM + rloc / RPI16);
 
     int i = 0;
     for (int bh = blockIdx.x; bh < BH; bh += gridDim.x, ++i) {
         const int s = i % S;
-        const float cur_alpha = pf_alpha, cur_beta = pf_beta, cur_L = pf_L, cur_Lprev = pf_Lprev;
-        const int cur_comp = pf_comp;
-        prefetch(bh + gridDim.x);
-        const bool ok = mbar_wait_bounded(&full[s], (i / S) & 1);
-
+        bool ok = mbar_wait_bounded(&prepared[s], (i / S) & 1);
+        if constexpr (COMMIT) ok = !consumer_sync_or<kConsumers>(!ok);
+        if (!ok) break;
         unsigned char *st = stages + (size_t)s * SL.bytes;
         const int8_t *codes_s = reinterpret_cast<const int8_t *>(st + SL.codes);
         const float *sig_s = reinterpret_cast<const float *>(st + SL.sig);
-        const float *cs_s = reinterpret_cast<const float *>(st + SL.cs);
-        const float *compv_s = reinterpret_cast<const float *>(st + SL.compv);
-        float *recK_s = reinterpret_cast<float *>(st + SL.recK);
+        const int *compr_s = reinterpret_cast<const int *>(st + SL.compr);
         float *recU_s = reinterpret_cast<float *>(st + SL.recU);
-        float *recL_s = reinterpret_cast<float *>(st + SL.recL);
-        int *compr_s = reinterpret_cast<int *>(st + SL.compr);
         const int b = bh / a.H, h = bh % a.H;
-        float *bufL = a.buf_gate + (size_t)bh * W * (GATE == 1 ? DK : 1);
-        float *bufK = a.buf_k + (size_t)bh * W * DK;
         float *bufU = a.buf_u + (size_t)bh * W * DV;
-        if (GATE == 0 && tid < pos) recL_s[tid] = cur_L;
-        if (tid < R) compr_s[tid] = cur_comp;
+        const int row = warp * RPW + rloc;
 
-        bool abort = false;
         for (int sidx = 0; sidx < nsteps; ++sidx) {
-            const int t = pos + sidx + 1;
+            const int t = pos + sidx + 1, nrec = t - 1;
             const size_t tok = ((size_t)b * nsteps + sidx) * a.H + h;
-            const float beta = sidx == 0 ? cur_beta : a.beta[tok];
-            float vi = 0.f;
-            // D1: inputs, running log gate, k~
-            if (tid < DK) {
-                float qj, kj, al;
-                if (sidx == 0) {
-                    qj = load_io<BF16>(st + SL.q, tid);
-                    kj = load_io<BF16>(st + SL.k, tid);
-                    al = GATE == 1 ? reinterpret_cast<const float *>(st + SL.al)[tid] : cur_alpha;
-                } else {
-                    qj = load_io<BF16>(a.q, tok * DK + tid);
-                    kj = load_io<BF16>(a.k, tok * DK + tid);
-                    al = GATE == 1 ? a.alpha[tok * DK + tid] : a.alpha[tok];
-                }
-                float Lt;
-                if (GATE == 1) {
-                    const float prev = t > 1 ? recL_s[(t - 2) * DK + tid] : 0.0f;
-                    Lt = prev + logf(al);
-                    recL_s[(t - 1) * DK + tid] = Lt;
-                    bufL[(size_t)(t - 1) * DK + tid] = Lt;
-                } else {
-                    // L_{t-1}: the prefetched register for the first token,
-                    // else the record thread 0 wrote one token earlier
-                    const float prev = sidx == 0 ? (t > 1 ? cur_Lprev : 0.0f) : recL_s[t - 2];
-                    Lt = prev + logf(al);
-                    if (tid == 0) {
-                        sc.misc[0] = Lt;
-                        recL_s[t - 1] = Lt;
-                        bufL[t - 1] = Lt;
-                    }
-                }
-                const float g = expf(Lt);
-                const float ktj = beta * kj;
-                sc.qf[tid] = qj;
-                sc.kf[tid] = kj;
-                sc.gk[tid] = g * kj;
-                sc.gq[tid] = g * qj;
-                const float xk = cs_s[tid] * (g * kj), xq = cs_s[tid] * (g * qj);
-                sc.xk[tid] = xk;
-                sc.xq[tid] = xq;
-                sc.kt[tid] = ktj;
-                split_limbs_t<DK>(xk, &sc.limb[0], sc.lscale[0], tid);
-                split_limbs_t<DK>(xq, &sc.limb[3], sc.lscale[1], tid);
-                recK_s[(t - 1) * DK + tid] = ktj;
-                bufK[(size_t)(t - 1) * DK + tid] = ktj;
-            }
-            if (tid < DV) vi = sidx == 0 ? load_io<BF16>(st + SL.v, tid) : load_io<BF16>(a.v, tok * DV + tid);
-            if (sidx == 0) {
-                if (consumer_sync_or<kConsumers>(!ok)) {
-                    abort = true;
-                    break;
-                }
-            } else {
-                consumer_sync<kConsumers>();
-            }
+            const unsigned char *slot = st + SL.prep + sidx * PL.bytes;
+            const int8_t *limb = reinterpret_cast<const int8_t *>(slot + PL.limb);
+            const float *lscale = reinterpret_cast<const float *>(slot + PL.lscale);
+            const float *coefA = reinterpret_cast<const float *>(slot + PL.coefA);
+            const float *coefG = reinterpret_cast<const float *>(slot + PL.coefG);
 
-            // D3 coefficients: records 1..t-1, compensators, own token.  Each
-            // warp takes up to four items per pass; the eight partial dot
-            // products are reduced together with a transposing reduction.
+            // D2: S^_0 x for this warp's rows: dp4a of the codes with the limbs
+            float y;
             {
-                const float Lt_s = GATE == 0 ? sc.misc[0] : 0.0f;
-                const int nrec = t - 1, nitems = nrec + R + 1;
-                for (int base = warp * 4; base < nitems; base += kConsumerWarps * 4) {
-                    float part[8];
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        const int it = base + q4;
-                        float da = 0.0f, dq = 0.0f;
-                        if (it < nrec) {
-                            const float *km = recK_s + it * DK;
-                            if (GATE == 1) {
-                                const float *Lm = recL_s + it * DK;
-                                const float *Lt = recL_s + (t - 1) * DK;
-#pragma unroll
-                                for (int e = 0; e < DK / 32; ++e) {
-                                    const int j = lane + 32 * e;
-                                    const float w = km[j] * expf(Lt[j] - Lm[j]);
-                                    da = fmaf(w, sc.kf[j], da);
-                                    dq = fmaf(w, sc.qf[j], dq);
-                                }
-                            } else {
-#pragma unroll
-                                for (int e = 0; e < DK / 32; ++e) {
-                                    const int j = lane + 32 * e;
-                                    da = fmaf(km[j], sc.kf[j], da);
-                                    dq = fmaf(km[j], sc.qf[j], dq);
-                                }
-                            }
-                        } else if (it < nrec + R) {
-                            const float *cv = compv_s + (it - nrec) * DK;
-#pragma unroll
-                            for (int e = 0; e < DK / 32; ++e) {
-                                const int j = lane + 32 * e;
-                                da = fmaf(cv[j], sc.gk[j], da);
-                                dq = fmaf(cv[j], sc.gq[j], dq);
-                            }
-                        } else if (it == nrec + R) {
-#pragma unroll
-                            for (int e = 0; e < DK / 32; ++e) {
-                                const int j = lane + 32 * e;
-                                dq = fmaf(sc.kt[j], sc.qf[j], dq);
-                            }
-                        }
-                        part[q4] = da;
-                        part[4 + q4] = dq;
-                    }
-                    transposed_sum<8, 32>(part, lane);
-                    const int idx = transposed_index<8, 32>(lane);
-                    const int it = base + (idx & 3);
-                    if (it < nitems && lane == transposed_owner<8, 32>(idx)) {
-                        float v = part[0];
-                        if (GATE == 0 && it < nrec) v *= expf(Lt_s - recL_s[it]);
-                        if (idx < 4) sc.coefA[it] = v;
-                        else sc.coefG[it] = v;
-                    }
-                }
-            }
-
-            // D2: y_k = Q (c e^L k), y_q = Q (c e^L q): integer dot products of
-            // the int8 codes with the int8 limbs of both vectors (dp4a), one
-            // 16-code chunk per lane, combined per chunk in FP32 and reduced
-            // across the row's lanes with a transposing reduction
-            {
-                constexpr int LPR16 = DK / 16, RPI16 = 32 / LPR16, RPW = DV / kConsumerWarps;
-                constexpr int NRM = RPW / RPI16;
-                static_assert(NRM >= 1 && RPW % RPI16 == 0, "matvec tiling");
-                const int cc = lane % LPR16, sub = lane / LPR16;
                 uint4 lw[6];
 #pragma unroll
-                for (int v = 0; v < 6; ++v) lw[v] = *reinterpret_cast<const uint4 *>(&sc.limb[v][16 * cc]);
+                for (int v = 0; v < 6; ++v)
+                    lw[v] = *reinterpret_cast<const uint4 *>(limb + v * DK + 16 * cc);
                 int acc[NRM][6];
 #pragma unroll
                 for (int n = 0; n < NRM; ++n) {
-                    const int row = warp * RPW + n * RPI16 + sub;
-                    const uint4 w = *reinterpret_cast<const uint4 *>(codes_s + row * DK + 16 * cc);
+                    const int r = warp * RPW + n * RPI16 + sub;
+                    const uint4 w = *reinterpret_cast<const uint4 *>(codes_s + r * DK + 16 * cc);
 #pragma unroll
                     for (int v = 0; v < 6; ++v) {
                         int x = __dp4a((int)w.x, (int)lw[v].x, 0);
@@ -394,56 +454,71 @@ __global__ void __launch_bounds__(kThreads, COMMIT ? 1 : 2) decode_kernel(const 
                         acc[n][v] = __dp4a((int)w.w, (int)lw[v].w, x);
                     }
                 }
-                const float sk = sc.lscale[0][cc], sq = sc.lscale[1][cc];
+                const float sk = lscale[0], sq = lscale[1];
                 float vals[2 * NRM];
 #pragma unroll
                 for (int n = 0; n < NRM; ++n) {
-                    vals[n] = sk * fmaf((float)acc[n][2], 6.103515625e-05f,
-                                        fmaf((float)acc[n][1], 0.0078125f, (float)acc[n][0]));
-                    vals[NRM + n] = sq * fmaf((float)acc[n][5], 6.103515625e-05f,
-                                              fmaf((float)acc[n][4], 0.0078125f, (float)acc[n][3]));
+                    // |acc| < 2^18: exact conversions without the conversion pipe
+                    vals[n] = sk * fmaf(small_int_to_f32(acc[n][2]), 6.103515625e-05f,
+                                        fmaf(small_int_to_f32(acc[n][1]), 0.0078125f,
+                                             small_int_to_f32(acc[n][0])));
+                    vals[NRM + n] = sq * fmaf(small_int_to_f32(acc[n][5]), 6.103515625e-05f,
+                                              fmaf(small_int_to_f32(acc[n][4]), 0.0078125f,
+                                                   small_int_to_f32(acc[n][3])));
                 }
                 transposed_sum<2 * NRM, LPR16>(vals, lane);
-                const int idx = transposed_index<2 * NRM, LPR16>(lane);
-                const int row = warp * RPW + (idx % NRM) * RPI16 + sub;
-                sc.y[(idx / NRM) * DV + row] = vals[0] * sig_s[row];
+                y = vals[0];
             }
-            consumer_sync<kConsumers>();
-
-            // D3-D6 per value channel: correction, u_t, o_t, record
-            if (tid < DV) {
-                const int nrec = t - 1;
-                float hb = sc.y[tid], p = sc.y[DV + tid];
-                for (int c = 0; c < R; ++c)
-                    if (compr_s[c] == tid) {
-                        hb += sc.coefA[nrec + c];
-                        p += sc.coefG[nrec + c];
-                    }
-                for (int m = 0; m < nrec; ++m) {
-                    const float um = recU_s[m * DV + tid];
-                    hb = fmaf(sc.coefA[m], um, hb);
-                    p = fmaf(sc.coefG[m], um, p);
+            // D3-D6 for row `row`: LPRD lanes share its buffered records
+            {
+                const float sg = sig_s[row];
+                const float yk = __shfl_sync(0xffffffffu, y, src_k) * sg;
+                const float yq = __shfl_sync(0xffffffffu, y, src_q) * sg;
+                float hb = part == 0 ? yk : 0.0f, p = part == 0 ? yq : 0.0f;
+                for (int m = part; m < nrec; m += LPRD) {
+                    const float um = recU_s[m * DV + row];
+                    hb = fmaf(coefA[m], um, hb);
+                    p = fmaf(coefG[m], um, p);
                 }
-                const float u = vi - hb;
-                const float o = fmaf(sc.coefG[nrec + R], u, p);
-                store_io<BF16>(a.o, tok * DV + tid, o);
-                recU_s[(t - 1) * DV + tid] = u;
-                bufU[(size_t)(t - 1) * DV + tid] = u;
+#pragma unroll
+                for (int o = LPRD / 2; o > 0; o >>= 1) {
+                    hb += __shfl_xor_sync(0xffffffffu, hb, o);
+                    p += __shfl_xor_sync(0xffffffffu, p, o);
+                }
+                if (part == 0) {
+                    for (int c = 0; c < R; ++c)
+                        if (compr_s[c] == row) {
+                            hb += coefA[nrec + c];
+                            p += coefG[nrec + c];
+                        }
+                    const float vi = sidx == 0 ? load_io<BF16>(st + SL.v, row)
+                                               : load_io<BF16>(a.v, tok * DV + row);
+                    const float u = vi - hb;
+                    const float o = fmaf(coefG[nrec + R], u, p);
+                    store_io<BF16>(a.o, tok * DV + row, o);
+                    recU_s[nrec * DV + row] = u;
+                    bufU[(size_t)nrec * DV + row] = u;
+                }
+                __syncwarp();
             }
         }
-        if (nsteps == 0 && consumer_sync_or<kConsumers>(!ok)) abort = true;
-        if (abort) break;
 
         if constexpr (COMMIT) {
+            using T = Tile<DK, DV, kConsumerWarps>;
+            auto &cs = *reinterpret_cast<CommitScratch<DK, DV> *>(stages + (size_t)S * SL.bytes);
+            const float *cs_s = reinterpret_cast<const float *>(st + SL.cs);
+            const float *compv_s = reinterpret_cast<const float *>(st + SL.compv);
+            float *recK_s = reinterpret_cast<float *>(st + SL.recK);
+            const float *recL_s = reinterpret_cast<const float *>(st + SL.recL);
+            const int c0 = T::col0(lane);
             consumer_sync<kConsumers>();
             // C1: S_n = S^_0 e^{L_n} + sum_m u_m (k~_m e^{L_n - L_m})^T  (FP32, registers)
             const int nrec = pos + nsteps;
-            float *gW_s = sc.gk, *cgW_s = sc.xk;
             for (int j = tid; j < DK; j += kConsumers) {
                 const float Ln = GATE == 1 ? recL_s[(nrec - 1) * DK + j] : recL_s[nrec - 1];
                 const float g = expf(Ln);
-                gW_s[j] = g;
-                cgW_s[j] = cs_s[j] * g;
+                cs.gW[j] = g;
+                cs.cgW[j] = cs_s[j] * g;
             }
             if (GATE == 1) {
                 for (int e = tid; e < nrec * DK; e += kConsumers) {
@@ -451,24 +526,21 @@ __global__ void __launch_bounds__(kThreads, COMMIT ? 1 : 2) decode_kernel(const 
                     recK_s[e] *= expf(recL_s[(nrec - 1) * DK + j] - recL_s[m * DK + j]);
                 }
             } else {
-                // one decay factor per record
-                for (int e = tid; e < nrec * DK; e += kConsumers) {
-                    const int m = e / DK;
-                    recK_s[e] *= expf(recL_s[nrec - 1] - recL_s[m]);
-                }
+                for (int e = tid; e < nrec * DK; e += kConsumers)
+                    recK_s[e] *= expf(recL_s[nrec - 1] - recL_s[e / DK]);
             }
             consumer_sync<kConsumers>();
             float Sreg[T::NR][4];
             {
                 float cg[4];
-                *reinterpret_cast<float4 *>(cg) = *reinterpret_cast<const float4 *>(cgW_s + c0);
+                *reinterpret_cast<float4 *>(cg) = *reinterpret_cast<const float4 *>(cs.cgW + c0);
 #pragma unroll
                 for (int n = 0; n < T::NR; ++n) {
-                    const int row = T::row(warp, lane, n);
-                    const uint32_t w = *reinterpret_cast<const uint32_t *>(codes_s + row * DK + c0);
+                    const int r = T::row(warp, lane, n);
+                    const uint32_t w = *reinterpret_cast<const uint32_t *>(codes_s + r * DK + c0);
                     float f[4];
                     codes4_to_f32(w, f);
-                    const float si = sig_s[row];
+                    const float si = sig_s[r];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) Sreg[n][e] = (si * f[e]) * cg[e];
                 }
@@ -479,7 +551,7 @@ __global__ void __launch_bounds__(kThreads, COMMIT ? 1 : 2) decode_kernel(const 
                         if (T::row(warp, lane, n) == rc)
 #pragma unroll
                             for (int e = 0; e < 4; ++e)
-                                Sreg[n][e] = fmaf(compv_s[c * DK + c0 + e], gW_s[c0 + e], Sreg[n][e]);
+                                Sreg[n][e] = fmaf(compv_s[c * DK + c0 + e], cs.gW[c0 + e], Sreg[n][e]);
                 }
 #pragma unroll 2
                 for (int m = 0; m < nrec; ++m) {
@@ -507,7 +579,7 @@ __global__ void __launch_bounds__(kThreads, COMMIT ? 1 : 2) decode_kernel(const 
                         a.col_smooth + (size_t)bh * DK,
                         a.comp_row ? a.comp_row + (size_t)bh * R : nullptr,
                         a.comp_val ? a.comp_val + (size_t)bh * R * DK : nullptr};
-            quantize_tile<DK, DV, kConsumerWarps>(Sreg, R, a.smoothing != 0, sc.quant, out);
+            quantize_tile<DK, DV, kConsumerWarps>(Sreg, R, a.smoothing != 0, cs.quant, out);
         }
         // release the stage to the producer
         fence_proxy_async_smem();
@@ -537,8 +609,10 @@ struct Launcher {
             sm_count[dev & 63] = sms;
             configured.fetch_or(bit, std::memory_order_acq_rel);
         }
-        const StageLayout SL = stage_layout(DK, DV, GATE, a.R, a.W, E);
-        const int fixed = header_bytes() + (int)sizeof(Scratch<DK, DV>);
+        // a stage holds the records this launch reads and writes (pos + n_steps)
+        const StageLayout SL =
+            stage_layout(DK, DV, GATE, a.R, a.pos + a.n_steps, a.n_steps, E);
+        const int fixed = header_bytes() + scratch_bytes<DK, DV, COMMIT>();
         // two CTAs per SM when registers allow it and each can hold at least
         // two stages, else one CTA per SM with as many stages as fit
         const int per_sm = 227 * 1024;

@@ -98,8 +98,9 @@ def test_decode_validation_without_launch():
     st = _fake_state(cfg)
     st.buf_k = st.buf_k + 4
     assert _decode(st, 1) == lq.LQ_ERR_MISALIGNED
-    # misaligned bf16 activation (odd address)
+    # misaligned activations: odd address, and element-aligned but not 16-byte aligned
     assert _decode(_fake_state(cfg), 1, q=0x20000001) == lq.LQ_ERR_MISALIGNED
+    assert _decode(_fake_state(cfg), 1, q=0x20000002) == lq.LQ_ERR_MISALIGNED
     # unsupported head size, bad window, too many compensators
     for field, val, want in (("d_k", 96, lq.LQ_ERR_UNSUPPORTED), ("window", 33, lq.LQ_ERR_INVALID_ARGUMENT),
                              ("window", 0, lq.LQ_ERR_INVALID_ARGUMENT),
