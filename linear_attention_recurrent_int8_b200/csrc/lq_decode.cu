@@ -110,13 +110,48 @@ template <int DK, int DV>
 struct alignas(16) CommitScratch {
     alignas(16) float gW[DK];
     alignas(16) float cgW[DK];
+    float dec[32];
     QuantSmem<DK, DV, kConsumerWarps> quant;
 };
+
+// Commit buffers sized by the launch: the FP32 rank term S [DV][DK + 4] and
+// the TF32 hi/lo operand K [kp][DK + 8] (kp = records + compensators rounded
+// up to the MMA's k = 8).
+struct CommitLayout {
+    int S, khi, klo, kp, bytes;
+};
+
+__host__ __device__ inline CommitLayout commit_layout(int DK, int DV, int items) {
+    CommitLayout C{};
+    C.kp = (items + 7) & ~7;
+    int o = 0;
+    C.S = o;   o += align16(4 * DV * (DK + 4));
+    C.khi = o; o += align16(4 * C.kp * (DK + 8));
+    C.klo = o; o += align16(4 * C.kp * (DK + 8));
+    C.bytes = o;
+    return C;
+}
 using CommitA = CommitScratch<128, 128>;
 static_assert(offsetof(CommitA, cgW) % 16 == 0 && offsetof(CommitA, quant) % 16 == 0,
               "vector-accessed commit scratch must be 16-byte aligned");
 
 __host__ __device__ constexpr int header_bytes() { return 3 * kMaxStages * 8; }
+
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
+// D += A B on a 16x8x8 tile, TF32 operands, FP32 accumulate (warp-wide).
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
 
 template <int DK, int DV, bool COMMIT>
 __host__ __device__ constexpr int scratch_bytes() {
@@ -506,30 +541,92 @@ __global__ void __launch_bounds__(kThreads, COMMIT ? 1 : 2) decode_kernel(const 
         if constexpr (COMMIT) {
             using T = Tile<DK, DV, kConsumerWarps>;
             auto &cs = *reinterpret_cast<CommitScratch<DK, DV> *>(stages + (size_t)S * SL.bytes);
+            const CommitLayout CL = commit_layout(DK, DV, pos + nsteps + R);
+            unsigned char *cbase = stages + (size_t)S * SL.bytes + sizeof(CommitScratch<DK, DV>);
+            float *Ssm = reinterpret_cast<float *>(cbase + CL.S);
+            uint32_t *Khi = reinterpret_cast<uint32_t *>(cbase + CL.khi);
+            uint32_t *Klo = reinterpret_cast<uint32_t *>(cbase + CL.klo);
             const float *cs_s = reinterpret_cast<const float *>(st + SL.cs);
             const float *compv_s = reinterpret_cast<const float *>(st + SL.compv);
-            float *recK_s = reinterpret_cast<float *>(st + SL.recK);
+            const float *recK_s = reinterpret_cast<const float *>(st + SL.recK);
             const float *recL_s = reinterpret_cast<const float *>(st + SL.recL);
             const int c0 = T::col0(lane);
+            const int nrec = pos + nsteps, Kp = CL.kp;
             consumer_sync<kConsumers>();
-            // C1: S_n = S^_0 e^{L_n} + sum_m u_m (k~_m e^{L_n - L_m})^T  (FP32, registers)
-            const int nrec = pos + nsteps;
+            // C1: S_n = S^_0 e^{L_n} + [U | E_comp] [K^ | comp e^{L_n}]^T with
+            // K^_m = k~_m e^{L_n - L_m}: the boundary term on CUDA cores, the
+            // rank-(n + r) term on tensor cores (TF32 with a hi/lo split of both
+            // operands, three products per tile: FP32-faithful).
             for (int j = tid; j < DK; j += kConsumers) {
                 const float Ln = GATE == 1 ? recL_s[(nrec - 1) * DK + j] : recL_s[nrec - 1];
                 const float g = expf(Ln);
                 cs.gW[j] = g;
                 cs.cgW[j] = cs_s[j] * g;
             }
-            if (GATE == 1) {
-                for (int e = tid; e < nrec * DK; e += kConsumers) {
-                    const int m = e / DK, j = e % DK;
-                    recK_s[e] *= expf(recL_s[(nrec - 1) * DK + j] - recL_s[m * DK + j]);
+            if (GATE == 0 && tid < nrec) cs.dec[tid] = expf(recL_s[nrec - 1] - recL_s[tid]);
+            consumer_sync<kConsumers>();
+            // B operand (Kp x DK, row m = one record or compensator), split into
+            // TF32 hi/lo, rows padded to DK + 8 words (conflict-free fragment loads)
+            for (int e = tid; e < Kp * DK; e += kConsumers) {
+                const int m = e / DK, j = e % DK;
+                float x = 0.0f;
+                if (m < nrec) {
+                    const float dcy = GATE == 1 ? expf(recL_s[(nrec - 1) * DK + j] - recL_s[m * DK + j])
+                                                : cs.dec[m];
+                    x = recK_s[m * DK + j] * dcy;
+                } else if (m < nrec + R) {
+                    x = compv_s[(m - nrec) * DK + j] * cs.gW[j];
                 }
-            } else {
-                for (int e = tid; e < nrec * DK; e += kConsumers)
-                    recK_s[e] *= expf(recL_s[nrec - 1] - recL_s[e / DK]);
+                const uint32_t hi = to_tf32(x);
+                Khi[m * (DK + 8) + j] = hi;
+                Klo[m * (DK + 8) + j] = to_tf32(x - __uint_as_float(hi));
             }
             consumer_sync<kConsumers>();
+            if (warp < DV / 16) {
+                // this warp's 16 value rows x all DK key channels
+                const int g = lane >> 2, tq = lane & 3, r0 = 16 * warp;
+                float acc[DK / 8][4];
+#pragma unroll
+                for (int jn = 0; jn < DK / 8; ++jn) acc[jn][0] = acc[jn][1] = acc[jn][2] = acc[jn][3] = 0.0f;
+                for (int k0 = 0; k0 < Kp; k0 += 8) {
+                    // A fragment: rows r0+g, r0+g+8; columns (records) k0+tq, k0+tq+4
+                    float av[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int r = r0 + g + 8 * (q & 1), m = k0 + tq + 4 * (q >> 1);
+                        float x = 0.0f;
+                        if (m < nrec) x = recU_s[m * DV + r];
+                        else if (m < nrec + R) x = compr_s[m - nrec] == r ? 1.0f : 0.0f;
+                        av[q] = x;
+                    }
+                    uint32_t ahi[4], alo[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        ahi[q] = to_tf32(av[q]);
+                        alo[q] = to_tf32(av[q] - __uint_as_float(ahi[q]));
+                    }
+#pragma unroll
+                    for (int jn = 0; jn < DK / 8; ++jn) {
+                        const int n = 8 * jn + g;
+                        const uint32_t bh0 = Khi[(k0 + tq) * (DK + 8) + n];
+                        const uint32_t bh1 = Khi[(k0 + tq + 4) * (DK + 8) + n];
+                        const uint32_t bl0 = Klo[(k0 + tq) * (DK + 8) + n];
+                        const uint32_t bl1 = Klo[(k0 + tq + 4) * (DK + 8) + n];
+                        mma_tf32(acc[jn], ahi, bh0, bh1);
+                        mma_tf32(acc[jn], ahi, bl0, bl1);
+                        mma_tf32(acc[jn], alo, bh0, bh1);
+                    }
+                }
+#pragma unroll
+                for (int jn = 0; jn < DK / 8; ++jn) {
+                    *reinterpret_cast<float2 *>(Ssm + (r0 + g) * (DK + 4) + 8 * jn + 2 * tq) =
+                        make_float2(acc[jn][0], acc[jn][1]);
+                    *reinterpret_cast<float2 *>(Ssm + (r0 + g + 8) * (DK + 4) + 8 * jn + 2 * tq) =
+                        make_float2(acc[jn][2], acc[jn][3]);
+                }
+            }
+            consumer_sync<kConsumers>();
+            // boundary term in the quantizer's tile layout, plus the rank term
             float Sreg[T::NR][4];
             {
                 float cg[4];
@@ -541,38 +638,11 @@ __global__ void __launch_bounds__(kThreads, COMMIT ? 1 : 2) decode_kernel(const 
                     float f[4];
                     codes4_to_f32(w, f);
                     const float si = sig_s[r];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) Sreg[n][e] = (si * f[e]) * cg[e];
-                }
-                for (int c = 0; c < R; ++c) {
-                    const int rc = compr_s[c];
-#pragma unroll
-                    for (int n = 0; n < T::NR; ++n)
-                        if (T::row(warp, lane, n) == rc)
-#pragma unroll
-                            for (int e = 0; e < 4; ++e)
-                                Sreg[n][e] = fmaf(compv_s[c * DK + c0 + e], cs.gW[c0 + e], Sreg[n][e]);
-                }
-#pragma unroll 2
-                for (int m = 0; m < nrec; ++m) {
-                    float kh[4];
-                    *reinterpret_cast<float4 *>(kh) =
-                        *reinterpret_cast<const float4 *>(recK_s + m * DK + c0);
-                    float u[T::NR];
-                    if constexpr (T::RPI == 1 && T::NR % 4 == 0) {
-                        // this lane's rows are consecutive: vector loads
-#pragma unroll
-                        for (int n = 0; n < T::NR; n += 4)
-                            *reinterpret_cast<float4 *>(&u[n]) = *reinterpret_cast<const float4 *>(
-                                recU_s + m * DV + T::row(warp, lane, n));
-                    } else {
-#pragma unroll
-                        for (int n = 0; n < T::NR; ++n) u[n] = recU_s[m * DV + T::row(warp, lane, n)];
-                    }
-#pragma unroll
-                    for (int n = 0; n < T::NR; ++n)
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) Sreg[n][e] = fmaf(u[n], kh[e], Sreg[n][e]);
+                    const float4 up = *reinterpret_cast<const float4 *>(Ssm + r * (DK + 4) + c0);
+                    Sreg[n][0] = fmaf(si * f[0], cg[0], up.x);
+                    Sreg[n][1] = fmaf(si * f[1], cg[1], up.y);
+                    Sreg[n][2] = fmaf(si * f[2], cg[2], up.z);
+                    Sreg[n][3] = fmaf(si * f[3], cg[3], up.w);
                 }
             }
             SnapPtr out{a.codes + (size_t)bh * DV * DK, a.row_scale + (size_t)bh * DV,
@@ -612,7 +682,8 @@ struct Launcher {
         // a stage holds the records this launch reads and writes (pos + n_steps)
         const StageLayout SL =
             stage_layout(DK, DV, GATE, a.R, a.pos + a.n_steps, a.n_steps, E);
-        const int fixed = header_bytes() + scratch_bytes<DK, DV, COMMIT>();
+        const int fixed = header_bytes() + scratch_bytes<DK, DV, COMMIT>() +
+                          (COMMIT ? commit_layout(DK, DV, a.pos + a.n_steps + a.R).bytes : 0);
         // two CTAs per SM when registers allow it and each can hold at least
         // two stages, else one CTA per SM with as many stages as fit
         const int per_sm = 227 * 1024;

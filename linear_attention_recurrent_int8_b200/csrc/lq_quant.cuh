@@ -192,12 +192,16 @@ __device__ __forceinline__ void quantize_tile(float (&S)[Tile<DK, DV, NWARPS>::N
         const float inv =
             __shfl_sync(0xffffffffu, inv_own, gbase + transposed_owner<T::NR, T::LPR>(n));
         const int row = T::row(warp, lane, n);
-        uint32_t packed = 0;
+        // round half to even by the magic-number addition (|y| <= 127 here),
+        // clamp, and pack the four low bytes
+        int iv[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            const float qv = fminf(fmaxf(rintf(__fmul_rn(S[n][e], inv)), -127.0f), 127.0f);
-            packed |= (static_cast<uint32_t>(static_cast<int>(qv)) & 0xFFu) << (8 * e);
+            const float y = fminf(fmaxf(__fmul_rn(S[n][e], inv), -127.0f), 127.0f);
+            iv[e] = __float_as_int(__fadd_rn(y, 12582912.0f)) - 0x4B400000;
         }
+        const uint32_t packed = __byte_perm(__byte_perm(iv[0], iv[1], 0x0040),
+                                            __byte_perm(iv[2], iv[3], 0x0040), 0x5410);
         *reinterpret_cast<uint32_t *>(out.codes + (size_t)row * DK + c0) = packed;
     }
 }

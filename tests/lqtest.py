@@ -224,3 +224,92 @@ class AnchoredRun:
         self.stats["near_ties"] += st["near_ties"]
         self.snap = new_snap
         return o_gpu, o_ref
+
+
+class SampledRun:
+    """Full-size run on the device (every sequence and head, the launch
+    configuration the benchmark times) with the oracle following a seeded
+    sample of (sequence, head) pairs.
+
+    Device inputs for all heads are drawn on the device with the same integer
+    streams; the sampled heads' inputs (and initial states) are overwritten
+    with the numpy draws that the oracle consumes, so both sides see identical
+    values there.  At each window start the sampled heads' snapshots are set
+    to the oracle's (anchoring); the other heads run free and are not checked
+    (every head is checked by AnchoredRun in the first windows).  Nothing the
+    device computes is given to the oracle."""
+
+    def __init__(self, wl: synth.DecodeWorkload, n_sample: int, seed: int = 1234, device="cuda"):
+        self.wl, self.device = wl, device
+        self.cfg = make_config(wl)
+        self.st = lq.State(self.cfg, device)
+        rng = np.random.default_rng(seed)
+        self.sample = np.sort(rng.choice(wl.nh, size=min(n_sample, wl.nh), replace=False))
+        self.sb, self.sh = self.sample // wl.heads, self.sample % wl.heads
+        self.idx = torch.from_numpy(self.sample).to(device)
+        self.stats = dict(windows=0, worst_out=0.0, code_flips=0, near_ties=0)
+
+    def _sample_tokens(self, t0, t1):
+        wl = self.wl
+        per = [synth.tokens(wl.seed, [b], [h], t0, t1, wl.d_k, wl.d_v, wl.gate, wl.io)
+               for b, h in zip(self.sb, self.sh)]
+        return {k: np.concatenate([p[k] for p in per], axis=2) for k in per[0]}  # [1, T, ns, ...]
+
+    def _sampled_snapshot(self):
+        return {k: v.index_select(0, self.idx).cpu().numpy() for k, v in self.st.snap.t.items()}
+
+    def init(self):
+        wl, dev = self.wl, self.device
+        S = synth.torch_initial_state(wl.seed, np.arange(wl.batch), np.arange(wl.heads), wl.d_k, wl.d_v,
+                                      wl.outlier_rows, wl.outlier_cols, wl.outlier_scale, dev)
+        S = S.reshape(wl.nh, wl.d_v, wl.d_k)
+        S_s = np.concatenate([synth.initial_state(wl.seed, [b], [h], wl.d_k, wl.d_v, wl.outlier_rows,
+                                                  wl.outlier_cols, wl.outlier_scale)[0]
+                              for b, h in zip(self.sb, self.sh)], axis=0)
+        S[self.idx] = torch.from_numpy(S_s).to(dev)
+        lq.lq_state_init(self.st, S)
+        torch.cuda.synchronize()
+        del S
+        ref = oracle.quantize(S_s, self.cfg.n_comp, bool(self.cfg.smoothing))
+        compare_snapshots(self._sampled_snapshot(), ref, ref["row_norm"], exact_codes=True)
+        self.snap = ref
+
+    def _anchor(self):
+        for key in ("codes", "row_scale", "col_smooth", "comp_row", "comp_val"):
+            if self.st.snap.t[key].numel():
+                src = torch.from_numpy(np.ascontiguousarray(self.snap[key])).to(self.device)
+                self.st.snap.t[key][self.idx] = src.to(self.st.snap.t[key].dtype)
+
+    def window(self, w: int):
+        wl, cfg, dev = self.wl, self.cfg, self.device
+        W = cfg.window
+        t0 = w * W
+        self._anchor()
+        dev_tok = synth.torch_tokens(wl.seed, wl.batch, wl.heads, t0, t0 + W, wl.d_k, wl.d_v, wl.gate,
+                                     wl.io, dev)
+        tok_s = self._sample_tokens(t0, t0 + W)
+        bi = torch.from_numpy(self.sb).to(dev)
+        hi = torch.from_numpy(self.sh).to(dev)
+        for k in ("q", "k", "v", "alpha", "beta"):
+            vals = torch.from_numpy(np.ascontiguousarray(np.swapaxes(tok_s[k][0], 0, 1))).to(dev)
+            dev_tok[k][bi, :, hi] = vals.to(dev_tok[k].dtype)
+        o = torch.empty((wl.batch, W, wl.heads, wl.d_v), dtype=io_dtype(wl.io), device=dev)
+        out = torch.empty((wl.batch, 1, wl.heads, wl.d_v), dtype=io_dtype(wl.io), device=dev)
+        for t in range(W):
+            args = [dev_tok[k][:, t:t + 1].contiguous() for k in ("q", "k", "v", "alpha", "beta")]
+            lq.lq_decode_window(self.st, *args, 1, out)
+            o[:, t:t + 1] = out
+        torch.cuda.synchronize()
+        assert self.st.pos == 0
+        d, kt, b, v, q = oracle_tokens(tok_s, wl.gate)
+        rec = oracle.empty_records(len(self.sample), W, wl.d_k, wl.d_v, cfg.gdim)
+        o_ref = oracle.window(self.snap, rec, 0, d, kt, b, v, q)
+        new_snap, _ = oracle.commit(self.snap, rec, W, cfg.n_comp, bool(cfg.smoothing))
+        o_gpu = o[bi, :, hi].float().cpu().numpy()  # [ns, W, dv]
+        worst = compare_outputs(o_gpu, o_ref, wl.io, f"outputs window {w}")
+        st = compare_snapshots(self._sampled_snapshot(), new_snap, new_snap["row_norm"])
+        self.stats["windows"] += 1
+        self.stats["worst_out"] = max(self.stats["worst_out"], worst)
+        self.stats["code_flips"] += st["code_flips"]
+        self.stats["near_ties"] += st["near_ties"]
+        self.snap = new_snap
