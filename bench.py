@@ -487,12 +487,171 @@ def run_e2e(args, wl, st, cfg, dev, world, group):
             "steps": n}
 
 
+def run_prefill(args):
+    """Prefill throughput: batch 2 x 32 heads, T tokens, bf16, a snapshot every
+    1024 tokens (prompt tokens/s)."""
+    import numpy as np
+    import torch
+
+    import linear_attention_recurrent_int8_b200 as lq
+    from linear_attention_recurrent_int8_b200 import synth
+    P = synth.PREFILL_WORKLOAD
+    B, H, dk, dv, every, r = P["batch"], P["heads"], P["d_k"], P["d_v"], P["snapshot_every"], P["n_comp"]
+    T = args.prefill_tokens or P["T"]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    cfg = lq.Config(batch=B, heads=H, d_k=dk, d_v=dv, window=P["window"], n_comp=r,
+                    gate=lq.LQ_GATE_SCALAR, io_dtype=lq.LQ_BF16, smoothing=1, auto_commit=1)
+    st = lq.State(cfg, dev)
+    lq.lq_state_init(st, None)
+    q = torch.empty((B, T, H, dk), dtype=torch.bfloat16, device=dev)
+    k, v = torch.empty_like(q), torch.empty((B, T, H, dv), dtype=torch.bfloat16, device=dev)
+    alpha = torch.empty((B, T, H), dtype=torch.float32, device=dev)
+    beta = torch.empty_like(alpha)
+    for t0 in range(0, T, 4096):
+        t1 = min(T, t0 + 4096)
+        tok = synth.torch_tokens(P["seed"], B, H, t0, t1, dk, dv, "scalar", "bf16", dev)
+        q[:, t0:t1], k[:, t0:t1], v[:, t0:t1] = tok["q"], tok["k"], tok["v"]
+        alpha[:, t0:t1], beta[:, t0:t1] = tok["alpha"], tok["beta"]
+    S = torch.zeros((B * H, dv, dk), dtype=torch.float32, device=dev)
+    o = torch.empty((B, T, H, dv), dtype=torch.bfloat16, device=dev)
+    snaps = [lq.Snapshot(cfg, dev) for _ in range(T // every)]
+
+    def one():
+        S.zero_()
+        lq.lq_prefill_chunk(st, S, q, k, v, alpha, beta, T, every, snaps, o)
+
+    for _ in range(args.warmup):
+        one()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        one()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / args.steps
+    nbytes = B * T * H * (2 * (2 * dk + dv) + 8 + 2 * dv)
+    flops = B * T * H * 3 * 2 * dk * dv
+    return {"metric": "prefill tokens/s (state update + output, snapshots every 1024 tokens)",
+            "value": B * T / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": f"gdn prefill batch {B} x {H} heads, d={dk}, T={T}, bf16, "
+                                   f"snapshot every {every} (r={r})"},
+            "detail": {"io_gbs": nbytes / (ms / 1e3) / 1e9, "fp32_tflops": flops / (ms / 1e3) / 1e12,
+                       "snapshots": T // every}}
+
+
+def run_fp32step(args, wl):
+    """FP32 per-step comparator: the whole FP32 state read and written every
+    token (one launch per token, all heads)."""
+    import torch
+
+    import linear_attention_recurrent_int8_b200 as lq
+    from linear_attention_recurrent_int8_b200 import synth
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    cfg = lq.Config(batch=wl.batch, heads=wl.heads, d_k=wl.d_k, d_v=wl.d_v,
+                    gate=lq.LQ_GATE_DIAG if wl.gate == "diag" else lq.LQ_GATE_SCALAR,
+                    io_dtype=lq.LQ_BF16 if wl.io == "bf16" else lq.LQ_F32)
+    S = torch.randn((wl.nh, wl.d_v, wl.d_k), dtype=torch.float32, device=dev)
+    toks = []
+    for t in range(8):
+        tok = synth.torch_tokens(wl.seed, wl.batch, wl.heads, t, t + 1, wl.d_k, wl.d_v, wl.gate,
+                                 wl.io, dev)
+        toks.append([tok[k2] for k2 in ("q", "k", "v", "alpha", "beta")])
+    o = torch.empty((wl.batch, 1, wl.heads, wl.d_v), dtype=cfg.io_torch_dtype, device=dev)
+    for i in range(args.warmup):
+        lq.lq_fp32_step(cfg, S, *toks[i % 8], 1, o)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for i in range(args.steps):
+        lq.lq_fp32_step(cfg, S, *toks[i % 8], 1, o)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / args.steps
+    e = 2 if wl.io == "bf16" else 4
+    nbytes = wl.nh * (8 * wl.d_v * wl.d_k + e * (2 * wl.d_k + 2 * wl.d_v) + 8)
+    peak, kind = measured_peaks()
+    return {"metric": "FP32 per-step comparator: decode tokens/s", "value": wl.batch / (ms / 1e3),
+            "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic", "config": workload_config(wl, args),
+            "roofline": {"bound": "hbm", "achieved": nbytes / (ms / 1e3) / 1e9, "peak": peak,
+                         "unit": "GB/s", "frac": nbytes / (ms / 1e3) / 1e9 / peak, "traffic": None}}
+
+
+def run_mse(args, wl):
+    """State MSE against the unquantized FP32 state (the FP32 per-step chain),
+    per-window (W, r, smoothing as configured) versus per-token (W = 1,
+    r = 0), over the same inputs, for a subset of sequences."""
+    import dataclasses
+
+    import torch
+
+    import linear_attention_recurrent_int8_b200 as lq
+    from linear_attention_recurrent_int8_b200 import synth
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    wl = dataclasses.replace(wl, batch=min(wl.batch, args.mse_batch))
+    steps = args.mse_steps
+    S0 = synth.torch_initial_state(wl.seed, range(wl.batch), range(wl.heads), wl.d_k, wl.d_v,
+                                   wl.outlier_rows, wl.outlier_cols, wl.outlier_scale, dev)
+    S0 = S0.reshape(wl.nh, wl.d_v, wl.d_k).contiguous()
+    variants = {"per_window": (wl.window, wl.n_comp, int(wl.smoothing)),
+                "per_token": (1, 0, int(wl.smoothing)), "per_token_plain": (1, 0, 0)}
+    states, cfgs = {}, {}
+    for name, (W, r, sm) in variants.items():
+        cfg = lq.Config(batch=wl.batch, heads=wl.heads, d_k=wl.d_k, d_v=wl.d_v, window=W, n_comp=r,
+                        gate=lq.LQ_GATE_DIAG if wl.gate == "diag" else lq.LQ_GATE_SCALAR,
+                        io_dtype=lq.LQ_BF16 if wl.io == "bf16" else lq.LQ_F32, smoothing=sm,
+                        auto_commit=1)
+        st = lq.State(cfg, dev)
+        lq.lq_state_init(st, S0)
+        states[name], cfgs[name] = st, cfg
+    S = S0.clone()
+    fcfg = cfgs["per_window"]
+    o = torch.empty((wl.batch, 1, wl.heads, wl.d_v), dtype=fcfg.io_torch_dtype, device=dev)
+
+    def dequant(st):
+        t = st.snap.t
+        Sh = (t["row_scale"][:, :, None] * t["codes"].float() * t["col_smooth"][:, None, :])
+        if t["comp_row"].numel():
+            Sh.scatter_add_(1, t["comp_row"].long()[:, :, None].expand(-1, -1, wl.d_k), t["comp_val"])
+        return Sh
+
+    curve = {n: [] for n in variants}
+    W = wl.window
+    for t in range(steps):
+        tok = synth.torch_tokens(wl.seed, wl.batch, wl.heads, t, t + 1, wl.d_k, wl.d_v, wl.gate, wl.io,
+                                 dev)
+        args_t = [tok[k2] for k2 in ("q", "k", "v", "alpha", "beta")]
+        lq.lq_fp32_step(fcfg, S, *args_t, 1, o)
+        for name, st in states.items():
+            lq.lq_decode_window(st, *args_t, 1, o)
+        if (t + 1) % W == 0:
+            ref_ms = float((S * S).mean())
+            for name, st in states.items():
+                curve[name].append(float(((dequant(st) - S) ** 2).mean()) / ref_ms)
+    out = {n: {"final_rel_mse": c[-1], "mean_rel_mse": sum(c) / len(c)} for n, c in curve.items()}
+    return {"report": "state MSE relative to the mean square of the FP32 state, at window ends",
+            "workload": wl.name, "batch": wl.batch, "heads": wl.heads, "steps": steps,
+            "window": W, "n_comp": wl.n_comp, "results": out}
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["lq", "reference"], default="lq")
+    ap.add_argument("--mode", choices=["decode", "prefill", "fp32step", "mse"], default="decode",
+                    help="decode (default, the headline) or a comparator / report")
+    ap.add_argument("--prefill-tokens", type=int, default=0)
+    ap.add_argument("--mse-batch", type=int, default=16)
+    ap.add_argument("--mse-steps", type=int, default=1024)
     ap.add_argument("--workload", default="gdn_256x32_d128_bf16")
     ap.add_argument("--window", type=int, default=None, help="override W (comparators / sweep)")
     ap.add_argument("--n-comp", type=int, default=None, help="override r")
@@ -521,7 +680,16 @@ def main(argv=None):
     if over:
         wl = dataclasses.replace(wl, **over)
 
-    line = run_reference(args, wl) if args.impl == "reference" else run_lq(args, wl)
+    if args.impl == "reference":
+        line = run_reference(args, wl)
+    elif args.mode == "prefill":
+        line = run_prefill(args)
+    elif args.mode == "fp32step":
+        line = run_fp32step(args, wl)
+    elif args.mode == "mse":
+        line = run_mse(args, wl)
+    else:
+        line = run_lq(args, wl)
     if line is not None:
         print(json.dumps(line), flush=True)
 
