@@ -90,6 +90,16 @@ def aggregate(elapsed_ms: float, tokens_per_rank: int, world: int, group=None):
     return elapsed_ms, tokens_per_rank * world / (elapsed_ms / 1e3)
 
 
+def shard(rank: int, world: int, batch_per_rank: int):
+    """This rank's sequences: a contiguous block of the global batch
+    (world * batch_per_rank sequences).  Each (sequence, head) state is
+    independent, so ranks share nothing but the final timing reduction."""
+    if not (0 <= rank < world) or batch_per_rank < 1:
+        raise ValueError("bad shard")
+    b0 = rank * batch_per_rank
+    return range(b0, b0 + batch_per_rank)
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -290,8 +300,7 @@ def run_lq(args, wl):
     e = 2 if wl.io == "bf16" else 4
     st = lq.State(cfg, dev)
     # this rank's shard of sequences: global sequence index offset
-    b0 = rank * wl.batch
-    bs, hs = np.arange(b0, b0 + wl.batch), np.arange(wl.heads)
+    bs, hs = np.array(shard(rank, world, wl.batch)), np.arange(wl.heads)
     S0 = synth.torch_initial_state(wl.seed, bs, hs, wl.d_k, wl.d_v, wl.outlier_rows, wl.outlier_cols,
                                    wl.outlier_scale, dev)
     lq.lq_state_init(st, S0.reshape(wl.nh, wl.d_v, wl.d_k))
