@@ -54,16 +54,19 @@ def record_bytes(dk, dv, gate):
     return 4 * ((dk if gate == "diag" else 1) + dk + dv)
 
 
-def decode_launch_bytes(dk, dv, r, gate, e, t, commit):
+def decode_launch_bytes(dk, dv, r, gate, e, t):
     """Bytes one decode launch at window position t must move per head:
     read the snapshot and the t-1 buffered records, read q, k, v, alpha,
-    beta, write o and record t; a fused commit also writes the new snapshot."""
+    beta, write o and record t."""
     G = dk if gate == "diag" else 1
     rec = record_bytes(dk, dv, gate)
-    b = snapshot_bytes(dk, dv, r) + (t - 1) * rec + e * (2 * dk + dv) + 4 * G + 4 + e * dv + rec
-    if commit:
-        b += snapshot_bytes(dk, dv, r)
-    return b
+    return snapshot_bytes(dk, dv, r) + (t - 1) * rec + e * (2 * dk + dv) + 4 * G + 4 + e * dv + rec
+
+
+def commit_launch_bytes(dk, dv, r, gate, n):
+    """Bytes the commit of a window of n records must move per head: read the
+    snapshot and the n records, write the new snapshot."""
+    return 2 * snapshot_bytes(dk, dv, r) + n * record_bytes(dk, dv, gate)
 
 
 # --------------------------------------------------------------------------
@@ -266,11 +269,11 @@ def workload_config(wl, args):
         "batch_per_gpu": wl.batch, "heads": wl.heads, "d_k": wl.d_k, "d_v": wl.d_v,
         "window": wl.window, "n_comp": wl.n_comp, "gate": wl.gate, "io": wl.io,
         "smoothing": bool(wl.smoothing), "state": "int8 codes + fp32 row scales",
-        "step": f"one window: {wl.window} decode launches (commit fused into the last)",
+        "step": f"one window: {wl.window} decode launches and the window commit",
         "tokens_per_step_per_gpu": wl.batch * wl.window,
         "l2": "inputs larger than L2: each decode launch reads ~%.0f MB vs 126 MB L2" % (
             wl.batch * wl.heads * decode_launch_bytes(wl.d_k, wl.d_v, wl.n_comp, wl.gate,
-                                                      2 if wl.io == "bf16" else 4, 1, False) / 1e6),
+                                                      2 if wl.io == "bf16" else 4, 1) / 1e6),
         "graph": not args.no_graph,
     }
 
@@ -295,7 +298,7 @@ def run_lq(args, wl):
     cfg = lq.Config(batch=wl.batch, heads=wl.heads, d_k=wl.d_k, d_v=wl.d_v, window=wl.window,
                     n_comp=wl.n_comp, gate=lq.LQ_GATE_DIAG if wl.gate == "diag" else lq.LQ_GATE_SCALAR,
                     io_dtype=lq.LQ_BF16 if wl.io == "bf16" else lq.LQ_F32,
-                    smoothing=int(wl.smoothing), auto_commit=1)
+                    smoothing=int(wl.smoothing), auto_commit=0)
     W = wl.window
     e = 2 if wl.io == "bf16" else 4
     st = lq.State(cfg, dev)
@@ -326,6 +329,9 @@ def run_lq(args, wl):
             lq.lq_decode_window(st, *per_t[t], 1, o)
             if events:
                 events[t + 1].record()
+        lq.lq_window_commit(st)
+        if events:
+            events[W + 1].record()
 
     # one eager window (also sets kernel attributes before any capture)
     run_window(slots[0])
@@ -336,7 +342,7 @@ def run_lq(args, wl):
         s = torch.cuda.Stream(device=dev)
         for slot in slots:
             # external events become event-record nodes of the graph
-            evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(W + 1)]
+            evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(W + 2)]
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=s):
                 run_window(slot, evs)
@@ -344,7 +350,7 @@ def run_lq(args, wl):
         assert st.pos == 0
     else:
         for slot in slots:
-            graphs.append((None, [torch.cuda.Event(enable_timing=True) for _ in range(W + 1)]))
+            graphs.append((None, [torch.cuda.Event(enable_timing=True) for _ in range(W + 2)]))
 
     def step(i):
         g, evs = graphs[i % len(graphs)]
@@ -378,46 +384,39 @@ def run_lq(args, wl):
     elapsed_max, value = aggregate(elapsed, wl.batch * W * args.steps, world, group)
 
     # per-launch times from the event nodes of the last replay of each graph
-    dec_ms, com_ms, dec_bytes, com_bytes = [], [], 0.0, 0.0
+    dec_ms, com_ms, dec_bytes = [], [], 0.0
     nh = wl.nh
     used = range(min(len(graphs), args.steps + args.warmup))
     for gi in used:
         evs = graphs[gi][1]
         for t in range(W):
-            ms = evs[t].elapsed_time(evs[t + 1])
-            commit = t == W - 1
-            nbytes = nh * decode_launch_bytes(wl.d_k, wl.d_v, wl.n_comp, wl.gate, e, t + 1, commit)
-            if commit:
-                com_ms.append(ms)
-                com_bytes += nbytes
-            else:
-                dec_ms.append(ms)
-                dec_bytes += nbytes
+            dec_ms.append(evs[t].elapsed_time(evs[t + 1]))
+            dec_bytes += nh * decode_launch_bytes(wl.d_k, wl.d_v, wl.n_comp, wl.gate, e, t + 1)
+        com_ms.append(evs[W].elapsed_time(evs[W + 1]))
     peak, peak_kind = measured_peaks()
-    if dec_ms:
-        dec_avg_ms = sum(dec_ms) / len(dec_ms)
-        achieved = dec_bytes / len(dec_ms) / (dec_avg_ms / 1e3) / 1e9
-        traffic = profiled_traffic(f"decode:{wl.name}")
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak, "traffic": traffic,
-                "kernel": "decode_kernel (non-commit launches, window positions 1..W-1)",
-                "bytes_per_launch": dec_bytes / len(dec_ms), "avg_launch_us": dec_avg_ms * 1e3,
-                "peak_source": f"{peak_kind} hbm_gbs (copy)"}
-    else:
-        roof = None
+    dec_avg_ms = sum(dec_ms) / len(dec_ms)
+    achieved = dec_bytes / len(dec_ms) / (dec_avg_ms / 1e3) / 1e9
+    traffic = profiled_traffic(f"decode:{wl.name}")
+    roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak, "traffic": traffic,
+            "kernel": "decode_kernel (window positions 1..W)",
+            "bytes_per_launch": dec_bytes / len(dec_ms), "avg_launch_us": dec_avg_ms * 1e3,
+            "peak_source": f"{peak_kind} hbm_gbs (copy)"}
     extra = {}
-    # average duration of the launch at each window position (us)
+    # average duration of the launch at each window position (us), then the commit
     pos_us = []
     for t in range(W):
         vals = [graphs[gi][1][t].elapsed_time(graphs[gi][1][t + 1]) for gi in used]
         pos_us.append(round(1e3 * sum(vals) / len(vals), 1))
     extra["launch_us_by_position"] = pos_us
-    if com_ms:
-        c_avg = sum(com_ms) / len(com_ms)
-        extra["commit_launch_us"] = c_avg * 1e3
-        extra["commit_launch_gbs"] = com_bytes / len(com_ms) / (c_avg / 1e3) / 1e9
-    step_bytes = nh * sum(decode_launch_bytes(wl.d_k, wl.d_v, wl.n_comp, wl.gate, e, t + 1,
-                                              t == W - 1) for t in range(W))
+    c_avg = sum(com_ms) / len(com_ms)
+    c_bytes = nh * commit_launch_bytes(wl.d_k, wl.d_v, wl.n_comp, wl.gate, W)
+    extra["commit"] = {"kernel": "commit_kernel", "avg_launch_us": c_avg * 1e3,
+                       "bytes_per_launch": c_bytes, "achieved_gbs": c_bytes / (c_avg / 1e3) / 1e9,
+                       "frac": c_bytes / (c_avg / 1e3) / 1e9 / peak,
+                       "traffic": profiled_traffic(f"commit:{wl.name}")}
+    step_bytes = c_bytes + nh * sum(decode_launch_bytes(wl.d_k, wl.d_v, wl.n_comp, wl.gate, e, t + 1)
+                                    for t in range(W))
     extra["step_gbs"] = step_bytes / (elapsed / args.steps / 1e3) / 1e9
 
     # end to end through the C ABI from pinned host buffers
@@ -430,7 +429,7 @@ def run_lq(args, wl):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed_max / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic", "config": workload_config(wl, args),
-        "roofline": roof, "gpu_launches": W * args.steps,
+        "roofline": roof, "gpu_launches": (W + 1) * args.steps,
         "detail": extra,
     }
     line["config"]["parallelism"] = f"dp{world} (independent sequence shards, no collective)"
@@ -476,6 +475,7 @@ def run_e2e(args, wl, st, cfg, dev, world, group):
             dbuf[k].copy_(host[k], non_blocking=True)
         for t in range(W):
             lq.lq_decode_window(st, *[dbuf[k][t] for k in keys], 1, o_dev[t])
+        lq.lq_window_commit(st)
         o_host.copy_(o_dev, non_blocking=True)
 
     for _ in range(3):

@@ -25,7 +25,8 @@
  *  - Calls are asynchronous on `stream` (NULL = the legacy default stream).
  *    They never synchronize, except lq_device_errors.
  *  - Arguments are validated before anything is launched.  A call that
- *    returns an error status has launched nothing and changed nothing.
+ *    returns an error status other than LQ_ERR_CUDA has launched nothing and
+ *    changed nothing (lq_decode_window states its one LQ_ERR_CUDA case).
  *  - A launch failure reported by the CUDA runtime returns LQ_ERR_CUDA.
  *  - No C++ exception crosses this boundary.
  *  - One lq_state is used by one stream at a time.
@@ -137,8 +138,11 @@ LQ_API lq_status lq_state_init(lq_state *st, const lq_config *cfg, const float *
  * is appended.  All n_steps tokens run inside one launch.
  * Requires 0 <= n_steps and pos + n_steps <= W (else LQ_ERR_WINDOW_FULL);
  * n_steps == 0 is a no-op.  When cfg.auto_commit is set and the window
- * becomes full, the same launch commits it (see lq_window_commit) and pos
- * returns to 0; otherwise pos += n_steps. */
+ * becomes full, the call also commits it (lq_window_commit, a second launch
+ * on the same stream) and pos returns to 0; otherwise pos += n_steps.  If the
+ * decode launch succeeded but the commit launch fails, the call returns
+ * LQ_ERR_CUDA with the tokens decoded and pos == W (window full, not
+ * committed); lq_window_commit completes it. */
 LQ_API lq_status lq_decode_window(lq_state *st, const void *q, const void *k, const void *v,
                            const float *alpha, const float *beta, int32_t n_steps,
                            void *o, lq_stream_t stream);

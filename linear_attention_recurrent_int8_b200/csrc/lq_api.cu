@@ -176,11 +176,11 @@ lq_status lq_decode_window(lq_state *st, const void *q, const void *k, const voi
     a.beta = beta;
     a.o = o;
     a.n_steps = n_steps;
-    const bool commit = st->cfg.auto_commit && st->pos + n_steps == st->cfg.window;
     e = cuda_status(lq::launch_decode(a, st->cfg.d_k, st->cfg.d_v, st->cfg.gate,
-                                      st->cfg.io_dtype == LQ_BF16, commit, (cudaStream_t)stream));
+                                      st->cfg.io_dtype == LQ_BF16, (cudaStream_t)stream));
     if (e != LQ_OK) return e;
-    st->pos = commit ? 0 : st->pos + n_steps;
+    st->pos += n_steps;
+    if (st->cfg.auto_commit && st->pos == st->cfg.window) return lq_window_commit(st, stream);
     return LQ_OK;
 }
 
@@ -190,8 +190,7 @@ lq_status lq_window_commit(lq_state *st, lq_stream_t stream) {
     if (st->pos == 0) return LQ_OK;
     lq::DecodeArgs a = decode_args(st);
     a.n_steps = 0;
-    e = cuda_status(lq::launch_decode(a, st->cfg.d_k, st->cfg.d_v, st->cfg.gate,
-                                      st->cfg.io_dtype == LQ_BF16, true, (cudaStream_t)stream));
+    e = cuda_status(lq::launch_commit(a, st->cfg.d_k, st->cfg.d_v, st->cfg.gate, (cudaStream_t)stream));
     if (e != LQ_OK) return e;
     st->pos = 0;
     return LQ_OK;

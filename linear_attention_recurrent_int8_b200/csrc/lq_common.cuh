@@ -98,6 +98,26 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
     return true;
 }
 
+// Named barrier ID over NT threads (ID 0 is __syncthreads).
+template <int ID, int NT>
+__device__ __forceinline__ void named_sync() {
+    asm volatile("bar.sync %0, %1;" ::"n"(ID), "n"(NT) : "memory");
+}
+
+// Named barrier ID over NT threads that also ORs `pred` over them: every
+// participant gets the same answer (so a group can leave a loop together).
+template <int ID, int NT>
+__device__ __forceinline__ bool named_sync_or(bool pred) {
+    uint32_t out;
+    asm volatile(
+        "{ .reg .pred p, q; setp.ne.u32 p, %1, 0; bar.red.or.pred q, %2, %3, p; selp.u32 %0, 1, 0, "
+        "q; }"
+        : "=r"(out)
+        : "r"((uint32_t)pred), "n"(ID), "n"(NT)
+        : "memory");
+    return out != 0;
+}
+
 // Named barrier 1 over the first NT threads of the CTA (the consumer warps of
 // a warp-specialised kernel; barrier 0 is __syncthreads).
 template <int NT>

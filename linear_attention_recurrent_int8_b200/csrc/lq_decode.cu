@@ -1,4 +1,4 @@
-// lq_decode.cu -- per-window int8 decode (and window commit) on sm_100a.
+// lq_decode.cu -- per-window int8 decode on sm_100a.
 //
 // "LeapQuant: Efficient Linear Attention with Accurate Recurrent State
 // Quantization", Figure 2: within a window the int8 boundary state S^_0 stays
@@ -16,7 +16,7 @@
 // pseudo-records at window position 0 (Figure 4; they share the update path
 // of real tokens), so they enter with decay e^{L_t}.
 //
-// Kernel structure (persistent, warp-specialised, 11 warps per CTA):
+// Kernel structure (persistent, warp-specialised, 12 warps per CTA):
 //  * the grid walks the (sequence, head) pairs with a grid stride; each head
 //    goes through a ring of shared-memory stages;
 //  * producer (warp 8, one lane): streams the head's int8 codes, scales,
@@ -25,17 +25,15 @@
 //  * prep A (warp 9): for every token of the call, the vectors
 //    x_k = c e^L k and x_q = c e^L q split into three int8 limbs per
 //    16-channel chunk, and k~_t . q_t -> "prepared";
-//  * prep B (warp 10): the records (L_t, k~_t) of the new tokens and every
-//    coefficient (k~_m e^{L_t-L_m}) . k_t, . q_t of the buffered records and
-//    compensators -> "prepared";
+//  * prep B (warps 10, 11): the records (L_t, k~_t) of the new tokens and
+//    every coefficient (k~_m e^{L_t-L_m}) . k_t, . q_t of the buffered records
+//    and compensators -> "prepared";
 //  * consumers (warps 0-7): warp w owns value rows [w*d_v/8, (w+1)*d_v/8).  It
 //    forms S^_0 x for its rows (dp4a of the codes with the limbs, FP32
 //    combine, transposing warp reduction), then u_t and o_t for the same rows
 //    from the coefficients and its own buffered u.  No CTA barrier is needed
-//    per head; the consumers release the stage through "empty";
-//  * when the window fills (or for a standalone commit, launched with no
-//    tokens) the consumers rebuild the FP32 state of the head in registers and
-//    re-quantize it in place (lq_quant.cuh).
+//    per head; the consumers release the stage through "empty".
+// The window commit is a separate kernel (lq_commit.cu).
 // Every wait is bounded (lq_common.cuh); a wait that expires sets the device
 // error word and the waiting warp stops.
 #include <atomic>
@@ -51,7 +49,6 @@ __device__ unsigned int g_dev_error = 0;
 namespace {
 
 constexpr int kConsumerWarps = 8;
-constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kProducerWarp = 8, kPrepAWarp = 9, kPrepBWarp = 10, kPrepBWarps = 2;
 constexpr int kPrepWarps = 1 + kPrepBWarps;
 constexpr int kThreads = (kConsumerWarps + 1 + kPrepWarps) * 32;
@@ -105,58 +102,7 @@ __host__ __device__ inline StageLayout stage_layout(int DK, int DV, int gate, in
     return L;
 }
 
-// Scratch of the commit (consumer warps only).
-template <int DK, int DV>
-struct alignas(16) CommitScratch {
-    alignas(16) float gW[DK];
-    alignas(16) float cgW[DK];
-    float dec[32];
-    QuantSmem<DK, DV, kConsumerWarps> quant;
-};
-
-// Commit buffers sized by the launch: the FP32 rank term S [DV][DK + 4] and
-// the TF32 hi/lo operand K [kp][DK + 8] (kp = records + compensators rounded
-// up to the MMA's k = 8).
-struct CommitLayout {
-    int S, khi, klo, kp, bytes;
-};
-
-__host__ __device__ inline CommitLayout commit_layout(int DK, int DV, int items) {
-    CommitLayout C{};
-    C.kp = (items + 7) & ~7;
-    int o = 0;
-    C.S = o;   o += align16(4 * DV * (DK + 4));
-    C.khi = o; o += align16(4 * C.kp * (DK + 8));
-    C.klo = o; o += align16(4 * C.kp * (DK + 8));
-    C.bytes = o;
-    return C;
-}
-using CommitA = CommitScratch<128, 128>;
-static_assert(offsetof(CommitA, cgW) % 16 == 0 && offsetof(CommitA, quant) % 16 == 0,
-              "vector-accessed commit scratch must be 16-byte aligned");
-
 __host__ __device__ constexpr int header_bytes() { return 3 * kMaxStages * 8; }
-
-__device__ __forceinline__ uint32_t to_tf32(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return r;
-}
-
-// D += A B on a 16x8x8 tile, TF32 operands, FP32 accumulate (warp-wide).
-__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
-                                         uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-        "{%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-template <int DK, int DV, bool COMMIT>
-__host__ __device__ constexpr int scratch_bytes() {
-    return COMMIT ? (int)sizeof(CommitScratch<DK, DV>) : 0;
-}
 
 // Splits the d_k-vector x (lane l holds x_j for the CPL channels
 // j = j0 .. j0+CPL-1) into three int8 limbs with one scale
@@ -194,8 +140,8 @@ __device__ __forceinline__ void split_limbs(const float (&x)[CPL], int8_t *limb,
     if (threadIdx.x % 32 == 0) *lscale = m * (1.0f / 127.0f);
 }
 
-template <int DK, int DV, int GATE, bool BF16, bool COMMIT>
-__global__ void __launch_bounds__(kThreads, COMMIT ? 1 : 2) decode_kernel(const DecodeArgs a, const int S) {
+template <int DK, int DV, int GATE, bool BF16>
+__global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a, const int S) {
     constexpr int E = BF16 ? 2 : 4;
     constexpr int RPW = DV / kConsumerWarps;  // value rows per consumer warp
     extern __shared__ __align__(128) unsigned char smem[];
@@ -448,9 +394,7 @@ __global__ void __launch_bounds__(kThreads, COMMIT ? 1 : 2) decode_kernel(const 
     int i = 0;
     for (int bh = blockIdx.x; bh < BH; bh += gridDim.x, ++i) {
         const int s = i % S;
-        bool ok = mbar_wait_bounded(&prepared[s], (i / S) & 1);
-        if constexpr (COMMIT) ok = !consumer_sync_or<kConsumers>(!ok);
-        if (!ok) break;
+        if (!mbar_wait_bounded(&prepared[s], (i / S) & 1)) break;
         unsigned char *st = stages + (size_t)s * SL.bytes;
         const int8_t *codes_s = reinterpret_cast<const int8_t *>(st + SL.codes);
         const float *sig_s = reinterpret_cast<const float *>(st + SL.sig);
@@ -538,119 +482,6 @@ __global__ void __launch_bounds__(kThreads, COMMIT ? 1 : 2) decode_kernel(const 
             }
         }
 
-        if constexpr (COMMIT) {
-            using T = Tile<DK, DV, kConsumerWarps>;
-            auto &cs = *reinterpret_cast<CommitScratch<DK, DV> *>(stages + (size_t)S * SL.bytes);
-            const CommitLayout CL = commit_layout(DK, DV, pos + nsteps + R);
-            unsigned char *cbase = stages + (size_t)S * SL.bytes + sizeof(CommitScratch<DK, DV>);
-            float *Ssm = reinterpret_cast<float *>(cbase + CL.S);
-            uint32_t *Khi = reinterpret_cast<uint32_t *>(cbase + CL.khi);
-            uint32_t *Klo = reinterpret_cast<uint32_t *>(cbase + CL.klo);
-            const float *cs_s = reinterpret_cast<const float *>(st + SL.cs);
-            const float *compv_s = reinterpret_cast<const float *>(st + SL.compv);
-            const float *recK_s = reinterpret_cast<const float *>(st + SL.recK);
-            const float *recL_s = reinterpret_cast<const float *>(st + SL.recL);
-            const int c0 = T::col0(lane);
-            const int nrec = pos + nsteps, Kp = CL.kp;
-            consumer_sync<kConsumers>();
-            // C1: S_n = S^_0 e^{L_n} + [U | E_comp] [K^ | comp e^{L_n}]^T with
-            // K^_m = k~_m e^{L_n - L_m}: the boundary term on CUDA cores, the
-            // rank-(n + r) term on tensor cores (TF32 with a hi/lo split of both
-            // operands, three products per tile: FP32-faithful).
-            for (int j = tid; j < DK; j += kConsumers) {
-                const float Ln = GATE == 1 ? recL_s[(nrec - 1) * DK + j] : recL_s[nrec - 1];
-                const float g = expf(Ln);
-                cs.gW[j] = g;
-                cs.cgW[j] = cs_s[j] * g;
-            }
-            if (GATE == 0 && tid < nrec) cs.dec[tid] = expf(recL_s[nrec - 1] - recL_s[tid]);
-            consumer_sync<kConsumers>();
-            // B operand (Kp x DK, row m = one record or compensator), split into
-            // TF32 hi/lo, rows padded to DK + 8 words (conflict-free fragment loads)
-            for (int e = tid; e < Kp * DK; e += kConsumers) {
-                const int m = e / DK, j = e % DK;
-                float x = 0.0f;
-                if (m < nrec) {
-                    const float dcy = GATE == 1 ? expf(recL_s[(nrec - 1) * DK + j] - recL_s[m * DK + j])
-                                                : cs.dec[m];
-                    x = recK_s[m * DK + j] * dcy;
-                } else if (m < nrec + R) {
-                    x = compv_s[(m - nrec) * DK + j] * cs.gW[j];
-                }
-                const uint32_t hi = to_tf32(x);
-                Khi[m * (DK + 8) + j] = hi;
-                Klo[m * (DK + 8) + j] = to_tf32(x - __uint_as_float(hi));
-            }
-            consumer_sync<kConsumers>();
-            if (warp < DV / 16) {
-                // this warp's 16 value rows x all DK key channels
-                const int g = lane >> 2, tq = lane & 3, r0 = 16 * warp;
-                float acc[DK / 8][4];
-#pragma unroll
-                for (int jn = 0; jn < DK / 8; ++jn) acc[jn][0] = acc[jn][1] = acc[jn][2] = acc[jn][3] = 0.0f;
-                for (int k0 = 0; k0 < Kp; k0 += 8) {
-                    // A fragment: rows r0+g, r0+g+8; columns (records) k0+tq, k0+tq+4
-                    float av[4];
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const int r = r0 + g + 8 * (q & 1), m = k0 + tq + 4 * (q >> 1);
-                        float x = 0.0f;
-                        if (m < nrec) x = recU_s[m * DV + r];
-                        else if (m < nrec + R) x = compr_s[m - nrec] == r ? 1.0f : 0.0f;
-                        av[q] = x;
-                    }
-                    uint32_t ahi[4], alo[4];
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        ahi[q] = to_tf32(av[q]);
-                        alo[q] = to_tf32(av[q] - __uint_as_float(ahi[q]));
-                    }
-#pragma unroll
-                    for (int jn = 0; jn < DK / 8; ++jn) {
-                        const int n = 8 * jn + g;
-                        const uint32_t bh0 = Khi[(k0 + tq) * (DK + 8) + n];
-                        const uint32_t bh1 = Khi[(k0 + tq + 4) * (DK + 8) + n];
-                        const uint32_t bl0 = Klo[(k0 + tq) * (DK + 8) + n];
-                        const uint32_t bl1 = Klo[(k0 + tq + 4) * (DK + 8) + n];
-                        mma_tf32(acc[jn], ahi, bh0, bh1);
-                        mma_tf32(acc[jn], ahi, bl0, bl1);
-                        mma_tf32(acc[jn], alo, bh0, bh1);
-                    }
-                }
-#pragma unroll
-                for (int jn = 0; jn < DK / 8; ++jn) {
-                    *reinterpret_cast<float2 *>(Ssm + (r0 + g) * (DK + 4) + 8 * jn + 2 * tq) =
-                        make_float2(acc[jn][0], acc[jn][1]);
-                    *reinterpret_cast<float2 *>(Ssm + (r0 + g + 8) * (DK + 4) + 8 * jn + 2 * tq) =
-                        make_float2(acc[jn][2], acc[jn][3]);
-                }
-            }
-            consumer_sync<kConsumers>();
-            // boundary term in the quantizer's tile layout, plus the rank term
-            float Sreg[T::NR][4];
-            {
-                float cg[4];
-                *reinterpret_cast<float4 *>(cg) = *reinterpret_cast<const float4 *>(cs.cgW + c0);
-#pragma unroll
-                for (int n = 0; n < T::NR; ++n) {
-                    const int r = T::row(warp, lane, n);
-                    const uint32_t w = *reinterpret_cast<const uint32_t *>(codes_s + r * DK + c0);
-                    float f[4];
-                    codes4_to_f32(w, f);
-                    const float si = sig_s[r];
-                    const float4 up = *reinterpret_cast<const float4 *>(Ssm + r * (DK + 4) + c0);
-                    Sreg[n][0] = fmaf(si * f[0], cg[0], up.x);
-                    Sreg[n][1] = fmaf(si * f[1], cg[1], up.y);
-                    Sreg[n][2] = fmaf(si * f[2], cg[2], up.z);
-                    Sreg[n][3] = fmaf(si * f[3], cg[3], up.w);
-                }
-            }
-            SnapPtr out{a.codes + (size_t)bh * DV * DK, a.row_scale + (size_t)bh * DV,
-                        a.col_smooth + (size_t)bh * DK,
-                        a.comp_row ? a.comp_row + (size_t)bh * R : nullptr,
-                        a.comp_val ? a.comp_val + (size_t)bh * R * DK : nullptr};
-            quantize_tile<DK, DV, kConsumerWarps>(Sreg, R, a.smoothing != 0, cs.quant, out);
-        }
         // release the stage to the producer
         fence_proxy_async_smem();
         __syncwarp();
@@ -658,82 +489,70 @@ __global__ void __launch_bounds__(kThreads, COMMIT ? 1 : 2) decode_kernel(const 
     }
 }
 
-template <int DK, int DV, int GATE, bool BF16, bool COMMIT>
-struct Launcher {
-    static cudaError_t run(const DecodeArgs &a, cudaStream_t stream) {
-        constexpr int E = BF16 ? 2 : 4;
-        static std::atomic<uint64_t> configured{0};  // devices already set up
-        static int sm_count[64];
-        int dev = 0;
-        cudaError_t e = cudaGetDevice(&dev);
-        if (e != cudaSuccess) return e;
-        auto kern = decode_kernel<DK, DV, GATE, BF16, COMMIT>;
-        const uint64_t bit = 1ull << (dev & 63);
-        if (!(configured.load(std::memory_order_acquire) & bit)) {
-            int optin = 0, sms = 0;
-            e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-            if (e == cudaSuccess)
-                e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
-            if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-            if (e != cudaSuccess) return e;
-            sm_count[dev & 63] = sms;
-            configured.fetch_or(bit, std::memory_order_acq_rel);
-        }
-        // a stage holds the records this launch reads and writes (pos + n_steps)
-        const StageLayout SL =
-            stage_layout(DK, DV, GATE, a.R, a.pos + a.n_steps, a.n_steps, E);
-        const int fixed = header_bytes() + scratch_bytes<DK, DV, COMMIT>() +
-                          (COMMIT ? commit_layout(DK, DV, a.pos + a.n_steps + a.R).bytes : 0);
-        // two CTAs per SM when registers allow it and each can hold at least
-        // two stages, else one CTA per SM with as many stages as fit
-        const int per_sm = 227 * 1024;
-        int ctas = 2, S = (per_sm / 2 - 1024 - fixed) / SL.bytes;
-        if (S > kMaxStages) S = kMaxStages;
-        int smem = fixed + S * SL.bytes;
-        int resident = 0;
-        if (S >= 2) {
-            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, kern, kThreads, smem);
-            if (e != cudaSuccess) return e;
-        }
-        if (S < 2 || resident < 2) {
-            ctas = 1;
-            S = (per_sm - 1024 - fixed) / SL.bytes;
-            if (S > kMaxStages) S = kMaxStages;
-            smem = fixed + S * SL.bytes;
-        }
-        if (S < 1) return cudaErrorInvalidConfiguration;
-        const int BH = a.B * a.H;
-        int grid = sm_count[dev & 63] * ctas;
-        if (grid > BH) grid = BH;
-        kern<<<grid, kThreads, smem, stream>>>(a, S);
-        return cudaGetLastError();
-    }
-};
-
 template <int DK, int DV, int GATE, bool BF16>
-cudaError_t launch_decode_c(const DecodeArgs &a, bool commit, cudaStream_t stream) {
-    return commit ? Launcher<DK, DV, GATE, BF16, true>::run(a, stream)
-                  : Launcher<DK, DV, GATE, BF16, false>::run(a, stream);
+cudaError_t launch_d(const DecodeArgs &a, cudaStream_t stream) {
+    constexpr int E = BF16 ? 2 : 4;
+    static std::atomic<uint64_t> configured{0};  // devices already set up
+    static int sm_count[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    auto kern = decode_kernel<DK, DV, GATE, BF16>;
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(configured.load(std::memory_order_acquire) & bit)) {
+        int optin = 0, sms = 0;
+        e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        sm_count[dev & 63] = sms;
+        configured.fetch_or(bit, std::memory_order_acq_rel);
+    }
+    // a stage holds the records this launch reads and writes (pos + n_steps)
+    const StageLayout SL = stage_layout(DK, DV, GATE, a.R, a.pos + a.n_steps, a.n_steps, E);
+    const int fixed = header_bytes();
+    // two CTAs per SM when registers allow it and each can hold at least
+    // two stages, else one CTA per SM with as many stages as fit
+    const int per_sm = 227 * 1024;
+    int ctas = 2, S = (per_sm / 2 - 1024 - fixed) / SL.bytes;
+    if (S > kMaxStages) S = kMaxStages;
+    int smem = fixed + S * SL.bytes;
+    int resident = 0;
+    if (S >= 2) {
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, kern, kThreads, smem);
+        if (e != cudaSuccess) return e;
+    }
+    if (S < 2 || resident < 2) {
+        ctas = 1;
+        S = (per_sm - 1024 - fixed) / SL.bytes;
+        if (S > kMaxStages) S = kMaxStages;
+        smem = fixed + S * SL.bytes;
+    }
+    if (S < 1) return cudaErrorInvalidConfiguration;
+    const int BH = a.B * a.H;
+    int grid = sm_count[dev & 63] * ctas;
+    if (grid > BH) grid = BH;
+    kern<<<grid, kThreads, smem, stream>>>(a, S);
+    return cudaGetLastError();
 }
 
 template <int DK, int DV>
-cudaError_t launch_decode_d(const DecodeArgs &a, int gate, bool bf16, bool commit,
-                            cudaStream_t stream) {
+cudaError_t launch_decode_d(const DecodeArgs &a, int gate, bool bf16, cudaStream_t stream) {
     if (gate == 1)
-        return bf16 ? launch_decode_c<DK, DV, 1, true>(a, commit, stream)
-                    : launch_decode_c<DK, DV, 1, false>(a, commit, stream);
-    return bf16 ? launch_decode_c<DK, DV, 0, true>(a, commit, stream)
-                : launch_decode_c<DK, DV, 0, false>(a, commit, stream);
+        return bf16 ? launch_d<DK, DV, 1, true>(a, stream) : launch_d<DK, DV, 1, false>(a, stream);
+    return bf16 ? launch_d<DK, DV, 0, true>(a, stream) : launch_d<DK, DV, 0, false>(a, stream);
 }
 
 }  // namespace
 
-cudaError_t launch_decode(const DecodeArgs &a, int d_k, int d_v, int gate, bool bf16, bool commit,
+cudaError_t launch_decode(const DecodeArgs &a, int d_k, int d_v, int gate, bool bf16,
                           cudaStream_t stream) {
-    if (d_k == 128 && d_v == 128) return launch_decode_d<128, 128>(a, gate, bf16, commit, stream);
-    if (d_k == 128 && d_v == 64) return launch_decode_d<128, 64>(a, gate, bf16, commit, stream);
-    if (d_k == 64 && d_v == 128) return launch_decode_d<64, 128>(a, gate, bf16, commit, stream);
-    if (d_k == 64 && d_v == 64) return launch_decode_d<64, 64>(a, gate, bf16, commit, stream);
+    if (a.n_steps < 1) return cudaErrorInvalidValue;
+    if (d_k == 128 && d_v == 128) return launch_decode_d<128, 128>(a, gate, bf16, stream);
+    if (d_k == 128 && d_v == 64) return launch_decode_d<128, 64>(a, gate, bf16, stream);
+    if (d_k == 64 && d_v == 128) return launch_decode_d<64, 128>(a, gate, bf16, stream);
+    if (d_k == 64 && d_v == 64) return launch_decode_d<64, 64>(a, gate, bf16, stream);
     return cudaErrorInvalidValue;
 }
 

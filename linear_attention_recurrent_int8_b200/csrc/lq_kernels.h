@@ -7,7 +7,7 @@
 
 namespace lq {
 
-// Arguments of the decode / commit kernel (one CTA per (b, h)).
+// Arguments of the decode and commit kernels.
 struct DecodeArgs {
     int8_t *codes;
     float *row_scale;
@@ -54,9 +54,13 @@ struct RecurArgs {
     int t0, nt;   // tokens [t0, t0+nt) processed by this launch
 };
 
-cudaError_t launch_decode(const DecodeArgs &a, int d_k, int d_v, int gate, bool bf16, bool commit,
+// Decodes a.n_steps >= 1 tokens (records a.pos .. a.pos + n_steps - 1).
+cudaError_t launch_decode(const DecodeArgs &a, int d_k, int d_v, int gate, bool bf16,
                           cudaStream_t stream);
-int decode_smem_bytes(int d_k, int d_v, int gate, int R, int W);
+
+// Commits the window of a.pos >= 1 buffered records (a.n_steps unused):
+// rebuild, compensators, smoothing, int8 codes, written over the snapshot.
+cudaError_t launch_commit(const DecodeArgs &a, int d_k, int d_v, int gate, cudaStream_t stream);
 
 // Reads the device error word and clears it (synchronizes the device).
 cudaError_t read_and_clear_dev_error(unsigned int *out);
