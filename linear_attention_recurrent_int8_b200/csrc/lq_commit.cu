@@ -29,8 +29,10 @@
 //  * producer (one lane): the head's records, compensators and scales into a
 //    ring of shared-memory stages by 1-D bulk copies (no multicast), and an L2
 //    prefetch of its int8 codes;
-//  * 4 builder warps: the TF32 hi/lo operands of the rank term, then one lane
-//    issues the MMAs into one of two TMEM accumulators;
+//  * 4 builder warps: the TF32 hi/lo operands of the rank term into one of
+//    two operand buffers;
+//  * MMA warp (one lane): the MMAs of a head into one of two TMEM
+//    accumulators once its operands are built and the accumulator is free;
 //  * 8 epilogue warps: C1-C4 from TMEM (lane quarter q = warp % 4 holds value
 //    rows 32q..32q+31, the two warps of a quarter split the key channels),
 //    while the builders already work on the next head.
@@ -47,14 +49,15 @@ namespace {
 
 constexpr int kEpiWarps = 8, kBldWarps = 4;
 constexpr int kEpi = kEpiWarps * 32, kBld = kBldWarps * 32;
-constexpr int kProducerWarp = kEpiWarps + kBldWarps;
-constexpr int kThreads = kEpi + kBld + 32;
+constexpr int kProducerWarp = kEpiWarps + kBldWarps, kMmaWarp = kProducerWarp + 1;
+constexpr int kThreads = kEpi + kBld + 64;
 constexpr int kMaxStages = 4;
 constexpr int kEpiBar = 1, kBldBar = 2;  // named barriers
 
 template <int DK, int DV>
 struct alignas(16) CommitSmem {
     uint64_t full[kMaxStages], empty[kMaxStages];  // stage ring
+    uint64_t ops_ready[2];                         // operand buffers filled
     uint64_t mma_done[2], tmem_free[2];            // TMEM accumulators
     uint32_t tmem;                                 // TMEM base address
     // builders
@@ -117,10 +120,18 @@ __host__ __device__ constexpr int scratch_bytes() {
     return align128((int)sizeof(CommitSmem<DK, DV>));
 }
 
+// x rounded to TF32 (10 explicit mantissa bits), to nearest with ties away
+// from zero, as a 32-bit pattern: add half a TF32 unit to the magnitude and
+// truncate (a carry into the exponent is the correct rounding; the values
+// here are finite).
 __device__ __forceinline__ uint32_t to_tf32(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return r;
+    return (__float_as_uint(x) + 0x1000u) & 0xFFFFE000u;
+}
+
+// The TF32 pair (hi, lo) with x = hi + lo + O(2^-22 |x|): lo = x - hi is exact.
+__device__ __forceinline__ void split_tf32(float x, uint32_t &hi, uint32_t &lo) {
+    hi = to_tf32(x);
+    lo = to_tf32(x - __uint_as_float(hi));
 }
 
 __device__ __forceinline__ uint32_t word_of(const uint4 &w, int k) {
@@ -162,6 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1) commit_kernel(const DecodeArgs a,
             mbar_init(&cs.empty[s], kEpiWarps + kBldWarps);
         }
         for (int b = 0; b < 2; ++b) {
+            mbar_init(&cs.ops_ready[b], kBldWarps);
             mbar_init(&cs.mma_done[b], 1);
             mbar_init(&cs.tmem_free[b], kEpiWarps);
         }
@@ -197,81 +209,21 @@ __global__ void __launch_bounds__(kThreads, 1) commit_kernel(const DecodeArgs a,
         return;
     }
 
-    // ------------------------------------------------------------ builders
-    if (warp >= kEpiWarps) {
-        const int bt = tid - kEpi;
-        int it = 0;
-        for (int bh = blockIdx.x; bh < BH; bh += gridDim.x, ++it) {
-            const int s = it % NS, b = it & 1;
-            bool ok = mbar_wait_bounded(&cs.full[s], (it / NS) & 1);
-            // the operand buffer is free once the MMAs that read it completed
-            if (ok && it >= NOPS) ok = mbar_wait_bounded(&cs.mma_done[(it - NOPS) & 1], ((it - NOPS) >> 1) & 1);
-            if (named_sync_or<kBldBar, kBld>(!ok)) break;  // the group leaves together
-            const unsigned char *st = stages + (size_t)s * SL.bytes;
-            const float *Ks = reinterpret_cast<const float *>(st + SL.K);
-            const float *Us = reinterpret_cast<const float *>(st + SL.U);
-            const float *Ls = reinterpret_cast<const float *>(st + SL.L);
-            const float *Cs = reinterpret_cast<const float *>(st + SL.comp);
-            const int *Cr = reinterpret_cast<const int *>(st + SL.compr);
-            unsigned char *ops = opsbase + (size_t)(it % NOPS) * OL.bytes;
-            unsigned char *Ahi = ops + OL.ahi, *Alo = ops + OL.alo, *Bhi = ops + OL.bhi, *Blo = ops + OL.blo;
-            for (int j = bt; j < DK; j += kBld) cs.gW[j] = expf(Ls[(nrec - 1) * G + (GATE == 1 ? j : 0)]);
-            if (GATE == 0 && bt < nrec) cs.dec[bt] = expf(Ls[nrec - 1] - Ls[bt]);
-            named_sync<kBldBar, kBld>();
-            // B: row j = key channel, element m = record m or compensator m - n
-            for (int e4 = bt; e4 < (Kp / 4) * DK; e4 += kBld) {
-                const int kc = e4 / DK, j = e4 % DK;
-                uint32_t hi[4], lo[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int m = 4 * kc + e;
-                    float x = 0.0f;
-                    if (m < nrec) {
-                        const float dcy = GATE == 1 ? expf(Ls[(nrec - 1) * DK + j] - Ls[m * DK + j]) : cs.dec[m];
-                        x = Ks[m * DK + j] * dcy;
-                    } else if (m < nrec + R) {
-                        x = Cs[(m - nrec) * DK + j] * cs.gW[j];
-                    }
-                    hi[e] = to_tf32(x);
-                    lo[e] = to_tf32(x - __uint_as_float(hi[e]));
-                }
-                const int off = (kc * DK + j) * 16;
-                *reinterpret_cast<uint4 *>(Bhi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                *reinterpret_cast<uint4 *>(Blo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-            }
-            // A: row r = value channel (zero beyond d_v), element m = u_m,r or
-            // the compensator's one-hot column (exact in TF32)
-            for (int kc = 0; kc < Kp / 4; ++kc) {
-                const int r = bt;
-                uint32_t hi[4], lo[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int m = 4 * kc + e;
-                    float x = 0.0f;
-                    if (r < DV) {
-                        if (m < nrec) x = Us[m * DV + r];
-                        else if (m < nrec + R) x = Cr[m - nrec] == r ? 1.0f : 0.0f;
-                    }
-                    hi[e] = to_tf32(x);
-                    lo[e] = to_tf32(x - __uint_as_float(hi[e]));
-                }
-                const int off = (kc * 128 + r) * 16;
-                *reinterpret_cast<uint4 *>(Ahi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                *reinterpret_cast<uint4 *>(Alo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&cs.empty[s]);
-            // the accumulator is free once the epilogue of head it - 2 is done
-            ok = true;
-            if (bt == 0 && it >= 2) ok = mbar_wait_bounded(&cs.tmem_free[b], ((it - 2) >> 1) & 1);
-            if (named_sync_or<kBldBar, kBld>(!ok)) break;
-            if (bt == 0) {
+    // ------------------------------------------------------------ MMA issuer
+    if (warp == kMmaWarp) {
+        if (lane == 0) {
+            int it = 0;
+            for (int bh = blockIdx.x; bh < BH; bh += gridDim.x, ++it) {
+                const int b = it & 1, ob = it % NOPS;
+                if (!mbar_wait_bounded(&cs.ops_ready[ob], (it / NOPS) & 1)) break;
+                // the accumulator is free once the epilogue of head it - 2 is done
+                if (it >= 2 && !mbar_wait_bounded(&cs.tmem_free[b], ((it - 2) >> 1) & 1)) break;
                 tc_fence_after_sync();
+                const unsigned char *ops = opsbase + (size_t)ob * OL.bytes;
                 constexpr uint32_t idesc = idesc_tf32(128, DK);
                 const uint32_t d = cs.tmem + b * DK;
-                const uint32_t ah = smem_u32(Ahi), al = smem_u32(Alo);
-                const uint32_t bhs = smem_u32(Bhi), bls = smem_u32(Blo);
+                const uint32_t ah = smem_u32(ops + OL.ahi), al = smem_u32(ops + OL.alo);
+                const uint32_t bhs = smem_u32(ops + OL.bhi), bls = smem_u32(ops + OL.blo);
                 for (int k8 = 0; k8 < Kp / 8; ++k8) {
                     const uint32_t ao = k8 * 2 * 128 * 16, bo = k8 * 2 * DK * 16;
                     const uint64_t dah = smem_desc(ah + ao, 128 * 16, 128);
@@ -288,10 +240,102 @@ __global__ void __launch_bounds__(kThreads, 1) commit_kernel(const DecodeArgs a,
         return;
     }
 
+    // ------------------------------------------------------------ builders
+    if (warp >= kEpiWarps) {
+        const int bt = tid - kEpi;
+        int it = 0;
+        for (int bh = blockIdx.x; bh < BH; bh += gridDim.x, ++it) {
+            const int s = it % NS;
+            bool ok = mbar_wait_bounded(&cs.full[s], (it / NS) & 1);
+            // the operand buffer is free once the MMAs that read it completed
+            if (ok && it >= NOPS) ok = mbar_wait_bounded(&cs.mma_done[(it - NOPS) & 1], ((it - NOPS) >> 1) & 1);
+            if (named_sync_or<kBldBar, kBld>(!ok)) break;  // the group leaves together
+            const unsigned char *st = stages + (size_t)s * SL.bytes;
+            const float *Ks = reinterpret_cast<const float *>(st + SL.K);
+            const float *Us = reinterpret_cast<const float *>(st + SL.U);
+            const float *Ls = reinterpret_cast<const float *>(st + SL.L);
+            const float *Cs = reinterpret_cast<const float *>(st + SL.comp);
+            const int *Cr = reinterpret_cast<const int *>(st + SL.compr);
+            unsigned char *ops = opsbase + (size_t)(it % NOPS) * OL.bytes;
+            unsigned char *Ahi = ops + OL.ahi, *Alo = ops + OL.alo, *Bhi = ops + OL.bhi, *Blo = ops + OL.blo;
+            for (int j = bt; j < DK; j += kBld) cs.gW[j] = expf(Ls[(nrec - 1) * G + (GATE == 1 ? j : 0)]);
+            if (GATE == 0 && bt < nrec) cs.dec[bt] = expf(Ls[nrec - 1] - Ls[bt]);
+            named_sync<kBldBar, kBld>();
+            // B: row j = key channel, element m = record m or compensator m - n.
+            // Every load is issued unconditionally from a clamped index (all
+            // inside the stage) and the element chosen by selects, so the
+            // loads of a slab are in flight together.
+            {
+                constexpr int SPJ = kBld / DK;        // threads per key channel
+                const int j = bt % DK;
+                const float Lnj = GATE == 1 ? Ls[(nrec - 1) * DK + j] : 0.0f;
+                const float gj = cs.gW[j];
+                for (int kc = bt / DK; kc < Kp / 4; kc += SPJ) {
+                    uint32_t hi[4], lo[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int m = 4 * kc + e;
+                        const int mr = m < nrec ? m : nrec - 1;
+                        const int mc = m - nrec < 0 ? 0 : (m - nrec < R ? m - nrec : (R > 0 ? R - 1 : 0));
+                        const float dcy = GATE == 1 ? expf(Lnj - Ls[mr * DK + j]) : cs.dec[mr];
+                        const float xr = Ks[mr * DK + j] * dcy;
+                        const float xc = R > 0 ? Cs[mc * DK + j] * gj : 0.0f;
+                        const float x = m < nrec ? xr : (m < nrec + R ? xc : 0.0f);
+                        split_tf32(x, hi[e], lo[e]);
+                    }
+                    const int off = (kc * DK + j) * 16;
+                    *reinterpret_cast<uint4 *>(Bhi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                    *reinterpret_cast<uint4 *>(Blo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                }
+            }
+            // A: row r = value channel (zero beyond d_v), element m = u_m,r or
+            // the compensator's one-hot column (exact in TF32)
+            {
+                const int r = bt;
+                const int rr = r < DV ? r : DV - 1;
+                for (int kc = 0; kc < Kp / 4; ++kc) {
+                    uint32_t hi[4], lo[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int m = 4 * kc + e;
+                        const int mr = m < nrec ? m : nrec - 1;
+                        const int mc = m - nrec < 0 ? 0 : (m - nrec < R ? m - nrec : (R > 0 ? R - 1 : 0));
+                        const float xu = Us[mr * DV + rr];
+                        const float xe = (R > 0 && Cr[mc] == r) ? 1.0f : 0.0f;
+                        float x = m < nrec ? xu : (m < nrec + R ? xe : 0.0f);
+                        if (r >= DV) x = 0.0f;
+                        split_tf32(x, hi[e], lo[e]);
+                    }
+                    const int off = (kc * 128 + r) * 16;
+                    *reinterpret_cast<uint4 *>(Ahi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                    *reinterpret_cast<uint4 *>(Alo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&cs.ops_ready[it % NOPS]);
+                mbar_arrive(&cs.empty[s]);
+            }
+        }
+        return;
+    }
+
     // ------------------------------------------------------------ epilogue
     const int qtr = warp & 3, half = warp >> 2;
     const bool has_row = qtr < NQ;  // warp-uniform
     const int row = 32 * qtr + lane, j0 = half * CPT;
+    // the row half's old codes, loaded one head ahead (the producer has
+    // prefetched them into L2)
+    uint4 cw[CPT / 16], cw_next[CPT / 16];
+    auto load_codes = [&](int bhx, uint4(&dst)[CPT / 16]) {
+        if (has_row && bhx < BH) {
+            const int8_t *src = a.codes + ((size_t)bhx * DV + row) * DK + j0;
+#pragma unroll
+            for (int c = 0; c < CPT / 16; ++c) dst[c] = *reinterpret_cast<const uint4 *>(src + 16 * c);
+        }
+    };
+    load_codes(blockIdx.x, cw_next);
     int it = 0;
     for (int bh = blockIdx.x; bh < BH; bh += gridDim.x, ++it) {
         const int s = it % NS, b = it & 1;
@@ -305,14 +349,10 @@ __global__ void __launch_bounds__(kThreads, 1) commit_kernel(const DecodeArgs a,
         const uint32_t tq = cs.tmem + ((uint32_t)(32 * qtr) << 16) + b * DK + j0;
         for (int j = tid; j < DK; j += kEpi) cs.cg[j] = Css[j] * expf(Ls[(nrec - 1) * G + (GATE == 1 ? j : 0)]);
         if (tid < DV) cs.comp_idx[tid] = -1;
-        // the row half's old codes (L2, prefetched) and scale
-        uint4 cw[CPT / 16];
-        float sig = 0.0f;
-        if (has_row) {
 #pragma unroll
-            for (int c = 0; c < CPT / 16; ++c) cw[c] = *reinterpret_cast<const uint4 *>(codes_row + 16 * c);
-            sig = Rss[row];
-        }
+        for (int c = 0; c < CPT / 16; ++c) cw[c] = cw_next[c];
+        load_codes(bh + gridDim.x, cw_next);
+        const float sig = has_row ? Rss[row] : 0.0f;
         const bool ok = mbar_wait_bounded(&cs.mma_done[b], (it >> 1) & 1);
         if (named_sync_or<kEpiBar, kEpi>(!ok)) break;  // also publishes cg and comp_idx
         tc_fence_after_sync();
@@ -353,33 +393,27 @@ __global__ void __launch_bounds__(kThreads, 1) commit_kernel(const DecodeArgs a,
         }
         named_sync<kEpiBar, kEpi>();
 
-        // C2: warp 0 selects the R rows of largest squared norm (ties to the
-        // smaller row)
+        // C2: warp 0 selects the R rows of largest squared norm, ties to the
+        // smaller row.  Keys are the norm's bit pattern + 1 (non-negative
+        // floats order like their bits); a selected row's key becomes 0.
         if (warp == 0 && R > 0) {
-            float val[NQ];
+            uint32_t key[NQ];
 #pragma unroll
-            for (int p = 0; p < NQ; ++p) val[p] = cs.rowpart[0][lane + 32 * p] + cs.rowpart[1][lane + 32 * p];
+            for (int p = 0; p < NQ; ++p)
+                key[p] = __float_as_uint(cs.rowpart[0][lane + 32 * p] + cs.rowpart[1][lane + 32 * p]) + 1u;
             for (int c = 0; c < R; ++c) {
-                float bv = -1.0f;
-                int bi = DV;
+                uint32_t km = key[0];
+#pragma unroll
+                for (int p = 1; p < NQ; ++p) km = km > key[p] ? km : key[p];
+                km = __reduce_max_sync(0xffffffffu, km);
+                uint32_t mine = DV;
+#pragma unroll
+                for (int p = NQ - 1; p >= 0; --p)
+                    if (key[p] == km) mine = lane + 32 * p;
+                const uint32_t bi = __reduce_min_sync(0xffffffffu, mine);
 #pragma unroll
                 for (int p = 0; p < NQ; ++p)
-                    if (val[p] > bv) {
-                        bv = val[p];
-                        bi = lane + 32 * p;
-                    }
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-                    if (ov > bv || (ov == bv && oi < bi)) {
-                        bv = ov;
-                        bi = oi;
-                    }
-                }
-#pragma unroll
-                for (int p = 0; p < NQ; ++p)
-                    if (lane + 32 * p == bi) val[p] = -1.0f;
+                    if (lane + 32 * p == (int)bi) key[p] = 0u;
                 if (lane == 0) {
                     cs.sel[c] = bi;
                     cs.comp_idx[bi] = c;
