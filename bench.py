@@ -112,11 +112,18 @@ def measured_peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
-def source_digest():
+# the sources of each kernel's translation unit (the .cu and the headers it includes)
+KERNEL_SOURCES = {
+    "decode": ["lq_decode.cu", "lq_common.cuh", "lq_quant.cuh", "lq_kernels.h"],
+    "commit": ["lq_commit.cu", "lq_common.cuh", "lq_quant.cuh", "lq_tc.cuh", "lq_kernels.h"],
+}
+
+
+def source_digest(kernel: str) -> str:
     h = hashlib.sha1()
-    for f in sorted(glob.glob(os.path.join(ROOT, "linear_attention_recurrent_int8_b200", "csrc", "*"))):
-        with open(f, "rb") as fh:
-            h.update(os.path.basename(f).encode())
+    for name in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "linear_attention_recurrent_int8_b200", "csrc", name), "rb") as fh:
+            h.update(name.encode())
             h.update(fh.read())
     return h.hexdigest()[:12]
 
@@ -124,7 +131,7 @@ def source_digest():
 def profiled_traffic(kernel_key: str):
     """dram bytes per launch recorded by an ncu capture summary under
     profiles/, if it was taken on the current kernel sources."""
-    digest = source_digest()
+    digest = source_digest(kernel_key.split(":")[0])
     for f in glob.glob(os.path.join(ROOT, "profiles", "*.md")):
         text = open(f).read()
         m_key = re.search(r"^traffic_key:\s*(\S+)", text, re.M)
@@ -427,7 +434,7 @@ def run_lq(args, wl):
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed_max / args.steps,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8+f32",
         "data": "synthetic", "config": workload_config(wl, args),
         "roofline": roof, "gpu_launches": (W + 1) * args.steps,
         "detail": extra,

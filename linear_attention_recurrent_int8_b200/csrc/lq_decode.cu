@@ -38,6 +38,7 @@
 // error word and the waiting warp stops.
 #include <atomic>
 #include <cstddef>
+#include <type_traits>
 
 #include "lq_kernels.h"
 #include "lq_quant.cuh"
@@ -105,10 +106,10 @@ __host__ __device__ inline StageLayout stage_layout(int DK, int DV, int gate, in
 __host__ __device__ constexpr int header_bytes() { return 3 * kMaxStages * 8; }
 
 // Splits the d_k-vector x (lane l holds x_j for the CPL channels
-// j = j0 .. j0+CPL-1) into three int8 limbs with one scale
-// s = max_j |x_j| / 127:  x ~= s (X0 + X1/2^7 + X2/2^14), |error| <= s / 2^15
-// (plus FP32 rounding).  Writes limb[0..2][j] and *lscale.
-template <int CPL>
+// j = j0 .. j0+CPL-1) into NL int8 limbs with one scale s = max_j |x_j| / 127:
+// x ~= s (X0 + X1/2^7 [+ X2/2^14]), |error| <= s / 2^(7 NL - 6) (plus FP32
+// rounding).  Writes limb[0..NL-1][j] and *lscale.
+template <int CPL, int NL>
 __device__ __forceinline__ void split_limbs(const float (&x)[CPL], int8_t *limb, int DK,
                                             float *lscale, int j0) {
     float m = 0.0f;
@@ -116,26 +117,23 @@ __device__ __forceinline__ void split_limbs(const float (&x)[CPL], int8_t *limb,
     for (int e = 0; e < CPL; ++e) m = fmaxf(m, fabsf(x[e]));
     m = group_max<32>(m);
     const float inv = m > 0.0f ? __fdiv_rn(127.0f, m) : 0.0f;
-    uint32_t w0 = 0, w1 = 0, w2 = 0;
+    uint32_t w[NL];
+#pragma unroll
+    for (int l = 0; l < NL; ++l) w[l] = 0;
 #pragma unroll
     for (int e = 0; e < CPL; ++e) {
-        const float t = x[e] * inv;
-        const float x0 = rintf(t);
-        const float r1 = (t - x0) * 128.0f;
-        const float x1 = rintf(r1);
-        const float x2 = rintf((r1 - x1) * 128.0f);
-        w0 |= (static_cast<uint32_t>(static_cast<int>(x0)) & 0xFFu) << (8 * e);
-        w1 |= (static_cast<uint32_t>(static_cast<int>(x1)) & 0xFFu) << (8 * e);
-        w2 |= (static_cast<uint32_t>(static_cast<int>(x2)) & 0xFFu) << (8 * e);
+        float r = x[e] * inv;
+#pragma unroll
+        for (int l = 0; l < NL; ++l) {
+            const float xl = rintf(r);
+            w[l] |= (static_cast<uint32_t>(static_cast<int>(xl)) & 0xFFu) << (8 * e);
+            r = (r - xl) * 128.0f;
+        }
     }
-    if constexpr (CPL == 4) {
-        *reinterpret_cast<uint32_t *>(limb + j0) = w0;
-        *reinterpret_cast<uint32_t *>(limb + DK + j0) = w1;
-        *reinterpret_cast<uint32_t *>(limb + 2 * DK + j0) = w2;
-    } else {
-        *reinterpret_cast<uint16_t *>(limb + j0) = (uint16_t)w0;
-        *reinterpret_cast<uint16_t *>(limb + DK + j0) = (uint16_t)w1;
-        *reinterpret_cast<uint16_t *>(limb + 2 * DK + j0) = (uint16_t)w2;
+#pragma unroll
+    for (int l = 0; l < NL; ++l) {
+        if constexpr (CPL == 4) *reinterpret_cast<uint32_t *>(limb + l * DK + j0) = w[l];
+        else *reinterpret_cast<uint16_t *>(limb + l * DK + j0) = (uint16_t)w[l];
     }
     if (threadIdx.x % 32 == 0) *lscale = m * (1.0f / 127.0f);
 }
@@ -298,8 +296,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a,
                         xq[e] = cj[e] * (gj[e] * qj[e]);
                         kq = fmaf(beta * kj[e], qj[e], kq);
                     }
-                    split_limbs<CPL>(xk, limb, DK, lscale, j0);
-                    split_limbs<CPL>(xq, limb + 3 * DK, DK, lscale + 1, j0);
+                    split_limbs<CPL, 3>(xk, limb, DK, lscale, j0);
+                    split_limbs<CPL, 3>(xq, limb + 3 * DK, DK, lscale + 1, j0);
                     kq = group_sum<32>(kq);
                     if (lane == 0) coefG[nrec + R] = kq;
                 } else {
@@ -320,15 +318,16 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a,
                         if (GATE == 0 && lane == 0) a.buf_gate[(size_t)bh * W + nrec] = Ls;
                     }
                     __syncwarp();
-                    // coefficients of records 0..nrec-1 and compensators,
-                    // eight items per pass, passes shared round-robin by the
-                    // prep-B warps; the 16 partial dot products of a pass are
-                    // reduced together with a transposing reduction
+                    // coefficients of records 0..nrec-1 and compensators, P = 8
+                    // items per pass, passes shared round-robin by the prep-B
+                    // warps; the 2P partial dot products of a pass are reduced
+                    // together with a transposing reduction
                     const int nitems = nrec + R;
-                    for (int base = 8 * bpart; base < nitems; base += 8 * kPrepBWarps) {
-                        float part[16];
+                    auto coef_pass = [&](auto PC, int base) {
+                        constexpr int P = decltype(PC)::value;
+                        float part[2 * P];
 #pragma unroll
-                        for (int q8 = 0; q8 < 8; ++q8) {
+                        for (int q8 = 0; q8 < P; ++q8) {
                             const int it = base + q8;
                             float da = 0.0f, dq = 0.0f;
                             if (it < nitems) {
@@ -356,18 +355,20 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a,
                                 }
                             }
                             part[q8] = da;
-                            part[8 + q8] = dq;
+                            part[P + q8] = dq;
                         }
-                        transposed_sum<16, 32>(part, lane);
-                        const int idx = transposed_index<16, 32>(lane);
-                        const int it = base + (idx & 7);
-                        if (it < nitems && lane == transposed_owner<16, 32>(idx)) {
+                        transposed_sum<2 * P, 32>(part, lane);
+                        const int idx = transposed_index<2 * P, 32>(lane);
+                        const int it = base + (idx % P);
+                        if (it < nitems && lane == transposed_owner<2 * P, 32>(idx)) {
                             float v = part[0];
                             if (GATE == 0 && it < nrec) v *= expf(Ls - recL_s[it]);
-                            if (idx < 8) coefA[it] = v;
+                            if (idx < P) coefA[it] = v;
                             else coefG[it] = v;
                         }
-                    }
+                    };
+                    for (int base = 8 * bpart; base < nitems; base += 8 * kPrepBWarps)
+                        coef_pass(std::integral_constant<int, 8>{}, base);
                 }
                 __syncwarp();
             }
@@ -413,37 +414,31 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a,
             const float *coefA = reinterpret_cast<const float *>(slot + PL.coefA);
             const float *coefG = reinterpret_cast<const float *>(slot + PL.coefG);
 
-            // D2: S^_0 x for this warp's rows: dp4a of the codes with the limbs
+            // D2: S^_0 x for this warp's rows: dp4a of the codes with the limbs.
+            // A0 2^7 + A1 is exact in int32 (|.| < 2^26) and converted once;
+            // the vector scales are applied after the cross-lane reduction.
             float y;
             {
                 uint4 lw[6];
 #pragma unroll
                 for (int v = 0; v < 6; ++v)
                     lw[v] = *reinterpret_cast<const uint4 *>(limb + v * DK + 16 * cc);
-                int acc[NRM][6];
+                float vals[2 * NRM];
 #pragma unroll
                 for (int n = 0; n < NRM; ++n) {
                     const int r = warp * RPW + n * RPI16 + sub;
                     const uint4 w = *reinterpret_cast<const uint4 *>(codes_s + r * DK + 16 * cc);
+                    int acc[6];
 #pragma unroll
                     for (int v = 0; v < 6; ++v) {
                         int x = __dp4a((int)w.x, (int)lw[v].x, 0);
                         x = __dp4a((int)w.y, (int)lw[v].y, x);
                         x = __dp4a((int)w.z, (int)lw[v].z, x);
-                        acc[n][v] = __dp4a((int)w.w, (int)lw[v].w, x);
+                        acc[v] = __dp4a((int)w.w, (int)lw[v].w, x);
                     }
-                }
-                const float sk = lscale[0], sq = lscale[1];
-                float vals[2 * NRM];
-#pragma unroll
-                for (int n = 0; n < NRM; ++n) {
-                    // |acc| < 2^18: exact conversions without the conversion pipe
-                    vals[n] = sk * fmaf(small_int_to_f32(acc[n][2]), 6.103515625e-05f,
-                                        fmaf(small_int_to_f32(acc[n][1]), 0.0078125f,
-                                             small_int_to_f32(acc[n][0])));
-                    vals[NRM + n] = sq * fmaf(small_int_to_f32(acc[n][5]), 6.103515625e-05f,
-                                              fmaf(small_int_to_f32(acc[n][4]), 0.0078125f,
-                                                   small_int_to_f32(acc[n][3])));
+                    // (A0 2^7 + A1) 2^7 + A2, in units of 2^-14 of the vector's scale
+                    vals[n] = fmaf(__int2float_rn(acc[0] * 128 + acc[1]), 128.0f, small_int_to_f32(acc[2]));
+                    vals[NRM + n] = fmaf(__int2float_rn(acc[3] * 128 + acc[4]), 128.0f, small_int_to_f32(acc[5]));
                 }
                 transposed_sum<2 * NRM, LPR16>(vals, lane);
                 y = vals[0];
@@ -451,8 +446,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a,
             // D3-D6 for row `row`: LPRD lanes share its buffered records
             {
                 const float sg = sig_s[row];
-                const float yk = __shfl_sync(0xffffffffu, y, src_k) * sg;
-                const float yq = __shfl_sync(0xffffffffu, y, src_q) * sg;
+                const float yk = __shfl_sync(0xffffffffu, y, src_k) * (sg * (lscale[0] * 6.103515625e-05f));
+                const float yq = __shfl_sync(0xffffffffu, y, src_q) * (sg * (lscale[1] * 6.103515625e-05f));
                 float hb = part == 0 ? yk : 0.0f, p = part == 0 ? yq : 0.0f;
                 for (int m = part; m < nrec; m += LPRD) {
                     const float um = recU_s[m * DV + row];
