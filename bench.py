@@ -40,6 +40,8 @@ if ROOT not in sys.path:
 
 METRIC = "decode tokens/s (state-update+output) and HBM GB/s as % of B200 peak"
 FALLBACK_HBM_GBS = 6650.0
+# FP32 FMA peak of one B200: 148 SMs x 128 FP32 lanes x 2 FLOP x 1.965 GHz
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
 # --------------------------------------------------------------------------
@@ -549,14 +551,90 @@ def run_prefill(args):
     ms = a.elapsed_time(b) / args.steps
     nbytes = B * T * H * (2 * (2 * dk + dv) + 8 + 2 * dv)
     flops = B * T * H * 3 * 2 * dk * dv
-    return {"metric": "prefill tokens/s (state update + output, snapshots every 1024 tokens)",
+    tflops = flops / (ms / 1e3) / 1e12
+    line = {"metric": "prefill tokens/s (state update + output, snapshots every 1024 tokens)",
             "value": B * T / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": f"gdn prefill batch {B} x {H} heads, d={dk}, T={T}, bf16, "
                                    f"snapshot every {every} (r={r})"},
-            "detail": {"io_gbs": nbytes / (ms / 1e3) / 1e9, "fp32_tflops": flops / (ms / 1e3) / 1e12,
-                       "snapshots": T // every}}
+            # the token-sequential FP32 recurrence is bound by FP32 FMA issue:
+            # 3 x 2 d_k d_v FLOP per (token, head) against 148 SMs x 128 FP32
+            # lanes x 2 FLOP x 1.965 GHz
+            "roofline": {"bound": "alu", "achieved": tflops, "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s",
+                         "frac": tflops / FP32_ALU_TFLOPS, "traffic": None,
+                         "kernel": "recur_kernel (FP32 recurrence) + quantize_kernel (snapshots)"},
+            "detail": {"io_gbs": nbytes / (ms / 1e3) / 1e9, "snapshots": T // every}}
+    if not args.no_cpu:
+        rate, dt, cores, sample = oracle_prefill_rate(P, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                "sample": sample}
+    return line
+
+
+def oracle_prefill_rate(P, target_s: float):
+    """The CPU oracle's prefill (FP64 recurrence, snapshots every 1024 tokens)
+    on a bounded sample of heads and tokens; tokens/s counts sequence tokens
+    (all heads of a sequence), scaled from the sampled heads."""
+    import numpy as np
+    cores = len(os.sched_getaffinity(0))
+    os.environ.setdefault("OMP_NUM_THREADS", str(cores))
+    import oracle
+    from linear_attention_recurrent_int8_b200 import synth
+    dk, dv, H, every, r = P["d_k"], P["d_v"], P["heads"], P["snapshot_every"], P["n_comp"]
+
+    def run(nh, T):
+        tok = synth.tokens(P["seed"], [0], list(range(nh)), 0, T, dk, dv, "scalar", "bf16")
+        hm = lambda x: np.ascontiguousarray(np.swapaxes(np.asarray(x), 1, 2).reshape(
+            (nh, T) + np.asarray(x).shape[3:]))
+        d, kt, b = oracle.gdn_instance(hm(tok["alpha"]), hm(tok["beta"]), hm(tok["k"]))
+        t0 = time.perf_counter()
+        oracle.prefill(np.zeros((nh, dv, dk)), d, kt, b, hm(tok["v"]), hm(tok["q"]), every, r)
+        return time.perf_counter() - t0
+
+    dt1 = run(H, every)
+    T = every * int(max(1, min(P["T"] // every, round(target_s / max(dt1, 1e-6)))))
+    dt = run(H, T)
+    return T / dt, dt, cores, f"one sequence (all {H} heads) x {T} tokens ({dt:.1f} s)"
+
+
+def run_init(args, wl):
+    """State initialisation (I1): quantize an FP32 state of every (sequence,
+    head) into the int8 snapshot (compensators, smoothing, codes)."""
+    import torch
+
+    import linear_attention_recurrent_int8_b200 as lq
+    from linear_attention_recurrent_int8_b200 import synth
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    cfg = lq.Config(batch=wl.batch, heads=wl.heads, d_k=wl.d_k, d_v=wl.d_v, window=wl.window,
+                    n_comp=wl.n_comp, gate=lq.LQ_GATE_DIAG if wl.gate == "diag" else lq.LQ_GATE_SCALAR,
+                    io_dtype=lq.LQ_BF16 if wl.io == "bf16" else lq.LQ_F32,
+                    smoothing=int(wl.smoothing))
+    st = lq.State(cfg, dev)
+    S0 = synth.torch_initial_state(wl.seed, range(wl.batch), range(wl.heads), wl.d_k, wl.d_v,
+                                   wl.outlier_rows, wl.outlier_cols, wl.outlier_scale, dev)
+    S0 = S0.reshape(wl.nh, wl.d_v, wl.d_k).contiguous()
+    for _ in range(args.warmup):
+        lq.lq_state_init(st, S0)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        lq.lq_state_init(st, S0)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / args.steps
+    nbytes = wl.nh * (4 * wl.d_v * wl.d_k + snapshot_bytes(wl.d_k, wl.d_v, wl.n_comp))
+    peak, kind = measured_peaks()
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"metric": "state init: heads quantized per second", "value": wl.nh / (ms / 1e3),
+            "unit": "heads/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic", "config": workload_config(wl, args),
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                         "traffic": None, "kernel": "quantize_kernel",
+                         "bytes_per_launch": nbytes, "peak_source": f"{kind} hbm_gbs (copy)"}}
 
 
 def run_fp32step(args, wl):
@@ -663,7 +741,7 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["lq", "reference"], default="lq")
-    ap.add_argument("--mode", choices=["decode", "prefill", "fp32step", "mse"], default="decode",
+    ap.add_argument("--mode", choices=["decode", "prefill", "fp32step", "mse", "init"], default="decode",
                     help="decode (default, the headline) or a comparator / report")
     ap.add_argument("--prefill-tokens", type=int, default=0)
     ap.add_argument("--mse-batch", type=int, default=16)
@@ -704,6 +782,8 @@ def main(argv=None):
         line = run_fp32step(args, wl)
     elif args.mode == "mse":
         line = run_mse(args, wl)
+    elif args.mode == "init":
+        line = run_init(args, wl)
     else:
         line = run_lq(args, wl)
     if line is not None:
