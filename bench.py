@@ -598,6 +598,68 @@ def oracle_prefill_rate(P, target_s: float):
     return T / dt, dt, cores, f"one sequence (all {H} heads) x {T} tokens ({dt:.1f} s)"
 
 
+def run_ragged(args, wl):
+    """Continuous batching: every sequence decodes one token per step at its
+    own window position (positions spread evenly over 0..W-1, so 1/W of the
+    sequences commit at each step) through lq_decode_ragged."""
+    import torch
+
+    import linear_attention_recurrent_int8_b200 as lq
+    from linear_attention_recurrent_int8_b200 import synth
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    W = wl.window
+    cfg = lq.Config(batch=wl.batch, heads=wl.heads, d_k=wl.d_k, d_v=wl.d_v, window=W, n_comp=wl.n_comp,
+                    gate=lq.LQ_GATE_DIAG if wl.gate == "diag" else lq.LQ_GATE_SCALAR,
+                    io_dtype=lq.LQ_BF16 if wl.io == "bf16" else lq.LQ_F32, smoothing=int(wl.smoothing))
+    st = lq.State(cfg, dev)
+    S0 = synth.torch_initial_state(wl.seed, range(wl.batch), range(wl.heads), wl.d_k, wl.d_v,
+                                   wl.outlier_rows, wl.outlier_cols, wl.outlier_scale, dev)
+    lq.lq_state_init(st, S0.reshape(wl.nh, wl.d_v, wl.d_k))
+    del S0
+    # staggered positions: the records below each position are those of a
+    # synthetic earlier stretch of the sequence (any finite values do)
+    seq_pos = (torch.arange(wl.batch, device=dev, dtype=torch.int32) % W).contiguous()
+    st.buf_u.normal_(0.0, 0.1)
+    st.buf_k.normal_(0.0, 0.05)
+    st.buf_gate.copy_(-0.1 * torch.arange(1, W + 1, device=dev, dtype=torch.float32).reshape(
+        (1, W) + (1,) * (st.buf_gate.dim() - 2)).expand_as(st.buf_gate))
+    slots = []
+    for sidx in range(4):
+        tok = synth.torch_tokens(wl.seed, wl.batch, wl.heads, sidx, sidx + 1, wl.d_k, wl.d_v, wl.gate,
+                                 wl.io, dev)
+        slots.append([tok[k].contiguous() for k in ("q", "k", "v", "alpha", "beta")])
+    o = torch.empty((wl.batch, 1, wl.heads, wl.d_v), dtype=cfg.io_torch_dtype, device=dev)
+    lq.lq_decode_ragged(st, seq_pos, *slots[0], o)  # sets kernel attributes before capture
+    torch.cuda.synchronize()
+    # one graph per input slot (the positions live on the device, so replays advance them)
+    graphs = []
+    cs = torch.cuda.Stream(device=dev)
+    for sl in slots:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cs):
+            lq.lq_decode_ragged(st, seq_pos, *sl, o)
+        graphs.append(g)
+    for i in range(args.warmup):
+        graphs[i % 4].replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    steps = args.steps * W
+    a.record()
+    for i in range(steps):
+        graphs[i % 4].replay()
+    b.record()
+    torch.cuda.synchronize()
+    assert lq.lq_device_errors() == 0
+    ms = a.elapsed_time(b) / steps
+    return {"metric": "decode tokens/s, per-sequence window positions", "value": wl.batch / (ms / 1e3),
+            "unit": "tokens/s", "n_gpus": 1, "steps": steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8+f32",
+            "data": "synthetic", "config": dict(workload_config(wl, args),
+                                                step="one token per sequence (decode, commit of the "
+                                                     "sequences whose window filled, position update)")}
+
+
 def run_init(args, wl):
     """State initialisation (I1): quantize an FP32 state of every (sequence,
     head) into the int8 snapshot (compensators, smoothing, codes)."""
@@ -741,7 +803,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["lq", "reference"], default="lq")
-    ap.add_argument("--mode", choices=["decode", "prefill", "fp32step", "mse", "init"], default="decode",
+    ap.add_argument("--mode", choices=["decode", "prefill", "fp32step", "mse", "init", "ragged"],
+                    default="decode",
                     help="decode (default, the headline) or a comparator / report")
     ap.add_argument("--prefill-tokens", type=int, default=0)
     ap.add_argument("--mse-batch", type=int, default=16)
@@ -784,6 +847,8 @@ def main(argv=None):
         line = run_mse(args, wl)
     elif args.mode == "init":
         line = run_init(args, wl)
+    elif args.mode == "ragged":
+        line = run_ragged(args, wl)
     else:
         line = run_lq(args, wl)
     if line is not None:

@@ -26,7 +26,8 @@
  *    They never synchronize, except lq_device_errors.
  *  - Arguments are validated before anything is launched.  A call that
  *    returns an error status other than LQ_ERR_CUDA has launched nothing and
- *    changed nothing (lq_decode_window states its one LQ_ERR_CUDA case).
+ *    changed nothing (lq_decode_window and lq_decode_ragged state their
+ *    LQ_ERR_CUDA cases).
  *  - A launch failure reported by the CUDA runtime returns LQ_ERR_CUDA.
  *  - No C++ exception crosses this boundary.
  *  - One lq_state is used by one stream at a time.
@@ -146,6 +147,27 @@ LQ_API lq_status lq_state_init(lq_state *st, const lq_config *cfg, const float *
 LQ_API lq_status lq_decode_window(lq_state *st, const void *q, const void *k, const void *v,
                            const float *alpha, const float *beta, int32_t n_steps,
                            void *o, lq_stream_t stream);
+
+/* Decode with per-sequence window positions (continuous batching): the
+ * batch's sequences need not share a window position.  seq_pos (device,
+ * int32 [B], 4-byte aligned, in/out) holds for each sequence b the number of
+ * tokens buffered in its open window, 0 <= seq_pos[b] < W, or a negative
+ * value for an idle slot.  One token per active sequence is decoded at window
+ * position seq_pos[b] + 1 (q, k, v, alpha, beta, o laid out as for
+ * lq_decode_window with n = 1; o of idle sequences is not written); every
+ * sequence whose window becomes full is committed in the same call
+ * (lq_window_commit's rule, on that sequence's heads only); then each active
+ * seq_pos[b] advances to (seq_pos[b] + 1) mod W.  Three launches on `stream`
+ * (decode, commit, position update).  Requires the batch-synchronous window
+ * to be closed (pos == 0, else LQ_ERR_WINDOW_OPEN); st->pos is not used
+ * afterwards.  A position >= W cannot be checked on the host: that sequence
+ * is skipped (its position is left as it is) and the device error word
+ * records it (lq_device_errors).
+ * If a later launch fails after an earlier one succeeded, LQ_ERR_CUDA is
+ * returned with the earlier launches' effects in place. */
+LQ_API lq_status lq_decode_ragged(lq_state *st, int32_t *seq_pos, const void *q, const void *k,
+                           const void *v, const float *alpha, const float *beta, void *o,
+                           lq_stream_t stream);
 
 /* Window commit ("LeapQuant: ...", Figures 2 and 4): rebuilds the FP32
  * state S_pos = S^_0 D_{1..pos} + sum_m u_m (D_{m+1..pos} k~_m)^T, keeps its

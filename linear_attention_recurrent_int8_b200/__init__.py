@@ -27,7 +27,8 @@ LQ_GATE_SCALAR, LQ_GATE_DIAG = 0, 1
 LQ_F32, LQ_BF16 = 0, 1
 
 # Every symbol include/lq.h declares.
-ABI_SYMBOLS = ("lq_buffer_elems", "lq_state_init", "lq_decode_window", "lq_window_commit",
+ABI_SYMBOLS = ("lq_buffer_elems", "lq_state_init", "lq_decode_window", "lq_decode_ragged",
+               "lq_window_commit",
                "lq_prefill_chunk", "lq_state_snapshot", "lq_state_restore", "lq_fp32_step",
                "lq_state_destroy", "lq_status_string", "lq_device_errors")
 
@@ -75,6 +76,7 @@ def load_library(build: bool = True):
                 "lq_buffer_elems": (ctypes.c_int64, [ctypes.POINTER(LqConfig), I32]),
                 "lq_state_init": (I32, [ctypes.POINTER(LqState), ctypes.POINTER(LqConfig), P, P]),
                 "lq_decode_window": (I32, [ctypes.POINTER(LqState), P, P, P, P, P, I32, P, P]),
+                "lq_decode_ragged": (I32, [ctypes.POINTER(LqState), P, P, P, P, P, P, P, P]),
                 "lq_window_commit": (I32, [ctypes.POINTER(LqState), P]),
                 "lq_prefill_chunk": (I32, [ctypes.POINTER(LqState), P, P, P, P, P, P, I32, I32,
                                            ctypes.POINTER(LqSnapshot), P, P]),
@@ -224,6 +226,14 @@ def lq_decode_window(st: State, q, k, v, alpha, beta, n_steps: int, o, stream=No
     _check(load_library().lq_decode_window(ctypes.byref(st.c), _ptr(q), _ptr(k), _ptr(v),
                                            _ptr(alpha), _ptr(beta), int(n_steps), _ptr(o),
                                            _stream(stream)), "lq_decode_window")
+
+
+def lq_decode_ragged(st: State, seq_pos, q, k, v, alpha, beta, o, stream=None) -> None:
+    """One token per active sequence at its own window position (seq_pos:
+    int32 device tensor [B], negative = idle slot; updated in place)."""
+    _check(load_library().lq_decode_ragged(ctypes.byref(st.c), _ptr(seq_pos), _ptr(q), _ptr(k),
+                                           _ptr(v), _ptr(alpha), _ptr(beta), _ptr(o),
+                                           _stream(stream)), "lq_decode_ragged")
 
 
 def lq_window_commit(st: State, stream=None) -> None:

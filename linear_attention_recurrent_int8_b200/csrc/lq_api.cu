@@ -184,6 +184,40 @@ lq_status lq_decode_window(lq_state *st, const void *q, const void *k, const voi
     return LQ_OK;
 }
 
+lq_status lq_decode_ragged(lq_state *st, int32_t *seq_pos, const void *q, const void *k,
+                           const void *v, const float *alpha, const float *beta, void *o,
+                           lq_stream_t stream) {
+    lq_status e = check_state(st);
+    if (e != LQ_OK) return e;
+    if (st->pos != 0) return LQ_ERR_WINDOW_OPEN;
+    if (!seq_pos) return LQ_ERR_INVALID_ARGUMENT;
+    if (!aligned_to(seq_pos, 4)) return LQ_ERR_MISALIGNED;
+    e = check_tokens(&st->cfg, q, k, v, alpha, beta, o);
+    if (e != LQ_OK) return e;
+    const int W = st->cfg.window;
+    lq::DecodeArgs a = decode_args(st);
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.alpha = alpha;
+    a.beta = beta;
+    a.o = o;
+    a.seq_pos = seq_pos;
+    // one token per active sequence; stages laid out for W - 1 buffered records
+    a.pos = W - 1;
+    a.n_steps = 1;
+    cudaStream_t s = (cudaStream_t)stream;
+    e = cuda_status(lq::launch_decode(a, st->cfg.d_k, st->cfg.d_v, st->cfg.gate,
+                                      st->cfg.io_dtype == LQ_BF16, s));
+    if (e != LQ_OK) return e;
+    // the sequences whose window is now full (seq_pos == W - 1) commit W records
+    a.pos = W;
+    a.n_steps = 0;
+    e = cuda_status(lq::launch_commit(a, st->cfg.d_k, st->cfg.d_v, st->cfg.gate, s));
+    if (e != LQ_OK) return e;
+    return cuda_status(lq::launch_advance_positions(seq_pos, st->cfg.batch, W, s));
+}
+
 lq_status lq_window_commit(lq_state *st, lq_stream_t stream) {
     lq_status e = check_state(st);
     if (e != LQ_OK) return e;

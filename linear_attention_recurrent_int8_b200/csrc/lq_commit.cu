@@ -148,6 +148,18 @@ __device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
+// The next head of this CTA's grid-stride walk at or after `bh` that commits
+// in this launch: every head with batch-synchronous positions; with
+// per-sequence positions the heads of sequences whose window has just
+// filled (seq_pos[b] == W - 1).  Every role walks the same sequence.
+__device__ __forceinline__ int next_commit_head(const DecodeArgs &a, int bh) {
+    const int BH = a.B * a.H;
+    if (!a.seq_pos) return bh;
+    for (; bh < BH; bh += gridDim.x)
+        if (a.seq_pos[bh / a.H] == a.W - 1) return bh;
+    return BH;
+}
+
 template <int DK, int DV, int GATE>
 __global__ void __launch_bounds__(kThreads, 1) commit_kernel(const DecodeArgs a, const int NS,
                                                              const int NOPS) {
@@ -186,7 +198,7 @@ __global__ void __launch_bounds__(kThreads, 1) commit_kernel(const DecodeArgs a,
     if (warp == kProducerWarp) {
         if (lane == 0) {
             int it = 0;
-            for (int bh = blockIdx.x; bh < BH; bh += gridDim.x, ++it) {
+            for (int bh = next_commit_head(a, blockIdx.x); bh < BH; bh = next_commit_head(a, bh + gridDim.x), ++it) {
                 const int s = it % NS;
                 if (it >= NS && !mbar_wait_bounded(&cs.empty[s], ((it / NS) - 1) & 1)) break;
                 unsigned char *st = stages + (size_t)s * SL.bytes;
@@ -213,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1) commit_kernel(const DecodeArgs a,
     if (warp == kMmaWarp) {
         if (lane == 0) {
             int it = 0;
-            for (int bh = blockIdx.x; bh < BH; bh += gridDim.x, ++it) {
+            for (int bh = next_commit_head(a, blockIdx.x); bh < BH; bh = next_commit_head(a, bh + gridDim.x), ++it) {
                 const int b = it & 1, ob = it % NOPS;
                 if (!mbar_wait_bounded(&cs.ops_ready[ob], (it / NOPS) & 1)) break;
                 // the accumulator is free once the epilogue of head it - 2 is done
@@ -244,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1) commit_kernel(const DecodeArgs a,
     if (warp >= kEpiWarps) {
         const int bt = tid - kEpi;
         int it = 0;
-        for (int bh = blockIdx.x; bh < BH; bh += gridDim.x, ++it) {
+        for (int bh = next_commit_head(a, blockIdx.x); bh < BH; bh = next_commit_head(a, bh + gridDim.x), ++it) {
             const int s = it % NS;
             bool ok = mbar_wait_bounded(&cs.full[s], (it / NS) & 1);
             // the operand buffer is free once the MMAs that read it completed
@@ -335,9 +347,9 @@ __global__ void __launch_bounds__(kThreads, 1) commit_kernel(const DecodeArgs a,
             for (int c = 0; c < CPT / 16; ++c) dst[c] = *reinterpret_cast<const uint4 *>(src + 16 * c);
         }
     };
-    load_codes(blockIdx.x, cw_next);
+    load_codes(next_commit_head(a, blockIdx.x), cw_next);
     int it = 0;
-    for (int bh = blockIdx.x; bh < BH; bh += gridDim.x, ++it) {
+    for (int bh = next_commit_head(a, blockIdx.x); bh < BH; bh = next_commit_head(a, bh + gridDim.x), ++it) {
         const int s = it % NS, b = it & 1;
         const bool okf = mbar_wait_bounded(&cs.full[s], (it / NS) & 1);
         if (named_sync_or<kEpiBar, kEpi>(!okf)) break;  // the group leaves together
@@ -351,7 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1) commit_kernel(const DecodeArgs a,
         if (tid < DV) cs.comp_idx[tid] = -1;
 #pragma unroll
         for (int c = 0; c < CPT / 16; ++c) cw[c] = cw_next[c];
-        load_codes(bh + gridDim.x, cw_next);
+        load_codes(next_commit_head(a, bh + gridDim.x), cw_next);
         const float sig = has_row ? Rss[row] : 0.0f;
         const bool ok = mbar_wait_bounded(&cs.mma_done[b], (it >> 1) & 1);
         if (named_sync_or<kEpiBar, kEpi>(!ok)) break;  // also publishes cg and comp_idx
@@ -579,6 +591,21 @@ cudaError_t launch_c_d(const DecodeArgs &a, int gate, cudaStream_t stream) {
 }
 
 }  // namespace
+
+namespace {
+__global__ void advance_positions_kernel(int32_t *seq_pos, int B, int W) {
+    const int b = blockIdx.x * blockDim.x + threadIdx.x;
+    if (b < B) {
+        const int p = seq_pos[b];
+        if (p >= 0 && p < W) seq_pos[b] = p + 1 == W ? 0 : p + 1;
+    }
+}
+}  // namespace
+
+cudaError_t launch_advance_positions(int32_t *seq_pos, int B, int W, cudaStream_t stream) {
+    advance_positions_kernel<<<(B + 255) / 256, 256, 0, stream>>>(seq_pos, B, W);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_commit(const DecodeArgs &a, int d_k, int d_v, int gate, cudaStream_t stream) {
     if (a.pos < 1 || a.pos > 32 || a.R < 0 || a.R > kMaxComp) return cudaErrorInvalidValue;

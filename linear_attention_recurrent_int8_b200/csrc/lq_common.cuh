@@ -15,6 +15,7 @@ namespace lq {
 // Device error word, read and cleared by lq_device_errors().
 extern __device__ unsigned int g_dev_error;
 constexpr unsigned int kErrWaitTimeout = 1u;
+constexpr unsigned int kErrBadPosition = 2u;  // a per-sequence window position >= W
 
 // A bounded wait gives up after this many nanoseconds of global time.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s

@@ -138,7 +138,29 @@ __device__ __forceinline__ void split_limbs(const float (&x)[CPL], int8_t *limb,
     if (threadIdx.x % 32 == 0) *lscale = m * (1.0f / 127.0f);
 }
 
-template <int DK, int DV, int GATE, bool BF16>
+// The next head (sequence-major index) of this CTA's grid-stride walk at or
+// after `bh` that decodes in this launch: every head with batch-synchronous
+// positions; with per-sequence positions the heads of sequences whose
+// position is in [0, W) (a position >= W is recorded as an error and skipped).
+// Every role of the CTA walks the same sequence.
+template <bool RAGGED>
+__device__ __forceinline__ int next_decode_head(const DecodeArgs &a, int bh) {
+    if constexpr (RAGGED) {
+        const int BH = a.B * a.H;
+        for (; bh < BH; bh += gridDim.x) {
+            const int p = a.seq_pos[bh / a.H];
+            if (p >= 0 && p < a.W) return bh;
+            if (p >= a.W) atomicOr(&g_dev_error, kErrBadPosition);
+        }
+        return BH;
+    } else {
+        return bh;
+    }
+}
+
+// RAGGED: per-sequence window positions (a.seq_pos); otherwise the window
+// position a.pos is the same for every head and stays a kernel constant.
+template <int DK, int DV, int GATE, bool BF16, bool RAGGED>
 __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a, const int S) {
     constexpr int E = BF16 ? 2 : 4;
     constexpr int RPW = DV / kConsumerWarps;  // value rows per consumer warp
@@ -146,8 +168,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a,
     uint64_t *full = reinterpret_cast<uint64_t *>(smem);
     uint64_t *prepared = full + kMaxStages;
     uint64_t *empty = prepared + kMaxStages;
-    const int nsteps = a.n_steps, pos = a.pos;
-    const StageLayout SL = stage_layout(DK, DV, GATE, a.R, pos + nsteps, nsteps, E);
+    const int nsteps = a.n_steps;
+    const StageLayout SL = stage_layout(DK, DV, GATE, a.R, a.pos + nsteps, nsteps, E);
     const PrepLayout PL = prep_layout(DK);
     unsigned char *stages = smem + header_bytes();
 
@@ -169,8 +191,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a,
         if (lane != 0) return;
         int i = 0;
         bool ok = true;
-        for (int bh = blockIdx.x; bh < BH; bh += gridDim.x, ++i) {
+        for (int bh = next_decode_head<RAGGED>(a, blockIdx.x); bh < BH; bh = next_decode_head<RAGGED>(a, bh + gridDim.x), ++i) {
             const int s = i % S, use = i / S;
+            const int pos = RAGGED ? a.seq_pos[bh / a.H] : a.pos;  // records buffered
             if (use > 0 && !mbar_wait_bounded(&empty[s], (use - 1) & 1)) {
                 ok = false;
                 break;
@@ -233,8 +256,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a,
         constexpr int CPL = DK / 32;          // contiguous key channels per lane
         const int j0 = CPL * lane;
         int i = 0;
-        for (int bh = blockIdx.x; bh < BH; bh += gridDim.x, ++i) {
+        for (int bh = next_decode_head<RAGGED>(a, blockIdx.x); bh < BH; bh = next_decode_head<RAGGED>(a, bh + gridDim.x), ++i) {
             const int s = i % S;
+            const int pos = RAGGED ? a.seq_pos[bh / a.H] : a.pos;  // records buffered
             if (!mbar_wait_bounded(&full[s], (i / S) & 1)) break;
             unsigned char *st = stages + (size_t)s * SL.bytes;
             const float *cs_s = reinterpret_cast<const float *>(st + SL.cs);
@@ -393,8 +417,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a,
     const int src_q = (rloc % RPI16) * LPR16 + transposed_owner<2 * NRM, LPR16>(NRM + rloc / RPI16);
 
     int i = 0;
-    for (int bh = blockIdx.x; bh < BH; bh += gridDim.x, ++i) {
+    for (int bh = next_decode_head<RAGGED>(a, blockIdx.x); bh < BH; bh = next_decode_head<RAGGED>(a, bh + gridDim.x), ++i) {
         const int s = i % S;
+        const int pos = RAGGED ? a.seq_pos[bh / a.H] : a.pos;  // records buffered
         if (!mbar_wait_bounded(&prepared[s], (i / S) & 1)) break;
         unsigned char *st = stages + (size_t)s * SL.bytes;
         const int8_t *codes_s = reinterpret_cast<const int8_t *>(st + SL.codes);
@@ -484,7 +509,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a,
     }
 }
 
-template <int DK, int DV, int GATE, bool BF16>
+template <int DK, int DV, int GATE, bool BF16, bool RAGGED>
 cudaError_t launch_d(const DecodeArgs &a, cudaStream_t stream) {
     constexpr int E = BF16 ? 2 : 4;
     static std::atomic<uint64_t> configured{0};  // devices already set up
@@ -492,7 +517,7 @@ cudaError_t launch_d(const DecodeArgs &a, cudaStream_t stream) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    auto kern = decode_kernel<DK, DV, GATE, BF16>;
+    auto kern = decode_kernel<DK, DV, GATE, BF16, RAGGED>;
     const uint64_t bit = 1ull << (dev & 63);
     if (!(configured.load(std::memory_order_acquire) & bit)) {
         int optin = 0, sms = 0;
@@ -532,11 +557,17 @@ cudaError_t launch_d(const DecodeArgs &a, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
+template <int DK, int DV, int GATE, bool BF16>
+cudaError_t launch_dr(const DecodeArgs &a, cudaStream_t stream) {
+    return a.seq_pos ? launch_d<DK, DV, GATE, BF16, true>(a, stream)
+                     : launch_d<DK, DV, GATE, BF16, false>(a, stream);
+}
+
 template <int DK, int DV>
 cudaError_t launch_decode_d(const DecodeArgs &a, int gate, bool bf16, cudaStream_t stream) {
     if (gate == 1)
-        return bf16 ? launch_d<DK, DV, 1, true>(a, stream) : launch_d<DK, DV, 1, false>(a, stream);
-    return bf16 ? launch_d<DK, DV, 0, true>(a, stream) : launch_d<DK, DV, 0, false>(a, stream);
+        return bf16 ? launch_dr<DK, DV, 1, true>(a, stream) : launch_dr<DK, DV, 1, false>(a, stream);
+    return bf16 ? launch_dr<DK, DV, 0, true>(a, stream) : launch_dr<DK, DV, 0, false>(a, stream);
 }
 
 }  // namespace

@@ -24,9 +24,16 @@ struct DecodeArgs {
     const float *beta;
     void *o;
     int B, H, W, R;
-    int pos;      // records already buffered
+    int pos;      // records already buffered (the same for every sequence)
     int n_steps;  // tokens decoded by this launch (0: commit only)
     int smoothing;
+    // per-sequence window positions [B] (device), or nullptr.  When set, the
+    // decode takes one token per sequence b with seq_pos[b] in [0, W) at
+    // window position seq_pos[b] + 1 (pos and n_steps are then W - 1 and 1,
+    // the sizes the stages are laid out for) and skips sequences with
+    // seq_pos[b] < 0; the commit takes the sequences with seq_pos[b] == W - 1
+    // (pos is then W).
+    const int32_t *seq_pos;
 };
 
 // Arguments of the quantize-from-FP32 kernel (init, prefill snapshots).
@@ -61,6 +68,9 @@ cudaError_t launch_decode(const DecodeArgs &a, int d_k, int d_v, int gate, bool 
 // Commits the window of a.pos >= 1 buffered records (a.n_steps unused):
 // rebuild, compensators, smoothing, int8 codes, written over the snapshot.
 cudaError_t launch_commit(const DecodeArgs &a, int d_k, int d_v, int gate, cudaStream_t stream);
+
+// seq_pos[b] <- (seq_pos[b] + 1) mod W for the sequences with 0 <= seq_pos[b] < W.
+cudaError_t launch_advance_positions(int32_t *seq_pos, int B, int W, cudaStream_t stream);
 
 // Reads the device error word and clears it (synchronizes the device).
 cudaError_t read_and_clear_dev_error(unsigned int *out);

@@ -161,3 +161,21 @@ def test_state_init_validation_without_launch():
     c = cfg.c()
     assert lib.lq_state_init(ctypes.byref(st), ctypes.byref(c), 0x1234, None) == lq.LQ_ERR_MISALIGNED
     assert lib.lq_state_init(None, ctypes.byref(c), None, None) == lq.LQ_ERR_INVALID_ARGUMENT
+
+
+def test_ragged_validation_without_launch():
+    lib = lq.load_library()
+    cfg = lq.Config(batch=2, heads=3, window=4, n_comp=2)
+    p = 0x50000000
+    toks = [p, p + 0x100000, p + 0x200000, p + 0x300000, p + 0x400000]
+    o = p + 0x500000
+    # no positions array, misaligned positions, an open synchronous window, null inputs
+    assert lib.lq_decode_ragged(ctypes.byref(_fake_state(cfg)), None, *toks, o, None) == \
+        lq.LQ_ERR_INVALID_ARGUMENT
+    assert lib.lq_decode_ragged(ctypes.byref(_fake_state(cfg)), p + 0x600002, *toks, o, None) == \
+        lq.LQ_ERR_MISALIGNED
+    assert lib.lq_decode_ragged(ctypes.byref(_fake_state(cfg, pos=1)), p + 0x600000, *toks, o,
+                                None) == lq.LQ_ERR_WINDOW_OPEN
+    assert lib.lq_decode_ragged(ctypes.byref(_fake_state(cfg)), p + 0x600000, None, *toks[1:], o,
+                                None) == lq.LQ_ERR_INVALID_ARGUMENT
+    assert lib.lq_decode_ragged(None, p + 0x600000, *toks, o, None) == lq.LQ_ERR_INVALID_ARGUMENT
