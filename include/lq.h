@@ -15,7 +15,10 @@
  * Table 4):  S_t = S_{t-1} D_t + (v_t - S_{t-1} b_t) k~_t^T,  o_t = S_t q_t,
  * with S in R^{d_v x d_k} (row = value channel), k~_t = beta_t k_t and
  *   scalar gate (Gated DeltaNet, Table 4):   D_t = alpha_t I,       b_t = alpha_t k_t
- *   diagonal gate (Kimi Delta Attention):    D_t = Diag(alpha_t),   b_t = alpha_t * k_t.
+ *   diagonal gate (Kimi Delta Attention):    D_t = Diag(alpha_t),   b_t = alpha_t * k_t
+ * and, with lq_config.delta = 0, b_t = 0 for either gate (the Table 4 rows of
+ * linear attention, RetNet, Mamba2 and GLA; k~_t = beta_t k_t, so those rows'
+ * k~ = k is beta = 1).
  *
  * Conventions of every call:
  *  - Every pointer argument named as device memory is caller-owned CUDA
@@ -82,7 +85,11 @@ typedef struct {
     int32_t io_dtype;    /* lq_dtype of q, k, v, o                          */
     int32_t smoothing;   /* 1: residual smoothing on; 0: c == 1             */
     int32_t auto_commit; /* 1: the decode call that fills the window also
-                            commits it, inside the same launch              */
+                            commits it (a second launch)                    */
+    int32_t delta;       /* 1: delta rule, b_t = D_t k_t (Gated DeltaNet,
+                            DeltaNet with alpha = 1, Kimi Delta Attention);
+                            0: b_t = 0, u_t = v_t (linear attention, RetNet,
+                            Mamba2, GLA: the b = 0 rows of Table 4)         */
 } lq_config;
 
 /* The quantized boundary state of every (b, h), all device memory:

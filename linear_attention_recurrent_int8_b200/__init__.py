@@ -41,7 +41,7 @@ class LQError(RuntimeError):
 
 class LqConfig(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("batch", "heads", "d_k", "d_v", "window", "n_comp",
-                                              "gate", "io_dtype", "smoothing", "auto_commit")]
+                                              "gate", "io_dtype", "smoothing", "auto_commit", "delta")]
 
 
 class LqSnapshot(ctypes.Structure):
@@ -130,10 +130,11 @@ class Config:
     io_dtype: int = LQ_BF16
     smoothing: int = 1
     auto_commit: int = 1
+    delta: int = 1
 
     def c(self) -> LqConfig:
         return LqConfig(self.batch, self.heads, self.d_k, self.d_v, self.window, self.n_comp,
-                        self.gate, self.io_dtype, self.smoothing, self.auto_commit)
+                        self.gate, self.io_dtype, self.smoothing, self.auto_commit, self.delta)
 
     @property
     def gdim(self) -> int:

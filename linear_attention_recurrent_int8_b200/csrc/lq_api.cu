@@ -25,7 +25,8 @@ lq_status check_config(const lq_config *c) {
     if (c->n_comp < 0 || c->n_comp > 16 || c->n_comp > c->d_v) return LQ_ERR_INVALID_ARGUMENT;
     if (c->gate != LQ_GATE_SCALAR && c->gate != LQ_GATE_DIAG) return LQ_ERR_INVALID_ARGUMENT;
     if (c->io_dtype != LQ_F32 && c->io_dtype != LQ_BF16) return LQ_ERR_INVALID_ARGUMENT;
-    if ((c->smoothing != 0 && c->smoothing != 1) || (c->auto_commit != 0 && c->auto_commit != 1))
+    if ((c->smoothing != 0 && c->smoothing != 1) || (c->auto_commit != 0 && c->auto_commit != 1) ||
+        (c->delta != 0 && c->delta != 1))
         return LQ_ERR_INVALID_ARGUMENT;
     return LQ_OK;
 }
@@ -78,6 +79,7 @@ lq::DecodeArgs decode_args(const lq_state *st) {
     a.B = st->cfg.batch;
     a.H = st->cfg.heads;
     a.W = st->cfg.window;
+    a.delta = st->cfg.delta;
     a.R = st->cfg.n_comp;
     a.pos = st->pos;
     a.smoothing = st->cfg.smoothing;
@@ -262,6 +264,7 @@ lq_status lq_prefill_chunk(lq_state *st, float *S_fp32, const void *q, const voi
     r.beta = beta;
     r.o = o;
     r.B = c->batch;
+    r.delta = c->delta;
     r.H = c->heads;
     r.T_total = T;
     for (int t0 = 0, i = 0; t0 < T; t0 += snapshot_every, ++i) {
@@ -318,6 +321,7 @@ lq_status lq_fp32_step(const lq_config *cfg, float *S, const void *q, const void
     r.beta = beta;
     r.o = o;
     r.B = cfg->batch;
+    r.delta = cfg->delta;
     r.H = cfg->heads;
     r.T_total = n_steps;
     r.t0 = 0;

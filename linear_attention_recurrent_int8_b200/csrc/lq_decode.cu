@@ -316,7 +316,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a,
                     load_vec<CPL>(cj, cs_s + j0);
 #pragma unroll
                     for (int e = 0; e < CPL; ++e) {
-                        xk[e] = cj[e] * (gj[e] * kj[e]);
+                        xk[e] = a.delta ? cj[e] * (gj[e] * kj[e]) : 0.0f;  // b = 0 rows: no S b term
                         xq[e] = cj[e] * (gj[e] * qj[e]);
                         kq = fmaf(beta * kj[e], qj[e], kq);
                     }
@@ -347,6 +347,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a,
                     // warps; the 2P partial dot products of a pass are reduced
                     // together with a transposing reduction
                     const int nitems = nrec + R;
+                    float kb[CPL];  // the b-side channels: k, or 0 for the b = 0 rows
+#pragma unroll
+                    for (int e = 0; e < CPL; ++e) kb[e] = a.delta ? kj[e] : 0.0f;
                     auto coef_pass = [&](auto PC, int base) {
                         constexpr int P = decltype(PC)::value;
                         float part[2 * P];
@@ -366,14 +369,14 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a,
                                     }
 #pragma unroll
                                     for (int e = 0; e < CPL; ++e) {
-                                        da = fmaf(w[e], kj[e], da);
+                                        da = fmaf(w[e], kb[e], da);
                                         dq = fmaf(w[e], qj[e], dq);
                                     }
                                 } else {
                                     load_vec<CPL>(w, compv_s + (it - nrec) * DK + j0);
 #pragma unroll
                                     for (int e = 0; e < CPL; ++e) {
-                                        da = fmaf(w[e], gj[e] * kj[e], da);
+                                        da = fmaf(w[e], gj[e] * kb[e], da);
                                         dq = fmaf(w[e], gj[e] * qj[e], dq);
                                     }
                                 }

@@ -24,6 +24,7 @@ struct DecodeArgs {
     const float *beta;
     void *o;
     int B, H, W, R;
+    int delta;    // 1: b_t = D_t k_t (delta rule); 0: b_t = 0
     int pos;      // records already buffered (the same for every sequence)
     int n_steps;  // tokens decoded by this launch (0: commit only)
     int smoothing;
@@ -57,6 +58,7 @@ struct RecurArgs {
     const float *beta;
     void *o;
     int B, H;
+    int delta;    // 1: b_t = D_t k_t (delta rule); 0: b_t = 0
     int T_total;  // tokens in the activation tensors (time stride)
     int t0, nt;   // tokens [t0, t0+nt) processed by this launch
 };

@@ -98,13 +98,16 @@ __global__ void __launch_bounds__(NWARPS * 32) recur_kernel(const RecurArgs a) {
             } else {
                 a4[0] = a4[1] = a4[2] = a4[3] = a_s[tt][0];
             }
+            float b4[4];  // b_t = alpha (.) k_t, or 0 for the b = 0 rows
+#pragma unroll
+            for (int e = 0; e < 4; ++e) b4[e] = a.delta ? a4[e] * k4[e] : 0.0f;
             float acc[2 * NR];
 #pragma unroll
             for (int n = 0; n < NR; ++n) {
-                float hb = S[n][0] * (a4[0] * k4[0]), pp = S[n][0] * (a4[0] * q4[0]);
+                float hb = S[n][0] * b4[0], pp = S[n][0] * (a4[0] * q4[0]);
 #pragma unroll
                 for (int e = 1; e < 4; ++e) {
-                    hb = fmaf(S[n][e], a4[e] * k4[e], hb);
+                    hb = fmaf(S[n][e], b4[e], hb);
                     pp = fmaf(S[n][e], a4[e] * q4[e], pp);
                 }
                 acc[n] = hb;

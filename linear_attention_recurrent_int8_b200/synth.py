@@ -146,6 +146,7 @@ class DecodeWorkload:
     outlier_cols: int = 0
     outlier_scale: float = 30.0
     seed: int = 0
+    delta: int = 1                # 1: delta rule (b = D k); 0: b = 0 (Mamba2 / GLA rows)
     extra: dict = field(default_factory=dict)
 
     @property

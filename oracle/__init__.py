@@ -102,6 +102,20 @@ def kda_instance(alpha, beta, k):
     return alpha, beta[..., None] * k, alpha * k
 
 
+def gated_linear_instance(alpha, beta, k, diagonal: bool):
+    """The b = 0 rows of Table 4 (linear attention with D = I, RetNet with a
+    constant decay, Mamba2 with a per-token scalar decay, GLA with a per-channel
+    decay): D = alpha I or Diag(alpha), k~ = beta k (those rows print k~ = k,
+    i.e. beta = 1), b = 0, so u_t = v_t.
+
+    alpha: [nh, n] (scalar) or [nh, n, d_k] (diagonal); beta: [nh, n]; k: [nh, n, d_k]."""
+    alpha = np.asarray(alpha, np.float64)
+    beta = np.asarray(beta, np.float64)
+    k = np.asarray(k, np.float64)
+    d = alpha if diagonal else alpha[..., None]
+    return d, beta[..., None] * k, np.zeros_like(k)
+
+
 # --------------------------------------------------------------------------
 # Equation 1, explicit stepping.
 # --------------------------------------------------------------------------

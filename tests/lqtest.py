@@ -38,7 +38,7 @@ def make_config(wl: synth.DecodeWorkload, **over) -> lq.Config:
     c = lq.Config(batch=wl.batch, heads=wl.heads, d_k=wl.d_k, d_v=wl.d_v, window=wl.window,
                   n_comp=wl.n_comp, gate=lq.LQ_GATE_DIAG if wl.gate == "diag" else lq.LQ_GATE_SCALAR,
                   io_dtype=lq.LQ_BF16 if wl.io == "bf16" else lq.LQ_F32,
-                  smoothing=int(wl.smoothing), auto_commit=1)
+                  smoothing=int(wl.smoothing), auto_commit=1, delta=wl.delta)
     for k, v in over.items():
         setattr(c, k, v)
     return c
@@ -51,11 +51,13 @@ def heads_major(x):
     return np.ascontiguousarray(np.swapaxes(x, 1, 2).reshape((B * H, T) + x.shape[3:]))
 
 
-def oracle_tokens(tok: dict, gate: str):
+def oracle_tokens(tok: dict, gate: str, delta: int = 1):
     """Oracle-side (d, k~, b, v, q) [nh, n, ...] from synth.tokens output."""
     q, k, v = heads_major(tok["q"]), heads_major(tok["k"]), heads_major(tok["v"])
     alpha, beta = heads_major(tok["alpha"]), heads_major(tok["beta"])
-    if gate == "diag":
+    if not delta:
+        d, kt, b = oracle.gated_linear_instance(alpha, beta, k, gate == "diag")
+    elif gate == "diag":
         d, kt, b = oracle.kda_instance(alpha, beta, k)
     else:
         d, kt, b = oracle.gdn_instance(alpha, beta, k)
@@ -203,7 +205,7 @@ class AnchoredRun:
         torch.cuda.synchronize()
         assert self.st.pos == 0
 
-        d, kt, b, v, q = oracle_tokens(tok, wl.gate)
+        d, kt, b, v, q = oracle_tokens(tok, wl.gate, wl.delta)
         rec = oracle.empty_records(wl.nh, W, wl.d_k, wl.d_v, cfg.gdim)
         o_ref = oracle.window(self.snap, rec, 0, d, kt, b, v, q)
         new_snap, S_n = oracle.commit(self.snap, rec, ntok, cfg.n_comp, bool(cfg.smoothing))
@@ -301,7 +303,7 @@ class SampledRun:
             o[:, t:t + 1] = out
         torch.cuda.synchronize()
         assert self.st.pos == 0
-        d, kt, b, v, q = oracle_tokens(tok_s, wl.gate)
+        d, kt, b, v, q = oracle_tokens(tok_s, wl.gate, wl.delta)
         rec = oracle.empty_records(len(self.sample), W, wl.d_k, wl.d_v, cfg.gdim)
         o_ref = oracle.window(self.snap, rec, 0, d, kt, b, v, q)
         new_snap, _ = oracle.commit(self.snap, rec, W, cfg.n_comp, bool(cfg.smoothing))

@@ -106,6 +106,7 @@ def test_decode_validation_without_launch():
                              ("window", 0, lq.LQ_ERR_INVALID_ARGUMENT),
                              ("n_comp", 17, lq.LQ_ERR_INVALID_ARGUMENT),
                              ("gate", 2, lq.LQ_ERR_INVALID_ARGUMENT),
+                             ("delta", 2, lq.LQ_ERR_INVALID_ARGUMENT),
                              ("batch", 0, lq.LQ_ERR_INVALID_ARGUMENT)):
         c2 = lq.Config(batch=2, heads=3, window=4, n_comp=2)
         setattr(c2, field, val)

@@ -511,3 +511,29 @@ def test_ragged_last_window_commits():
     seen = []
     oracle.decode_run(snap, d, kt, b, v, q, W=8, n_comp=4, on_commit=lambda i, s: seen.append(i))
     assert seen == [0, 1, 2]
+
+
+@pytest.mark.parametrize("diagonal", [False, True])
+def test_gated_linear_instance_matches_published_updates(diagonal):
+    """oracle.gated_linear_instance + eq1 = the Mamba2 (scalar decay) or GLA
+    (per-channel decay) update alpha S + v k^T with beta = 1, and
+    alpha S + beta v k^T in general; the outputs are S_t q_t."""
+    dv, dk, n = 3, 5, 8
+    r = _rng(7)
+    S = r.normal(size=(dv, dk))
+    nh = 1
+    alpha = 1.0 / (1.0 + np.exp(r.normal(size=(nh, n, dk) if diagonal else (nh, n))))
+    for beta_is_one in (True, False):
+        beta = np.ones((nh, n)) if beta_is_one else 1.0 / (1.0 + np.exp(-r.normal(size=(nh, n))))
+        k = np.stack([_unit(r.normal(size=dk)) for _ in range(n)])[None]
+        v = r.normal(size=(nh, n, dv))
+        q = r.normal(size=(nh, n, dk))
+        d, kt, b = oracle.gated_linear_instance(alpha, beta, k, diagonal)
+        assert np.all(b == 0.0)
+        o, S_eq1 = oracle.eq1_steps(S[None], d, kt, b, v, q)
+        S_pub = S.copy()
+        for t in range(n):
+            decay = np.diag(alpha[0, t]) if diagonal else alpha[0, t] * np.eye(dk)
+            S_pub = S_pub @ decay + beta[0, t] * np.outer(v[0, t], k[0, t])
+            assert _rel(o[0, t], S_pub @ q[0, t]) < 1e-13
+        assert _rel(S_eq1[0], S_pub) < 1e-13
