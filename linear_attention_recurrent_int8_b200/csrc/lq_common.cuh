@@ -62,6 +62,17 @@ __device__ __forceinline__ void cp_async4(void *dst_smem, const void *src_gmem) 
                  : "memory");
 }
 
+// 16-byte global -> shared copy (both addresses 16-byte aligned), bypassing L1.
+__device__ __forceinline__ void cp_async16(void *dst_smem, const void *src_gmem) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst_smem)), "l"(src_gmem)
+                 : "memory");
+}
+
+// Closes the group of this thread's cp.async copies issued so far; waits
+// until all of its groups have completed.
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 // Makes `bar` track completion of this thread's earlier cp.async copies: its
 // pending arrival count is raised by one now and lowered when they complete.
 __device__ __forceinline__ void cp_async_mbar_arrive(uint64_t *bar) {

@@ -16,6 +16,8 @@
 // formed in one pass and reduced with a transposing warp reduction; then
 // u = v - S b, o = S_{t-1}(alpha*q) + u (k~ . q), S = S Diag(alpha) + u k~^T.
 // Inputs are staged through shared memory in chunks of tokens.
+#include <atomic>
+
 #include "lq_common.cuh"
 #include "lq_kernels.h"
 
@@ -144,13 +146,207 @@ __global__ void __launch_bounds__(NWARPS * 32) recur_kernel(const RecurArgs a) {
             make_float4(S[n][0], S[n][1], S[n][2], S[n][3]);
 }
 
+// Long runs (prefill): the same ownership (a lane holds 4 key channels of
+// each of its warp's rows, so each token vector is read once per warp with
+// one load per lane), 8 rows per warp, and no shared-memory round trip
+// inside the token loop: after the transposing reduction the lane that holds
+// S_{t-1} b_t of a row forms u_t, passes it by shuffle to the lane that holds
+// S_{t-1} (alpha q_t) (which writes o_t), and every lane fetches the rows'
+// u_t by shuffle for its update.  The tokens' raw inputs arrive in chunks of
+// 16 by 16-byte cp.async copies into a second buffer while the current
+// chunk is computed, so no load latency sits on the token loop.
+template <int DK, int DV, int GATE, bool BF16, int NWARPS>
+struct RowsSmem {
+    static constexpr int E = BF16 ? 2 : 4, G = GATE == 1 ? DK : 1, RPC = NWARPS * 8;
+    alignas(16) unsigned char k[2][kChunk][DK * E];
+    alignas(16) unsigned char q[2][kChunk][DK * E];
+    alignas(16) unsigned char v[2][kChunk][RPC * E];
+    alignas(16) float al[2][kChunk][G];
+    alignas(16) float beta[2][kChunk];
+    float kq[2][kChunk];
+};
+
+template <int DK, int DV, int GATE, bool BF16, int NWARPS>
+__global__ void __launch_bounds__(NWARPS * 32) recur_rows_kernel(const RecurArgs a) {
+    using Sm = RowsSmem<DK, DV, GATE, BF16, NWARPS>;
+    constexpr int E = Sm::E;
+    constexpr int LPR = DK / 4, RPI = 32 / LPR, RW = 8, NR = RW / RPI, RPC = NWARPS * RW;
+    constexpr int NT = NWARPS * 32;
+    static_assert(DV % RPC == 0, "bad row split");
+    extern __shared__ __align__(16) unsigned char rows_smem[];
+    Sm &sm = *reinterpret_cast<Sm *>(rows_smem);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    constexpr int cph = DV / RPC;
+    const int bh = blockIdx.x / cph;
+    const int rbase = (blockIdx.x % cph) * RPC;
+    const int b = bh / a.H, h = bh % a.H;
+    const int c0 = 4 * (lane % LPR);
+    const int rs = lane / LPR;
+    const int idx = transposed_index<2 * NR, LPR>(lane);  // the value this lane holds after the reduction
+    const int gbase = lane & ~(LPR - 1);
+
+    auto tok_of = [&](int t) { return ((size_t)b * a.T_total + a.t0 + t) * a.H + h; };
+    // raw copies of tokens [t, t + n) into buffer p
+    auto stage = [&](int p, int t, int n) {
+        const unsigned char *kg = static_cast<const unsigned char *>(a.k);
+        const unsigned char *qg = static_cast<const unsigned char *>(a.q);
+        const unsigned char *vg = static_cast<const unsigned char *>(a.v);
+        constexpr int KC = DK * E / 16, VC = RPC * E / 16;
+        for (int i = tid; i < n * KC; i += NT) {
+            const int tt = i / KC, c = i % KC;
+            const size_t tok = tok_of(t + tt);
+            cp_async16(&sm.k[p][tt][16 * c], kg + tok * DK * E + 16 * c);
+            cp_async16(&sm.q[p][tt][16 * c], qg + tok * DK * E + 16 * c);
+        }
+        for (int i = tid; i < n * VC; i += NT) {
+            const int tt = i / VC, c = i % VC;
+            cp_async16(&sm.v[p][tt][16 * c], vg + (tok_of(t + tt) * DV + rbase) * E + 16 * c);
+        }
+        if (GATE == 1) {
+            for (int i = tid; i < n * (DK / 4); i += NT) {
+                const int tt = i / (DK / 4), c = i % (DK / 4);
+                cp_async16(&sm.al[p][tt][4 * c], a.alpha + tok_of(t + tt) * DK + 4 * c);
+            }
+        } else {
+            for (int tt = tid; tt < n; tt += NT) cp_async4(&sm.al[p][tt][0], a.alpha + tok_of(t + tt));
+        }
+        for (int tt = tid; tt < n; tt += NT) cp_async4(&sm.beta[p][tt], a.beta + tok_of(t + tt));
+        cp_async_commit();
+    };
+    auto load4 = [&](const unsigned char *row, int j, float (&x)[4]) {
+        if constexpr (BF16) {
+            const uint2 w = *reinterpret_cast<const uint2 *>(row + 2 * j);
+            x[0] = __uint_as_float(w.x << 16);
+            x[1] = __uint_as_float(w.x & 0xFFFF0000u);
+            x[2] = __uint_as_float(w.y << 16);
+            x[3] = __uint_as_float(w.y & 0xFFFF0000u);
+        } else {
+            *reinterpret_cast<float4 *>(x) = *reinterpret_cast<const float4 *>(row + 4 * j);
+        }
+    };
+    auto load1 = [&](const unsigned char *row, int j) -> float {
+        if constexpr (BF16)
+            return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(row)[j]);
+        else
+            return reinterpret_cast<const float *>(row)[j];
+    };
+    // k~ . q of the staged tokens: one warp per token
+    auto kq_of = [&](int p, int n) {
+        for (int tt = warp; tt < n; tt += NWARPS) {
+            float d = 0.0f;
+#pragma unroll
+            for (int e = 0; e < DK / 32; ++e)
+                d = fmaf(load1(sm.k[p][tt], lane + 32 * e), load1(sm.q[p][tt], lane + 32 * e), d);
+            d = group_sum<32>(d);
+            if (lane == 0) sm.kq[p][tt] = sm.beta[p][tt] * d;
+        }
+    };
+
+    float S[NR][4];
+    float *Sg = a.S + ((size_t)bh * DV + rbase) * DK;
+#pragma unroll
+    for (int n = 0; n < NR; ++n) {
+        const float4 x = *reinterpret_cast<const float4 *>(Sg + (size_t)(warp * RW + n * RPI + rs) * DK + c0);
+        S[n][0] = x.x;
+        S[n][1] = x.y;
+        S[n][2] = x.z;
+        S[n][3] = x.w;
+    }
+
+    const int nt = a.nt;
+    if (nt > 0) {
+        stage(0, 0, min(kChunk, nt));
+        cp_async_wait_all();
+        __syncthreads();
+        kq_of(0, min(kChunk, nt));
+        __syncthreads();
+    }
+    for (int tc0 = 0, p = 0; tc0 < nt; tc0 += kChunk, p ^= 1) {
+        const int nc = min(kChunk, nt - tc0);
+        const int nn = min(kChunk, nt - tc0 - nc);
+        if (nn > 0) stage(p ^ 1, tc0 + nc, nn);
+        for (int tt = 0; tt < nc; ++tt) {
+            float k4[4], q4[4], a4[4], b4[4];
+            load4(sm.k[p][tt], c0, k4);
+            load4(sm.q[p][tt], c0, q4);
+            if (GATE == 1) {
+                *reinterpret_cast<float4 *>(a4) = *reinterpret_cast<const float4 *>(&sm.al[p][tt][c0]);
+            } else {
+                a4[0] = a4[1] = a4[2] = a4[3] = sm.al[p][tt][0];
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                b4[e] = a.delta ? a4[e] * k4[e] : 0.0f;
+                q4[e] *= a4[e];
+            }
+            float acc[2 * NR];
+            const float2 b01 = make_float2(b4[0], b4[1]), b23 = make_float2(b4[2], b4[3]);
+            const float2 q01 = make_float2(q4[0], q4[1]), q23 = make_float2(q4[2], q4[3]);
+#pragma unroll
+            for (int n = 0; n < NR; ++n) {
+                const float2 s01 = make_float2(S[n][0], S[n][1]), s23 = make_float2(S[n][2], S[n][3]);
+                const float2 hb = __ffma2_rn(s23, b23, __fmul2_rn(s01, b01));
+                const float2 pp = __ffma2_rn(s23, q23, __fmul2_rn(s01, q01));
+                acc[n] = hb.x + hb.y;
+                acc[NR + n] = pp.x + pp.y;
+            }
+            transposed_sum<2 * NR, LPR>(acc, lane);
+            const int rloc = (idx % NR) * RPI + rs;  // warp-local row of this lane's value
+            float u = 0.0f;
+            if (idx < NR) u = load1(sm.v[p][tt], warp * RW + rloc) - acc[0];
+            const float u_row = __shfl_sync(0xffffffffu, u, gbase + transposed_owner<2 * NR, LPR>(idx % NR));
+            if (idx >= NR && lane == gbase + transposed_owner<2 * NR, LPR>(idx))
+                store_io<BF16>(a.o, tok_of(tc0 + tt) * DV + rbase + warp * RW + rloc,
+                               fmaf(sm.kq[p][tt], u_row, acc[0]));
+            const float beta = sm.beta[p][tt];
+            const float2 kt01 = make_float2(beta * k4[0], beta * k4[1]);
+            const float2 kt23 = make_float2(beta * k4[2], beta * k4[3]);
+            const float2 a01 = make_float2(a4[0], a4[1]), a23 = make_float2(a4[2], a4[3]);
+#pragma unroll
+            for (int n = 0; n < NR; ++n) {
+                const float un = __shfl_sync(0xffffffffu, u, gbase + transposed_owner<2 * NR, LPR>(n));
+                const float2 u2 = make_float2(un, un);
+                const float2 s01 = __ffma2_rn(make_float2(S[n][0], S[n][1]), a01, __fmul2_rn(u2, kt01));
+                const float2 s23 = __ffma2_rn(make_float2(S[n][2], S[n][3]), a23, __fmul2_rn(u2, kt23));
+                S[n][0] = s01.x;
+                S[n][1] = s01.y;
+                S[n][2] = s23.x;
+                S[n][3] = s23.y;
+            }
+        }
+        if (nn > 0) {
+            cp_async_wait_all();
+            __syncthreads();  // the next chunk has arrived; this chunk's buffer is free
+            kq_of(p ^ 1, nn);
+            __syncthreads();
+        }
+    }
+
+#pragma unroll
+    for (int n = 0; n < NR; ++n)
+        *reinterpret_cast<float4 *>(Sg + (size_t)(warp * RW + n * RPI + rs) * DK + c0) =
+            make_float4(S[n][0], S[n][1], S[n][2], S[n][3]);
+}
+
 template <int DK, int DV, int GATE, bool BF16>
 cudaError_t launch_r(const RecurArgs &a, bool long_run, cudaStream_t stream) {
     if (long_run) {
-        // 4 warps x 4 rows: DV/16 CTAs per head
-        constexpr int NW = 4, RW = 4;
-        recur_kernel<DK, DV, GATE, BF16, NW, RW>
-            <<<a.B * a.H * (DV / (NW * RW)), NW * 32, 0, stream>>>(a);
+        // 4 warps x 8 rows: DV/32 CTAs per head
+        constexpr int NW = 4;
+        constexpr int smem = (int)sizeof(RowsSmem<DK, DV, GATE, BF16, NW>);
+        auto kern = recur_rows_kernel<DK, DV, GATE, BF16, NW>;
+        static std::atomic<uint64_t> configured{0};  // devices already set up
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        const uint64_t bit = 1ull << (dev & 63);
+        if (!(configured.load(std::memory_order_acquire) & bit)) {
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            if (e != cudaSuccess) return e;
+            configured.fetch_or(bit, std::memory_order_acq_rel);
+        }
+        kern<<<a.B * a.H * (DV / (NW * 8)), NW * 32, smem, stream>>>(a);
     } else {
         // one CTA of 8 warps per head
         constexpr int NW = 8, RW = DV / 8;
