@@ -130,11 +130,11 @@ def source_digest(kernel: str) -> str:
     return h.hexdigest()[:12]
 
 
-def profiled_traffic(kernel_key: str):
+def profiled_traffic(kernel_key: str, directory: str | None = None):
     """dram bytes per launch recorded by an ncu capture summary under
     profiles/, if it was taken on the current kernel sources."""
     digest = source_digest(kernel_key.split(":")[0])
-    for f in glob.glob(os.path.join(ROOT, "profiles", "*.md")):
+    for f in glob.glob(os.path.join(directory or os.path.join(ROOT, "profiles"), "*.md")):
         text = open(f).read()
         m_key = re.search(r"^traffic_key:\s*(\S+)", text, re.M)
         m_src = re.search(r"^source_sha1:\s*(\S+)", text, re.M)
