@@ -4,14 +4,16 @@
 Workload (default): Gated DeltaNet decode, batch 256 x 32 heads, d_k = d_v =
 128, bf16 q/k/v/o, int8 state with per-row scales, window W = 16, r = 4
 Compensator Tokens, smoothing on.  One STEP is one window: W decode launches
-through the C ABI (the commit fused into the last), i.e. batch * W tokens.
+and the window commit through the C ABI, i.e. batch * W tokens.
 
 Timing: W_warm untimed steps, then exactly K steps bracketed by a barrier and
 torch.cuda.synchronize() on both sides, timed with CUDA events on the
 launching stream, max over ranks.  Each step replays a CUDA graph of the
 window's launches; event-record nodes inside the graph time every launch for
-the roofline.  Each decode launch reads about 250 MB (int8 state, records,
-inputs), twice the 126 MB L2, so every launch streams from HBM.
+the roofline.  Each decode launch reads 160-300 MB (int8 state, records,
+inputs), above the 126 MB L2, so every launch streams from HBM.
+
+Other modes: --mode prefill | fp32step | init | ragged | mse (see --help).
 
 Multi-GPU (torchrun): every rank decodes its own shard of sequences (batch
 per rank fixed: weak scaling); no collective on the data path; the host
