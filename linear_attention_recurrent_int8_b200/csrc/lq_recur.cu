@@ -155,9 +155,9 @@ __global__ void __launch_bounds__(NWARPS * 32) recur_kernel(const RecurArgs a) {
 // u_t by shuffle for its update.  The tokens' raw inputs arrive in chunks of
 // 16 by 16-byte cp.async copies into a second buffer while the current
 // chunk is computed, so no load latency sits on the token loop.
-template <int DK, int DV, int GATE, bool BF16, int NWARPS>
+template <int DK, int DV, int GATE, bool BF16, int NWARPS, int RW>
 struct RowsSmem {
-    static constexpr int E = BF16 ? 2 : 4, G = GATE == 1 ? DK : 1, RPC = NWARPS * 8;
+    static constexpr int E = BF16 ? 2 : 4, G = GATE == 1 ? DK : 1, RPC = NWARPS * RW;
     alignas(16) unsigned char k[2][kChunk][DK * E];
     alignas(16) unsigned char q[2][kChunk][DK * E];
     alignas(16) unsigned char v[2][kChunk][RPC * E];
@@ -166,11 +166,11 @@ struct RowsSmem {
     float kq[2][kChunk];
 };
 
-template <int DK, int DV, int GATE, bool BF16, int NWARPS>
+template <int DK, int DV, int GATE, bool BF16, int NWARPS, int RW>
 __global__ void __launch_bounds__(NWARPS * 32) recur_rows_kernel(const RecurArgs a) {
-    using Sm = RowsSmem<DK, DV, GATE, BF16, NWARPS>;
+    using Sm = RowsSmem<DK, DV, GATE, BF16, NWARPS, RW>;
     constexpr int E = Sm::E;
-    constexpr int LPR = DK / 4, RPI = 32 / LPR, RW = 8, NR = RW / RPI, RPC = NWARPS * RW;
+    constexpr int LPR = DK / 4, RPI = 32 / LPR, NR = RW / RPI, RPC = NWARPS * RW;
     constexpr int NT = NWARPS * 32;
     static_assert(DV % RPC == 0, "bad row split");
     extern __shared__ __align__(16) unsigned char rows_smem[];
@@ -332,10 +332,10 @@ __global__ void __launch_bounds__(NWARPS * 32) recur_rows_kernel(const RecurArgs
 template <int DK, int DV, int GATE, bool BF16>
 cudaError_t launch_r(const RecurArgs &a, bool long_run, cudaStream_t stream) {
     if (long_run) {
-        // 4 warps x 8 rows: DV/32 CTAs per head
-        constexpr int NW = 4;
-        constexpr int smem = (int)sizeof(RowsSmem<DK, DV, GATE, BF16, NW>);
-        auto kern = recur_rows_kernel<DK, DV, GATE, BF16, NW>;
+        // 4 warps x 8 rows: DV/32 CTAs per head (4 rows per warp measured slower)
+        constexpr int NW = 4, RW = 8;
+        constexpr int smem = (int)sizeof(RowsSmem<DK, DV, GATE, BF16, NW, RW>);
+        auto kern = recur_rows_kernel<DK, DV, GATE, BF16, NW, RW>;
         static std::atomic<uint64_t> configured{0};  // devices already set up
         int dev = 0;
         cudaError_t e = cudaGetDevice(&dev);
@@ -346,7 +346,7 @@ cudaError_t launch_r(const RecurArgs &a, bool long_run, cudaStream_t stream) {
             if (e != cudaSuccess) return e;
             configured.fetch_or(bit, std::memory_order_acq_rel);
         }
-        kern<<<a.B * a.H * (DV / (NW * 8)), NW * 32, smem, stream>>>(a);
+        kern<<<a.B * a.H * (DV / (NW * RW)), NW * 32, smem, stream>>>(a);
     } else {
         // one CTA of 8 warps per head
         constexpr int NW = 8, RW = DV / 8;
