@@ -59,7 +59,7 @@ def _load():
             P = ctypes.c_void_p
             I = ctypes.c_int
             lib.lqo_eq1_steps.argtypes = [I, I, I, I, P, P, P, P, P, P, P]
-            lib.lqo_quantize.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P]
+            lib.lqo_quantize.argtypes = [I, I, I, I, I, I, P, P, P, P, P, P, P]
             lib.lqo_dequantize.argtypes = [I, I, I, I, P, P, P, P, P, P]
             lib.lqo_window.argtypes = [I] * 9 + [P] * 14
             lib.lqo_rebuild.argtypes = [I] * 7 + [P] * 9
@@ -152,12 +152,18 @@ class Snapshot(dict):
         return self["comp_row"].shape[1]
 
 
-def quantize(S, n_comp: int, smoothing: bool = True) -> Snapshot:
-    """Compensator selection, residual smoothing and per-row int8 codes of an
-    FP32 state ``S`` [nh, dv, dk] (rounded to FP32 first if it is not)."""
+BITS = (8, 6, 4)  # code widths: q_max = 2^(bits-1) - 1 = 127, 31, 7
+
+
+def quantize(S, n_comp: int, smoothing: bool = True, bits: int = 8) -> Snapshot:
+    """Compensator selection, residual smoothing and per-row codes of an FP32
+    state ``S`` [nh, dv, dk] (rounded to FP32 first if it is not); the codes
+    are ``bits`` wide (8, or the 6- and 4-bit widths of the lower-precision
+    groups of [LQ] Table 1) and returned one per int8."""
     S = _c(S, np.float32)
     nh, dv, dk = S.shape
     assert 0 <= n_comp <= dv
+    assert bits in BITS
     out = Snapshot(
         codes=np.zeros((nh, dv, dk), np.int8),
         row_scale=np.zeros((nh, dv), np.float32),
@@ -166,7 +172,7 @@ def quantize(S, n_comp: int, smoothing: bool = True) -> Snapshot:
         comp_val=np.zeros((nh, n_comp, dk), np.float32),
         row_norm=np.zeros((nh, dv), np.float64),
     )
-    _load().lqo_quantize(nh, dv, dk, n_comp, int(bool(smoothing)), _p(S), _p(out["codes"]),
+    _load().lqo_quantize(nh, dv, dk, n_comp, int(bool(smoothing)), int(bits), _p(S), _p(out["codes"]),
                          _p(out["row_scale"]), _p(out["col_smooth"]), _p(out["comp_row"]),
                          _p(out["comp_val"]), _p(out["row_norm"]))
     return out
@@ -239,16 +245,16 @@ def rebuild(snap, records: Records, n: int) -> np.ndarray:
     return out
 
 
-def commit(snap, records: Records, n: int, n_comp: int, smoothing: bool = True):
+def commit(snap, records: Records, n: int, n_comp: int, smoothing: bool = True, bits: int = 8):
     """Window commit: rebuild S_n (kept as an FP32 state), then quantize.
 
     Returns (new snapshot, S_n as float32)."""
     S = rebuild(snap, records, n).astype(np.float32)
-    return quantize(S, n_comp, smoothing), S
+    return quantize(S, n_comp, smoothing, bits), S
 
 
 def decode_run(snap, d, kt, b, v, q, W: int, n_comp: int, smoothing: bool = True,
-               on_commit=None):
+               on_commit=None, bits: int = 8):
     """Free-running per-window decode of T tokens: windows of W tokens, each
     committed at its end (the last, possibly short, window too).
 
@@ -265,14 +271,15 @@ def decode_run(snap, d, kt, b, v, q, W: int, n_comp: int, smoothing: bool = True
         rec = empty_records(nh, W, dk, dv, gdim)
         sl = slice(t0, t1)
         o[:, sl] = window(snap, rec, 0, d[:, sl], kt[:, sl], b[:, sl], v[:, sl], q[:, sl])
-        snap, _ = commit(snap, rec, t1 - t0, n_comp, smoothing)
+        snap, _ = commit(snap, rec, t1 - t0, n_comp, smoothing, bits)
         if on_commit is not None:
             on_commit(widx, snap)
         widx += 1
     return o, snap
 
 
-def prefill(S0, d, kt, b, v, q, snapshot_every: int, n_comp: int, smoothing: bool = True):
+def prefill(S0, d, kt, b, v, q, snapshot_every: int, n_comp: int, smoothing: bool = True,
+            bits: int = 8):
     """Prefill by the token recurrence (equation 1, FP64 state) with a
     quantized snapshot of the state, rounded to FP32, after every
     ``snapshot_every`` tokens (one state per that many cached tokens).
@@ -288,5 +295,5 @@ def prefill(S0, d, kt, b, v, q, snapshot_every: int, n_comp: int, smoothing: boo
         sl = slice(t0, t1)
         o[:, sl], S = eq1_steps(S, d[:, sl], kt[:, sl], b[:, sl], v[:, sl], q[:, sl])
         if t1 - t0 == snapshot_every:
-            snaps.append(quantize(S.astype(np.float32), n_comp, smoothing))
+            snaps.append(quantize(S.astype(np.float32), n_comp, smoothing, bits))
     return o, snaps, S

@@ -126,10 +126,13 @@ void lqo_eq1_steps(int nh, int dv, int dk, int n, double *S, const double *d,
  *      smoothing is off (SmoothQuant-style migration with strength 1/2 along
  *      the key channels).  Each factor is inverted once, ic_j = fp32(1 / c_j),
  *      and R'_ij = fp32(R_ij * ic_j).
- *  C4  mx_i = max_j |R'_ij|;  sigma_i = fp32(mx_i / 127) (the stored scale);
- *      is_i = fp32(127 / mx_i);  Q_ij = clamp(rne(fp32(R'_ij * is_i)), -127,
- *      127), Q_i. = 0 when mx_i = 0.  Round half to even; no zero point;
- *      -128 unused.
+ *  C4  with q = 2^(bits-1) - 1 (127 for 8 bits; the 6- and 4-bit states of
+ *      [LQ] Table 1's lower-precision groups give 31 and 7):
+ *      mx_i = max_j |R'_ij|;  sigma_i = fp32(mx_i / q) (the stored scale);
+ *      is_i = fp32(q / mx_i);  Q_ij = clamp(rne(fp32(R'_ij * is_i)), -q, q),
+ *      Q_i. = 0 when mx_i = 0.  Round half to even; no zero point; -q-1
+ *      unused.  The codes come back one per int8 whatever the width (the
+ *      packing of a narrower code is a storage format, not arithmetic).
  *
  * Every division, square root and product above is one IEEE FP32 operation
  * on FP32 operands (an FP64 operation rounded once to FP32 gives the same
@@ -139,10 +142,11 @@ void lqo_eq1_steps(int nh, int dv, int dk, int n, double *S, const double *d,
  * correct.
  *
  * row_norm [nh][dv] (optional) receives n_i.                               */
-void lqo_quantize(int nh, int dv, int dk, int r, int smoothing, const float *S,
+void lqo_quantize(int nh, int dv, int dk, int r, int smoothing, int bits, const float *S,
                   int8_t *codes, float *row_scale, float *col_smooth,
                   int32_t *comp_row, float *comp_val, double *row_norm)
 {
+    const double qmax = (double)((1 << (bits - 1)) - 1);
 #pragma omp parallel for schedule(dynamic)
     for (int h = 0; h < nh; ++h) {
         const float *Sh = S + (size_t)h * dv * dk;
@@ -186,22 +190,22 @@ void lqo_quantize(int nh, int dv, int dk, int r, int smoothing, const float *S,
             for (int i = 0; i < dv; ++i)
                 R[(size_t)i * dk + j] = f32(R[(size_t)i * dk + j] * ic);
         }
-        /* C4: per-row symmetric int8. */
+        /* C4: per-row symmetric codes in [-qmax, qmax]. */
         for (int i = 0; i < dv; ++i) {
             double mx = 0.0;
             for (int j = 0; j < dk; ++j) {
                 double a = fabs(R[(size_t)i * dk + j]);
                 if (a > mx) mx = a;
             }
-            double sigma = f32(mx / 127.0);
-            double is = mx > 0.0 ? f32(127.0 / mx) : 0.0;
+            double sigma = f32(mx / qmax);
+            double is = mx > 0.0 ? f32(qmax / mx) : 0.0;
             row_scale[(size_t)h * dv + i] = (float)sigma;
             for (int j = 0; j < dk; ++j) {
                 double qv = 0.0;
                 if (mx > 0.0) {
                     qv = rint(f32(R[(size_t)i * dk + j] * is)); /* ties to even */
-                    if (qv > 127.0) qv = 127.0;
-                    if (qv < -127.0) qv = -127.0;
+                    if (qv > qmax) qv = qmax;
+                    if (qv < -qmax) qv = -qmax;
                 }
                 codes[((size_t)h * dv + i) * dk + j] = (int8_t)qv;
             }

@@ -29,9 +29,13 @@ MUTATIONS = {
     "ties_to_larger_row": ("norm[i] > norm[best]", "norm[i] >= norm[best]"),
     "smoothing_without_sqrt": ("(float)sqrt(m) : 1.0f", "(float)m : 1.0f"),
     "round_half_away": ("qv = rint(f32(", "qv = round(f32("),
-    "no_inverse_scale_rounding": ("double is = mx > 0.0 ? f32(127.0 / mx) : 0.0;",
-                                  "double is = mx > 0.0 ? 127.0 / mx : 0.0;"),
-    "scale_255": ("double sigma = f32(mx / 127.0);", "double sigma = f32(mx / 255.0);"),
+    "no_inverse_scale_rounding": ("double is = mx > 0.0 ? f32(qmax / mx) : 0.0;",
+                                  "double is = mx > 0.0 ? qmax / mx : 0.0;"),
+    "scale_255": ("double sigma = f32(mx / qmax);", "double sigma = f32(mx / (2.0 * qmax + 1.0));"),
+    "code_range_one_too_wide": ("const double qmax = (double)((1 << (bits - 1)) - 1);",
+                                "const double qmax = (double)(1 << (bits - 1));"),
+    "code_width_fixed_at_8": ("const double qmax = (double)((1 << (bits - 1)) - 1);",
+                              "const double qmax = 127.0;"),
 }
 
 

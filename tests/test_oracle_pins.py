@@ -365,11 +365,14 @@ def _outlier_state(nh=4, dv=40, dk=24, seed=7):
     return S.astype(np.float32)
 
 
+@pytest.mark.parametrize("bits", [8, 6, 4])
 @pytest.mark.parametrize("smoothing", [True, False])
 @pytest.mark.parametrize("r", [0, 1, 4])
-def test_quantizer_error_bound_and_compensators(r, smoothing):
+def test_quantizer_error_bound_and_compensators(r, smoothing, bits):
+    """Round to nearest: every residual element is within half a code step
+    (sigma_i c_j / 2) of the original, at every code width."""
     S = _outlier_state()
-    snap = oracle.quantize(S, r, smoothing)
+    snap = oracle.quantize(S, r, smoothing, bits)
     S_hat = oracle.dequantize(snap)
     sig = snap["row_scale"].astype(np.float64)
     c = snap["col_smooth"].astype(np.float64)
@@ -399,10 +402,11 @@ def test_quantizer_selects_top_r_rows(r):
     np.testing.assert_allclose(snap["row_norm"], norms, rtol=1e-15)
 
 
-def test_quantizer_smoothing_and_code_range():
+@pytest.mark.parametrize("bits,qmax", [(8, 127), (6, 31), (4, 7)])
+def test_quantizer_smoothing_and_code_range(bits, qmax):
     S = _outlier_state(seed=9)
     r = 2
-    snap = oracle.quantize(S, r)
+    snap = oracle.quantize(S, r, bits=bits)
     for h in range(S.shape[0]):
         R = S[h].astype(np.float64).copy()
         R[snap["comp_row"][h]] = 0
@@ -413,9 +417,14 @@ def test_quantizer_smoothing_and_code_range():
         assert np.all(np.abs(c * c - m) <= 2.0 ** -22 * m)
         codes = snap["codes"][h].astype(int)
         nz = snap["row_scale"][h] > 0
-        assert np.all(np.abs(codes[nz]).max(axis=1) == 127)
-        assert codes.min() >= -127
+        # every nonzero row reaches the end of the code range, none passes it
+        assert np.all(np.abs(codes[nz]).max(axis=1) == qmax)
+        assert codes.min() >= -qmax and codes.max() <= qmax
         assert not codes[~nz].any()
+        # sigma = row max / qmax: the largest code reconstructs the row max
+        Rp = R * (np.float32(1) / snap["col_smooth"][h]).astype(np.float64)[None, :]
+        np.testing.assert_allclose(snap["row_scale"][h][nz] * qmax,
+                                   np.abs(Rp).max(axis=1)[nz], rtol=2e-7)
 
 
 def test_quantizer_hand_cases():
@@ -447,32 +456,53 @@ def test_quantizer_hand_cases():
     assert abs(oracle.dequantize(s)[0, 1, 5] - 7.0) < 1e-5
 
 
-def test_quantizer_golden_hand_case():
+@pytest.mark.parametrize("bits,qmax,name", [(8, 127, "quantizer_hand_case.txt"),
+                                             (6, 31, "quantizer_hand_case_6bit.txt"),
+                                             (4, 7, "quantizer_hand_case_4bit.txt")])
+def test_quantizer_golden_hand_case(bits, qmax, name):
     vals = {}
-    with open(os.path.join(GOLDEN, "quantizer_hand_case.txt")) as f:
+    with open(os.path.join(GOLDEN, name)) as f:
         for line in f:
             if line.strip() and not line.startswith("#"):
                 key, *rest = line.split()
                 vals[key] = [float(x) for x in rest]
     dv, dk = (int(x) for x in vals["shape"])
     S = np.array(vals["state"], np.float32).reshape(1, dv, dk)
-    s = oracle.quantize(S, int(vals["n_comp"][0]))
+    s = oracle.quantize(S, int(vals["n_comp"][0]), bits=bits)
     assert s["comp_row"][0].tolist() == [int(x) for x in vals["comp_row"]]
     np.testing.assert_array_equal(s["comp_val"][0].ravel(), np.float32(vals["comp_val"]))
     np.testing.assert_array_equal(s["col_smooth"][0], np.float32(vals["col_smooth"]))
     np.testing.assert_array_equal(s["codes"][0].ravel(), np.int8(vals["codes"]))
-    np.testing.assert_allclose(s["row_scale"][0] * 127, vals["row_scale_times_127"], rtol=1e-6)
+    np.testing.assert_allclose(s["row_scale"][0] * qmax, vals[f"row_scale_times_{qmax}"], rtol=1e-6)
 
 
-def test_quantizer_decision_is_fp32():
+def test_quantizer_narrow_codes_hand_cases():
+    """4-bit: sigma = 1 exactly for a row of maximum 7; quotients 2.5 -> 2,
+    -0.5 -> 0, 1.5 -> 2, 3.5 -> 4 (half to even), -6.5 -> -6.  6-bit: a row of
+    maximum 31 likewise."""
+    dv, dk = 4, 8
+    S = np.zeros((1, dv, dk), np.float32)
+    S[0, 1, :6] = [7.0, 2.5, -0.5, 1.5, 3.5, -6.5]
+    s = oracle.quantize(S, 0, smoothing=False, bits=4)
+    assert s["row_scale"][0, 1] == 1.0
+    assert s["codes"][0, 1, :6].tolist() == [7, 2, 0, 2, 4, -6]
+    S[0, 1, :6] = [31.0, 2.5, -0.5, 1.5, 30.5, -29.5]
+    s = oracle.quantize(S, 0, smoothing=False, bits=6)
+    assert s["row_scale"][0, 1] == 1.0
+    assert s["codes"][0, 1, :6].tolist() == [31, 2, 0, 2, 30, -30]
+
+
+@pytest.mark.parametrize("bits", [8, 6, 4])
+def test_quantizer_decision_is_fp32(bits):
     """Codes are rne of FP32 products of FP32 operands (inverse smoothing
     factor and inverse scale each rounded once): recompute the decision with
     numpy float32 arithmetic (IEEE single) and compare bit for bit."""
     # large enough (5e5 codes) that rounding the inverse scale differently
     # moves some quotient across a .5 boundary
     S = _outlier_state(nh=32, dv=128, dk=128, seed=10)
-    snap = oracle.quantize(S, 2)
-    one, q127 = np.float32(1), np.float32(127)
+    snap = oracle.quantize(S, 2, bits=bits)
+    qm = 2 ** (bits - 1) - 1
+    one, q127 = np.float32(1), np.float32(qm)
     for h in range(S.shape[0]):
         R = S[h].copy()
         R[snap["comp_row"][h]] = 0
@@ -483,7 +513,7 @@ def test_quantizer_decision_is_fp32():
         with np.errstate(divide="ignore", invalid="ignore"):
             inv = np.where(mx > 0, q127 / mx, np.float32(0)).astype(np.float32)
         Q = np.where(mx[:, None] > 0, np.rint((Rp * inv[:, None]).astype(np.float32)), 0)
-        np.testing.assert_array_equal(np.clip(Q, -127, 127).astype(np.int8), snap["codes"][h])
+        np.testing.assert_array_equal(np.clip(Q, -qm, qm).astype(np.int8), snap["codes"][h])
 
 
 # --------------------------------------------------------------------------
