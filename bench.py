@@ -50,27 +50,31 @@ FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # Algorithmic bytes (per (sequence, head) and launch)
 # --------------------------------------------------------------------------
 
-def snapshot_bytes(dk, dv, r):
-    return dv * dk + 4 * dv + 4 * dk + r * (4 + 4 * dk)
+def snapshot_bytes(dk, dv, r, bits=8):
+    """Codes (one byte per code, half a byte at 4 bits), row scales,
+    smoothing factors and compensators of one head."""
+    codes = dv * dk // 2 if bits == 4 else dv * dk
+    return codes + 4 * dv + 4 * dk + r * (4 + 4 * dk)
 
 
 def record_bytes(dk, dv, gate):
     return 4 * ((dk if gate == "diag" else 1) + dk + dv)
 
 
-def decode_launch_bytes(dk, dv, r, gate, e, t):
+def decode_launch_bytes(dk, dv, r, gate, e, t, bits=8):
     """Bytes one decode launch at window position t must move per head:
     read the snapshot and the t-1 buffered records, read q, k, v, alpha,
     beta, write o and record t."""
     G = dk if gate == "diag" else 1
     rec = record_bytes(dk, dv, gate)
-    return snapshot_bytes(dk, dv, r) + (t - 1) * rec + e * (2 * dk + dv) + 4 * G + 4 + e * dv + rec
+    return (snapshot_bytes(dk, dv, r, bits) + (t - 1) * rec + e * (2 * dk + dv) + 4 * G + 4 + e * dv
+            + rec)
 
 
-def commit_launch_bytes(dk, dv, r, gate, n):
+def commit_launch_bytes(dk, dv, r, gate, n, bits=8):
     """Bytes the commit of a window of n records must move per head: read the
     snapshot and the n records, write the new snapshot."""
-    return 2 * snapshot_bytes(dk, dv, r) + n * record_bytes(dk, dv, gate)
+    return 2 * snapshot_bytes(dk, dv, r, bits) + n * record_bytes(dk, dv, gate)
 
 
 # --------------------------------------------------------------------------
@@ -201,9 +205,10 @@ class ClockSampler:
 # CPU oracle timing (cpu_baseline and the reference arm)
 # --------------------------------------------------------------------------
 
-def oracle_window_rate(wl, n_seq: int, w_index: int = 0):
+def oracle_window_rate(wl, n_seq: int, w_index: int = 0, bits: int = 8):
     """Times the CPU oracle on n_seq sequences x all heads for one window of
-    decode plus its commit.  Returns (tokens/s, seconds, threads)."""
+    decode plus its commit (codes of width `bits`).  Returns (tokens/s,
+    seconds, threads)."""
     import numpy as np
     cores = len(os.sched_getaffinity(0))
     os.environ.setdefault("OMP_NUM_THREADS", str(cores))
@@ -224,18 +229,18 @@ def oracle_window_rate(wl, n_seq: int, w_index: int = 0):
     inst = oracle.kda_instance if wl.gate == "diag" else oracle.gdn_instance
     d, kt, b = inst(hm(tok["alpha"]), hm(tok["beta"]), hm(tok["k"]))
     v, q = hm(tok["v"]), hm(tok["q"])
-    snap = oracle.quantize(S0, wl.n_comp, wl.smoothing)
+    snap = oracle.quantize(S0, wl.n_comp, wl.smoothing, bits)
     gdim = wl.d_k if wl.gate == "diag" else 1
     t0 = time.perf_counter()
     rec = oracle.empty_records(n_seq * wl.heads, wl.window, wl.d_k, wl.d_v, gdim)
     oracle.window(snap, rec, 0, d, kt, b, v, q)
-    oracle.commit(snap, rec, wl.window, wl.n_comp, wl.smoothing)
+    oracle.commit(snap, rec, wl.window, wl.n_comp, wl.smoothing, bits)
     dt = time.perf_counter() - t0
     return n_seq * wl.window / dt, dt, int(os.environ["OMP_NUM_THREADS"])
 
 
-def calibrated_sample(wl, target_s: float):
-    _, dt1, _ = oracle_window_rate(wl, 1)
+def calibrated_sample(wl, target_s: float, bits: int = 8):
+    _, dt1, _ = oracle_window_rate(wl, 1, bits=bits)
     n = int(max(1, min(wl.batch, math.floor(target_s / max(dt1, 1e-6)))))
     return n
 
@@ -248,12 +253,12 @@ def run_reference(args, wl):
     rank, world, _ = _dist()
     if rank != 0:
         return None
-    n_seq = calibrated_sample(wl, args.ref_seconds)
+    n_seq = calibrated_sample(wl, args.ref_seconds, args.bits)
     for i in range(args.warmup):
-        oracle_window_rate(wl, n_seq, i)
+        oracle_window_rate(wl, n_seq, i, args.bits)
     total_tok, total_s = 0, 0.0
     for i in range(args.steps):
-        rate, dt, cores = oracle_window_rate(wl, n_seq, args.warmup + i)
+        rate, dt, cores = oracle_window_rate(wl, n_seq, args.warmup + i, args.bits)
         total_tok += n_seq * wl.window
         total_s += dt
     value = total_tok / total_s
@@ -271,20 +276,42 @@ def run_reference(args, wl):
     }
 
 
+def state_words(bits):
+    return {8: "int8 codes", 6: "6-bit codes (one per byte)", 4: "4-bit codes (two per byte)"}[bits]
+
+
+def profile_key(kernel, wl, args):
+    """Key of the ncu summary under profiles/ that holds this kernel's DRAM
+    traffic: the workload's name, plus every override of its window,
+    compensators, smoothing or code width (no summary exists for those)."""
+    base = synth_workload(wl.name)
+    key = f"{kernel}:{wl.name}"
+    if (wl.window, wl.n_comp, bool(wl.smoothing)) != (base.window, base.n_comp, bool(base.smoothing)) \
+            or args.bits != 8:
+        key += f"_W{wl.window}_r{wl.n_comp}_s{int(bool(wl.smoothing))}_b{args.bits}"
+    return key
+
+
+def synth_workload(name):
+    from linear_attention_recurrent_int8_b200 import synth
+    return synth.WORKLOADS[name]
+
+
 def workload_config(wl, args):
     return {
         "workload": (f"{wl.name}: {'KDA per-channel' if wl.gate == 'diag' else 'GDN scalar'}-gate "
                      f"decode, batch {wl.batch} x {wl.heads} heads, d_k={wl.d_k}, d_v={wl.d_v}, "
                      f"window W={wl.window}, r={wl.n_comp} compensators, {wl.io} q/k/v/o, "
-                     f"int8 state with per-row scales"),
+                     f"{state_words(args.bits)} state with per-row scales"),
         "batch_per_gpu": wl.batch, "heads": wl.heads, "d_k": wl.d_k, "d_v": wl.d_v,
         "window": wl.window, "n_comp": wl.n_comp, "gate": wl.gate, "io": wl.io,
-        "smoothing": bool(wl.smoothing), "state": "int8 codes + fp32 row scales",
+        "smoothing": bool(wl.smoothing), "bits": args.bits,
+        "state": f"{state_words(args.bits)} + fp32 row scales",
         "step": f"one window: {wl.window} decode launches and the window commit",
         "tokens_per_step_per_gpu": wl.batch * wl.window,
         "l2": "inputs larger than L2: each decode launch reads ~%.0f MB vs 126 MB L2" % (
             wl.batch * wl.heads * decode_launch_bytes(wl.d_k, wl.d_v, wl.n_comp, wl.gate,
-                                                      2 if wl.io == "bf16" else 4, 1) / 1e6),
+                                                      2 if wl.io == "bf16" else 4, 1, args.bits) / 1e6),
         "graph": not args.no_graph,
     }
 
@@ -309,7 +336,7 @@ def run_lq(args, wl):
     cfg = lq.Config(batch=wl.batch, heads=wl.heads, d_k=wl.d_k, d_v=wl.d_v, window=wl.window,
                     n_comp=wl.n_comp, gate=lq.LQ_GATE_DIAG if wl.gate == "diag" else lq.LQ_GATE_SCALAR,
                     io_dtype=lq.LQ_BF16 if wl.io == "bf16" else lq.LQ_F32,
-                    smoothing=int(wl.smoothing), auto_commit=0)
+                    smoothing=int(wl.smoothing), auto_commit=0, bits=args.bits)
     W = wl.window
     e = 2 if wl.io == "bf16" else 4
     st = lq.State(cfg, dev)
@@ -402,12 +429,12 @@ def run_lq(args, wl):
         evs = graphs[gi][1]
         for t in range(W):
             dec_ms.append(evs[t].elapsed_time(evs[t + 1]))
-            dec_bytes += nh * decode_launch_bytes(wl.d_k, wl.d_v, wl.n_comp, wl.gate, e, t + 1)
+            dec_bytes += nh * decode_launch_bytes(wl.d_k, wl.d_v, wl.n_comp, wl.gate, e, t + 1, args.bits)
         com_ms.append(evs[W].elapsed_time(evs[W + 1]))
     peak, peak_kind = measured_peaks()
     dec_avg_ms = sum(dec_ms) / len(dec_ms)
     achieved = dec_bytes / len(dec_ms) / (dec_avg_ms / 1e3) / 1e9
-    traffic = profiled_traffic(f"decode:{wl.name}")
+    traffic = profiled_traffic(profile_key("decode", wl, args))
     roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
             "frac": achieved / peak, "traffic": traffic,
             "kernel": "decode_kernel (window positions 1..W)",
@@ -421,13 +448,13 @@ def run_lq(args, wl):
         pos_us.append(round(1e3 * sum(vals) / len(vals), 1))
     extra["launch_us_by_position"] = pos_us
     c_avg = sum(com_ms) / len(com_ms)
-    c_bytes = nh * commit_launch_bytes(wl.d_k, wl.d_v, wl.n_comp, wl.gate, W)
+    c_bytes = nh * commit_launch_bytes(wl.d_k, wl.d_v, wl.n_comp, wl.gate, W, args.bits)
     extra["commit"] = {"kernel": "commit_kernel", "avg_launch_us": c_avg * 1e3,
                        "bytes_per_launch": c_bytes, "achieved_gbs": c_bytes / (c_avg / 1e3) / 1e9,
                        "frac": c_bytes / (c_avg / 1e3) / 1e9 / peak,
-                       "traffic": profiled_traffic(f"commit:{wl.name}")}
-    step_bytes = c_bytes + nh * sum(decode_launch_bytes(wl.d_k, wl.d_v, wl.n_comp, wl.gate, e, t + 1)
-                                    for t in range(W))
+                       "traffic": profiled_traffic(profile_key("commit", wl, args))}
+    step_bytes = c_bytes + nh * sum(decode_launch_bytes(wl.d_k, wl.d_v, wl.n_comp, wl.gate, e, t + 1,
+                                                        args.bits) for t in range(W))
     extra["step_gbs"] = step_bytes / (elapsed / args.steps / 1e3) / 1e9
 
     # end to end through the C ABI from pinned host buffers
@@ -449,8 +476,8 @@ def run_lq(args, wl):
     if sampler:
         line["clocks"] = sampler.summary(t0, t1, t_warm0)
     if rank == 0 and world == 1 and not args.no_cpu:
-        n_seq = calibrated_sample(wl, args.cpu_seconds)
-        rate, dt, cores = oracle_window_rate(wl, n_seq)
+        n_seq = calibrated_sample(wl, args.cpu_seconds, args.bits)
+        rate, dt, cores = oracle_window_rate(wl, n_seq, bits=args.bits)
         line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                                 "sample": f"{n_seq} of {wl.batch} sequences x {wl.heads} heads, one "
                                           f"window of {W} decode tokens plus its commit ({dt:.1f} s)"}
@@ -613,7 +640,8 @@ def run_ragged(args, wl):
     W = wl.window
     cfg = lq.Config(batch=wl.batch, heads=wl.heads, d_k=wl.d_k, d_v=wl.d_v, window=W, n_comp=wl.n_comp,
                     gate=lq.LQ_GATE_DIAG if wl.gate == "diag" else lq.LQ_GATE_SCALAR,
-                    io_dtype=lq.LQ_BF16 if wl.io == "bf16" else lq.LQ_F32, smoothing=int(wl.smoothing))
+                    io_dtype=lq.LQ_BF16 if wl.io == "bf16" else lq.LQ_F32, smoothing=int(wl.smoothing),
+                    bits=args.bits)
     st = lq.State(cfg, dev)
     S0 = synth.torch_initial_state(wl.seed, range(wl.batch), range(wl.heads), wl.d_k, wl.d_v,
                                    wl.outlier_rows, wl.outlier_cols, wl.outlier_scale, dev)
@@ -674,7 +702,7 @@ def run_init(args, wl):
     cfg = lq.Config(batch=wl.batch, heads=wl.heads, d_k=wl.d_k, d_v=wl.d_v, window=wl.window,
                     n_comp=wl.n_comp, gate=lq.LQ_GATE_DIAG if wl.gate == "diag" else lq.LQ_GATE_SCALAR,
                     io_dtype=lq.LQ_BF16 if wl.io == "bf16" else lq.LQ_F32,
-                    smoothing=int(wl.smoothing))
+                    smoothing=int(wl.smoothing), bits=args.bits)
     st = lq.State(cfg, dev)
     S0 = synth.torch_initial_state(wl.seed, range(wl.batch), range(wl.heads), wl.d_k, wl.d_v,
                                    wl.outlier_rows, wl.outlier_cols, wl.outlier_scale, dev)
@@ -689,7 +717,7 @@ def run_init(args, wl):
     b.record()
     torch.cuda.synchronize()
     ms = a.elapsed_time(b) / args.steps
-    nbytes = wl.nh * (4 * wl.d_v * wl.d_k + snapshot_bytes(wl.d_k, wl.d_v, wl.n_comp))
+    nbytes = wl.nh * (4 * wl.d_v * wl.d_k + snapshot_bytes(wl.d_k, wl.d_v, wl.n_comp, args.bits))
     peak, kind = measured_peaks()
     gbs = nbytes / (ms / 1e3) / 1e9
     return {"metric": "state init: heads quantized per second", "value": wl.nh / (ms / 1e3),
@@ -758,14 +786,17 @@ def run_mse(args, wl):
     S0 = synth.torch_initial_state(wl.seed, range(wl.batch), range(wl.heads), wl.d_k, wl.d_v,
                                    wl.outlier_rows, wl.outlier_cols, wl.outlier_scale, dev)
     S0 = S0.reshape(wl.nh, wl.d_v, wl.d_k).contiguous()
-    variants = {"per_window": (wl.window, wl.n_comp, int(wl.smoothing)),
-                "per_token": (1, 0, int(wl.smoothing)), "per_token_plain": (1, 0, 0)}
+    sm0 = int(wl.smoothing)
+    variants = {"per_window": (wl.window, wl.n_comp, sm0, 8),
+                "per_token": (1, 0, sm0, 8), "per_token_plain": (1, 0, 0, 8),
+                "per_window_6bit": (wl.window, wl.n_comp, sm0, 6), "per_token_6bit": (1, 0, sm0, 6),
+                "per_window_4bit": (wl.window, wl.n_comp, sm0, 4), "per_token_4bit": (1, 0, sm0, 4)}
     states, cfgs = {}, {}
-    for name, (W, r, sm) in variants.items():
+    for name, (W, r, sm, bits) in variants.items():
         cfg = lq.Config(batch=wl.batch, heads=wl.heads, d_k=wl.d_k, d_v=wl.d_v, window=W, n_comp=r,
                         gate=lq.LQ_GATE_DIAG if wl.gate == "diag" else lq.LQ_GATE_SCALAR,
                         io_dtype=lq.LQ_BF16 if wl.io == "bf16" else lq.LQ_F32, smoothing=sm,
-                        auto_commit=1)
+                        auto_commit=1, bits=bits)
         st = lq.State(cfg, dev)
         lq.lq_state_init(st, S0)
         states[name], cfgs[name] = st, cfg
@@ -773,9 +804,20 @@ def run_mse(args, wl):
     fcfg = cfgs["per_window"]
     o = torch.empty((wl.batch, 1, wl.heads, wl.d_v), dtype=fcfg.io_torch_dtype, device=dev)
 
+    def codes_float(st):
+        c = st.snap.t["codes"]
+        if st.cfg.bits != 4:
+            return c.float()
+        # two per byte: in each 8-channel group, byte b holds channel b (low
+        # nibble) and channel 4 + b (high nibble), two's complement
+        p = c.to(torch.int16).reshape(c.shape[0], c.shape[1], -1, 4)
+        nib = torch.stack([p & 0xF, (p >> 4) & 0xF], dim=-2)
+        nib = torch.where(nib >= 8, nib - 16, nib)
+        return nib.reshape(c.shape[0], c.shape[1], -1).float()
+
     def dequant(st):
         t = st.snap.t
-        Sh = (t["row_scale"][:, :, None] * t["codes"].float() * t["col_smooth"][:, None, :])
+        Sh = (t["row_scale"][:, :, None] * codes_float(st) * t["col_smooth"][:, None, :])
         if t["comp_row"].numel():
             Sh.scatter_add_(1, t["comp_row"].long()[:, :, None].expand(-1, -1, wl.d_k), t["comp_val"])
         return Sh
@@ -796,7 +838,9 @@ def run_mse(args, wl):
     out = {n: {"final_rel_mse": c[-1], "mean_rel_mse": sum(c) / len(c)} for n, c in curve.items()}
     return {"report": "state MSE relative to the mean square of the FP32 state, at window ends",
             "workload": wl.name, "batch": wl.batch, "heads": wl.heads, "steps": steps,
-            "window": W, "n_comp": wl.n_comp, "results": out}
+            "window": W, "n_comp": wl.n_comp, "results": out,
+            "variants": {n: {"window": v[0], "n_comp": v[1], "smoothing": bool(v[2]), "bits": v[3]}
+                         for n, v in variants.items()}}
 
 
 def main(argv=None):
@@ -815,6 +859,8 @@ def main(argv=None):
     ap.add_argument("--window", type=int, default=None, help="override W (comparators / sweep)")
     ap.add_argument("--n-comp", type=int, default=None, help="override r")
     ap.add_argument("--no-smoothing", action="store_true")
+    ap.add_argument("--bits", type=int, choices=[8, 6, 4], default=8,
+                    help="code width of the state (8; 6 and 4 are the narrow variants)")
     ap.add_argument("--slots", type=int, default=8, help="distinct input windows (graphs)")
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")

@@ -90,10 +90,24 @@ typedef struct {
                             DeltaNet with alpha = 1, Kimi Delta Attention);
                             0: b_t = 0, u_t = v_t (linear attention, RetNet,
                             Mamba2, GLA: the b = 0 rows of Table 4)         */
+    int32_t bits;        /* code width of the snapshot: 8 (0 also means 8), 6
+                            or 4.  Codes lie in [-q, q], q = 2^(bits-1) - 1
+                            (127, 31, 7); the paper reports 8-, 6- and 4-bit
+                            state groups (Table 1) and fixes no format, so
+                            the narrower widths are this library's variant of
+                            the same quantizer.  8 and 6 store one code per
+                            byte, 4 stores two (see lq_snapshot).          */
 } lq_config;
 
 /* The quantized boundary state of every (b, h), all device memory:
- *   codes      int8    [B*H][d_v][d_k]  (16B)  Q, residual codes in [-127,127]
+ *   codes      int8    [B*H][d_v][d_k]  (16B)  Q, residual codes in [-q, q]
+ *                                              (bits 8 or 6);
+ *              uint8   [B*H][d_v][d_k/2] (16B) at bits = 4: in each group of
+ *                                              8 key channels 8g..8g+7 of a
+ *                                              row, byte 4g+b (b = 0..3) holds
+ *                                              channel 8g+b in its low nibble
+ *                                              and 8g+4+b in its high nibble,
+ *                                              both two's complement
  *   row_scale  float   [B*H][d_v]       (16B)  sigma_i (0 for a zero row)
  *   col_smooth float   [B*H][d_k]       (16B)  c_j (1 when smoothing is off)
  *   comp_row   int32   [B*H][r]                row index of each compensator,

@@ -41,7 +41,8 @@ class LQError(RuntimeError):
 
 class LqConfig(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("batch", "heads", "d_k", "d_v", "window", "n_comp",
-                                              "gate", "io_dtype", "smoothing", "auto_commit", "delta")]
+                                              "gate", "io_dtype", "smoothing", "auto_commit", "delta",
+                                              "bits")]
 
 
 class LqSnapshot(ctypes.Structure):
@@ -131,10 +132,17 @@ class Config:
     smoothing: int = 1
     auto_commit: int = 1
     delta: int = 1
+    bits: int = 8  # code width: 8, 6 (one code per byte) or 4 (two per byte)
 
     def c(self) -> LqConfig:
         return LqConfig(self.batch, self.heads, self.d_k, self.d_v, self.window, self.n_comp,
-                        self.gate, self.io_dtype, self.smoothing, self.auto_commit, self.delta)
+                        self.gate, self.io_dtype, self.smoothing, self.auto_commit, self.delta,
+                        self.bits)
+
+    @property
+    def code_cols(self) -> int:
+        """Bytes of one value row of codes (d_k, or d_k / 2 at 4 bits)."""
+        return self.d_k // 2 if self.bits == 4 else self.d_k
 
     @property
     def gdim(self) -> int:
@@ -154,7 +162,8 @@ class Snapshot:
         bh = cfg.batch * cfg.heads
         if tensors is None:
             tensors = dict(
-                codes=torch.zeros((bh, cfg.d_v, cfg.d_k), dtype=torch.int8, device=device),
+                codes=torch.zeros((bh, cfg.d_v, cfg.code_cols),
+                                  dtype=torch.uint8 if cfg.bits == 4 else torch.int8, device=device),
                 row_scale=torch.zeros((bh, cfg.d_v), dtype=torch.float32, device=device),
                 col_smooth=torch.ones((bh, cfg.d_k), dtype=torch.float32, device=device),
                 comp_row=torch.zeros((bh, cfg.n_comp), dtype=torch.int32, device=device),

@@ -28,7 +28,16 @@ lq_status check_config(const lq_config *c) {
     if ((c->smoothing != 0 && c->smoothing != 1) || (c->auto_commit != 0 && c->auto_commit != 1) ||
         (c->delta != 0 && c->delta != 1))
         return LQ_ERR_INVALID_ARGUMENT;
+    if (c->bits != 0 && c->bits != 8 && c->bits != 6 && c->bits != 4) return LQ_ERR_INVALID_ARGUMENT;
     return LQ_OK;
+}
+
+// Code width of a valid configuration (0 means 8).
+int code_bits(const lq_config *c) { return c->bits == 0 ? 8 : c->bits; }
+
+// Bytes of one head's codes: one per code, or two codes per byte at 4 bits.
+size_t code_bytes_per_head(const lq_config *c) {
+    return (size_t)c->d_v * (code_bits(c) == 4 ? c->d_k / 2 : c->d_k);
 }
 
 lq_status check_snapshot(const lq_config *c, const lq_snapshot *s) {
@@ -83,6 +92,7 @@ lq::DecodeArgs decode_args(const lq_state *st) {
     a.R = st->cfg.n_comp;
     a.pos = st->pos;
     a.smoothing = st->cfg.smoothing;
+    a.bits = code_bits(&st->cfg);
     return a;
 }
 
@@ -97,6 +107,7 @@ lq::QuantArgs quant_args(const lq_config *c, const float *S, const lq_snapshot *
     a.BH = c->batch * c->heads;
     a.R = c->n_comp;
     a.smoothing = c->smoothing;
+    a.bits = code_bits(c);
     return a;
 }
 
@@ -106,7 +117,7 @@ lq_status copy_snapshot(const lq_config *c, const lq_snapshot *dst, const lq_sna
                         cudaStream_t stream) {
     const size_t bh = (size_t)c->batch * c->heads;
     const cudaMemcpyKind kind = cudaMemcpyDeviceToDevice;
-    cudaError_t e = cudaMemcpyAsync(dst->codes, src->codes, bh * c->d_v * c->d_k, kind, stream);
+    cudaError_t e = cudaMemcpyAsync(dst->codes, src->codes, bh * code_bytes_per_head(c), kind, stream);
     if (e == cudaSuccess)
         e = cudaMemcpyAsync(dst->row_scale, src->row_scale, bh * c->d_v * 4, kind, stream);
     if (e == cudaSuccess)
@@ -128,7 +139,7 @@ int64_t lq_buffer_elems(const lq_config *cfg, int32_t which) {
     const int64_t bh = (int64_t)cfg->batch * cfg->heads;
     const int64_t G = cfg->gate == LQ_GATE_DIAG ? cfg->d_k : 1;
     switch (which) {
-        case 0: return bh * cfg->d_v * cfg->d_k;
+        case 0: return bh * (int64_t)code_bytes_per_head(cfg);
         case 1: return bh * cfg->d_v;
         case 2: return bh * cfg->d_k;
         case 3: return bh * cfg->n_comp;

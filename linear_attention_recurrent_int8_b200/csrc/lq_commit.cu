@@ -1,6 +1,6 @@
 // lq_commit.cu -- the window commit on sm_100a: rebuild of the FP32 state at
-// the window end, Compensator Tokens, residual smoothing and per-row int8
-// re-quantization ("LeapQuant: Efficient Linear Attention with Accurate
+// the window end, Compensator Tokens, residual smoothing and per-row
+// re-quantization to 8-bit (or 6- or 4-bit) codes ("LeapQuant: Efficient Linear Attention with Accurate
 // Recurrent State Quantization", Figure 2: the state is quantized once per
 // window; Figure 4 and the Abstract: the largest outliers are kept as
 // high-precision Compensator Tokens and the residual is smoothed across
@@ -12,7 +12,7 @@
 //   S_n = S^_0 Diag(e^{L_n}) + [U | E_comp] [K^ | comp Diag(e^{L_n})]^T,
 //   K^_m = k~_m * e^{L_n - L_m},
 //
-// where S^_0 = Diag(sigma) Q Diag(c) is the int8 residual of the snapshot,
+// where S^_0 = Diag(sigma) Q Diag(c) is the quantized residual of the snapshot,
 // U = [u_1 .. u_n] the buffered updates and E_comp the one-hot columns of the
 // compensator rows.  The rank-(n + r) term is a dense contraction and runs on
 // the 5th-generation tensor core: kind::tf32 with both operands split into a
@@ -28,7 +28,7 @@
 // quantization of consecutive heads overlap:
 //  * producer (one lane): the head's records, compensators and scales into a
 //    ring of shared-memory stages by 1-D bulk copies (no multicast), and an L2
-//    prefetch of its int8 codes;
+//    prefetch of its codes;
 //  * 4 builder warps: the TF32 hi/lo operands of the rank term into one of
 //    two operand buffers;
 //  * MMA warp (one lane): the MMAs of a head into one of two TMEM
@@ -160,13 +160,16 @@ __device__ __forceinline__ int next_commit_head(const DecodeArgs &a, int bh) {
     return BH;
 }
 
-template <int DK, int DV, int GATE>
+// PACK4: 4-bit codes, two per byte (lq_quant.cuh); otherwise one per byte.
+template <int DK, int DV, int GATE, bool PACK4>
 __global__ void __launch_bounds__(kThreads, 1) commit_kernel(const DecodeArgs a, const int NS,
                                                              const int NOPS) {
     static_assert(DV == 64 || DV == 128, "d_v must be 64 or 128");
     constexpr int NQ = DV / 32;        // lane quarters that hold rows
     constexpr int CPT = DK / 2;        // key channels per epilogue thread
     constexpr int NCH = CPT / 32;      // 32-column TMEM chunks per thread
+    constexpr int CRB = PACK4 ? DK / 2 : DK;  // code bytes per value row
+    constexpr int NCW = PACK4 ? CPT / 32 : CPT / 16;  // 16-byte code words per thread
     constexpr int G = GATE == 1 ? DK : 1;
     extern __shared__ __align__(128) unsigned char smem[];
     auto &cs = *reinterpret_cast<CommitSmem<DK, DV> *>(smem);
@@ -215,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1) commit_kernel(const DecodeArgs a,
                 if (R > 0) bulk_g2s(st + SL.comp, a.comp_val + (size_t)bh * R * DK, 4 * R * DK, &cs.full[s]);
                 bulk_g2s(st + SL.cs, a.col_smooth + (size_t)bh * DK, 4 * DK, &cs.full[s]);
                 bulk_g2s(st + SL.rs, a.row_scale + (size_t)bh * DV, 4 * DV, &cs.full[s]);
-                prefetch_l2(a.codes + (size_t)bh * DV * DK, DV * DK);
+                prefetch_l2(a.codes + (size_t)bh * DV * CRB, DV * CRB);
             }
         }
         return;
@@ -339,12 +342,12 @@ __global__ void __launch_bounds__(kThreads, 1) commit_kernel(const DecodeArgs a,
     const int row = 32 * qtr + lane, j0 = half * CPT;
     // the row half's old codes, loaded one head ahead (the producer has
     // prefetched them into L2)
-    uint4 cw[CPT / 16], cw_next[CPT / 16];
-    auto load_codes = [&](int bhx, uint4(&dst)[CPT / 16]) {
+    uint4 cw[NCW], cw_next[NCW];
+    auto load_codes = [&](int bhx, uint4(&dst)[NCW]) {
         if (has_row && bhx < BH) {
-            const int8_t *src = a.codes + ((size_t)bhx * DV + row) * DK + j0;
+            const int8_t *src = a.codes + ((size_t)bhx * DV + row) * CRB + (PACK4 ? j0 / 2 : j0);
 #pragma unroll
-            for (int c = 0; c < CPT / 16; ++c) dst[c] = *reinterpret_cast<const uint4 *>(src + 16 * c);
+            for (int c = 0; c < NCW; ++c) dst[c] = *reinterpret_cast<const uint4 *>(src + 16 * c);
         }
     };
     load_codes(next_commit_head(a, blockIdx.x), cw_next);
@@ -357,12 +360,12 @@ __global__ void __launch_bounds__(kThreads, 1) commit_kernel(const DecodeArgs a,
         const float *Ls = reinterpret_cast<const float *>(st + SL.L);
         const float *Css = reinterpret_cast<const float *>(st + SL.cs);
         const float *Rss = reinterpret_cast<const float *>(st + SL.rs);
-        int8_t *codes_row = a.codes + ((size_t)bh * DV + (has_row ? row : 0)) * DK + j0;
+        int8_t *codes_row = a.codes + ((size_t)bh * DV + (has_row ? row : 0)) * CRB + (PACK4 ? j0 / 2 : j0);
         const uint32_t tq = cs.tmem + ((uint32_t)(32 * qtr) << 16) + b * DK + j0;
         for (int j = tid; j < DK; j += kEpi) cs.cg[j] = Css[j] * expf(Ls[(nrec - 1) * G + (GATE == 1 ? j : 0)]);
         if (tid < DV) cs.comp_idx[tid] = -1;
 #pragma unroll
-        for (int c = 0; c < CPT / 16; ++c) cw[c] = cw_next[c];
+        for (int c = 0; c < NCW; ++c) cw[c] = cw_next[c];
         load_codes(next_commit_head(a, bh + gridDim.x), cw_next);
         const float sig = has_row ? Rss[row] : 0.0f;
         const bool ok = mbar_wait_bounded(&cs.mma_done[b], (it >> 1) & 1);
@@ -374,21 +377,39 @@ __global__ void __launch_bounds__(kThreads, 1) commit_kernel(const DecodeArgs a,
             float2 ss = make_float2(0.0f, 0.0f);
             const float2 sg2 = make_float2(sig, sig);
             const float2 off2 = make_float2(-8388736.0f, -8388736.0f);
+            // 4-bit: each biased byte is 16 Q + 128; x / 16 - (2^23 + 128) / 16 = Q exactly
+            const float2 sixteenth2 = make_float2(0.0625f, 0.0625f);
+            const float2 off16_2 = make_float2(-524296.0f, -524296.0f);
 #pragma unroll
             for (int c = 0; c < NCH; ++c) {
                 float x[32];
                 tmem_load<32>(tq + 32 * c, x);
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
-                    const uint32_t u = word_of(cw[2 * c + q / 4], q % 4) ^ 0x80808080u;
+                    uint32_t cword;
+                    if constexpr (PACK4) {
+                        // channels 8h..8h+3 sit in the low nibbles of word h,
+                        // 8h+4..8h+7 in the high ones: move the nibble into
+                        // the high half of each byte, giving 16 Q as an int8
+                        const uint32_t w = word_of(cw[c], q / 2);
+                        cword = (q & 1) ? (w & 0xF0F0F0F0u) : ((w << 4) & 0xF0F0F0F0u);
+                    } else {
+                        cword = word_of(cw[2 * c + q / 4], q % 4);
+                    }
+                    const uint32_t u = cword ^ 0x80808080u;
                     const float4 g = *reinterpret_cast<const float4 *>(cs.cg + j0 + 32 * c + 4 * q);
                     // code + 128 in the low mantissa bits of 2^23, minus (2^23 + 128)
                     float2 f01 = make_float2(__uint_as_float(__byte_perm(u, 0x4B000000u, 0x7650)),
                                              __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7651)));
                     float2 f23 = make_float2(__uint_as_float(__byte_perm(u, 0x4B000000u, 0x7652)),
                                              __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7653)));
-                    f01 = __fmul2_rn(__fadd2_rn(f01, off2), sg2);
-                    f23 = __fmul2_rn(__fadd2_rn(f23, off2), sg2);
+                    if constexpr (PACK4) {
+                        f01 = __fmul2_rn(__ffma2_rn(f01, sixteenth2, off16_2), sg2);
+                        f23 = __fmul2_rn(__ffma2_rn(f23, sixteenth2, off16_2), sg2);
+                    } else {
+                        f01 = __fmul2_rn(__fadd2_rn(f01, off2), sg2);
+                        f23 = __fmul2_rn(__fadd2_rn(f23, off2), sg2);
+                    }
                     const float2 y01 = __ffma2_rn(f01, make_float2(g.x, g.y), make_float2(x[4 * q], x[4 * q + 1]));
                     const float2 y23 = __ffma2_rn(f23, make_float2(g.z, g.w), make_float2(x[4 * q + 2], x[4 * q + 3]));
                     ss = __ffma2_rn(y01, y01, ss);
@@ -502,14 +523,16 @@ __global__ void __launch_bounds__(kThreads, 1) commit_kernel(const DecodeArgs a,
             tmem_wait_st();
         }
         named_sync<kEpiBar, kEpi>();
-        // C4: sigma = max / 127 and the codes.  |R'_ij| <= max_j |R'_ij| makes
-        // |R'_ij * (127 / max)| <= 127 (1 + 2^-23), which rounds to at most
-        // 127: no clamp.  The magic-number addition rounds half to even; the
-        // low byte of its bits is the two's-complement code.
+        // C4: sigma = max / q and the codes (q = 127, 31 or 7).  |R'_ij| <=
+        // max_j |R'_ij| makes |R'_ij * (q / max)| <= q (1 + 2^-23), which
+        // rounds to at most q: no clamp.  The magic-number addition rounds
+        // half to even; the low byte of its bits is the two's-complement code
+        // (its low nibble the 4-bit code).
         if (has_row) {
+            const float qmax = (float)((1 << (a.bits - 1)) - 1);  // 127, 31 or 7
             const float mxr = fmaxf(cs.rowpart[0][row], cs.rowpart[1][row]);
-            if (half == 0) a.row_scale[(size_t)bh * DV + row] = __fdiv_rn(mxr, 127.0f);
-            const float inv = mxr > 0.0f ? __fdiv_rn(127.0f, mxr) : 0.0f;
+            if (half == 0) a.row_scale[(size_t)bh * DV + row] = __fdiv_rn(mxr, qmax);
+            const float inv = mxr > 0.0f ? __fdiv_rn(qmax, mxr) : 0.0f;
             const float2 inv2 = make_float2(inv, inv), mg2 = make_float2(12582912.0f, 12582912.0f);
 #pragma unroll
             for (int c = 0; c < NCH; ++c) {
@@ -524,8 +547,17 @@ __global__ void __launch_bounds__(kThreads, 1) commit_kernel(const DecodeArgs a,
                                         __byte_perm(__float_as_uint(y23.x), __float_as_uint(y23.y), 0x0040),
                                         0x5410);
                 }
-                *reinterpret_cast<uint4 *>(codes_row + 32 * c) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-                *reinterpret_cast<uint4 *>(codes_row + 32 * c + 16) = make_uint4(wv[4], wv[5], wv[6], wv[7]);
+                if constexpr (PACK4) {
+                    // word h: channels 8h..8h+3 low nibbles, 8h+4..8h+7 high
+                    uint32_t pw[4];
+#pragma unroll
+                    for (int h = 0; h < 4; ++h)
+                        pw[h] = (wv[2 * h] & 0x0F0F0F0Fu) | ((wv[2 * h + 1] & 0x0F0F0F0Fu) << 4);
+                    *reinterpret_cast<uint4 *>(codes_row + 16 * c) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+                } else {
+                    *reinterpret_cast<uint4 *>(codes_row + 32 * c) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                    *reinterpret_cast<uint4 *>(codes_row + 32 * c + 16) = make_uint4(wv[4], wv[5], wv[6], wv[7]);
+                }
             }
         }
         // this head's TMEM reads are complete: release the accumulator and the stage
@@ -549,14 +581,14 @@ struct DeviceInfo {
     int sms, smem_optin;
 };
 
-template <int DK, int DV, int GATE>
+template <int DK, int DV, int GATE, bool PACK4>
 cudaError_t launch_c(const DecodeArgs &a, cudaStream_t stream) {
     static std::atomic<uint64_t> configured{0};  // devices already set up
     static DeviceInfo info[64];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    auto kern = commit_kernel<DK, DV, GATE>;
+    auto kern = commit_kernel<DK, DV, GATE, PACK4>;
     const uint64_t bit = 1ull << (dev & 63);
     if (!(configured.load(std::memory_order_acquire) & bit)) {
         DeviceInfo I{};
@@ -587,7 +619,9 @@ cudaError_t launch_c(const DecodeArgs &a, cudaStream_t stream) {
 }
 template <int DK, int DV>
 cudaError_t launch_c_d(const DecodeArgs &a, int gate, cudaStream_t stream) {
-    return gate == 1 ? launch_c<DK, DV, 1>(a, stream) : launch_c<DK, DV, 0>(a, stream);
+    if (a.bits == 4)
+        return gate == 1 ? launch_c<DK, DV, 1, true>(a, stream) : launch_c<DK, DV, 0, true>(a, stream);
+    return gate == 1 ? launch_c<DK, DV, 1, false>(a, stream) : launch_c<DK, DV, 0, false>(a, stream);
 }
 
 }  // namespace
@@ -609,6 +643,7 @@ cudaError_t launch_advance_positions(int32_t *seq_pos, int B, int W, cudaStream_
 
 cudaError_t launch_commit(const DecodeArgs &a, int d_k, int d_v, int gate, cudaStream_t stream) {
     if (a.pos < 1 || a.pos > 32 || a.R < 0 || a.R > kMaxComp) return cudaErrorInvalidValue;
+    if (a.bits != 8 && a.bits != 6 && a.bits != 4) return cudaErrorInvalidValue;
     if (d_k == 128 && d_v == 128) return launch_c_d<128, 128>(a, gate, stream);
     if (d_k == 128 && d_v == 64) return launch_c_d<128, 64>(a, gate, stream);
     if (d_k == 64 && d_v == 128) return launch_c_d<64, 128>(a, gate, stream);

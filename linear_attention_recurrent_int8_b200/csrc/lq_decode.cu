@@ -1,4 +1,4 @@
-// lq_decode.cu -- per-window int8 decode on sm_100a.
+// lq_decode.cu -- per-window decode from a quantized state on sm_100a.
 //
 // "LeapQuant: Efficient Linear Attention with Accurate Recurrent State
 // Quantization", Figure 2: within a window the int8 boundary state S^_0 stays
@@ -16,10 +16,13 @@
 // pseudo-records at window position 0 (Figure 4; they share the update path
 // of real tokens), so they enter with decay e^{L_t}.
 //
+// The boundary state's codes are 8-bit (or 6-bit) one per byte, or 4-bit two
+// per byte (PACK4; layout in lq_quant.cuh).
+//
 // Kernel structure (persistent, warp-specialised, 12 warps per CTA):
 //  * the grid walks the (sequence, head) pairs with a grid stride; each head
 //    goes through a ring of shared-memory stages;
-//  * producer (warp 8, one lane): streams the head's int8 codes, scales,
+//  * producer (warp 8, one lane): streams the head's codes, scales,
 //    smoothing factors, compensators, buffered records and the first token's
 //    q/k/v into a stage with 1-D bulk copies (no multicast) -> "full";
 //  * prep A (warp 9): for every token of the call, the vectors
@@ -76,16 +79,16 @@ __host__ __device__ inline PrepLayout prep_layout(int DK) {
 
 // Byte offsets inside one stage (one head's operands).  `nrec` is the number
 // of record slots the stage holds (records read plus records written), `n`
-// the number of tokens of the call.
+// the number of tokens of the call; `pack4`: 4-bit codes, two per byte.
 struct StageLayout {
     int codes, sig, cs, compv, compr, recK, recU, recL, q, k, v, al, scal, prep, bytes;
 };
 
 __host__ __device__ inline StageLayout stage_layout(int DK, int DV, int gate, int R, int nrec,
-                                                   int n, int e) {
+                                                   int n, int e, bool pack4) {
     StageLayout L{};
     int o = 0;
-    L.codes = o; o += align16(DV * DK);
+    L.codes = o; o += align16(DV * (pack4 ? DK / 2 : DK));
     L.sig = o;   o += align16(4 * DV);
     L.cs = o;    o += align16(4 * DK);
     L.compv = o; o += align16(4 * R * DK);
@@ -160,16 +163,18 @@ __device__ __forceinline__ int next_decode_head(const DecodeArgs &a, int bh) {
 
 // RAGGED: per-sequence window positions (a.seq_pos); otherwise the window
 // position a.pos is the same for every head and stays a kernel constant.
-template <int DK, int DV, int GATE, bool BF16, bool RAGGED>
+// PACK4: 4-bit codes, two per byte.
+template <int DK, int DV, int GATE, bool BF16, bool RAGGED, bool PACK4>
 __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a, const int S) {
     constexpr int E = BF16 ? 2 : 4;
     constexpr int RPW = DV / kConsumerWarps;  // value rows per consumer warp
+    constexpr int CRB = PACK4 ? DK / 2 : DK;  // code bytes per value row
     extern __shared__ __align__(128) unsigned char smem[];
     uint64_t *full = reinterpret_cast<uint64_t *>(smem);
     uint64_t *prepared = full + kMaxStages;
     uint64_t *empty = prepared + kMaxStages;
     const int nsteps = a.n_steps;
-    const StageLayout SL = stage_layout(DK, DV, GATE, a.R, a.pos + nsteps, nsteps, E);
+    const StageLayout SL = stage_layout(DK, DV, GATE, a.R, a.pos + nsteps, nsteps, E, PACK4);
     const PrepLayout PL = prep_layout(DK);
     unsigned char *stages = smem + header_bytes();
 
@@ -203,7 +208,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a,
             const size_t tok = (size_t)b * nsteps * a.H + h;  // token 0 of this call
             const uint32_t in_bytes =
                 nsteps > 0 ? (uint32_t)(E * (2 * DK + DV) + (GATE == 1 ? 4 * DK : 0)) : 0u;
-            const uint32_t bytes = DV * DK + 4 * DV + 4 * DK + 4 * R * DK + 4 * pos * (DK + DV) +
+            const uint32_t bytes = DV * CRB + 4 * DV + 4 * DK + 4 * R * DK + 4 * pos * (DK + DV) +
                                    (GATE == 1 ? 4 * pos * DK : 0) + in_bytes;
             // small operands by 4-byte copies, tracked by the same barrier:
             // alpha and beta of token 0, the scalar-gate records, the
@@ -220,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a,
                 cp_async4(st + SL.compr + 4 * c, a.comp_row + (size_t)bh * R + c);
             cp_async_mbar_arrive(&full[s]);
             mbar_arrive_expect_tx(&full[s], bytes);
-            bulk_g2s(st + SL.codes, a.codes + (size_t)bh * DV * DK, DV * DK, &full[s]);
+            bulk_g2s(st + SL.codes, a.codes + (size_t)bh * DV * CRB, DV * CRB, &full[s]);
             bulk_g2s(st + SL.sig, a.row_scale + (size_t)bh * DV, 4 * DV, &full[s]);
             bulk_g2s(st + SL.cs, a.col_smooth + (size_t)bh * DK, 4 * DK, &full[s]);
             if (R > 0) bulk_g2s(st + SL.compv, a.comp_val + (size_t)bh * R * DK, 4 * R * DK, &full[s]);
@@ -445,6 +450,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a,
             // D2: S^_0 x for this warp's rows: dp4a of the codes with the limbs.
             // A0 2^7 + A1 is exact in int32 (|.| < 2^26) and converted once;
             // the vector scales are applied after the cross-lane reduction.
+            // 4-bit codes enter as 16 Q (the nibble in the high half of an
+            // int8), so every sum is 16 times larger and the unit is 2^-18.
             float y;
             {
                 uint4 lw[6];
@@ -455,7 +462,16 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a,
 #pragma unroll
                 for (int n = 0; n < NRM; ++n) {
                     const int r = warp * RPW + n * RPI16 + sub;
-                    const uint4 w = *reinterpret_cast<const uint4 *>(codes_s + r * DK + 16 * cc);
+                    uint4 w;
+                    if constexpr (PACK4) {
+                        // 8 bytes = channels 16cc..16cc+15: word h holds
+                        // 8h..8h+3 in its low nibbles and 8h+4..8h+7 in its high
+                        const uint2 p = *reinterpret_cast<const uint2 *>(codes_s + r * CRB + 8 * cc);
+                        w = make_uint4((p.x << 4) & 0xF0F0F0F0u, p.x & 0xF0F0F0F0u,
+                                       (p.y << 4) & 0xF0F0F0F0u, p.y & 0xF0F0F0F0u);
+                    } else {
+                        w = *reinterpret_cast<const uint4 *>(codes_s + r * DK + 16 * cc);
+                    }
                     int acc[6];
 #pragma unroll
                     for (int v = 0; v < 6; ++v) {
@@ -474,8 +490,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a,
             // D3-D6 for row `row`: LPRD lanes share its buffered records
             {
                 const float sg = sig_s[row];
-                const float yk = __shfl_sync(0xffffffffu, y, src_k) * (sg * (lscale[0] * 6.103515625e-05f));
-                const float yq = __shfl_sync(0xffffffffu, y, src_q) * (sg * (lscale[1] * 6.103515625e-05f));
+                constexpr float kUnit = PACK4 ? 3.814697265625e-06f : 6.103515625e-05f;  // 2^-18, 2^-14
+                const float yk = __shfl_sync(0xffffffffu, y, src_k) * (sg * (lscale[0] * kUnit));
+                const float yq = __shfl_sync(0xffffffffu, y, src_q) * (sg * (lscale[1] * kUnit));
                 float hb = part == 0 ? yk : 0.0f, p = part == 0 ? yq : 0.0f;
                 for (int m = part; m < nrec; m += LPRD) {
                     const float um = recU_s[m * DV + row];
@@ -512,7 +529,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a,
     }
 }
 
-template <int DK, int DV, int GATE, bool BF16, bool RAGGED>
+template <int DK, int DV, int GATE, bool BF16, bool RAGGED, bool PACK4>
 cudaError_t launch_d(const DecodeArgs &a, cudaStream_t stream) {
     constexpr int E = BF16 ? 2 : 4;
     static std::atomic<uint64_t> configured{0};  // devices already set up
@@ -520,7 +537,7 @@ cudaError_t launch_d(const DecodeArgs &a, cudaStream_t stream) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    auto kern = decode_kernel<DK, DV, GATE, BF16, RAGGED>;
+    auto kern = decode_kernel<DK, DV, GATE, BF16, RAGGED, PACK4>;
     const uint64_t bit = 1ull << (dev & 63);
     if (!(configured.load(std::memory_order_acquire) & bit)) {
         int optin = 0, sms = 0;
@@ -533,7 +550,7 @@ cudaError_t launch_d(const DecodeArgs &a, cudaStream_t stream) {
         configured.fetch_or(bit, std::memory_order_acq_rel);
     }
     // a stage holds the records this launch reads and writes (pos + n_steps)
-    const StageLayout SL = stage_layout(DK, DV, GATE, a.R, a.pos + a.n_steps, a.n_steps, E);
+    const StageLayout SL = stage_layout(DK, DV, GATE, a.R, a.pos + a.n_steps, a.n_steps, E, PACK4);
     const int fixed = header_bytes();
     // two CTAs per SM when registers allow it and each can hold at least
     // two stages, else one CTA per SM with as many stages as fit
@@ -562,8 +579,11 @@ cudaError_t launch_d(const DecodeArgs &a, cudaStream_t stream) {
 
 template <int DK, int DV, int GATE, bool BF16>
 cudaError_t launch_dr(const DecodeArgs &a, cudaStream_t stream) {
-    return a.seq_pos ? launch_d<DK, DV, GATE, BF16, true>(a, stream)
-                     : launch_d<DK, DV, GATE, BF16, false>(a, stream);
+    if (a.bits == 4)
+        return a.seq_pos ? launch_d<DK, DV, GATE, BF16, true, true>(a, stream)
+                         : launch_d<DK, DV, GATE, BF16, false, true>(a, stream);
+    return a.seq_pos ? launch_d<DK, DV, GATE, BF16, true, false>(a, stream)
+                     : launch_d<DK, DV, GATE, BF16, false, false>(a, stream);
 }
 
 template <int DK, int DV>
@@ -578,6 +598,7 @@ cudaError_t launch_decode_d(const DecodeArgs &a, int gate, bool bf16, cudaStream
 cudaError_t launch_decode(const DecodeArgs &a, int d_k, int d_v, int gate, bool bf16,
                           cudaStream_t stream) {
     if (a.n_steps < 1) return cudaErrorInvalidValue;
+    if (a.bits != 8 && a.bits != 6 && a.bits != 4) return cudaErrorInvalidValue;
     if (d_k == 128 && d_v == 128) return launch_decode_d<128, 128>(a, gate, bf16, stream);
     if (d_k == 128 && d_v == 64) return launch_decode_d<128, 64>(a, gate, bf16, stream);
     if (d_k == 64 && d_v == 128) return launch_decode_d<64, 128>(a, gate, bf16, stream);

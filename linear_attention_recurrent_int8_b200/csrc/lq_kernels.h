@@ -28,6 +28,7 @@ struct DecodeArgs {
     int pos;      // records already buffered (the same for every sequence)
     int n_steps;  // tokens decoded by this launch (0: commit only)
     int smoothing;
+    int bits;     // code width: 8 or 6 (one code per byte) or 4 (two per byte)
     // per-sequence window positions [B] (device), or nullptr.  When set, the
     // decode takes one token per sequence b with seq_pos[b] in [0, W) at
     // window position seq_pos[b] + 1 (pos and n_steps are then W - 1 and 1,
@@ -46,6 +47,7 @@ struct QuantArgs {
     int32_t *comp_row;
     float *comp_val;
     int BH, R, smoothing;
+    int bits;  // code width: 8 or 6 (one code per byte) or 4 (two per byte)
 };
 
 // Arguments of the FP32-state recurrence kernel (prefill, FP32 per-step).
@@ -68,7 +70,7 @@ cudaError_t launch_decode(const DecodeArgs &a, int d_k, int d_v, int gate, bool 
                           cudaStream_t stream);
 
 // Commits the window of a.pos >= 1 buffered records (a.n_steps unused):
-// rebuild, compensators, smoothing, int8 codes, written over the snapshot.
+// rebuild, compensators, smoothing, codes, written over the snapshot.
 cudaError_t launch_commit(const DecodeArgs &a, int d_k, int d_v, int gate, cudaStream_t stream);
 
 // seq_pos[b] <- (seq_pos[b] + 1) mod W for the sequences with 0 <= seq_pos[b] < W.

@@ -1,4 +1,4 @@
-// lq_quant.cu -- quantization of FP32 states into int8 snapshots: state
+// lq_quant.cu -- quantization of FP32 states into snapshots: state
 // initialisation and the prefill's prefix-cache snapshots ("LeapQuant:
 // Efficient Linear Attention with Accurate Recurrent State Quantization",
 // Figure 1(b): one state per 1,024 cached tokens).  One CTA per head loads the
@@ -31,10 +31,11 @@ __global__ void __launch_bounds__(kWarps * 32) quantize_kernel(const QuantArgs a
         S[n][2] = x.z;
         S[n][3] = x.w;
     }
-    SnapPtr out{a.codes + (size_t)bh * DV * DK, a.row_scale + (size_t)bh * DV,
+    const size_t code_bytes = a.bits == 4 ? (size_t)DV * DK / 2 : (size_t)DV * DK;
+    SnapPtr out{a.codes + (size_t)bh * code_bytes, a.row_scale + (size_t)bh * DV,
                 a.col_smooth + (size_t)bh * DK, a.comp_row ? a.comp_row + (size_t)bh * a.R : nullptr,
                 a.comp_val ? a.comp_val + (size_t)bh * a.R * DK : nullptr};
-    quantize_tile<DK, DV, kWarps>(S, a.R, a.smoothing != 0, qsm, out);
+    quantize_tile<DK, DV, kWarps>(S, a.R, a.smoothing != 0, a.bits, qsm, out);
 }
 
 template <int DK, int DV>

@@ -11,8 +11,12 @@
 //       in the residual R;
 //   C3  c_j = sqrt(max_i |R_ij|) (1 for a zero column or with smoothing off),
 //       R'_ij = R_ij * (1 / c_j);
-//   C4  mx_i = max_j |R'_ij|, sigma_i = mx_i / 127 (stored),
-//       Q_ij = rne(R'_ij * (127 / mx_i)) in [-127, 127], Q = 0 where mx_i = 0.
+//   C4  mx_i = max_j |R'_ij|, sigma_i = mx_i / q (stored),
+//       Q_ij = rne(R'_ij * (q / mx_i)) in [-q, q], Q = 0 where mx_i = 0,
+//       with q = 2^(bits-1) - 1: 127 for 8-bit codes, 31 and 7 for the 6- and
+//       4-bit widths of the paper's lower-precision groups (Table 1); 4-bit
+//       codes are stored two per byte (low nibble: channel 8g+b, high
+//       nibble: channel 8g+4+b, in byte 4g+b of a row).
 // Each smoothing factor and each row is inverted once; every element then
 // costs one FP32 product per step.  Every division, square root and product
 // is one IEEE round-to-nearest FP32 operation (__fdiv_rn, __fsqrt_rn, __fmul_rn),
@@ -45,7 +49,7 @@ struct Tile {
 
 // Device pointers of one head's snapshot.
 struct SnapPtr {
-    int8_t *codes;      // [DV][DK]
+    int8_t *codes;      // [DV][DK], or [DV][DK/2] bytes of packed 4-bit codes
     float *row_scale;   // [DV]
     float *col_smooth;  // [DK]
     int32_t *comp_row;  // [R]
@@ -64,18 +68,20 @@ struct alignas(16) QuantSmem {
 };
 
 // C2-C4 on the register tile S (the FP32 state of one head, owned as Tile
-// describes), writing the snapshot to `out`.  The NWARPS*32 threads that own
-// the tile (threads 0 .. NWARPS*32-1) call it; it synchronises them on named
-// barrier 1.
+// describes), writing the snapshot to `out` with codes of width `bits` (8, 6
+// or 4).  The NWARPS*32 threads that own the tile (threads 0 .. NWARPS*32-1)
+// call it; it synchronises them on named barrier 1.
 template <int DK, int DV, int NWARPS>
 __device__ __forceinline__ void quantize_tile(float (&S)[Tile<DK, DV, NWARPS>::NR][4], int R,
-                                              bool smoothing, QuantSmem<DK, DV, NWARPS> &sm,
-                                              const SnapPtr &out) {
+                                              bool smoothing, int bits,
+                                              QuantSmem<DK, DV, NWARPS> &sm, const SnapPtr &out) {
     using T = Tile<DK, DV, NWARPS>;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int c0 = T::col0(lane);
 
     const int gbase = lane & ~(T::LPR - 1);  // first lane of this lane's row group
+    const float qmax = (float)((1 << (bits - 1)) - 1);
+    const bool pack4 = bits == 4;
     // C2 (1/2): squared row norms (order-preserving for the selection),
     // reduced across the row's lanes with a transposing reduction
     {
@@ -183,26 +189,36 @@ __device__ __forceinline__ void quantize_tile(float (&S)[Tile<DK, DV, NWARPS>::N
         }
         transposed_max<T::NR, T::LPR>(mx, lane);
         const int n = transposed_index<T::NR, T::LPR>(lane);
-        inv_own = mx[0] > 0.0f ? __fdiv_rn(127.0f, mx[0]) : 0.0f;
+        inv_own = mx[0] > 0.0f ? __fdiv_rn(qmax, mx[0]) : 0.0f;
         if ((lane & (T::LPR - 1)) == transposed_owner<T::NR, T::LPR>(n))
-            out.row_scale[T::row(warp, lane, n)] = __fdiv_rn(mx[0], 127.0f);
+            out.row_scale[T::row(warp, lane, n)] = __fdiv_rn(mx[0], qmax);
     }
 #pragma unroll
     for (int n = 0; n < T::NR; ++n) {
         const float inv =
             __shfl_sync(0xffffffffu, inv_own, gbase + transposed_owner<T::NR, T::LPR>(n));
         const int row = T::row(warp, lane, n);
-        // round half to even by the magic-number addition (|y| <= 127 here),
+        // round half to even by the magic-number addition (|y| <= q here),
         // clamp, and pack the four low bytes
         int iv[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            const float y = fminf(fmaxf(__fmul_rn(S[n][e], inv), -127.0f), 127.0f);
+            const float y = fminf(fmaxf(__fmul_rn(S[n][e], inv), -qmax), qmax);
             iv[e] = __float_as_int(__fadd_rn(y, 12582912.0f)) - 0x4B400000;
         }
         const uint32_t packed = __byte_perm(__byte_perm(iv[0], iv[1], 0x0040),
                                             __byte_perm(iv[2], iv[3], 0x0040), 0x5410);
-        *reinterpret_cast<uint32_t *>(out.codes + (size_t)row * DK + c0) = packed;
+        if (pack4) {
+            // two's-complement nibbles; lanes 2p and 2p+1 of a row hold the
+            // channels 8g..8g+3 and 8g+4..8g+7 of one 8-channel group
+            const uint32_t nib = packed & 0x0F0F0F0Fu;
+            const uint32_t hi = __shfl_xor_sync(0xffffffffu, nib, 1);
+            if ((c0 & 4) == 0)
+                *reinterpret_cast<uint32_t *>(out.codes + (size_t)row * (DK / 2) + c0 / 2) =
+                    nib | (hi << 4);
+        } else {
+            *reinterpret_cast<uint32_t *>(out.codes + (size_t)row * DK + c0) = packed;
+        }
     }
 }
 

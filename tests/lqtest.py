@@ -75,8 +75,37 @@ def to_device_tokens(tok: dict, io: str, device="cuda"):
     return out
 
 
+def pack_codes4(codes) -> np.ndarray:
+    """int8 codes [..., d_k] with |Q| <= 7 -> bytes [..., d_k / 2] in the
+    4-bit storage format that lq.h states for lq_snapshot.codes: in each group
+    of 8 key channels 8g..8g+7, byte 4g+b holds channel 8g+b in its low nibble
+    and 8g+4+b in its high nibble, two's complement."""
+    c = np.asarray(codes).astype(np.int16)
+    g = c.reshape(c.shape[:-1] + (-1, 2, 4))  # [..., group, half, b]
+    lo, hi = g[..., 0, :] & 0xF, g[..., 1, :] & 0xF
+    return (lo | (hi << 4)).astype(np.uint8).reshape(c.shape[:-1] + (-1,))
+
+
+def unpack_codes4(packed) -> np.ndarray:
+    """Inverse of pack_codes4: bytes [..., d_k / 2] -> int8 codes [..., d_k]."""
+    p = np.asarray(packed).astype(np.uint8)
+    g = p.reshape(p.shape[:-1] + (-1, 4)).astype(np.int16)  # [..., group, b]
+    nib = np.stack([g & 0xF, g >> 4], axis=-2)             # [..., group, half, b]
+    nib = np.where(nib >= 8, nib - 16, nib)
+    return nib.reshape(p.shape[:-1] + (-1,)).astype(np.int8)
+
+
+def codes_to_device_format(cfg: lq.Config, codes) -> np.ndarray:
+    return pack_codes4(codes) if cfg.bits == 4 else np.asarray(codes, np.int8)
+
+
+def codes_from_device_format(cfg: lq.Config, codes) -> np.ndarray:
+    return unpack_codes4(codes) if cfg.bits == 4 else np.asarray(codes)
+
+
 def upload_snapshot(cfg: lq.Config, snap: dict, device="cuda") -> lq.Snapshot:
-    t = dict(codes=torch.from_numpy(np.ascontiguousarray(snap["codes"])).to(device),
+    codes = np.ascontiguousarray(codes_to_device_format(cfg, snap["codes"]))
+    t = dict(codes=torch.from_numpy(codes).to(device),
              row_scale=torch.from_numpy(np.ascontiguousarray(snap["row_scale"])).to(device),
              col_smooth=torch.from_numpy(np.ascontiguousarray(snap["col_smooth"])).to(device),
              comp_row=torch.from_numpy(np.ascontiguousarray(snap["comp_row"], np.int32)).to(device),
@@ -84,8 +113,15 @@ def upload_snapshot(cfg: lq.Config, snap: dict, device="cuda") -> lq.Snapshot:
     return lq.Snapshot(cfg, device, t)
 
 
+def snapshot_to_host(cfg: lq.Config, snap: lq.Snapshot) -> dict:
+    """A device snapshot as numpy arrays, codes one int8 per code."""
+    out = {k: v.detach().cpu().numpy() for k, v in snap.t.items()}
+    out["codes"] = codes_from_device_format(cfg, out["codes"])
+    return out
+
+
 def download_snapshot(st: lq.State) -> dict:
-    return {k: v.detach().cpu().numpy() for k, v in st.snap.t.items()}
+    return snapshot_to_host(st.cfg, st.snap)
 
 
 def rel_l2(a, b, axis=-1):
@@ -174,7 +210,7 @@ class AnchoredRun:
         S0 = S0.reshape(wl.nh, wl.d_v, wl.d_k)
         lq.lq_state_init(self.st, torch.from_numpy(S0).to(self.device))
         torch.cuda.synchronize()
-        ref = oracle.quantize(S0, cfg.n_comp, bool(cfg.smoothing))
+        ref = oracle.quantize(S0, cfg.n_comp, bool(cfg.smoothing), cfg.bits)
         st = compare_snapshots(download_snapshot(self.st), ref, ref["row_norm"], exact_codes=True)
         self.stats["near_ties"] += st["near_ties"]
         self.snap = ref
@@ -208,7 +244,7 @@ class AnchoredRun:
         d, kt, b, v, q = oracle_tokens(tok, wl.gate, wl.delta)
         rec = oracle.empty_records(wl.nh, W, wl.d_k, wl.d_v, cfg.gdim)
         o_ref = oracle.window(self.snap, rec, 0, d, kt, b, v, q)
-        new_snap, S_n = oracle.commit(self.snap, rec, ntok, cfg.n_comp, bool(cfg.smoothing))
+        new_snap, S_n = oracle.commit(self.snap, rec, ntok, cfg.n_comp, bool(cfg.smoothing), cfg.bits)
 
         o_gpu = heads_major(o.float().cpu().numpy())
         worst = compare_outputs(o_gpu, o_ref, wl.io, f"outputs window {w}")
@@ -241,9 +277,10 @@ class SampledRun:
     (every head is checked by AnchoredRun in the first windows).  Nothing the
     device computes is given to the oracle."""
 
-    def __init__(self, wl: synth.DecodeWorkload, n_sample: int, seed: int = 1234, device="cuda"):
+    def __init__(self, wl: synth.DecodeWorkload, n_sample: int, seed: int = 1234, device="cuda",
+                 bits: int = 8):
         self.wl, self.device = wl, device
-        self.cfg = make_config(wl)
+        self.cfg = make_config(wl, bits=bits)
         self.st = lq.State(self.cfg, device)
         rng = np.random.default_rng(seed)
         self.sample = np.sort(rng.choice(wl.nh, size=min(n_sample, wl.nh), replace=False))
@@ -258,7 +295,9 @@ class SampledRun:
         return {k: np.concatenate([p[k] for p in per], axis=2) for k in per[0]}  # [1, T, ns, ...]
 
     def _sampled_snapshot(self):
-        return {k: v.index_select(0, self.idx).cpu().numpy() for k, v in self.st.snap.t.items()}
+        out = {k: v.index_select(0, self.idx).cpu().numpy() for k, v in self.st.snap.t.items()}
+        out["codes"] = codes_from_device_format(self.cfg, out["codes"])
+        return out
 
     def init(self):
         wl, dev = self.wl, self.device
@@ -272,14 +311,15 @@ class SampledRun:
         lq.lq_state_init(self.st, S)
         torch.cuda.synchronize()
         del S
-        ref = oracle.quantize(S_s, self.cfg.n_comp, bool(self.cfg.smoothing))
+        ref = oracle.quantize(S_s, self.cfg.n_comp, bool(self.cfg.smoothing), self.cfg.bits)
         compare_snapshots(self._sampled_snapshot(), ref, ref["row_norm"], exact_codes=True)
         self.snap = ref
 
     def _anchor(self):
         for key in ("codes", "row_scale", "col_smooth", "comp_row", "comp_val"):
             if self.st.snap.t[key].numel():
-                src = torch.from_numpy(np.ascontiguousarray(self.snap[key])).to(self.device)
+                val = codes_to_device_format(self.cfg, self.snap[key]) if key == "codes" else self.snap[key]
+                src = torch.from_numpy(np.ascontiguousarray(val)).to(self.device)
                 self.st.snap.t[key][self.idx] = src.to(self.st.snap.t[key].dtype)
 
     def window(self, w: int):
@@ -306,7 +346,7 @@ class SampledRun:
         d, kt, b, v, q = oracle_tokens(tok_s, wl.gate, wl.delta)
         rec = oracle.empty_records(len(self.sample), W, wl.d_k, wl.d_v, cfg.gdim)
         o_ref = oracle.window(self.snap, rec, 0, d, kt, b, v, q)
-        new_snap, _ = oracle.commit(self.snap, rec, W, cfg.n_comp, bool(cfg.smoothing))
+        new_snap, _ = oracle.commit(self.snap, rec, W, cfg.n_comp, bool(cfg.smoothing), cfg.bits)
         o_gpu = o[bi, :, hi].float().cpu().numpy()  # [ns, W, dv]
         worst = compare_outputs(o_gpu, o_ref, wl.io, f"outputs window {w}")
         st = compare_snapshots(self._sampled_snapshot(), new_snap, new_snap["row_norm"])

@@ -49,8 +49,32 @@ def test_buffer_elems():
     assert lq.lq_buffer_elems(cfg, 8) == -1
     cfg.gate = lq.LQ_GATE_SCALAR
     assert lq.lq_buffer_elems(cfg, 5) == bh * 16
+    # code bytes: one per code at 8 and 6 bits (0 means 8), half a byte at 4
+    for bits, want0 in ((0, bh * 64 * 128), (8, bh * 64 * 128), (6, bh * 64 * 128),
+                        (4, bh * 64 * 64)):
+        cfg.bits = bits
+        assert lq.lq_buffer_elems(cfg, 0) == want0, bits
+    cfg.bits = 5
+    assert lq.lq_buffer_elems(cfg, 0) == -1
+    cfg.bits = 8
     cfg.d_k = 96
     assert lq.lq_buffer_elems(cfg, 0) == -1
+
+
+def test_four_bit_packing_helpers_follow_the_header():
+    """lq.h: in each group of 8 key channels 8g..8g+7 of a row, byte 4g+b
+    holds channel 8g+b in its low nibble and 8g+4+b in its high nibble, two's
+    complement.  Hand-packed example, then a random round trip."""
+    import numpy as np
+    from lqtest import pack_codes4, unpack_codes4
+    row = np.array([1, 2, 3, 4, 5, 6, 7, -7, 0, -1, -8 + 1, 0, 3, -2, 0, 7], np.int8)
+    packed = pack_codes4(row)
+    assert packed.tolist() == [0x51, 0x62, 0x73, 0x94, 0x30, 0xEF, 0x09, 0x70]
+    assert unpack_codes4(packed).tolist() == row.tolist()
+    r = np.random.default_rng(0).integers(-7, 8, size=(3, 5, 64)).astype(np.int8)
+    p = pack_codes4(r)
+    assert p.shape == (3, 5, 32) and p.dtype == np.uint8
+    assert np.array_equal(unpack_codes4(p), r)
 
 
 class _Buf:
@@ -107,6 +131,8 @@ def test_decode_validation_without_launch():
                              ("n_comp", 17, lq.LQ_ERR_INVALID_ARGUMENT),
                              ("gate", 2, lq.LQ_ERR_INVALID_ARGUMENT),
                              ("delta", 2, lq.LQ_ERR_INVALID_ARGUMENT),
+                             ("bits", 5, lq.LQ_ERR_INVALID_ARGUMENT),
+                             ("bits", 16, lq.LQ_ERR_INVALID_ARGUMENT),
                              ("batch", 0, lq.LQ_ERR_INVALID_ARGUMENT)):
         c2 = lq.Config(batch=2, heads=3, window=4, n_comp=2)
         setattr(c2, field, val)

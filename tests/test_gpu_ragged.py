@@ -11,8 +11,8 @@ import oracle
 import linear_attention_recurrent_int8_b200 as lq
 from linear_attention_recurrent_int8_b200 import synth
 
-from lqtest import (compare_outputs, compare_snapshots, download_snapshot, heads_major, io_dtype,
-                    make_config, oracle_tokens)
+from lqtest import (codes_to_device_format, compare_outputs, compare_snapshots, download_snapshot,
+                    heads_major, io_dtype, make_config, oracle_tokens)
 
 pytestmark = pytest.mark.gpu
 
@@ -27,20 +27,21 @@ def _write_heads(st, snap, heads):
     """Device state's snapshot of `heads` <- snap (oracle arrays for those heads)."""
     idx = torch.as_tensor(heads, device="cuda")
     for key in ("codes", "row_scale", "col_smooth", "comp_row", "comp_val"):
-        src = np.ascontiguousarray(snap[key], np.int32 if key == "comp_row" else None)
+        val = codes_to_device_format(st.cfg, snap[key]) if key == "codes" else snap[key]
+        src = np.ascontiguousarray(val, np.int32 if key == "comp_row" else None)
         st.snap.t[key][idx] = torch.from_numpy(src).to("cuda")
 
 
-def _run(dk, dv, gate, io, W, r, B, H, steps, start_of):
+def _run(dk, dv, gate, io, W, r, B, H, steps, start_of, bits=8):
     wl = synth.DecodeWorkload(f"ragged_{dk}_{dv}_{gate}", B, H, dk, dv, steps, W, r, gate, io, True,
                               max(1, dv // 100), max(1, dk // 100), 30.0)
-    cfg = make_config(wl, auto_commit=0)
+    cfg = make_config(wl, auto_commit=0, bits=bits)
     st = lq.State(cfg, "cuda")
     bs, hs = np.arange(B), np.arange(H)
     S0 = synth.initial_state(wl.seed, bs, hs, dk, dv, wl.outlier_rows, wl.outlier_cols,
                              wl.outlier_scale).reshape(B * H, dv, dk)
     lq.lq_state_init(st, torch.from_numpy(S0).to("cuda"))
-    ref0 = oracle.quantize(S0, r, True)
+    ref0 = oracle.quantize(S0, r, True, bits)
     anchor = {b: _slice_snap(ref0, np.arange(b * H, (b + 1) * H)) for b in range(B)}
     seq_pos = torch.full((B,), -1, dtype=torch.int32, device="cuda")
     count = [0] * B            # tokens decoded so far by each sequence
@@ -88,7 +89,7 @@ def _run(dk, dv, gate, io, W, r, B, H, steps, start_of):
                 o_ref = oracle.window(anchor[b], rec, 0, d, kt, bb, vv, qq)
                 o_gpu = heads_major(np.concatenate([x for _, x in win], axis=1))
                 compare_outputs(o_gpu, o_ref, io, f"sequence {b} window ending at token {count[b]}")
-                new, _ = oracle.commit(anchor[b], rec, W, r, True)
+                new, _ = oracle.commit(anchor[b], rec, W, r, True, bits)
                 if snap_gpu is None:
                     snap_gpu = download_snapshot(st)
                 compare_snapshots(_slice_snap(snap_gpu, np.arange(b * H, (b + 1) * H)), new,
@@ -110,6 +111,11 @@ def test_ragged_staggered_windows(dk, dv, gate, io, W, r, B, H):
     start_of = [b % W for b in range(B)]  # every window phase present at once
     checked = _run(dk, dv, gate, io, W, r, B, H, steps=3 * W + 2, start_of=start_of)
     assert checked >= B * 2
+
+
+def test_ragged_staggered_windows_4bit():
+    _run(128, 128, "scalar", "bf16", 4, 2, 5, 3, steps=3 * 4 + 2, start_of=[b % 4 for b in range(5)],
+         bits=4)
 
 
 def test_ragged_matches_synchronous_when_aligned():
