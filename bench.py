@@ -13,7 +13,8 @@ window's launches; event-record nodes inside the graph time every launch for
 the roofline.  Each decode launch reads 160-300 MB (int8 state, records,
 inputs), above the 126 MB L2, so every launch streams from HBM.
 
-Other modes: --mode prefill | fp32step | init | ragged | mse (see --help).
+Other modes: --mode prefill | fp32step | init | ragged | mse (see --help);
+--bits 6 | 4 runs any decode mode on the narrow-code state variants.
 
 Multi-GPU (torchrun): every rank decodes its own shard of sequences (batch
 per rank fixed: weak scaling); no collective on the data path; the host

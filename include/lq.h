@@ -148,14 +148,15 @@ LQ_API int64_t lq_buffer_elems(const lq_config *cfg, int32_t which);
 
 /* Initialises `st` with configuration `cfg` and quantizes the FP32 state
  * S_init [B*H][d_v][d_k] (device, (16B)) into st->snap: compensator
- * selection, residual smoothing, per-row int8 codes (the commit quantizer).
+ * selection, residual smoothing, per-row codes of lq_config.bits (the commit
+ * quantizer).
  * S_init == NULL means the zero state.  Sets pos = 0. */
 LQ_API lq_status lq_state_init(lq_state *st, const lq_config *cfg, const float *S_init,
                         lq_stream_t stream);
 
 /* Decodes n_steps tokens (window positions pos+1 .. pos+n_steps) for every
  * sequence and head: for each token, u_t = v_t - S_{t-1} b_t and
- * o_t = S_t q_t computed from the fixed int8 boundary state plus the buffered
+ * o_t = S_t q_t computed from the fixed quantized boundary state plus the buffered
  * FP32 records ("LeapQuant: ...", Figure 2), and the record (L_t, k~_t, u_t)
  * is appended.  All n_steps tokens run inside one launch.
  * Requires 0 <= n_steps and pos + n_steps <= W (else LQ_ERR_WINDOW_FULL);
@@ -193,7 +194,8 @@ LQ_API lq_status lq_decode_ragged(lq_state *st, int32_t *seq_pos, const void *q,
 /* Window commit ("LeapQuant: ...", Figures 2 and 4): rebuilds the FP32
  * state S_pos = S^_0 D_{1..pos} + sum_m u_m (D_{m+1..pos} k~_m)^T, keeps its
  * r largest-norm rows as Compensator Tokens, smooths the residual across key
- * channels and re-quantizes it to int8 into st->snap; pos returns to 0.
+ * channels and re-quantizes it (codes of lq_config.bits) into st->snap; pos
+ * returns to 0.
  * A no-op when pos == 0. */
 LQ_API lq_status lq_window_commit(lq_state *st, lq_stream_t stream);
 

@@ -33,3 +33,30 @@ def test_profiled_traffic_requires_matching_sources(tmp_path):
     assert bench.profiled_traffic("commit:wl", str(tmp_path)) is None   # stale sources
     assert bench.profiled_traffic("decode:other", str(tmp_path)) is None
     assert bench.source_digest("decode") != bench.source_digest("commit")
+
+
+def test_profile_key_names_overrides():
+    """The headline workload keeps its plain key (its ncu summary applies);
+    any override of W, r, smoothing or the code width gets its own key."""
+    import dataclasses
+    from linear_attention_recurrent_int8_b200 import synth
+
+    class A:
+        bits = 8
+
+    wl = synth.WORKLOADS["gdn_256x32_d128_bf16"]
+    assert bench.profile_key("decode", wl, A) == "decode:gdn_256x32_d128_bf16"
+    A.bits = 4
+    assert bench.profile_key("decode", wl, A) == "decode:gdn_256x32_d128_bf16_W16_r4_s1_b4"
+    A.bits = 8
+    w8 = dataclasses.replace(wl, window=8)
+    assert bench.profile_key("commit", w8, A) == "commit:gdn_256x32_d128_bf16_W8_r4_s1_b8"
+
+
+def test_narrow_code_byte_models():
+    # 4-bit codes: d_v d_k / 2 code bytes per head; 6-bit: one byte per code
+    assert bench.snapshot_bytes(128, 128, 4, 4) == 19472 - 8192
+    assert bench.snapshot_bytes(128, 128, 4, 6) == 19472
+    assert bench.decode_launch_bytes(128, 128, 4, "scalar", 2, 8, 4) == \
+        bench.decode_launch_bytes(128, 128, 4, "scalar", 2, 8) - 8192
+    assert bench.commit_launch_bytes(128, 128, 4, "scalar", 16, 4) == 2 * 11280 + 16 * 1028
