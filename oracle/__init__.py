@@ -59,10 +59,10 @@ def _load():
             P = ctypes.c_void_p
             I = ctypes.c_int
             lib.lqo_eq1_steps.argtypes = [I, I, I, I, P, P, P, P, P, P, P]
-            lib.lqo_quantize.argtypes = [I, I, I, I, I, I, P, P, P, P, P, P, P]
-            lib.lqo_dequantize.argtypes = [I, I, I, I, P, P, P, P, P, P]
-            lib.lqo_window.argtypes = [I] * 9 + [P] * 14
-            lib.lqo_rebuild.argtypes = [I] * 7 + [P] * 9
+            lib.lqo_quantize.argtypes = [I, I, I, I, I, I, P, P, P, P, P, P, P, P]
+            lib.lqo_dequantize.argtypes = [I, I, I, I, P, P, P, P, P, P, P]
+            lib.lqo_window.argtypes = [I] * 9 + [P] * 15
+            lib.lqo_rebuild.argtypes = [I] * 7 + [P] * 10
             for f in (lib.lqo_eq1_steps, lib.lqo_quantize, lib.lqo_dequantize,
                       lib.lqo_window, lib.lqo_rebuild):
                 f.restype = None
@@ -145,21 +145,24 @@ def eq1_steps(S0, d, kt, b, v, q=None):
 class Snapshot(dict):
     """codes int8 [nh,dv,dk], row_scale f32 [nh,dv], col_smooth f32 [nh,dk],
     comp_row i32 [nh,r], comp_val f32 [nh,r,dk] (+ row_norm f64 [nh,dv] when
-    produced by quantize)."""
+    produced by quantize); a BF16 state (bits = 16) also holds dense f32
+    [nh,dv,dk], the BF16-rounded residual, which replaces codes x scales."""
 
     @property
     def n_comp(self):
         return self["comp_row"].shape[1]
 
 
-BITS = (8, 6, 4)  # code widths: q_max = 2^(bits-1) - 1 = 127, 31, 7
+BITS = (8, 6, 4, 16)  # code widths: q_max = 2^(bits-1) - 1 = 127, 31, 7; 16 = BF16 state
 
 
 def quantize(S, n_comp: int, smoothing: bool = True, bits: int = 8) -> Snapshot:
     """Compensator selection, residual smoothing and per-row codes of an FP32
     state ``S`` [nh, dv, dk] (rounded to FP32 first if it is not); the codes
     are ``bits`` wide (8, or the 6- and 4-bit widths of the lower-precision
-    groups of [LQ] Table 1) and returned one per int8."""
+    groups of [LQ] Table 1) and returned one per int8.  ``bits = 16`` is the
+    BF16 state of [LQ] Table 2: compensators as above, the residual rounded
+    to BF16 into ``dense`` (no smoothing, unit scales, zero codes)."""
     S = _c(S, np.float32)
     nh, dv, dk = S.shape
     assert 0 <= n_comp <= dv
@@ -172,9 +175,11 @@ def quantize(S, n_comp: int, smoothing: bool = True, bits: int = 8) -> Snapshot:
         comp_val=np.zeros((nh, n_comp, dk), np.float32),
         row_norm=np.zeros((nh, dv), np.float64),
     )
+    if bits == 16:
+        out["dense"] = np.zeros((nh, dv, dk), np.float32)
     _load().lqo_quantize(nh, dv, dk, n_comp, int(bool(smoothing)), int(bits), _p(S), _p(out["codes"]),
                          _p(out["row_scale"]), _p(out["col_smooth"]), _p(out["comp_row"]),
-                         _p(out["comp_val"]), _p(out["row_norm"]))
+                         _p(out["comp_val"]), _p(out["row_norm"]), _p(out.get("dense")))
     return out
 
 
@@ -183,15 +188,18 @@ def _snap_arrays(snap):
     nh, dv, dk = codes.shape
     comp_row = _c(snap["comp_row"], np.int32).reshape(nh, -1)
     r = comp_row.shape[1]
+    dense = snap.get("dense")
+    dense = None if dense is None else _c(dense, np.float32)
     return (codes, _c(snap["row_scale"], np.float32), _c(snap["col_smooth"], np.float32),
-            comp_row, _c(snap["comp_val"], np.float32).reshape(nh, r, dk), nh, dv, dk, r)
+            comp_row, _c(snap["comp_val"], np.float32).reshape(nh, r, dk), dense, nh, dv, dk, r)
 
 
 def dequantize(snap) -> np.ndarray:
-    """S^_0 = Diag(sigma) Q Diag(c) + compensator rows, FP64 [nh, dv, dk]."""
-    codes, rs, cs, cr, cv, nh, dv, dk, r = _snap_arrays(snap)
+    """S^_0 = Diag(sigma) Q Diag(c) (or the BF16 residual) + compensator rows,
+    FP64 [nh, dv, dk]."""
+    codes, rs, cs, cr, cv, dn, nh, dv, dk, r = _snap_arrays(snap)
     out = np.zeros((nh, dv, dk), np.float64)
-    _load().lqo_dequantize(nh, dv, dk, r, _p(codes), _p(rs), _p(cs), _p(cr), _p(cv), _p(out))
+    _load().lqo_dequantize(nh, dv, dk, r, _p(codes), _p(rs), _p(cs), _p(cr), _p(cv), _p(dn), _p(out))
     return out
 
 
@@ -215,7 +223,7 @@ def window(snap, records: Records, pos: int, d, kt, b, v, q, exact: bool = False
 
     d [nh, n, gdim] (gdim 1 = scalar gate, d_k = diagonal gate); kt, b, q
     [nh, n, dk]; v [nh, n, dv].  Returns o [nh, n, dv] (FP64)."""
-    codes, rs, cs, cr, cv, nh, dv, dk, r = _snap_arrays(snap)
+    codes, rs, cs, cr, cv, dn, nh, dv, dk, r = _snap_arrays(snap)
     W = records["k"].shape[1]
     gdim = records["L"].shape[2]
     d = _c(d, np.float64)
@@ -227,21 +235,21 @@ def window(snap, records: Records, pos: int, d, kt, b, v, q, exact: bool = False
     kt, b, v, q = (_c(a, np.float64) for a in (kt, b, v, q))
     o = np.zeros((nh, n, dv), np.float64)
     _load().lqo_window(nh, dv, dk, r, gdim, W, pos, n, int(bool(exact)), _p(codes), _p(rs), _p(cs),
-                       _p(cr), _p(cv), _p(records["L"]), _p(records["k"]), _p(records["u"]),
+                       _p(cr), _p(cv), _p(dn), _p(records["L"]), _p(records["k"]), _p(records["u"]),
                        _p(d), _p(kt), _p(b), _p(v), _p(q), _p(o))
     return o
 
 
 def rebuild(snap, records: Records, n: int) -> np.ndarray:
     """S_n = S^_0 D_{1..n} + sum_{m<=n} u_m (D_{m+1..n} k~_m)^T, FP64 [nh, dv, dk]."""
-    codes, rs, cs, cr, cv, nh, dv, dk, r = _snap_arrays(snap)
+    codes, rs, cs, cr, cv, dn, nh, dv, dk, r = _snap_arrays(snap)
     W = records["k"].shape[1]
     gdim = records["L"].shape[2]
     assert 0 <= n <= W
     L, K, U = (_c(records[key], np.float64) for key in ("L", "k", "u"))
     out = np.zeros((nh, dv, dk), np.float64)
     _load().lqo_rebuild(nh, dv, dk, r, gdim, W, n, _p(codes), _p(rs), _p(cs), _p(cr), _p(cv),
-                        _p(L), _p(K), _p(U), _p(out))
+                        _p(dn), _p(L), _p(K), _p(U), _p(out))
     return out
 
 

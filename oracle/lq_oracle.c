@@ -58,6 +58,17 @@
 /* Round an FP64 value to the nearest FP32 value (ties to even). */
 static double f32(double x) { return (double)(float)x; }
 
+/* Round a finite value to the nearest value with 8 significant bits (the
+ * BF16 significand), ties to even: x = m 2^e with 0.5 <= |m| < 1, so
+ * rint(m 2^8) 2^(e-8) keeps 8 bits (rint rounds half to even).  Values in
+ * the FP32 normal range only (BF16 shares FP32's exponent range). */
+static double bf16(double x)
+{
+    int e;
+    double m = frexp(x, &e);
+    return ldexp(rint(ldexp(m, 8)), e - 8);
+}
+
 /* ------------------------------------------------------------------------ */
 /* Equation 1, explicit stepping ([LQ] Table 4).                             */
 /* ------------------------------------------------------------------------ */
@@ -133,6 +144,10 @@ void lqo_eq1_steps(int nh, int dv, int dk, int n, double *S, const double *d,
  *      Q_i. = 0 when mx_i = 0.  Round half to even; no zero point; -q-1
  *      unused.  The codes come back one per int8 whatever the width (the
  *      packing of a narrower code is a storage format, not arithmetic).
+ *  bits = 16 is the BF16 state of [LQ] Table 2 ("BF16 per-step" and its
+ *      per-window row): C2 as above, then no smoothing (c = 1) and no integer
+ *      codes (sigma = 1): the residual itself is stored rounded to BF16,
+ *      dense_ij = bf16(R_ij), in `dense` [nh][dv][dk] (FP32 array).
  *
  * Every division, square root and product above is one IEEE FP32 operation
  * on FP32 operands (an FP64 operation rounded once to FP32 gives the same
@@ -144,7 +159,7 @@ void lqo_eq1_steps(int nh, int dv, int dk, int n, double *S, const double *d,
  * row_norm [nh][dv] (optional) receives n_i.                               */
 void lqo_quantize(int nh, int dv, int dk, int r, int smoothing, int bits, const float *S,
                   int8_t *codes, float *row_scale, float *col_smooth,
-                  int32_t *comp_row, float *comp_val, double *row_norm)
+                  int32_t *comp_row, float *comp_val, double *row_norm, float *dense)
 {
     const double qmax = (double)((1 << (bits - 1)) - 1);
 #pragma omp parallel for schedule(dynamic)
@@ -174,6 +189,21 @@ void lqo_quantize(int nh, int dv, int dk, int r, int smoothing, int bits, const 
                 comp_val[((size_t)h * r + c) * dk + j] = Sh[(size_t)best * dk + j];
                 R[(size_t)best * dk + j] = 0.0;
             }
+        }
+        if (bits == 16) {
+            /* BF16 residual: no smoothing, unit scales, rounded values. */
+            for (int j = 0; j < dk; ++j) col_smooth[(size_t)h * dk + j] = 1.0f;
+            for (int i = 0; i < dv; ++i) {
+                row_scale[(size_t)h * dv + i] = 1.0f;
+                for (int j = 0; j < dk; ++j) {
+                    codes[((size_t)h * dv + i) * dk + j] = 0;
+                    dense[((size_t)h * dv + i) * dk + j] = (float)bf16(R[(size_t)i * dk + j]);
+                }
+            }
+            free(R);
+            free(norm);
+            free(taken);
+            continue;
         }
         /* C3: smoothing factor per key channel. */
         float *c = col_smooth + (size_t)h * dk;
@@ -225,13 +255,14 @@ void lqo_quantize(int nh, int dv, int dk, int r, int smoothing, int bits, const 
 static void dequantize_head(int dv, int dk, int r, const int8_t *codes,
                             const float *row_scale, const float *col_smooth,
                             const int32_t *comp_row, const float *comp_val,
-                            double *Sh)
+                            const float *dense, double *Sh)
 {
     for (int i = 0; i < dv; ++i)
         for (int j = 0; j < dk; ++j)
-            Sh[(size_t)i * dk + j] = (double)row_scale[i] *
-                                     (double)codes[(size_t)i * dk + j] *
-                                     (double)col_smooth[j];
+            Sh[(size_t)i * dk + j] = dense ? (double)dense[(size_t)i * dk + j]
+                                           : (double)row_scale[i] *
+                                                 (double)codes[(size_t)i * dk + j] *
+                                                 (double)col_smooth[j];
     for (int c = 0; c < r; ++c) {
         int row = comp_row[c];
         for (int j = 0; j < dk; ++j)
@@ -241,13 +272,15 @@ static void dequantize_head(int dv, int dk, int r, const int8_t *codes,
 
 void lqo_dequantize(int nh, int dv, int dk, int r, const int8_t *codes,
                     const float *row_scale, const float *col_smooth,
-                    const int32_t *comp_row, const float *comp_val, double *S_hat)
+                    const int32_t *comp_row, const float *comp_val,
+                    const float *dense, double *S_hat)
 {
 #pragma omp parallel for schedule(dynamic)
     for (int h = 0; h < nh; ++h)
         dequantize_head(dv, dk, r, codes + (size_t)h * dv * dk,
                         row_scale + (size_t)h * dv, col_smooth + (size_t)h * dk,
                         comp_row + (size_t)h * r, comp_val + (size_t)h * r * dk,
+                        dense ? dense + (size_t)h * dv * dk : NULL,
                         S_hat + (size_t)h * dv * dk);
 }
 
@@ -295,7 +328,7 @@ static double decay(const double *L, int gdim, int t, int m, int j)
 void lqo_window(int nh, int dv, int dk, int r, int gdim, int W, int pos, int n,
                 int exact, const int8_t *codes, const float *row_scale,
                 const float *col_smooth, const int32_t *comp_row,
-                const float *comp_val, double *rec_L, double *rec_k,
+                const float *comp_val, const float *dense, double *rec_L, double *rec_k,
                 double *rec_u, const double *d, const double *kt,
                 const double *b, const double *v, const double *q, double *o)
 {
@@ -306,7 +339,8 @@ void lqo_window(int nh, int dv, int dk, int r, int gdim, int W, int pos, int n,
         double *hb = malloc(sizeof(double) * dv);
         dequantize_head(dv, dk, r, codes + (size_t)h * dv * dk,
                         row_scale + (size_t)h * dv, col_smooth + (size_t)h * dk,
-                        comp_row + (size_t)h * r, comp_val + (size_t)h * r * dk, S0);
+                        comp_row + (size_t)h * r, comp_val + (size_t)h * r * dk,
+                        dense ? dense + (size_t)h * dv * dk : NULL, S0);
         double *L = rec_L + (size_t)h * W * gdim;
         double *K = rec_k + (size_t)h * W * dk;
         double *U = rec_u + (size_t)h * W * dv;
@@ -373,7 +407,7 @@ void lqo_window(int nh, int dv, int dk, int r, int gdim, int W, int pos, int n,
 void lqo_rebuild(int nh, int dv, int dk, int r, int gdim, int W, int n,
                  const int8_t *codes, const float *row_scale,
                  const float *col_smooth, const int32_t *comp_row,
-                 const float *comp_val, const double *rec_L,
+                 const float *comp_val, const float *dense, const double *rec_L,
                  const double *rec_k, const double *rec_u, double *S_out)
 {
 #pragma omp parallel for schedule(dynamic)
@@ -381,7 +415,8 @@ void lqo_rebuild(int nh, int dv, int dk, int r, int gdim, int W, int n,
         double *Sh = S_out + (size_t)h * dv * dk;
         dequantize_head(dv, dk, r, codes + (size_t)h * dv * dk,
                         row_scale + (size_t)h * dv, col_smooth + (size_t)h * dk,
-                        comp_row + (size_t)h * r, comp_val + (size_t)h * r * dk, Sh);
+                        comp_row + (size_t)h * r, comp_val + (size_t)h * r * dk,
+                        dense ? dense + (size_t)h * dv * dk : NULL, Sh);
         const double *L = rec_L + (size_t)h * W * gdim;
         const double *K = rec_k + (size_t)h * W * dk;
         const double *U = rec_u + (size_t)h * W * dv;

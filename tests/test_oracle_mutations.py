@@ -34,6 +34,10 @@ MUTATIONS = {
     "scale_255": ("double sigma = f32(mx / qmax);", "double sigma = f32(mx / (2.0 * qmax + 1.0));"),
     "code_range_one_too_wide": ("const double qmax = (double)((1 << (bits - 1)) - 1);",
                                 "const double qmax = (double)(1 << (bits - 1));"),
+    "bf16_truncates": ("return ldexp(rint(ldexp(m, 8)), e - 8);",
+                       "return ldexp(trunc(ldexp(m, 8)), e - 8);"),
+    "bf16_keeps_9_bits": ("return ldexp(rint(ldexp(m, 8)), e - 8);",
+                          "return ldexp(rint(ldexp(m, 9)), e - 9);"),
     "code_width_fixed_at_8": ("const double qmax = (double)((1 << (bits - 1)) - 1);",
                               "const double qmax = 127.0;"),
 }

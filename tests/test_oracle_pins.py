@@ -266,9 +266,10 @@ def _config1_like(gate="scalar", T=16, dk=64, dv=48, nh=3, io="fp32"):
     return S0, d, kt, b, v, q
 
 
+@pytest.mark.parametrize("bits", [8, 16])
 @pytest.mark.parametrize("exact,tol", [(True, 1e-11), (False, 1e-5)])
 @pytest.mark.parametrize("gate", ["scalar", "diag"])
-def test_window_equals_explicit_stepping(gate, exact, tol):
+def test_window_equals_explicit_stepping(gate, exact, tol, bits):
     """In-window outputs from the fixed S^_0 plus buffered updates equal
     explicitly stepping S^_0 ([LQ] Figure 2).  With FP64 records the two
     agree to rounding of FP64; with FP32 records the gap is the records'
@@ -276,7 +277,7 @@ def test_window_equals_explicit_stepping(gate, exact, tol):
     has shrunk)."""
     S0, d, kt, b, v, q = _config1_like(gate)
     W = d.shape[1]
-    snap = oracle.quantize(S0, 4)
+    snap = oracle.quantize(S0, 4, bits=bits)
     rec = oracle.empty_records(S0.shape[0], W, S0.shape[2], S0.shape[1], d.shape[2])
     o_buf = oracle.window(snap, rec, 0, d, kt, b, v, q, exact=exact)
     o_exp, S_exp = oracle.eq1_steps(oracle.dequantize(snap), d, kt, b, v, q)
@@ -567,3 +568,47 @@ def test_gated_linear_instance_matches_published_updates(diagonal):
             S_pub = S_pub @ decay + beta[0, t] * np.outer(v[0, t], k[0, t])
             assert _rel(o[0, t], S_pub @ q[0, t]) < 1e-13
         assert _rel(S_eq1[0], S_pub) < 1e-13
+
+
+# --------------------------------------------------------------------------
+# BF16 state ([LQ] Table 2, "BF16 per-step" and its per-window row)
+# --------------------------------------------------------------------------
+
+def test_bf16_state_is_round_to_nearest_even_of_the_residual():
+    """The BF16 residual equals torch's float32 -> bfloat16 conversion (round
+    to nearest, ties to even) of the state with its compensator rows zeroed;
+    scales are 1, codes 0, compensators the top-r rows as at 8 bits."""
+    import torch
+    S = _outlier_state(seed=21)
+    r = 3
+    snap = oracle.quantize(S, r, bits=16)
+    ref8 = oracle.quantize(S, r)
+    for h in range(S.shape[0]):
+        assert snap["comp_row"][h].tolist() == ref8["comp_row"][h].tolist()
+        R = S[h].copy()
+        R[snap["comp_row"][h]] = 0
+        want = torch.from_numpy(R).to(torch.bfloat16).to(torch.float32).numpy()
+        np.testing.assert_array_equal(snap["dense"][h], want)
+        np.testing.assert_array_equal(snap["comp_val"][h], S[h][snap["comp_row"][h]])
+    assert np.all(snap["row_scale"] == 1.0) and np.all(snap["col_smooth"] == 1.0)
+    assert not snap["codes"].any()
+    # dequantized: the BF16 residual plus the exact compensator rows
+    Sh = oracle.dequantize(snap)
+    for h in range(S.shape[0]):
+        rows = snap["comp_row"][h]
+        np.testing.assert_array_equal(Sh[h][rows], S[h][rows].astype(np.float64))
+        keep = np.setdiff1d(np.arange(S.shape[1]), rows)
+        np.testing.assert_array_equal(Sh[h][keep], snap["dense"][h][keep].astype(np.float64))
+
+
+def test_bf16_state_hand_cases():
+    """8 significant bits: 1 + 2^-8 is a tie between 1 and 1 + 2^-7 and goes
+    to the even 1; 1 + 3 2^-8 goes to the even 1 + 2^-6; just above a tie
+    rounds up; values with 8 bits are kept; negatives are symmetric."""
+    vals = [1 + 2 ** -8, 1 + 3 * 2 ** -8, 1 + 2 ** -8 + 2 ** -20, 3.0, -(1 + 2 ** -8 + 2 ** -20),
+            0.0, 255.0, 257.0, 2 ** -30 * (1 + 2 ** -9)]
+    want = [1.0, 1 + 2 ** -6, 1 + 2 ** -7, 3.0, -(1 + 2 ** -7), 0.0, 255.0, 256.0, 2 ** -30]
+    S = np.zeros((1, 4, 16), np.float32)
+    S[0, 1, :len(vals)] = vals
+    snap = oracle.quantize(S, 0, bits=16)
+    assert snap["dense"][0, 1, :len(vals)].tolist() == [float(np.float32(w)) for w in want]
