@@ -14,7 +14,7 @@ the roofline.  Each decode launch reads 160-300 MB (int8 state, records,
 inputs), above the 126 MB L2, so every launch streams from HBM.
 
 Other modes: --mode prefill | fp32step | init | ragged | mse (see --help);
---bits 6 | 4 runs any decode mode on the narrow-code state variants.
+--bits 6 | 4 | 16 runs any decode mode on the narrow-code or BF16 state variants.
 
 Multi-GPU (torchrun): every rank decodes its own shard of sequences (batch
 per rank fixed: weak scaling); no collective on the data path; the host
@@ -52,9 +52,9 @@ FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # --------------------------------------------------------------------------
 
 def snapshot_bytes(dk, dv, r, bits=8):
-    """Codes (one byte per code, half a byte at 4 bits), row scales,
-    smoothing factors and compensators of one head."""
-    codes = dv * dk // 2 if bits == 4 else dv * dk
+    """Codes (one byte per code, half a byte at 4 bits, two bytes per BF16
+    value at 16), row scales, smoothing factors and compensators of one head."""
+    codes = dv * dk // 2 if bits == 4 else 2 * dv * dk if bits == 16 else dv * dk
     return codes + 4 * dv + 4 * dk + r * (4 + 4 * dk)
 
 
@@ -278,7 +278,8 @@ def run_reference(args, wl):
 
 
 def state_words(bits):
-    return {8: "int8 codes", 6: "6-bit codes (one per byte)", 4: "4-bit codes (two per byte)"}[bits]
+    return {8: "int8 codes", 6: "6-bit codes (one per byte)", 4: "4-bit codes (two per byte)",
+            16: "bf16 residual"}[bits]
 
 
 def profile_key(kernel, wl, args):
@@ -791,7 +792,8 @@ def run_mse(args, wl):
     variants = {"per_window": (wl.window, wl.n_comp, sm0, 8),
                 "per_token": (1, 0, sm0, 8), "per_token_plain": (1, 0, 0, 8),
                 "per_window_6bit": (wl.window, wl.n_comp, sm0, 6), "per_token_6bit": (1, 0, sm0, 6),
-                "per_window_4bit": (wl.window, wl.n_comp, sm0, 4), "per_token_4bit": (1, 0, sm0, 4)}
+                "per_window_4bit": (wl.window, wl.n_comp, sm0, 4), "per_token_4bit": (1, 0, sm0, 4),
+                "per_window_bf16": (wl.window, 0, 0, 16), "per_token_bf16": (1, 0, 0, 16)}
     states, cfgs = {}, {}
     for name, (W, r, sm, bits) in variants.items():
         cfg = lq.Config(batch=wl.batch, heads=wl.heads, d_k=wl.d_k, d_v=wl.d_v, window=W, n_comp=r,
@@ -860,8 +862,8 @@ def main(argv=None):
     ap.add_argument("--window", type=int, default=None, help="override W (comparators / sweep)")
     ap.add_argument("--n-comp", type=int, default=None, help="override r")
     ap.add_argument("--no-smoothing", action="store_true")
-    ap.add_argument("--bits", type=int, choices=[8, 6, 4], default=8,
-                    help="code width of the state (8; 6 and 4 are the narrow variants)")
+    ap.add_argument("--bits", type=int, choices=[8, 6, 4, 16], default=8,
+                    help="code width of the state (8; 6 and 4 are the narrow variants; 16 = BF16)")
     ap.add_argument("--slots", type=int, default=8, help="distinct input windows (graphs)")
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")

@@ -96,7 +96,11 @@ typedef struct {
                             state groups (Table 1) and fixes no format, so
                             the narrower widths are this library's variant of
                             the same quantizer.  8 and 6 store one code per
-                            byte, 4 stores two (see lq_snapshot).          */
+                            byte, 4 stores two (see lq_snapshot).
+                            16: the BF16 state of the paper's Table 2
+                            ablation: compensators as above, the residual
+                            stored as BF16 values (round to nearest even),
+                            no smoothing, row_scale = col_smooth = 1.      */
 } lq_config;
 
 /* The quantized boundary state of every (b, h), all device memory:
@@ -107,7 +111,8 @@ typedef struct {
  *                                              row, byte 4g+b (b = 0..3) holds
  *                                              channel 8g+b in its low nibble
  *                                              and 8g+4+b in its high nibble,
- *                                              both two's complement
+ *                                              both two's complement;
+ *              bf16    [B*H][d_v][d_k]  (16B)  at bits = 16: the residual
  *   row_scale  float   [B*H][d_v]       (16B)  sigma_i (0 for a zero row)
  *   col_smooth float   [B*H][d_k]       (16B)  c_j (1 when smoothing is off)
  *   comp_row   int32   [B*H][r]                row index of each compensator,
@@ -141,7 +146,9 @@ typedef struct {
 } lq_state;
 
 /* Number of elements of one buffer of a state with configuration `cfg`
- * (for sizing allocations); -1 for an invalid configuration.
+ * (for sizing allocations; codes count elements of their storage type:
+ * int8, uint8 at bits = 4, bf16 at bits = 16); -1 for an invalid
+ * configuration.
  * which: 0 codes, 1 row_scale, 2 col_smooth, 3 comp_row, 4 comp_val,
  *        5 buf_gate, 6 buf_k, 7 buf_u. */
 LQ_API int64_t lq_buffer_elems(const lq_config *cfg, int32_t which);

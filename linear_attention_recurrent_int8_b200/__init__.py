@@ -132,7 +132,7 @@ class Config:
     smoothing: int = 1
     auto_commit: int = 1
     delta: int = 1
-    bits: int = 8  # code width: 8, 6 (one code per byte) or 4 (two per byte)
+    bits: int = 8  # code width: 8, 6 (one code per byte), 4 (two per byte), 16 (BF16 residual)
 
     def c(self) -> LqConfig:
         return LqConfig(self.batch, self.heads, self.d_k, self.d_v, self.window, self.n_comp,
@@ -141,8 +141,13 @@ class Config:
 
     @property
     def code_cols(self) -> int:
-        """Bytes of one value row of codes (d_k, or d_k / 2 at 4 bits)."""
+        """Elements of one value row of the residual (d_k, or d_k / 2 bytes at 4 bits)."""
         return self.d_k // 2 if self.bits == 4 else self.d_k
+
+    @property
+    def code_torch_dtype(self):
+        import torch
+        return {4: torch.uint8, 16: torch.bfloat16}.get(self.bits, torch.int8)
 
     @property
     def gdim(self) -> int:
@@ -162,8 +167,8 @@ class Snapshot:
         bh = cfg.batch * cfg.heads
         if tensors is None:
             tensors = dict(
-                codes=torch.zeros((bh, cfg.d_v, cfg.code_cols),
-                                  dtype=torch.uint8 if cfg.bits == 4 else torch.int8, device=device),
+                codes=torch.zeros((bh, cfg.d_v, cfg.code_cols), dtype=cfg.code_torch_dtype,
+                                  device=device),
                 row_scale=torch.zeros((bh, cfg.d_v), dtype=torch.float32, device=device),
                 col_smooth=torch.ones((bh, cfg.d_k), dtype=torch.float32, device=device),
                 comp_row=torch.zeros((bh, cfg.n_comp), dtype=torch.int32, device=device),

@@ -28,16 +28,24 @@ lq_status check_config(const lq_config *c) {
     if ((c->smoothing != 0 && c->smoothing != 1) || (c->auto_commit != 0 && c->auto_commit != 1) ||
         (c->delta != 0 && c->delta != 1))
         return LQ_ERR_INVALID_ARGUMENT;
-    if (c->bits != 0 && c->bits != 8 && c->bits != 6 && c->bits != 4) return LQ_ERR_INVALID_ARGUMENT;
+    if (c->bits != 0 && c->bits != 8 && c->bits != 6 && c->bits != 4 && c->bits != 16)
+        return LQ_ERR_INVALID_ARGUMENT;
     return LQ_OK;
 }
 
 // Code width of a valid configuration (0 means 8).
 int code_bits(const lq_config *c) { return c->bits == 0 ? 8 : c->bits; }
 
-// Bytes of one head's codes: one per code, or two codes per byte at 4 bits.
+// Bytes of one head's residual: one per code, two codes per byte at 4 bits,
+// two bytes per BF16 value at 16.
 size_t code_bytes_per_head(const lq_config *c) {
-    return (size_t)c->d_v * (code_bits(c) == 4 ? c->d_k / 2 : c->d_k);
+    return (size_t)c->d_v * lq::code_row_bytes(lq::code_format(code_bits(c)), c->d_k);
+}
+
+// Elements of one head's residual in its storage type (int8, uint8 or bf16).
+int64_t code_elems_per_head(const lq_config *c) {
+    const int b = code_bits(c);
+    return (int64_t)c->d_v * (b == 4 ? c->d_k / 2 : c->d_k);
 }
 
 lq_status check_snapshot(const lq_config *c, const lq_snapshot *s) {
@@ -139,7 +147,7 @@ int64_t lq_buffer_elems(const lq_config *cfg, int32_t which) {
     const int64_t bh = (int64_t)cfg->batch * cfg->heads;
     const int64_t G = cfg->gate == LQ_GATE_DIAG ? cfg->d_k : 1;
     switch (which) {
-        case 0: return bh * (int64_t)code_bytes_per_head(cfg);
+        case 0: return bh * code_elems_per_head(cfg);
         case 1: return bh * cfg->d_v;
         case 2: return bh * cfg->d_k;
         case 3: return bh * cfg->n_comp;

@@ -1,6 +1,6 @@
 // lq_commit.cu -- the window commit on sm_100a: rebuild of the FP32 state at
 // the window end, Compensator Tokens, residual smoothing and per-row
-// re-quantization to 8-bit (or 6- or 4-bit) codes ("LeapQuant: Efficient Linear Attention with Accurate
+// re-quantization to 8-bit (or 6- or 4-bit) codes, or BF16 ("LeapQuant: Efficient Linear Attention with Accurate
 // Recurrent State Quantization", Figure 2: the state is quantized once per
 // window; Figure 4 and the Abstract: the largest outliers are kept as
 // high-precision Compensator Tokens and the residual is smoothed across
@@ -160,16 +160,21 @@ __device__ __forceinline__ int next_commit_head(const DecodeArgs &a, int bh) {
     return BH;
 }
 
-// PACK4: 4-bit codes, two per byte (lq_quant.cuh); otherwise one per byte.
-template <int DK, int DV, int GATE, bool PACK4>
+// FMT: the residual's storage (lq_kernels.h): codes one per byte, 4-bit codes
+// two per byte (layout in lq_quant.cuh), or BF16 values.
+template <int DK, int DV, int GATE, int FMT>
 __global__ void __launch_bounds__(kThreads, 1) commit_kernel(const DecodeArgs a, const int NS,
                                                              const int NOPS) {
     static_assert(DV == 64 || DV == 128, "d_v must be 64 or 128");
     constexpr int NQ = DV / 32;        // lane quarters that hold rows
     constexpr int CPT = DK / 2;        // key channels per epilogue thread
     constexpr int NCH = CPT / 32;      // 32-column TMEM chunks per thread
-    constexpr int CRB = PACK4 ? DK / 2 : DK;  // code bytes per value row
-    constexpr int NCW = PACK4 ? CPT / 32 : CPT / 16;  // 16-byte code words per thread
+    constexpr bool PACK4 = FMT == kCodesI4, BF16S = FMT == kCodesBF16;
+    constexpr int CRB = code_row_bytes(FMT, DK);  // residual bytes per value row
+    // 16-byte code words per thread, loaded one head ahead (a BF16 row half
+    // is loaded chunk by chunk where it is used instead)
+    constexpr int NCW = PACK4 ? CPT / 32 : BF16S ? 1 : CPT / 16;
+    constexpr int JB = CRB / (DK / 2);  // residual bytes per 2 key channels
     constexpr int G = GATE == 1 ? DK : 1;
     extern __shared__ __align__(128) unsigned char smem[];
     auto &cs = *reinterpret_cast<CommitSmem<DK, DV> *>(smem);
@@ -344,8 +349,8 @@ __global__ void __launch_bounds__(kThreads, 1) commit_kernel(const DecodeArgs a,
     // prefetched them into L2)
     uint4 cw[NCW], cw_next[NCW];
     auto load_codes = [&](int bhx, uint4(&dst)[NCW]) {
-        if (has_row && bhx < BH) {
-            const int8_t *src = a.codes + ((size_t)bhx * DV + row) * CRB + (PACK4 ? j0 / 2 : j0);
+        if (!BF16S && has_row && bhx < BH) {
+            const int8_t *src = a.codes + ((size_t)bhx * DV + row) * CRB + j0 * JB / 2;
 #pragma unroll
             for (int c = 0; c < NCW; ++c) dst[c] = *reinterpret_cast<const uint4 *>(src + 16 * c);
         }
@@ -360,7 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1) commit_kernel(const DecodeArgs a,
         const float *Ls = reinterpret_cast<const float *>(st + SL.L);
         const float *Css = reinterpret_cast<const float *>(st + SL.cs);
         const float *Rss = reinterpret_cast<const float *>(st + SL.rs);
-        int8_t *codes_row = a.codes + ((size_t)bh * DV + (has_row ? row : 0)) * CRB + (PACK4 ? j0 / 2 : j0);
+        int8_t *codes_row = a.codes + ((size_t)bh * DV + (has_row ? row : 0)) * CRB + j0 * JB / 2;
         const uint32_t tq = cs.tmem + ((uint32_t)(32 * qtr) << 16) + b * DK + j0;
         for (int j = tid; j < DK; j += kEpi) cs.cg[j] = Css[j] * expf(Ls[(nrec - 1) * G + (GATE == 1 ? j : 0)]);
         if (tid < DV) cs.comp_idx[tid] = -1;
@@ -383,41 +388,64 @@ __global__ void __launch_bounds__(kThreads, 1) commit_kernel(const DecodeArgs a,
 #pragma unroll
             for (int c = 0; c < NCH; ++c) {
                 float x[32];
+                uint4 bw[BF16S ? 4 : 1];  // BF16: this chunk's 32 values (64 bytes)
+                if constexpr (BF16S) {
+#pragma unroll
+                    for (int v = 0; v < 4; ++v)
+                        bw[v] = *reinterpret_cast<const uint4 *>(codes_row + 64 * c + 16 * v);
+                }
                 tmem_load<32>(tq + 32 * c, x);
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
-                    uint32_t cword;
-                    if constexpr (PACK4) {
-                        // channels 8h..8h+3 sit in the low nibbles of word h,
-                        // 8h+4..8h+7 in the high ones: move the nibble into
-                        // the high half of each byte, giving 16 Q as an int8
-                        const uint32_t w = word_of(cw[c], q / 2);
-                        cword = (q & 1) ? (w & 0xF0F0F0F0u) : ((w << 4) & 0xF0F0F0F0u);
+                    if constexpr (BF16S) {
+                        // BF16 -> FP32 is a 16-bit shift; sigma = c = 1
+                        const uint32_t wa = word_of(bw[q / 2], 2 * (q % 2));
+                        const uint32_t wb = word_of(bw[q / 2], 2 * (q % 2) + 1);
+                        const float4 g = *reinterpret_cast<const float4 *>(cs.cg + j0 + 32 * c + 4 * q);
+                        const float2 f01 = make_float2(__uint_as_float(wa << 16), __uint_as_float(wa & 0xFFFF0000u));
+                        const float2 f23 = make_float2(__uint_as_float(wb << 16), __uint_as_float(wb & 0xFFFF0000u));
+                        const float2 y01 = __ffma2_rn(f01, make_float2(g.x, g.y), make_float2(x[4 * q], x[4 * q + 1]));
+                        const float2 y23 = __ffma2_rn(f23, make_float2(g.z, g.w), make_float2(x[4 * q + 2], x[4 * q + 3]));
+                        ss = __ffma2_rn(y01, y01, ss);
+                        ss = __ffma2_rn(y23, y23, ss);
+                        x[4 * q] = y01.x;
+                        x[4 * q + 1] = y01.y;
+                        x[4 * q + 2] = y23.x;
+                        x[4 * q + 3] = y23.y;
                     } else {
-                        cword = word_of(cw[2 * c + q / 4], q % 4);
+                        uint32_t cword;
+                        if constexpr (PACK4) {
+                            // channels 8h..8h+3 sit in the low nibbles of word h,
+                            // 8h+4..8h+7 in the high ones: move the nibble into
+                            // the high half of each byte, giving 16 Q as an int8
+                            const uint32_t w = word_of(cw[c], q / 2);
+                            cword = (q & 1) ? (w & 0xF0F0F0F0u) : ((w << 4) & 0xF0F0F0F0u);
+                        } else {
+                            cword = word_of(cw[2 * c + q / 4], q % 4);
+                        }
+                        const uint32_t u = cword ^ 0x80808080u;
+                        const float4 g = *reinterpret_cast<const float4 *>(cs.cg + j0 + 32 * c + 4 * q);
+                        // code + 128 in the low mantissa bits of 2^23, minus (2^23 + 128)
+                        float2 f01 = make_float2(__uint_as_float(__byte_perm(u, 0x4B000000u, 0x7650)),
+                                                 __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7651)));
+                        float2 f23 = make_float2(__uint_as_float(__byte_perm(u, 0x4B000000u, 0x7652)),
+                                                 __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7653)));
+                        if constexpr (PACK4) {
+                            f01 = __fmul2_rn(__ffma2_rn(f01, sixteenth2, off16_2), sg2);
+                            f23 = __fmul2_rn(__ffma2_rn(f23, sixteenth2, off16_2), sg2);
+                        } else {
+                            f01 = __fmul2_rn(__fadd2_rn(f01, off2), sg2);
+                            f23 = __fmul2_rn(__fadd2_rn(f23, off2), sg2);
+                        }
+                        const float2 y01 = __ffma2_rn(f01, make_float2(g.x, g.y), make_float2(x[4 * q], x[4 * q + 1]));
+                        const float2 y23 = __ffma2_rn(f23, make_float2(g.z, g.w), make_float2(x[4 * q + 2], x[4 * q + 3]));
+                        ss = __ffma2_rn(y01, y01, ss);
+                        ss = __ffma2_rn(y23, y23, ss);
+                        x[4 * q] = y01.x;
+                        x[4 * q + 1] = y01.y;
+                        x[4 * q + 2] = y23.x;
+                        x[4 * q + 3] = y23.y;
                     }
-                    const uint32_t u = cword ^ 0x80808080u;
-                    const float4 g = *reinterpret_cast<const float4 *>(cs.cg + j0 + 32 * c + 4 * q);
-                    // code + 128 in the low mantissa bits of 2^23, minus (2^23 + 128)
-                    float2 f01 = make_float2(__uint_as_float(__byte_perm(u, 0x4B000000u, 0x7650)),
-                                             __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7651)));
-                    float2 f23 = make_float2(__uint_as_float(__byte_perm(u, 0x4B000000u, 0x7652)),
-                                             __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7653)));
-                    if constexpr (PACK4) {
-                        f01 = __fmul2_rn(__ffma2_rn(f01, sixteenth2, off16_2), sg2);
-                        f23 = __fmul2_rn(__ffma2_rn(f23, sixteenth2, off16_2), sg2);
-                    } else {
-                        f01 = __fmul2_rn(__fadd2_rn(f01, off2), sg2);
-                        f23 = __fmul2_rn(__fadd2_rn(f23, off2), sg2);
-                    }
-                    const float2 y01 = __ffma2_rn(f01, make_float2(g.x, g.y), make_float2(x[4 * q], x[4 * q + 1]));
-                    const float2 y23 = __ffma2_rn(f23, make_float2(g.z, g.w), make_float2(x[4 * q + 2], x[4 * q + 3]));
-                    ss = __ffma2_rn(y01, y01, ss);
-                    ss = __ffma2_rn(y23, y23, ss);
-                    x[4 * q] = y01.x;
-                    x[4 * q + 1] = y01.y;
-                    x[4 * q + 2] = y23.x;
-                    x[4 * q + 3] = y23.y;
                 }
                 tmem_store32(tq + 32 * c, x);
             }
@@ -477,11 +505,13 @@ __global__ void __launch_bounds__(kThreads, 1) commit_kernel(const DecodeArgs a,
                     __syncwarp();
                     tmem_store32(tq + 32 * c, x);
                 }
+                if constexpr (!BF16S) {  // BF16: no smoothing, no column maxima
 #pragma unroll
-                for (int e = 0; e < 32; e += 4) {
-                    const float4 m = make_float4(warp_max_abs(x[e]), warp_max_abs(x[e + 1]),
-                                                 warp_max_abs(x[e + 2]), warp_max_abs(x[e + 3]));
-                    if (lane == 0) *reinterpret_cast<float4 *>(&cs.colpart[qtr][j0 + 32 * c + e]) = m;
+                    for (int e = 0; e < 32; e += 4) {
+                        const float4 m = make_float4(warp_max_abs(x[e]), warp_max_abs(x[e + 1]),
+                                                     warp_max_abs(x[e + 2]), warp_max_abs(x[e + 3]));
+                        if (lane == 0) *reinterpret_cast<float4 *>(&cs.colpart[qtr][j0 + 32 * c + e]) = m;
+                    }
                 }
             }
             if (any_comp) tmem_wait_st();
@@ -489,17 +519,41 @@ __global__ void __launch_bounds__(kThreads, 1) commit_kernel(const DecodeArgs a,
         named_sync<kEpiBar, kEpi>();
         // C3 (2/2): smoothing factor c_j and its inverse
         for (int j = tid; j < DK; j += kEpi) {
-            float mj = cs.colpart[0][j];
+            float mj = 0.0f;
+            if constexpr (!BF16S) {
+                mj = cs.colpart[0][j];
 #pragma unroll
-            for (int q = 1; q < NQ; ++q) mj = fmaxf(mj, cs.colpart[q][j]);
+                for (int q = 1; q < NQ; ++q) mj = fmaxf(mj, cs.colpart[q][j]);
+            }
             const float c = (a.smoothing && mj > 0.0f) ? __fsqrt_rn(mj) : 1.0f;
             a.col_smooth[(size_t)bh * DK + j] = c;
             cs.icol[j] = __fdiv_rn(1.0f, c);
         }
         named_sync<kEpiBar, kEpi>();
 
+        // BF16 residual: unit scale and the values rounded to BF16 (nearest even)
+        if constexpr (BF16S) {
+            if (has_row) {
+                if (half == 0) a.row_scale[(size_t)bh * DV + row] = 1.0f;
+#pragma unroll
+                for (int c = 0; c < NCH; ++c) {
+                    float x[32];
+                    tmem_load<32>(tq + 32 * c, x);
+                    uint32_t hv[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const __nv_bfloat162 p = __floats2bfloat162_rn(x[2 * e], x[2 * e + 1]);
+                        hv[e] = *reinterpret_cast<const uint32_t *>(&p);
+                    }
+#pragma unroll
+                    for (int v = 0; v < 4; ++v)
+                        *reinterpret_cast<uint4 *>(codes_row + 64 * c + 16 * v) =
+                            make_uint4(hv[4 * v], hv[4 * v + 1], hv[4 * v + 2], hv[4 * v + 3]);
+                }
+            }
+        }
         // C4: R' = R (1/c) (kept in TMEM) and its row maximum
-        if (has_row) {
+        if (!BF16S && has_row) {
             float mx = 0.0f;
 #pragma unroll
             for (int c = 0; c < NCH; ++c) {
@@ -528,7 +582,7 @@ __global__ void __launch_bounds__(kThreads, 1) commit_kernel(const DecodeArgs a,
         // rounds to at most q: no clamp.  The magic-number addition rounds
         // half to even; the low byte of its bits is the two's-complement code
         // (its low nibble the 4-bit code).
-        if (has_row) {
+        if (!BF16S && has_row) {
             const float qmax = (float)((1 << (a.bits - 1)) - 1);  // 127, 31 or 7
             const float mxr = fmaxf(cs.rowpart[0][row], cs.rowpart[1][row]);
             if (half == 0) a.row_scale[(size_t)bh * DV + row] = __fdiv_rn(mxr, qmax);
@@ -581,14 +635,14 @@ struct DeviceInfo {
     int sms, smem_optin;
 };
 
-template <int DK, int DV, int GATE, bool PACK4>
+template <int DK, int DV, int GATE, int FMT>
 cudaError_t launch_c(const DecodeArgs &a, cudaStream_t stream) {
     static std::atomic<uint64_t> configured{0};  // devices already set up
     static DeviceInfo info[64];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    auto kern = commit_kernel<DK, DV, GATE, PACK4>;
+    auto kern = commit_kernel<DK, DV, GATE, FMT>;
     const uint64_t bit = 1ull << (dev & 63);
     if (!(configured.load(std::memory_order_acquire) & bit)) {
         DeviceInfo I{};
@@ -619,9 +673,13 @@ cudaError_t launch_c(const DecodeArgs &a, cudaStream_t stream) {
 }
 template <int DK, int DV>
 cudaError_t launch_c_d(const DecodeArgs &a, int gate, cudaStream_t stream) {
-    if (a.bits == 4)
-        return gate == 1 ? launch_c<DK, DV, 1, true>(a, stream) : launch_c<DK, DV, 0, true>(a, stream);
-    return gate == 1 ? launch_c<DK, DV, 1, false>(a, stream) : launch_c<DK, DV, 0, false>(a, stream);
+    const int fmt = code_format(a.bits);
+    if (fmt == kCodesI4)
+        return gate == 1 ? launch_c<DK, DV, 1, kCodesI4>(a, stream) : launch_c<DK, DV, 0, kCodesI4>(a, stream);
+    if (fmt == kCodesBF16)
+        return gate == 1 ? launch_c<DK, DV, 1, kCodesBF16>(a, stream)
+                         : launch_c<DK, DV, 0, kCodesBF16>(a, stream);
+    return gate == 1 ? launch_c<DK, DV, 1, kCodesI8>(a, stream) : launch_c<DK, DV, 0, kCodesI8>(a, stream);
 }
 
 }  // namespace
@@ -643,7 +701,7 @@ cudaError_t launch_advance_positions(int32_t *seq_pos, int B, int W, cudaStream_
 
 cudaError_t launch_commit(const DecodeArgs &a, int d_k, int d_v, int gate, cudaStream_t stream) {
     if (a.pos < 1 || a.pos > 32 || a.R < 0 || a.R > kMaxComp) return cudaErrorInvalidValue;
-    if (a.bits != 8 && a.bits != 6 && a.bits != 4) return cudaErrorInvalidValue;
+    if (a.bits != 8 && a.bits != 6 && a.bits != 4 && a.bits != 16) return cudaErrorInvalidValue;
     if (d_k == 128 && d_v == 128) return launch_c_d<128, 128>(a, gate, stream);
     if (d_k == 128 && d_v == 64) return launch_c_d<128, 64>(a, gate, stream);
     if (d_k == 64 && d_v == 128) return launch_c_d<64, 128>(a, gate, stream);

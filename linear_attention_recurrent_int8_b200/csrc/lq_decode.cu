@@ -16,8 +16,9 @@
 // pseudo-records at window position 0 (Figure 4; they share the update path
 // of real tokens), so they enter with decay e^{L_t}.
 //
-// The boundary state's codes are 8-bit (or 6-bit) one per byte, or 4-bit two
-// per byte (PACK4; layout in lq_quant.cuh).
+// The boundary state's residual is stored as 8-bit (or 6-bit) codes one per
+// byte, 4-bit codes two per byte (layout in lq_quant.cuh), or BF16 values
+// (the format FMT of lq_kernels.h).
 //
 // Kernel structure (persistent, warp-specialised, 12 warps per CTA):
 //  * the grid walks the (sequence, head) pairs with a grid stride; each head
@@ -27,7 +28,8 @@
 //    q/k/v into a stage with 1-D bulk copies (no multicast) -> "full";
 //  * prep A (warp 9): for every token of the call, the vectors
 //    x_k = c e^L k and x_q = c e^L q split into three int8 limbs per
-//    16-channel chunk, and k~_t . q_t -> "prepared";
+//    16-channel chunk (kept in FP32 for a BF16 residual), and k~_t . q_t
+//    -> "prepared";
 //  * prep B (warps 10, 11): the records (L_t, k~_t) of the new tokens and
 //    every coefficient (k~_m e^{L_t-L_m}) . k_t, . q_t of the buffered records
 //    and compensators -> "prepared";
@@ -66,10 +68,11 @@ struct PrepLayout {
     int limb, lscale, coefA, coefG, bytes;
 };
 
-__host__ __device__ inline PrepLayout prep_layout(int DK) {
+__host__ __device__ inline PrepLayout prep_layout(int DK, int fmt) {
     PrepLayout P{};
     int o = 0;
-    P.limb = o;   o += 6 * DK;            // int8 [6][DK]: x_k limbs 0..2, x_q limbs 0..2
+    P.limb = o;                            // int8 [6][DK]: x_k limbs 0..2, x_q limbs 0..2,
+    o += fmt == kCodesBF16 ? 8 * DK : 6 * DK;  // or (BF16 residual) float [2][DK]: x_k, x_q
     P.lscale = o; o += 16;                 // float [2]: scales of x_k, x_q
     P.coefA = o;  o += 4 * kCoef;          // records, compensators
     P.coefG = o;  o += 4 * kCoef;          // records, compensators, own token (k~.q)
@@ -79,16 +82,16 @@ __host__ __device__ inline PrepLayout prep_layout(int DK) {
 
 // Byte offsets inside one stage (one head's operands).  `nrec` is the number
 // of record slots the stage holds (records read plus records written), `n`
-// the number of tokens of the call; `pack4`: 4-bit codes, two per byte.
+// the number of tokens of the call; `fmt` the residual's storage.
 struct StageLayout {
     int codes, sig, cs, compv, compr, recK, recU, recL, q, k, v, al, scal, prep, bytes;
 };
 
 __host__ __device__ inline StageLayout stage_layout(int DK, int DV, int gate, int R, int nrec,
-                                                   int n, int e, bool pack4) {
+                                                   int n, int e, int fmt) {
     StageLayout L{};
     int o = 0;
-    L.codes = o; o += align16(DV * (pack4 ? DK / 2 : DK));
+    L.codes = o; o += align16(DV * code_row_bytes(fmt, DK));
     L.sig = o;   o += align16(4 * DV);
     L.cs = o;    o += align16(4 * DK);
     L.compv = o; o += align16(4 * R * DK);
@@ -101,7 +104,7 @@ __host__ __device__ inline StageLayout stage_layout(int DK, int DV, int gate, in
     L.v = o;     o += align16(e * DV);
     L.al = o;    o += gate == 1 ? align16(4 * DK) : 0;
     L.scal = o;  o += 16;                  // float: alpha (scalar gate), beta of token 0
-    L.prep = o;  o += n * prep_layout(DK).bytes;
+    L.prep = o;  o += n * prep_layout(DK, fmt).bytes;
     L.bytes = align16(o);
     return L;
 }
@@ -163,19 +166,20 @@ __device__ __forceinline__ int next_decode_head(const DecodeArgs &a, int bh) {
 
 // RAGGED: per-sequence window positions (a.seq_pos); otherwise the window
 // position a.pos is the same for every head and stays a kernel constant.
-// PACK4: 4-bit codes, two per byte.
-template <int DK, int DV, int GATE, bool BF16, bool RAGGED, bool PACK4>
+// FMT: the residual's storage (lq_kernels.h).
+template <int DK, int DV, int GATE, bool BF16, bool RAGGED, int FMT>
 __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a, const int S) {
     constexpr int E = BF16 ? 2 : 4;
     constexpr int RPW = DV / kConsumerWarps;  // value rows per consumer warp
-    constexpr int CRB = PACK4 ? DK / 2 : DK;  // code bytes per value row
+    constexpr bool PACK4 = FMT == kCodesI4, BF16S = FMT == kCodesBF16;
+    constexpr int CRB = code_row_bytes(FMT, DK);  // residual bytes per value row
     extern __shared__ __align__(128) unsigned char smem[];
     uint64_t *full = reinterpret_cast<uint64_t *>(smem);
     uint64_t *prepared = full + kMaxStages;
     uint64_t *empty = prepared + kMaxStages;
     const int nsteps = a.n_steps;
-    const StageLayout SL = stage_layout(DK, DV, GATE, a.R, a.pos + nsteps, nsteps, E, PACK4);
-    const PrepLayout PL = prep_layout(DK);
+    const StageLayout SL = stage_layout(DK, DV, GATE, a.R, a.pos + nsteps, nsteps, E, FMT);
+    const PrepLayout PL = prep_layout(DK, FMT);
     unsigned char *stages = smem + header_bytes();
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -325,8 +329,16 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a,
                         xq[e] = cj[e] * (gj[e] * qj[e]);
                         kq = fmaf(beta * kj[e], qj[e], kq);
                     }
-                    split_limbs<CPL, 3>(xk, limb, DK, lscale, j0);
-                    split_limbs<CPL, 3>(xq, limb + 3 * DK, DK, lscale + 1, j0);
+                    if constexpr (BF16S) {
+                        // the FP32 vectors themselves, unit scales
+                        float *xs = reinterpret_cast<float *>(limb);
+                        store_vec<CPL>(xs + j0, xk);
+                        store_vec<CPL>(xs + DK + j0, xq);
+                        if (lane == 0) lscale[0] = lscale[1] = 1.0f;
+                    } else {
+                        split_limbs<CPL, 3>(xk, limb, DK, lscale, j0);
+                        split_limbs<CPL, 3>(xq, limb + 3 * DK, DK, lscale + 1, j0);
+                    }
                     kq = group_sum<32>(kq);
                     if (lane == 0) coefG[nrec + R] = kq;
                 } else {
@@ -453,7 +465,47 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a,
             // 4-bit codes enter as 16 Q (the nibble in the high half of an
             // int8), so every sum is 16 times larger and the unit is 2^-18.
             float y;
-            {
+            if constexpr (BF16S) {
+                // BF16 residual: FP32 FMAs with the FP32 vectors.  Lane cc
+                // takes key channels [8cc, 8cc+8) and [d_k/2 + 8cc, d_k/2 +
+                // 8cc + 8), so each 16-byte read is contiguous across a row's lanes.
+                const float *xs = reinterpret_cast<const float *>(limb);
+                float xk[16], xq[16];
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int v = 0; v < 2; ++v) {
+                        const float4 a4 = *reinterpret_cast<const float4 *>(xs + h * (DK / 2) + 8 * cc + 4 * v);
+                        const float4 b4 = *reinterpret_cast<const float4 *>(xs + DK + h * (DK / 2) + 8 * cc + 4 * v);
+                        const int o = 8 * h + 4 * v;
+                        xk[o] = a4.x; xk[o + 1] = a4.y; xk[o + 2] = a4.z; xk[o + 3] = a4.w;
+                        xq[o] = b4.x; xq[o + 1] = b4.y; xq[o + 2] = b4.z; xq[o + 3] = b4.w;
+                    }
+                float vals[2 * NRM];
+#pragma unroll
+                for (int n = 0; n < NRM; ++n) {
+                    const int r = warp * RPW + n * RPI16 + sub;
+                    const int8_t *rowp = codes_s + r * CRB;
+                    const uint4 w0 = *reinterpret_cast<const uint4 *>(rowp + 16 * cc);
+                    const uint4 w1 = *reinterpret_cast<const uint4 *>(rowp + DK + 16 * cc);
+                    const uint32_t ww[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                    float ak = 0.0f, aq = 0.0f;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        // element 2i in the low half of word i, 2i+1 in the high half
+                        const float lo = __uint_as_float(ww[i] << 16);
+                        const float hi = __uint_as_float(ww[i] & 0xFFFF0000u);
+                        ak = fmaf(lo, xk[2 * i], ak);
+                        ak = fmaf(hi, xk[2 * i + 1], ak);
+                        aq = fmaf(lo, xq[2 * i], aq);
+                        aq = fmaf(hi, xq[2 * i + 1], aq);
+                    }
+                    vals[n] = ak;
+                    vals[NRM + n] = aq;
+                }
+                transposed_sum<2 * NRM, LPR16>(vals, lane);
+                y = vals[0];
+            } else {
                 uint4 lw[6];
 #pragma unroll
                 for (int v = 0; v < 6; ++v)
@@ -490,7 +542,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a,
             // D3-D6 for row `row`: LPRD lanes share its buffered records
             {
                 const float sg = sig_s[row];
-                constexpr float kUnit = PACK4 ? 3.814697265625e-06f : 6.103515625e-05f;  // 2^-18, 2^-14
+                // 2^-18 (4-bit codes enter as 16 Q), 2^-14, or 1 (FP32 sums of a BF16 residual)
+                constexpr float kUnit = PACK4 ? 3.814697265625e-06f : BF16S ? 1.0f : 6.103515625e-05f;
                 const float yk = __shfl_sync(0xffffffffu, y, src_k) * (sg * (lscale[0] * kUnit));
                 const float yq = __shfl_sync(0xffffffffu, y, src_q) * (sg * (lscale[1] * kUnit));
                 float hb = part == 0 ? yk : 0.0f, p = part == 0 ? yq : 0.0f;
@@ -529,7 +582,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a,
     }
 }
 
-template <int DK, int DV, int GATE, bool BF16, bool RAGGED, bool PACK4>
+template <int DK, int DV, int GATE, bool BF16, bool RAGGED, int FMT>
 cudaError_t launch_d(const DecodeArgs &a, cudaStream_t stream) {
     constexpr int E = BF16 ? 2 : 4;
     static std::atomic<uint64_t> configured{0};  // devices already set up
@@ -537,7 +590,7 @@ cudaError_t launch_d(const DecodeArgs &a, cudaStream_t stream) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    auto kern = decode_kernel<DK, DV, GATE, BF16, RAGGED, PACK4>;
+    auto kern = decode_kernel<DK, DV, GATE, BF16, RAGGED, FMT>;
     const uint64_t bit = 1ull << (dev & 63);
     if (!(configured.load(std::memory_order_acquire) & bit)) {
         int optin = 0, sms = 0;
@@ -550,7 +603,7 @@ cudaError_t launch_d(const DecodeArgs &a, cudaStream_t stream) {
         configured.fetch_or(bit, std::memory_order_acq_rel);
     }
     // a stage holds the records this launch reads and writes (pos + n_steps)
-    const StageLayout SL = stage_layout(DK, DV, GATE, a.R, a.pos + a.n_steps, a.n_steps, E, PACK4);
+    const StageLayout SL = stage_layout(DK, DV, GATE, a.R, a.pos + a.n_steps, a.n_steps, E, FMT);
     const int fixed = header_bytes();
     // two CTAs per SM when registers allow it and each can hold at least
     // two stages, else one CTA per SM with as many stages as fit
@@ -579,11 +632,15 @@ cudaError_t launch_d(const DecodeArgs &a, cudaStream_t stream) {
 
 template <int DK, int DV, int GATE, bool BF16>
 cudaError_t launch_dr(const DecodeArgs &a, cudaStream_t stream) {
-    if (a.bits == 4)
-        return a.seq_pos ? launch_d<DK, DV, GATE, BF16, true, true>(a, stream)
-                         : launch_d<DK, DV, GATE, BF16, false, true>(a, stream);
-    return a.seq_pos ? launch_d<DK, DV, GATE, BF16, true, false>(a, stream)
-                     : launch_d<DK, DV, GATE, BF16, false, false>(a, stream);
+    const int fmt = code_format(a.bits);
+    if (fmt == kCodesI4)
+        return a.seq_pos ? launch_d<DK, DV, GATE, BF16, true, kCodesI4>(a, stream)
+                         : launch_d<DK, DV, GATE, BF16, false, kCodesI4>(a, stream);
+    if (fmt == kCodesBF16)
+        return a.seq_pos ? launch_d<DK, DV, GATE, BF16, true, kCodesBF16>(a, stream)
+                         : launch_d<DK, DV, GATE, BF16, false, kCodesBF16>(a, stream);
+    return a.seq_pos ? launch_d<DK, DV, GATE, BF16, true, kCodesI8>(a, stream)
+                     : launch_d<DK, DV, GATE, BF16, false, kCodesI8>(a, stream);
 }
 
 template <int DK, int DV>
@@ -598,7 +655,7 @@ cudaError_t launch_decode_d(const DecodeArgs &a, int gate, bool bf16, cudaStream
 cudaError_t launch_decode(const DecodeArgs &a, int d_k, int d_v, int gate, bool bf16,
                           cudaStream_t stream) {
     if (a.n_steps < 1) return cudaErrorInvalidValue;
-    if (a.bits != 8 && a.bits != 6 && a.bits != 4) return cudaErrorInvalidValue;
+    if (a.bits != 8 && a.bits != 6 && a.bits != 4 && a.bits != 16) return cudaErrorInvalidValue;
     if (d_k == 128 && d_v == 128) return launch_decode_d<128, 128>(a, gate, bf16, stream);
     if (d_k == 128 && d_v == 64) return launch_decode_d<128, 64>(a, gate, bf16, stream);
     if (d_k == 64 && d_v == 128) return launch_decode_d<64, 128>(a, gate, bf16, stream);

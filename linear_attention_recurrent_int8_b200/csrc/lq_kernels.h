@@ -7,6 +7,17 @@
 
 namespace lq {
 
+// Storage of a snapshot's residual: integer codes one per byte (8- and 6-bit
+// widths), two per byte (4-bit), or BF16 values (bits = 16).
+enum CodeFormat { kCodesI8 = 0, kCodesI4 = 1, kCodesBF16 = 2 };
+__host__ __device__ constexpr int code_format(int bits) {
+    return bits == 4 ? kCodesI4 : bits == 16 ? kCodesBF16 : kCodesI8;
+}
+// Bytes of one value row of the residual with d_k key channels.
+__host__ __device__ constexpr int code_row_bytes(int fmt, int dk) {
+    return fmt == kCodesI4 ? dk / 2 : fmt == kCodesBF16 ? 2 * dk : dk;
+}
+
 // Arguments of the decode and commit kernels.
 struct DecodeArgs {
     int8_t *codes;
@@ -28,7 +39,7 @@ struct DecodeArgs {
     int pos;      // records already buffered (the same for every sequence)
     int n_steps;  // tokens decoded by this launch (0: commit only)
     int smoothing;
-    int bits;     // code width: 8 or 6 (one code per byte) or 4 (two per byte)
+    int bits;     // code width: 8 or 6 (one code per byte), 4 (two per byte), 16 (BF16)
     // per-sequence window positions [B] (device), or nullptr.  When set, the
     // decode takes one token per sequence b with seq_pos[b] in [0, W) at
     // window position seq_pos[b] + 1 (pos and n_steps are then W - 1 and 1,
@@ -47,7 +58,7 @@ struct QuantArgs {
     int32_t *comp_row;
     float *comp_val;
     int BH, R, smoothing;
-    int bits;  // code width: 8 or 6 (one code per byte) or 4 (two per byte)
+    int bits;  // code width: 8 or 6 (one code per byte), 4 (two per byte), 16 (BF16)
 };
 
 // Arguments of the FP32-state recurrence kernel (prefill, FP32 per-step).

@@ -31,7 +31,7 @@ __global__ void __launch_bounds__(kWarps * 32) quantize_kernel(const QuantArgs a
         S[n][2] = x.z;
         S[n][3] = x.w;
     }
-    const size_t code_bytes = a.bits == 4 ? (size_t)DV * DK / 2 : (size_t)DV * DK;
+    const size_t code_bytes = (size_t)DV * code_row_bytes(code_format(a.bits), DK);
     SnapPtr out{a.codes + (size_t)bh * code_bytes, a.row_scale + (size_t)bh * DV,
                 a.col_smooth + (size_t)bh * DK, a.comp_row ? a.comp_row + (size_t)bh * a.R : nullptr,
                 a.comp_val ? a.comp_val + (size_t)bh * a.R * DK : nullptr};

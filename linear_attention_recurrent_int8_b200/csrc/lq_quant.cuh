@@ -17,6 +17,8 @@
 //       4-bit widths of the paper's lower-precision groups (Table 1); 4-bit
 //       codes are stored two per byte (low nibble: channel 8g+b, high
 //       nibble: channel 8g+4+b, in byte 4g+b of a row).
+// bits = 16 is the paper's BF16 state (Table 2): C2 as above, then c = 1,
+// sigma = 1 and the residual itself rounded to BF16 (nearest, ties to even).
 // Each smoothing factor and each row is inverted once; every element then
 // costs one FP32 product per step.  Every division, square root and product
 // is one IEEE round-to-nearest FP32 operation (__fdiv_rn, __fsqrt_rn, __fmul_rn),
@@ -49,7 +51,7 @@ struct Tile {
 
 // Device pointers of one head's snapshot.
 struct SnapPtr {
-    int8_t *codes;      // [DV][DK], or [DV][DK/2] bytes of packed 4-bit codes
+    int8_t *codes;      // [DV][DK], [DV][DK/2] bytes of packed 4-bit codes, or BF16 [DV][DK]
     float *row_scale;   // [DV]
     float *col_smooth;  // [DK]
     int32_t *comp_row;  // [R]
@@ -69,8 +71,8 @@ struct alignas(16) QuantSmem {
 
 // C2-C4 on the register tile S (the FP32 state of one head, owned as Tile
 // describes), writing the snapshot to `out` with codes of width `bits` (8, 6
-// or 4).  The NWARPS*32 threads that own the tile (threads 0 .. NWARPS*32-1)
-// call it; it synchronises them on named barrier 1.
+// or 4; 16 = BF16 residual).  The NWARPS*32 threads that own the tile
+// (threads 0 .. NWARPS*32-1) call it; it synchronises them on named barrier 1.
 template <int DK, int DV, int NWARPS>
 __device__ __forceinline__ void quantize_tile(float (&S)[Tile<DK, DV, NWARPS>::NR][4], int R,
                                               bool smoothing, int bits,
@@ -81,7 +83,8 @@ __device__ __forceinline__ void quantize_tile(float (&S)[Tile<DK, DV, NWARPS>::N
 
     const int gbase = lane & ~(T::LPR - 1);  // first lane of this lane's row group
     const float qmax = (float)((1 << (bits - 1)) - 1);
-    const bool pack4 = bits == 4;
+    const bool pack4 = bits == 4, bf16s = bits == 16;
+    if (bf16s) smoothing = false;  // c = 1 for the BF16 residual
     // C2 (1/2): squared row norms (order-preserving for the selection),
     // reduced across the row's lanes with a transposing reduction
     {
@@ -191,13 +194,22 @@ __device__ __forceinline__ void quantize_tile(float (&S)[Tile<DK, DV, NWARPS>::N
         const int n = transposed_index<T::NR, T::LPR>(lane);
         inv_own = mx[0] > 0.0f ? __fdiv_rn(qmax, mx[0]) : 0.0f;
         if ((lane & (T::LPR - 1)) == transposed_owner<T::NR, T::LPR>(n))
-            out.row_scale[T::row(warp, lane, n)] = __fdiv_rn(mx[0], qmax);
+            out.row_scale[T::row(warp, lane, n)] = bf16s ? 1.0f : __fdiv_rn(mx[0], qmax);
     }
 #pragma unroll
     for (int n = 0; n < T::NR; ++n) {
         const float inv =
             __shfl_sync(0xffffffffu, inv_own, gbase + transposed_owner<T::NR, T::LPR>(n));
         const int row = T::row(warp, lane, n);
+        if (bf16s) {
+            // the residual itself, rounded to BF16 (c = 1, so S is unscaled)
+            const __nv_bfloat162 p0 = __floats2bfloat162_rn(S[n][0], S[n][1]);
+            const __nv_bfloat162 p1 = __floats2bfloat162_rn(S[n][2], S[n][3]);
+            *reinterpret_cast<uint2 *>(out.codes + ((size_t)row * DK + c0) * 2) =
+                make_uint2(*reinterpret_cast<const uint32_t *>(&p0),
+                           *reinterpret_cast<const uint32_t *>(&p1));
+            continue;
+        }
         // round half to even by the magic-number addition (|y| <= q here),
         // clamp, and pack the four low bytes
         int iv[4];

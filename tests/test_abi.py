@@ -51,7 +51,7 @@ def test_buffer_elems():
     assert lq.lq_buffer_elems(cfg, 5) == bh * 16
     # code bytes: one per code at 8 and 6 bits (0 means 8), half a byte at 4
     for bits, want0 in ((0, bh * 64 * 128), (8, bh * 64 * 128), (6, bh * 64 * 128),
-                        (4, bh * 64 * 64)):
+                        (4, bh * 64 * 64), (16, bh * 64 * 128)):
         cfg.bits = bits
         assert lq.lq_buffer_elems(cfg, 0) == want0, bits
     cfg.bits = 5
@@ -132,7 +132,8 @@ def test_decode_validation_without_launch():
                              ("gate", 2, lq.LQ_ERR_INVALID_ARGUMENT),
                              ("delta", 2, lq.LQ_ERR_INVALID_ARGUMENT),
                              ("bits", 5, lq.LQ_ERR_INVALID_ARGUMENT),
-                             ("bits", 16, lq.LQ_ERR_INVALID_ARGUMENT),
+                             ("bits", 12, lq.LQ_ERR_INVALID_ARGUMENT),
+                             ("bits", 32, lq.LQ_ERR_INVALID_ARGUMENT),
                              ("batch", 0, lq.LQ_ERR_INVALID_ARGUMENT)):
         c2 = lq.Config(batch=2, heads=3, window=4, n_comp=2)
         setattr(c2, field, val)

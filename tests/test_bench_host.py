@@ -60,3 +60,8 @@ def test_narrow_code_byte_models():
     assert bench.decode_launch_bytes(128, 128, 4, "scalar", 2, 8, 4) == \
         bench.decode_launch_bytes(128, 128, 4, "scalar", 2, 8) - 8192
     assert bench.commit_launch_bytes(128, 128, 4, "scalar", 16, 4) == 2 * 11280 + 16 * 1028
+
+
+def test_bf16_state_byte_model():
+    # BF16 residual: two bytes per value
+    assert bench.snapshot_bytes(128, 128, 0, 16) == 2 * 128 * 128 + 4 * 128 + 4 * 128

@@ -1,6 +1,7 @@
-"""The 6- and 4-bit code widths (lq_config.bits): the same parity bar as the
-8-bit state -- initialisation codes bit-exact, anchored windows (outputs,
-records, next snapshot with codes within one step), the prefill's snapshots,
+"""The 6- and 4-bit code widths and the BF16 state (lq_config.bits = 6, 4,
+16): the same parity bar as the 8-bit state -- initialisation bit-exact,
+anchored windows (outputs, records, next snapshot with codes within one
+step, a BF16 residual within one BF16 step), the prefill's snapshots,
 per-sequence positions and a full-size sampled run -- against the oracle's
 quantizer at the same width.  4-bit codes are packed two per byte on the
 device (lq.h); the helpers unpack them before comparing."""
@@ -25,7 +26,7 @@ def _check_no_device_errors():
     assert lq.lq_device_errors() == 0
 
 
-@pytest.mark.parametrize("bits", [4, 6])
+@pytest.mark.parametrize("bits", [4, 6, 16])
 @pytest.mark.parametrize("name", ["gdn_1x1_d64_fp32", "gdn_64x16_d128_bf16"])
 def test_state_init_bit_exact(name, bits):
     wl = synth.WORKLOADS[name]
@@ -43,6 +44,10 @@ VARIANTS = [
     (64, 64, "scalar", "bf16", 1, 0, False, 5, 1, 4),
     (128, 128, "scalar", "fp32", 16, 4, True, 2, 3, 6),
     (64, 128, "diag", "bf16", 8, 2, True, 3, 1, 6),
+    (128, 128, "scalar", "bf16", 16, 0, True, 3, 5, 16),
+    (128, 128, "diag", "fp32", 8, 4, True, 2, 3, 16),
+    (64, 64, "scalar", "bf16", 1, 0, True, 4, 2, 16),
+    (128, 64, "scalar", "fp32", 32, 2, False, 1, 3, 16),
 ]
 
 
@@ -57,7 +62,7 @@ def test_variants(dk, dv, gate, io, W, r, smooth, B, H, bits):
     _check_no_device_errors()
 
 
-@pytest.mark.parametrize("bits", [4, 6])
+@pytest.mark.parametrize("bits", [4, 6, 16])
 def test_explicit_commit_short_window(bits):
     wl = synth.WORKLOADS["gdn_1x1_d64_fp32"]
     run = AnchoredRun(wl, cfg=make_config(wl, bits=bits), steps_per_call=3, commit_mode="explicit")
@@ -67,7 +72,7 @@ def test_explicit_commit_short_window(bits):
     _check_no_device_errors()
 
 
-@pytest.mark.parametrize("bits", [4, 6])
+@pytest.mark.parametrize("bits", [4, 6, 16])
 def test_prefill_snapshots(bits):
     B, H, dk, dv, T, every, r, io = 2, 3, 128, 128, 192, 64, 4, "bf16"
     cfg = lq.Config(batch=B, heads=H, d_k=dk, d_v=dv, window=16, n_comp=r, gate=0,
@@ -117,5 +122,31 @@ def test_gdn_256x32_4bit_sampled():
     run = SampledRun(wl, n_sample=16, seed=44, bits=4)
     run.init()
     for w in range(8):
+        run.window(w)
+    _check_no_device_errors()
+
+
+def test_snapshot_copy_moves_bf16_residual():
+    wl = synth.WORKLOADS["gdn_1x1_d64_fp32"]
+    cfg = make_config(wl, bits=16)
+    assert lq.lq_buffer_elems(cfg, 0) == wl.nh * wl.d_v * wl.d_k  # bf16 elements
+    run = AnchoredRun(wl, cfg=cfg)
+    ref = run.init()
+    dst = lq.Snapshot(cfg, "cuda")
+    lq.lq_state_snapshot(run.st, dst)
+    torch.cuda.synchronize()
+    assert dst.t["codes"].dtype == torch.bfloat16
+    assert torch.equal(dst.t["codes"], run.st.snap.t["codes"])
+    compare_snapshots(snapshot_to_host(cfg, dst), ref, ref["row_norm"], exact_codes=True)
+
+
+def test_gdn_256x32_bf16_state_sampled():
+    """The large-batch GDN workload with a BF16 state and no compensators (the
+    BF16 per-window row of the paper's Table 2 ablation), in the benchmark's
+    launch configuration, against the oracle on a seeded sample of heads."""
+    wl = dataclasses.replace(synth.WORKLOADS["gdn_256x32_d128_bf16"], n_comp=0)
+    run = SampledRun(wl, n_sample=16, seed=45, bits=16)
+    run.init()
+    for w in range(6):
         run.window(w)
     _check_no_device_errors()

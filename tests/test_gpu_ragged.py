@@ -11,8 +11,8 @@ import oracle
 import linear_attention_recurrent_int8_b200 as lq
 from linear_attention_recurrent_int8_b200 import synth
 
-from lqtest import (codes_to_device_format, compare_outputs, compare_snapshots, download_snapshot,
-                    heads_major, io_dtype, make_config, oracle_tokens)
+from lqtest import (compare_outputs, compare_snapshots, download_snapshot, heads_major, io_dtype,
+                    make_config, oracle_tokens, residual_to_device)
 
 pytestmark = pytest.mark.gpu
 
@@ -27,8 +27,10 @@ def _write_heads(st, snap, heads):
     """Device state's snapshot of `heads` <- snap (oracle arrays for those heads)."""
     idx = torch.as_tensor(heads, device="cuda")
     for key in ("codes", "row_scale", "col_smooth", "comp_row", "comp_val"):
-        val = codes_to_device_format(st.cfg, snap[key]) if key == "codes" else snap[key]
-        src = np.ascontiguousarray(val, np.int32 if key == "comp_row" else None)
+        if key == "codes":
+            st.snap.t[key][idx] = residual_to_device(st.cfg, snap)
+            continue
+        src = np.ascontiguousarray(snap[key], np.int32 if key == "comp_row" else None)
         st.snap.t[key][idx] = torch.from_numpy(src).to("cuda")
 
 
@@ -116,6 +118,11 @@ def test_ragged_staggered_windows(dk, dv, gate, io, W, r, B, H):
 def test_ragged_staggered_windows_4bit():
     _run(128, 128, "scalar", "bf16", 4, 2, 5, 3, steps=3 * 4 + 2, start_of=[b % 4 for b in range(5)],
          bits=4)
+
+
+def test_ragged_staggered_windows_bf16_state():
+    _run(64, 128, "diag", "fp32", 3, 1, 4, 2, steps=3 * 3 + 2, start_of=[b % 3 for b in range(4)],
+         bits=16)
 
 
 def test_ragged_matches_synchronous_when_aligned():
