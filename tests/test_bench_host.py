@@ -1,6 +1,13 @@
 """Host-side logic of the benchmark: the algorithmic byte models used for the
-roofline, and the lookup of ncu-measured traffic keyed on kernel sources."""
+roofline, the lookup of ncu-measured traffic keyed on kernel sources, and
+the reference arm's JSON line (it runs the CPU oracle only)."""
+import os
+
+import pytest
+
 import bench
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def test_decode_bytes_per_head():
@@ -65,3 +72,25 @@ def test_narrow_code_byte_models():
 def test_bf16_state_byte_model():
     # BF16 residual: two bytes per value
     assert bench.snapshot_bytes(128, 128, 0, 16) == 2 * 128 * 128 + 4 * 128 + 4 * 128
+
+
+@pytest.mark.parametrize("bits", [8, 4, 16])
+def test_reference_arm_line_on_cpu(bits):
+    """The reference arm (the oracle on the host cores) prints one JSON line
+    with the contract's keys, on a tiny workload, at every state width."""
+    import json
+    import subprocess
+    import sys
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "gdn_1x1_d64_fp32", "--steps", "1", "--warmup", "3",
+                        "--ref-seconds", "0.05", "--bits", str(bits)],
+                       cwd=ROOT, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["value"] > 0 and line["warmup"] >= 3
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["config"]["bits"] == bits
