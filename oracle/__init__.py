@@ -60,9 +60,9 @@ def _load():
             I = ctypes.c_int
             lib.lqo_eq1_steps.argtypes = [I, I, I, I, P, P, P, P, P, P, P]
             lib.lqo_quantize.argtypes = [I, I, I, I, I, I, P, P, P, P, P, P, P, P]
-            lib.lqo_dequantize.argtypes = [I, I, I, I, P, P, P, P, P, P, P]
-            lib.lqo_window.argtypes = [I] * 9 + [P] * 15
-            lib.lqo_rebuild.argtypes = [I] * 7 + [P] * 10
+            lib.lqo_dequantize.argtypes = [I, I, I, I, P, P, P, P, P, P, P, P]
+            lib.lqo_window.argtypes = [I] * 9 + [P] * 16
+            lib.lqo_rebuild.argtypes = [I] * 7 + [P] * 11
             for f in (lib.lqo_eq1_steps, lib.lqo_quantize, lib.lqo_dequantize,
                       lib.lqo_window, lib.lqo_rebuild):
                 f.restype = None
@@ -146,7 +146,10 @@ class Snapshot(dict):
     """codes int8 [nh,dv,dk], row_scale f32 [nh,dv], col_smooth f32 [nh,dk],
     comp_row i32 [nh,r], comp_val f32 [nh,r,dk] (+ row_norm f64 [nh,dv] when
     produced by quantize); a BF16 state (bits = 16) also holds dense f32
-    [nh,dv,dk], the BF16-rounded residual, which replaces codes x scales."""
+    [nh,dv,dk], the BF16-rounded residual, which replaces codes x scales;
+    the rank-r SVD compensator rule also holds comp_u f32 [nh,r,dv]: the
+    compensators are then the rank-one terms comp_u[c] comp_val[c]^T instead
+    of the rows comp_row[c] = comp_val[c]."""
 
     @property
     def n_comp(self):
@@ -156,17 +159,51 @@ class Snapshot(dict):
 BITS = (8, 6, 4, 16)  # code widths: q_max = 2^(bits-1) - 1 = 127, 31, 7; 16 = BF16 state
 
 
-def quantize(S, n_comp: int, smoothing: bool = True, bits: int = 8) -> Snapshot:
+def svd_compensators(S, r: int):
+    """The rank-r SVD compensator rule (the scope table's variant of the
+    row rule): for each head the r largest singular triplets of the FP32
+    state (an FP64 SVD), u_c = s_c U_c and k~_c = V_c, the sign chosen so that
+    the largest-magnitude entry of k~_c is positive, both rounded to FP32.
+    Returns (u [nh, r, dv], k~ [nh, r, dk], singular values [nh, min(dv, dk)])."""
+    S = _c(S, np.float32)
+    nh, dv, dk = S.shape
+    cu = np.zeros((nh, r, dv), np.float32)
+    ck = np.zeros((nh, r, dk), np.float32)
+    sv_all = np.zeros((nh, min(dv, dk)))
+    for h in range(nh):
+        U, sv, Vt = np.linalg.svd(S[h].astype(np.float64))
+        sv_all[h] = sv
+        for c in range(r):
+            u, v = U[:, c] * sv[c], Vt[c]
+            if v[np.argmax(np.abs(v))] < 0:
+                u, v = -u, -v
+            cu[h, c], ck[h, c] = u, v
+    return cu, ck, sv_all
+
+
+def quantize(S, n_comp: int, smoothing: bool = True, bits: int = 8, rule: str = "rows") -> Snapshot:
     """Compensator selection, residual smoothing and per-row codes of an FP32
     state ``S`` [nh, dv, dk] (rounded to FP32 first if it is not); the codes
     are ``bits`` wide (8, or the 6- and 4-bit widths of the lower-precision
     groups of [LQ] Table 1) and returned one per int8.  ``bits = 16`` is the
     BF16 state of [LQ] Table 2: compensators as above, the residual rounded
-    to BF16 into ``dense`` (no smoothing, unit scales, zero codes)."""
+    to BF16 into ``dense`` (no smoothing, unit scales, zero codes).
+    ``rule = "svd"`` takes the compensators by :func:`svd_compensators` and
+    quantizes the residual S - sum_c u_c k~_c^T (rounded to FP32) with the
+    same C3-C4."""
     S = _c(S, np.float32)
     nh, dv, dk = S.shape
     assert 0 <= n_comp <= dv
-    assert bits in BITS
+    assert bits in BITS and rule in ("rows", "svd")
+    if rule == "svd":
+        cu, ck, sv = svd_compensators(S, n_comp)
+        R = S.astype(np.float64) - np.einsum("hci,hcj->hij", cu.astype(np.float64), ck.astype(np.float64))
+        out = quantize(R.astype(np.float32), 0, smoothing, bits)
+        out["comp_row"] = np.zeros((nh, n_comp), np.int32)
+        out["comp_val"] = ck
+        out["comp_u"] = cu
+        out["singular_values"] = sv
+        return out
     out = Snapshot(
         codes=np.zeros((nh, dv, dk), np.int8),
         row_scale=np.zeros((nh, dv), np.float32),
@@ -190,16 +227,19 @@ def _snap_arrays(snap):
     r = comp_row.shape[1]
     dense = snap.get("dense")
     dense = None if dense is None else _c(dense, np.float32)
+    cu = snap.get("comp_u")
+    cu = None if cu is None else _c(cu, np.float32).reshape(nh, r, dv)
     return (codes, _c(snap["row_scale"], np.float32), _c(snap["col_smooth"], np.float32),
-            comp_row, _c(snap["comp_val"], np.float32).reshape(nh, r, dk), dense, nh, dv, dk, r)
+            comp_row, _c(snap["comp_val"], np.float32).reshape(nh, r, dk), dense, cu, nh, dv, dk, r)
 
 
 def dequantize(snap) -> np.ndarray:
     """S^_0 = Diag(sigma) Q Diag(c) (or the BF16 residual) + compensator rows,
     FP64 [nh, dv, dk]."""
-    codes, rs, cs, cr, cv, dn, nh, dv, dk, r = _snap_arrays(snap)
+    codes, rs, cs, cr, cv, dn, cu, nh, dv, dk, r = _snap_arrays(snap)
     out = np.zeros((nh, dv, dk), np.float64)
-    _load().lqo_dequantize(nh, dv, dk, r, _p(codes), _p(rs), _p(cs), _p(cr), _p(cv), _p(dn), _p(out))
+    _load().lqo_dequantize(nh, dv, dk, r, _p(codes), _p(rs), _p(cs), _p(cr), _p(cv), _p(dn), _p(cu),
+                           _p(out))
     return out
 
 
@@ -223,7 +263,7 @@ def window(snap, records: Records, pos: int, d, kt, b, v, q, exact: bool = False
 
     d [nh, n, gdim] (gdim 1 = scalar gate, d_k = diagonal gate); kt, b, q
     [nh, n, dk]; v [nh, n, dv].  Returns o [nh, n, dv] (FP64)."""
-    codes, rs, cs, cr, cv, dn, nh, dv, dk, r = _snap_arrays(snap)
+    codes, rs, cs, cr, cv, dn, cu, nh, dv, dk, r = _snap_arrays(snap)
     W = records["k"].shape[1]
     gdim = records["L"].shape[2]
     d = _c(d, np.float64)
@@ -235,30 +275,31 @@ def window(snap, records: Records, pos: int, d, kt, b, v, q, exact: bool = False
     kt, b, v, q = (_c(a, np.float64) for a in (kt, b, v, q))
     o = np.zeros((nh, n, dv), np.float64)
     _load().lqo_window(nh, dv, dk, r, gdim, W, pos, n, int(bool(exact)), _p(codes), _p(rs), _p(cs),
-                       _p(cr), _p(cv), _p(dn), _p(records["L"]), _p(records["k"]), _p(records["u"]),
+                       _p(cr), _p(cv), _p(dn), _p(cu), _p(records["L"]), _p(records["k"]), _p(records["u"]),
                        _p(d), _p(kt), _p(b), _p(v), _p(q), _p(o))
     return o
 
 
 def rebuild(snap, records: Records, n: int) -> np.ndarray:
     """S_n = S^_0 D_{1..n} + sum_{m<=n} u_m (D_{m+1..n} k~_m)^T, FP64 [nh, dv, dk]."""
-    codes, rs, cs, cr, cv, dn, nh, dv, dk, r = _snap_arrays(snap)
+    codes, rs, cs, cr, cv, dn, cu, nh, dv, dk, r = _snap_arrays(snap)
     W = records["k"].shape[1]
     gdim = records["L"].shape[2]
     assert 0 <= n <= W
     L, K, U = (_c(records[key], np.float64) for key in ("L", "k", "u"))
     out = np.zeros((nh, dv, dk), np.float64)
     _load().lqo_rebuild(nh, dv, dk, r, gdim, W, n, _p(codes), _p(rs), _p(cs), _p(cr), _p(cv),
-                        _p(dn), _p(L), _p(K), _p(U), _p(out))
+                        _p(dn), _p(cu), _p(L), _p(K), _p(U), _p(out))
     return out
 
 
-def commit(snap, records: Records, n: int, n_comp: int, smoothing: bool = True, bits: int = 8):
+def commit(snap, records: Records, n: int, n_comp: int, smoothing: bool = True, bits: int = 8,
+           rule: str = "rows"):
     """Window commit: rebuild S_n (kept as an FP32 state), then quantize.
 
     Returns (new snapshot, S_n as float32)."""
     S = rebuild(snap, records, n).astype(np.float32)
-    return quantize(S, n_comp, smoothing, bits), S
+    return quantize(S, n_comp, smoothing, bits, rule), S
 
 
 def decode_run(snap, d, kt, b, v, q, W: int, n_comp: int, smoothing: bool = True,

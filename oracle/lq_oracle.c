@@ -252,10 +252,13 @@ void lqo_quantize(int nh, int dv, int dk, int r, int smoothing, int bits, const 
  * window position 0 ([LQ] Abstract: the Compensator Tokens share the update
  * path of real tokens; Figure 4: the state is the quantized residual plus the
  * Compensator Tokens plus the buffered real-token updates).                */
+/* Compensators are rank-one pseudo-tokens u_c k~_c^T at window position 0.
+ * The row rule stores k~_c = comp_val[c] and u_c = e_{comp_row[c]}; the
+ * rank-r SVD rule stores u_c = comp_u[c] [dv] (comp_u != NULL) as well.    */
 static void dequantize_head(int dv, int dk, int r, const int8_t *codes,
                             const float *row_scale, const float *col_smooth,
                             const int32_t *comp_row, const float *comp_val,
-                            const float *dense, double *Sh)
+                            const float *dense, const float *comp_u, double *Sh)
 {
     for (int i = 0; i < dv; ++i)
         for (int j = 0; j < dk; ++j)
@@ -264,6 +267,13 @@ static void dequantize_head(int dv, int dk, int r, const int8_t *codes,
                                                  (double)codes[(size_t)i * dk + j] *
                                                  (double)col_smooth[j];
     for (int c = 0; c < r; ++c) {
+        if (comp_u) {
+            for (int i = 0; i < dv; ++i)
+                for (int j = 0; j < dk; ++j)
+                    Sh[(size_t)i * dk + j] += (double)comp_u[(size_t)c * dv + i] *
+                                              (double)comp_val[(size_t)c * dk + j];
+            continue;
+        }
         int row = comp_row[c];
         for (int j = 0; j < dk; ++j)
             Sh[(size_t)row * dk + j] += (double)comp_val[(size_t)c * dk + j];
@@ -273,7 +283,7 @@ static void dequantize_head(int dv, int dk, int r, const int8_t *codes,
 void lqo_dequantize(int nh, int dv, int dk, int r, const int8_t *codes,
                     const float *row_scale, const float *col_smooth,
                     const int32_t *comp_row, const float *comp_val,
-                    const float *dense, double *S_hat)
+                    const float *dense, const float *comp_u, double *S_hat)
 {
 #pragma omp parallel for schedule(dynamic)
     for (int h = 0; h < nh; ++h)
@@ -281,6 +291,7 @@ void lqo_dequantize(int nh, int dv, int dk, int r, const int8_t *codes,
                         row_scale + (size_t)h * dv, col_smooth + (size_t)h * dk,
                         comp_row + (size_t)h * r, comp_val + (size_t)h * r * dk,
                         dense ? dense + (size_t)h * dv * dk : NULL,
+                        comp_u ? comp_u + (size_t)h * r * dv : NULL,
                         S_hat + (size_t)h * dv * dk);
 }
 
@@ -328,8 +339,8 @@ static double decay(const double *L, int gdim, int t, int m, int j)
 void lqo_window(int nh, int dv, int dk, int r, int gdim, int W, int pos, int n,
                 int exact, const int8_t *codes, const float *row_scale,
                 const float *col_smooth, const int32_t *comp_row,
-                const float *comp_val, const float *dense, double *rec_L, double *rec_k,
-                double *rec_u, const double *d, const double *kt,
+                const float *comp_val, const float *dense, const float *comp_u,
+                double *rec_L, double *rec_k, double *rec_u, const double *d, const double *kt,
                 const double *b, const double *v, const double *q, double *o)
 {
 #pragma omp parallel for schedule(dynamic)
@@ -340,7 +351,8 @@ void lqo_window(int nh, int dv, int dk, int r, int gdim, int W, int pos, int n,
         dequantize_head(dv, dk, r, codes + (size_t)h * dv * dk,
                         row_scale + (size_t)h * dv, col_smooth + (size_t)h * dk,
                         comp_row + (size_t)h * r, comp_val + (size_t)h * r * dk,
-                        dense ? dense + (size_t)h * dv * dk : NULL, S0);
+                        dense ? dense + (size_t)h * dv * dk : NULL,
+                        comp_u ? comp_u + (size_t)h * r * dv : NULL, S0);
         double *L = rec_L + (size_t)h * W * gdim;
         double *K = rec_k + (size_t)h * W * dk;
         double *U = rec_u + (size_t)h * W * dv;
@@ -407,8 +419,8 @@ void lqo_window(int nh, int dv, int dk, int r, int gdim, int W, int pos, int n,
 void lqo_rebuild(int nh, int dv, int dk, int r, int gdim, int W, int n,
                  const int8_t *codes, const float *row_scale,
                  const float *col_smooth, const int32_t *comp_row,
-                 const float *comp_val, const float *dense, const double *rec_L,
-                 const double *rec_k, const double *rec_u, double *S_out)
+                 const float *comp_val, const float *dense, const float *comp_u,
+                 const double *rec_L, const double *rec_k, const double *rec_u, double *S_out)
 {
 #pragma omp parallel for schedule(dynamic)
     for (int h = 0; h < nh; ++h) {
@@ -416,7 +428,8 @@ void lqo_rebuild(int nh, int dv, int dk, int r, int gdim, int W, int n,
         dequantize_head(dv, dk, r, codes + (size_t)h * dv * dk,
                         row_scale + (size_t)h * dv, col_smooth + (size_t)h * dk,
                         comp_row + (size_t)h * r, comp_val + (size_t)h * r * dk,
-                        dense ? dense + (size_t)h * dv * dk : NULL, Sh);
+                        dense ? dense + (size_t)h * dv * dk : NULL,
+                        comp_u ? comp_u + (size_t)h * r * dv : NULL, Sh);
         const double *L = rec_L + (size_t)h * W * gdim;
         const double *K = rec_k + (size_t)h * W * dk;
         const double *U = rec_u + (size_t)h * W * dv;

@@ -34,6 +34,10 @@ MUTATIONS = {
     "scale_255": ("double sigma = f32(mx / qmax);", "double sigma = f32(mx / (2.0 * qmax + 1.0));"),
     "code_range_one_too_wide": ("const double qmax = (double)((1 << (bits - 1)) - 1);",
                                 "const double qmax = (double)(1 << (bits - 1));"),
+    "svd_compensators_dropped": ("Sh[(size_t)i * dk + j] += (double)comp_u[(size_t)c * dv + i] *",
+                                 "Sh[(size_t)i * dk + j] += 0.0 * comp_u[(size_t)c * dv + i] *"),
+    "svd_compensator_transposed": ("(double)comp_val[(size_t)c * dk + j];\n            continue;",
+                                   "(double)comp_val[(size_t)c * dk + (j + 1) % dk];\n            continue;"),
     "bf16_truncates": ("return ldexp(rint(ldexp(m, 8)), e - 8);",
                        "return ldexp(trunc(ldexp(m, 8)), e - 8);"),
     "bf16_keeps_9_bits": ("return ldexp(rint(ldexp(m, 8)), e - 8);",

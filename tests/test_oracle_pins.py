@@ -612,3 +612,79 @@ def test_bf16_state_hand_cases():
     S[0, 1, :len(vals)] = vals
     snap = oracle.quantize(S, 0, bits=16)
     assert snap["dense"][0, 1, :len(vals)].tolist() == [float(np.float32(w)) for w in want]
+
+
+# --------------------------------------------------------------------------
+# Rank-r SVD compensators (the variant of the row rule)
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("r", [1, 3, 6])
+def test_svd_compensators_are_the_best_rank_r_part(r):
+    """Eckart-Young: the residual S - sum_c u_c k~_c^T has spectral norm
+    s_{r+1} and squared Frobenius norm sum_{c>r} s_c^2 (up to the FP32
+    rounding of the factors); each pair satisfies S k~_c = u_c and
+    S^T u_c = s_c^2 k~_c with |k~_c| = 1; and no rank-r row selection leaves a
+    smaller residual."""
+    S = _outlier_state(seed=31)
+    cu, ck, sv = oracle.svd_compensators(S, r)
+    for h in range(S.shape[0]):
+        A = S[h].astype(np.float64)
+        P = cu[h].astype(np.float64).T @ ck[h].astype(np.float64)
+        R = A - P
+        scale = sv[h][0]
+        assert abs(np.linalg.norm(R, 2) - sv[h][r]) <= 1e-5 * scale
+        assert abs(np.linalg.norm(R) ** 2 - np.sum(sv[h][r:] ** 2)) <= 1e-5 * scale ** 2
+        for c in range(r):
+            k = ck[h, c].astype(np.float64)
+            u = cu[h, c].astype(np.float64)
+            assert abs(np.linalg.norm(k) - 1.0) < 1e-6
+            assert np.linalg.norm(A @ k - u) <= 1e-5 * scale
+            assert np.linalg.norm(A.T @ u - sv[h][c] ** 2 * k) <= 1e-5 * scale ** 2
+            assert k[np.argmax(np.abs(k))] > 0  # the sign convention
+        rows = np.argsort(-np.linalg.norm(A, axis=1), kind="stable")[:r]
+        Rrow = A.copy()
+        Rrow[rows] = 0
+        assert np.linalg.norm(R) <= np.linalg.norm(Rrow) * (1 + 1e-6)
+
+
+def test_svd_rule_on_a_rank_r_state_leaves_no_residual():
+    """A state of rank r is held entirely by r SVD compensators: the residual
+    is FP32 rounding only, far below the state's scale."""
+    rng = _rng(32)
+    r, dv, dk = 3, 24, 32
+    S = (rng.normal(size=(2, dv, r)) @ rng.normal(size=(2, r, dk))).astype(np.float32)
+    snap = oracle.quantize(S, r, smoothing=False, rule="svd")
+    # without smoothing sigma_i * 127 is the residual row's largest magnitude
+    assert np.abs(snap["row_scale"]).max() * 127 <= 1e-5 * np.abs(S).max()
+    np.testing.assert_allclose(oracle.dequantize(snap), S.astype(np.float64), atol=1e-5 * np.abs(S).max())
+
+
+def test_svd_rule_with_no_compensators_is_the_row_rule():
+    S = _outlier_state(seed=33)
+    a, b = oracle.quantize(S, 0, rule="svd"), oracle.quantize(S, 0)
+    for key in ("codes", "row_scale", "col_smooth"):
+        np.testing.assert_array_equal(a[key], b[key])
+
+
+@pytest.mark.parametrize("gate", ["scalar", "diag"])
+def test_svd_compensators_share_the_update_path(gate):
+    """Decoding a window from an SVD-compensated snapshot equals explicit
+    stepping of its dequantized state (the compensators are pseudo-tokens at
+    window position 0 with u = u_c, k~ = k~_c), and the rebuild equals the
+    stepped state."""
+    S0, d, kt, b, v, q = _config1_like(gate)
+    W = d.shape[1]
+    snap = oracle.quantize(S0, 4, rule="svd")
+    rec = oracle.empty_records(S0.shape[0], W, S0.shape[2], S0.shape[1], d.shape[2])
+    o_buf = oracle.window(snap, rec, 0, d, kt, b, v, q, exact=True)
+    o_exp, S_exp = oracle.eq1_steps(oracle.dequantize(snap), d, kt, b, v, q)
+    for h in range(S0.shape[0]):
+        for t in range(W):
+            assert _rel(o_buf[h, t], o_exp[h, t]) < 1e-11
+    assert _rel(oracle.rebuild(snap, rec, W), S_exp) < 1e-11
+    # and the dequantized state is the quantized residual plus the rank-r part
+    P = np.einsum("hci,hcj->hij", snap["comp_u"].astype(np.float64), snap["comp_val"].astype(np.float64))
+    res = oracle.dequantize({k2: v2 for k2, v2 in snap.items() if k2 != "comp_u"} | {
+        "comp_row": np.zeros((S0.shape[0], 0), np.int32),
+        "comp_val": np.zeros((S0.shape[0], 0, S0.shape[2]), np.float32)})
+    np.testing.assert_allclose(oracle.dequantize(snap), res + P, rtol=0, atol=1e-12)
