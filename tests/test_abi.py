@@ -207,3 +207,29 @@ def test_ragged_validation_without_launch():
     assert lib.lq_decode_ragged(ctypes.byref(_fake_state(cfg)), p + 0x600000, None, *toks[1:], o,
                                 None) == lq.LQ_ERR_INVALID_ARGUMENT
     assert lib.lq_decode_ragged(None, p + 0x600000, *toks, o, None) == lq.LQ_ERR_INVALID_ARGUMENT
+
+
+def test_binding_structs_match_the_header_layout(tmp_path):
+    """The ctypes mirrors of lq_config, lq_snapshot and lq_state have the
+    C header's field names, offsets and sizes (a C program compiled against
+    include/lq.h prints them)."""
+    import os
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    structs = {"lq_config": lq.LqConfig, "lq_snapshot": lq.LqSnapshot, "lq_state": lq.LqState}
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "lq.h"', 'int main(void) {']
+    for cname, py in structs.items():
+        lines.append(f'printf("{cname} sizeof %zu\\n", sizeof({cname}));')
+        for fname, _ in py._fields_:
+            lines.append(f'printf("{cname} {fname} %zu\\n", offsetof({cname}, {fname}));')
+    lines += ["return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines))
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-std=c11", "-I", os.path.join(root, "include"), str(src), "-o", str(exe)],
+                   check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split("\n")
+    got = {(a, b): int(c) for a, b, c in (ln.split() for ln in out if ln.strip())}
+    for cname, py in structs.items():
+        assert got[(cname, "sizeof")] == ctypes.sizeof(py), cname
+        for fname, _ in py._fields_:
+            assert got[(cname, fname)] == getattr(py, fname).offset, (cname, fname)
