@@ -94,3 +94,8 @@ def test_reference_arm_line_on_cpu(bits):
     assert line["impl"] == "reference" and line["value"] > 0 and line["warmup"] >= 3
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["config"]["bits"] == bits
+
+
+def test_l2_note_says_which():
+    assert bench.l2_note(160e6).startswith("inputs larger than L2")
+    assert "L2-resident" in bench.l2_note(28e6)
