@@ -116,6 +116,29 @@ def gated_linear_instance(alpha, beta, k, diagonal: bool):
     return d, beta[..., None] * k, np.zeros_like(k)
 
 
+def deltaproduct_instance(alpha, beta, k, v):
+    """DeltaProduct ([LQ] Table 4 caption: n delta-rule sub-steps per token,
+    each an instance of equation 1) as micro-tokens in sub-step order: the
+    token's gate alpha acts once, at its first sub-step (the Gated DeltaNet
+    row: D = alpha I, k~ = beta_1 k_1, b = alpha k_1), the other sub-steps are
+    DeltaNet rows (D = I, k~ = beta_j k_j, b = k_j).  The token's output is
+    the output of its last sub-step.
+
+    alpha [nh, T]; beta [nh, T, n]; k [nh, T, n, dk]; v [nh, T, n, dv].
+    Returns d [nh, T n, 1], k~ [nh, T n, dk], b [nh, T n, dk], v [nh, T n, dv]."""
+    alpha = np.asarray(alpha, np.float64)
+    beta = np.asarray(beta, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    nh, T, n, dk = k.shape
+    g = np.ones((nh, T, n))
+    g[:, :, 0] = alpha
+    d = g.reshape(nh, T * n, 1)
+    kt = (beta[..., None] * k).reshape(nh, T * n, dk)
+    b = (g[..., None] * k).reshape(nh, T * n, dk)
+    return d, kt, b, v.reshape(nh, T * n, -1)
+
+
 # --------------------------------------------------------------------------
 # Equation 1, explicit stepping.
 # --------------------------------------------------------------------------

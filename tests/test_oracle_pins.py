@@ -688,3 +688,56 @@ def test_svd_compensators_share_the_update_path(gate):
         "comp_row": np.zeros((S0.shape[0], 0), np.int32),
         "comp_val": np.zeros((S0.shape[0], 0, S0.shape[2]), np.float32)})
     np.testing.assert_allclose(oracle.dequantize(snap), res + P, rtol=0, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# DeltaProduct: n delta-rule sub-steps per token ([LQ] Table 4 caption)
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("n", [1, 2, 3])
+def test_deltaproduct_micro_tokens_equal_the_householder_product(n):
+    """Equation 1 over the micro-tokens equals the published DeltaProduct
+    update, written here with explicit matrices: S_t = alpha_t S_{t-1} H_t +
+    sum_j beta_j v_j k_j^T prod_{l>j} (I - beta_l k_l k_l^T), with H_t the
+    product of the n Householder-like factors (I - beta_j k_j k_j^T); the
+    token's output is S_t q_t.  The window (buffered) decode of the same
+    micro-tokens from a quantized state gives the same outputs as stepping
+    its dequantized state."""
+    rng = _rng(40 + n)
+    nh, T, dk, dv = 2, 5, 6, 4
+    S0 = rng.normal(size=(nh, dv, dk))
+    alpha = rng.uniform(0.5, 1.0, size=(nh, T))
+    beta = rng.uniform(0.1, 1.0, size=(nh, T, n))
+    k = rng.normal(size=(nh, T, n, dk))
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.normal(size=(nh, T, n, dv))
+    q = rng.normal(size=(nh, T, dk))
+    d, kt, b, vm = oracle.deltaproduct_instance(alpha, beta, k, v)
+    qm = np.repeat(q, n, axis=1)  # any q for the inner sub-steps; only the last output is used
+    o_m, S_m = oracle.eq1_steps(S0, d, kt, b, vm, qm)
+    I = np.eye(dk)
+    for h in range(nh):
+        S = S0[h].copy()
+        for t in range(T):
+            H = [I - beta[h, t, j] * np.outer(k[h, t, j], k[h, t, j]) for j in range(n)]
+            P = I.copy()
+            for j in range(n):
+                P = P @ H[j]
+            add = np.zeros((dv, dk))
+            for j in range(n):
+                tail = I.copy()
+                for l in range(j + 1, n):
+                    tail = tail @ H[l]
+                add += beta[h, t, j] * np.outer(v[h, t, j], k[h, t, j]) @ tail
+            S = alpha[h, t] * S @ P + add
+            assert _rel(o_m[h, t * n + n - 1], S @ q[h, t]) < 1e-12
+        assert _rel(S_m[h], S) < 1e-12
+    # the buffered window over the micro-tokens (W = T n) equals stepping the
+    # dequantized boundary state
+    snap = oracle.quantize(S0.astype(np.float32), 1)
+    rec = oracle.empty_records(nh, T * n, dk, dv, 1)
+    o_w = oracle.window(snap, rec, 0, d, kt, b, vm, qm, exact=True)
+    o_s, _ = oracle.eq1_steps(oracle.dequantize(snap), d, kt, b, vm, qm)
+    for h in range(nh):
+        for t in range(T):
+            assert _rel(o_w[h, t * n + n - 1], o_s[h, t * n + n - 1]) < 1e-11
