@@ -19,7 +19,12 @@
 // TF32 high and low part and three products (hi*hi + hi*lo + lo*hi), which
 // keeps it FP32-faithful; the accumulator lives in tensor memory (TMEM).
 // Then C2-C4 (the rule stated in lq_quant.cuh) run with one value row per
-// thread: TMEM lane i holds row i, so row norms and row maxima are
+// thread.  Where the rule divides (R / c_j, R' / sigma_i) this kernel
+// multiplies by the FP32 inverse (1 / c_j, q / max_j |R'_ij|): one rounding
+// more per element, so a code can differ by one step from the rule's where
+// the quotient lies within an FP32 step of a half-integer, and sigma and c
+// agree to about 1e-7 relative; the window's code tolerance (one step)
+// admits it, and every element costs one product instead of a division. TMEM lane i holds row i, so row norms and row maxima are
 // reductions inside a thread, and column maxima are warp reductions
 // (redux.sync) plus one shared-memory pass over the four lane quarters.
 //

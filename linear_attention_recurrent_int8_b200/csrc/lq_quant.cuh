@@ -10,19 +10,19 @@
 //       exact tie to the smaller row), stored exactly in FP32, and are zeroed
 //       in the residual R;
 //   C3  c_j = sqrt(max_i |R_ij|) (1 for a zero column or with smoothing off),
-//       R'_ij = R_ij * (1 / c_j);
-//   C4  mx_i = max_j |R'_ij|, sigma_i = mx_i / q (stored),
-//       Q_ij = rne(R'_ij * (q / mx_i)) in [-q, q], Q = 0 where mx_i = 0,
+//       R'_ij = R_ij / c_j;
+//   C4  sigma_i = max_j |R'_ij| / q (stored),
+//       Q_ij = rne(R'_ij / sigma_i) in [-q, q], Q = 0 where sigma_i = 0,
 //       with q = 2^(bits-1) - 1: 127 for 8-bit codes, 31 and 7 for the 6- and
 //       4-bit widths of the paper's lower-precision groups (Table 1); 4-bit
 //       codes are stored two per byte (low nibble: channel 8g+b, high
 //       nibble: channel 8g+4+b, in byte 4g+b of a row).
 // bits = 16 is the paper's BF16 state (Table 2): C2 as above, then c = 1,
 // sigma = 1 and the residual itself rounded to BF16 (nearest, ties to even).
-// Each smoothing factor and each row is inverted once; every element then
-// costs one FP32 product per step.  Every division, square root and product
-// is one IEEE round-to-nearest FP32 operation (__fdiv_rn, __fsqrt_rn, __fmul_rn),
-// so the codes of a given FP32 state are exactly determined.
+// Every division and square root is one IEEE round-to-nearest FP32 operation
+// (__fdiv_rn, __fsqrt_rn), so the codes of a given FP32 state are exactly
+// determined.  (The window commit, lq_commit.cu, multiplies by the FP32
+// inverses instead: one more rounding, codes within one step of these.)
 #pragma once
 
 #include "lq_common.cuh"
@@ -168,17 +168,17 @@ __device__ __forceinline__ void quantize_tile(float (&S)[Tile<DK, DV, NWARPS>::N
         for (int p = 0; p < NWARPS * T::RPI; ++p) m = fmaxf(m, sm.colpart[p][j]);
         const float c = (smoothing && m > 0.0f) ? __fsqrt_rn(m) : 1.0f;
         out.col_smooth[j] = c;
-        sm.cs[j] = __fdiv_rn(1.0f, c);  // the inverse, used below
+        sm.cs[j] = c;
     }
     consumer_sync<T::NTHREADS>();
-    float ic[4];
+    float cj[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) ic[e] = sm.cs[c0 + e];
+    for (int e = 0; e < 4; ++e) cj[e] = sm.cs[c0 + e];
 
-    // C4: per-row scale and codes of R' = R * (1/c).  Row maxima are reduced
-    // with a transposing reduction; each row's scale and inverse scale are
-    // computed once, by the lane that holds the row's maximum, and broadcast.
-    float inv_own;
+    // C4: per-row scale and codes of R' = R / c.  Row maxima are reduced with
+    // a transposing reduction; each row's scale is computed once, by the lane
+    // that holds the row's maximum, and broadcast.
+    float sig_own;
     {
         float mx[T::NR];
 #pragma unroll
@@ -186,20 +186,20 @@ __device__ __forceinline__ void quantize_tile(float (&S)[Tile<DK, DV, NWARPS>::N
             mx[n] = 0.0f;
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                S[n][e] = __fmul_rn(S[n][e], ic[e]);
+                S[n][e] = __fdiv_rn(S[n][e], cj[e]);
                 mx[n] = fmaxf(mx[n], fabsf(S[n][e]));
             }
         }
         transposed_max<T::NR, T::LPR>(mx, lane);
         const int n = transposed_index<T::NR, T::LPR>(lane);
-        inv_own = mx[0] > 0.0f ? __fdiv_rn(qmax, mx[0]) : 0.0f;
+        sig_own = __fdiv_rn(mx[0], qmax);
         if ((lane & (T::LPR - 1)) == transposed_owner<T::NR, T::LPR>(n))
-            out.row_scale[T::row(warp, lane, n)] = bf16s ? 1.0f : __fdiv_rn(mx[0], qmax);
+            out.row_scale[T::row(warp, lane, n)] = bf16s ? 1.0f : sig_own;
     }
 #pragma unroll
     for (int n = 0; n < T::NR; ++n) {
-        const float inv =
-            __shfl_sync(0xffffffffu, inv_own, gbase + transposed_owner<T::NR, T::LPR>(n));
+        const float sig =
+            __shfl_sync(0xffffffffu, sig_own, gbase + transposed_owner<T::NR, T::LPR>(n));
         const int row = T::row(warp, lane, n);
         if (bf16s) {
             // the residual itself, rounded to BF16 (c = 1, so S is unscaled)
@@ -215,7 +215,9 @@ __device__ __forceinline__ void quantize_tile(float (&S)[Tile<DK, DV, NWARPS>::N
         int iv[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            const float y = fminf(fmaxf(__fmul_rn(S[n][e], inv), -qmax), qmax);
+            // Q = 0 where sigma = 0 (a zero row, or a maximum below q times
+            // the smallest FP32 value)
+            const float y = sig > 0.0f ? fminf(fmaxf(__fdiv_rn(S[n][e], sig), -qmax), qmax) : 0.0f;
             iv[e] = __float_as_int(__fadd_rn(y, 12582912.0f)) - 0x4B400000;
         }
         const uint32_t packed = __byte_perm(__byte_perm(iv[0], iv[1], 0x0040),

@@ -135,24 +135,25 @@ void lqo_eq1_steps(int nh, int dv, int dk, int n, double *S, const double *d,
  *      R = S with those rows set to zero.
  *  C3  m_j = max_i |R_ij|;  c_j = fp32(sqrt(m_j)), or 1 when m_j = 0 or when
  *      smoothing is off (SmoothQuant-style migration with strength 1/2 along
- *      the key channels).  Each factor is inverted once, ic_j = fp32(1 / c_j),
- *      and R'_ij = fp32(R_ij * ic_j).
+ *      the key channels).  R'_ij = fp32(R_ij / c_j).
  *  C4  with q = 2^(bits-1) - 1 (127 for 8 bits; the 6- and 4-bit states of
  *      [LQ] Table 1's lower-precision groups give 31 and 7):
- *      mx_i = max_j |R'_ij|;  sigma_i = fp32(mx_i / q) (the stored scale);
- *      is_i = fp32(q / mx_i);  Q_ij = clamp(rne(fp32(R'_ij * is_i)), -q, q),
- *      Q_i. = 0 when mx_i = 0.  Round half to even; no zero point; -q-1
- *      unused.  The codes come back one per int8 whatever the width (the
- *      packing of a narrower code is a storage format, not arithmetic).
+ *      sigma_i = fp32(max_j |R'_ij| / q) (the stored scale);
+ *      Q_ij = clamp(rne(fp32(R'_ij / sigma_i)), -q, q), Q_i. = 0 when
+ *      sigma_i = 0.  Round half to even; no zero point; -q-1 unused.  The
+ *      codes come back one per int8 whatever the width (the packing of a
+ *      narrower code is a storage format, not arithmetic).
  *  bits = 16 is the BF16 state of [LQ] Table 2 ("BF16 per-step" and its
  *      per-window row): C2 as above, then no smoothing (c = 1) and no integer
  *      codes (sigma = 1): the residual itself is stored rounded to BF16,
  *      dense_ij = bf16(R_ij), in `dense` [nh][dv][dk] (FP32 array).
  *
- * Every division, square root and product above is one IEEE FP32 operation
- * on FP32 operands (an FP64 operation rounded once to FP32 gives the same
- * result), so the quantization decision is taken in FP32, the precision of
- * the stored format.  The row norms (an argmax decision) are computed in
+ * Every division and square root above is one IEEE FP32 operation on FP32
+ * operands: the FP64 result rounded once to FP32 is the correctly rounded
+ * FP32 result, because FP64 carries more than 2 x 24 + 2 significant bits
+ * (double rounding is then innocuous for a quotient or a square root).  So
+ * the quantization decision is taken in FP32, the precision of the stored
+ * format.  The row norms (an argmax decision) are computed in
  * FP64; when two norms are within rounding of each other either selection is
  * correct.
  *
@@ -215,11 +216,9 @@ void lqo_quantize(int nh, int dv, int dk, int r, int smoothing, int bits, const 
             }
             c[j] = (smoothing && m > 0.0) ? (float)sqrt(m) : 1.0f;
         }
-        for (int j = 0; j < dk; ++j) {
-            double ic = f32(1.0 / (double)c[j]);
-            for (int i = 0; i < dv; ++i)
-                R[(size_t)i * dk + j] = f32(R[(size_t)i * dk + j] * ic);
-        }
+        for (int i = 0; i < dv; ++i)
+            for (int j = 0; j < dk; ++j)
+                R[(size_t)i * dk + j] = f32(R[(size_t)i * dk + j] / (double)c[j]);
         /* C4: per-row symmetric codes in [-qmax, qmax]. */
         for (int i = 0; i < dv; ++i) {
             double mx = 0.0;
@@ -228,12 +227,11 @@ void lqo_quantize(int nh, int dv, int dk, int r, int smoothing, int bits, const 
                 if (a > mx) mx = a;
             }
             double sigma = f32(mx / qmax);
-            double is = mx > 0.0 ? f32(qmax / mx) : 0.0;
             row_scale[(size_t)h * dv + i] = (float)sigma;
             for (int j = 0; j < dk; ++j) {
                 double qv = 0.0;
-                if (mx > 0.0) {
-                    qv = rint(f32(R[(size_t)i * dk + j] * is)); /* ties to even */
+                if (sigma > 0.0) {
+                    qv = rint(f32(R[(size_t)i * dk + j] / sigma)); /* ties to even */
                     if (qv > qmax) qv = qmax;
                     if (qv < -qmax) qv = -qmax;
                 }

@@ -29,8 +29,11 @@ MUTATIONS = {
     "ties_to_larger_row": ("norm[i] > norm[best]", "norm[i] >= norm[best]"),
     "smoothing_without_sqrt": ("(float)sqrt(m) : 1.0f", "(float)m : 1.0f"),
     "round_half_away": ("qv = rint(f32(", "qv = round(f32("),
-    "no_inverse_scale_rounding": ("double is = mx > 0.0 ? f32(qmax / mx) : 0.0;",
-                                  "double is = mx > 0.0 ? qmax / mx : 0.0;"),
+    "inverse_scale_product": ("qv = rint(f32(R[(size_t)i * dk + j] / sigma));",
+                              "qv = rint(f32(R[(size_t)i * dk + j] * f32(1.0 / sigma)));"),
+    "inverse_smoothing_product": (
+        "R[(size_t)i * dk + j] = f32(R[(size_t)i * dk + j] / (double)c[j]);",
+        "R[(size_t)i * dk + j] = f32(R[(size_t)i * dk + j] * f32(1.0 / (double)c[j]));"),
     "scale_255": ("double sigma = f32(mx / qmax);", "double sigma = f32(mx / (2.0 * qmax + 1.0));"),
     "code_range_one_too_wide": ("const double qmax = (double)((1 << (bits - 1)) - 1);",
                                 "const double qmax = (double)(1 << (bits - 1));"),

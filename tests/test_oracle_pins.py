@@ -423,7 +423,7 @@ def test_quantizer_smoothing_and_code_range(bits, qmax):
         assert codes.min() >= -qmax and codes.max() <= qmax
         assert not codes[~nz].any()
         # sigma = row max / qmax: the largest code reconstructs the row max
-        Rp = R * (np.float32(1) / snap["col_smooth"][h]).astype(np.float64)[None, :]
+        Rp = R / snap["col_smooth"][h].astype(np.float64)[None, :]
         np.testing.assert_allclose(snap["row_scale"][h][nz] * qmax,
                                    np.abs(Rp).max(axis=1)[nz], rtol=2e-7)
 
@@ -493,28 +493,30 @@ def test_quantizer_narrow_codes_hand_cases():
     assert s["codes"][0, 1, :6].tolist() == [31, 2, 0, 2, 30, -30]
 
 
-@pytest.mark.parametrize("bits", [8, 6, 4])
-def test_quantizer_decision_is_fp32(bits):
-    """Codes are rne of FP32 products of FP32 operands (inverse smoothing
-    factor and inverse scale each rounded once): recompute the decision with
-    numpy float32 arithmetic (IEEE single) and compare bit for bit."""
-    # large enough (5e5 codes) that rounding the inverse scale differently
-    # moves some quotient across a .5 boundary
-    S = _outlier_state(nh=32, dv=128, dk=128, seed=10)
-    snap = oracle.quantize(S, 2, bits=bits)
-    qm = 2 ** (bits - 1) - 1
-    one, q127 = np.float32(1), np.float32(qm)
-    for h in range(S.shape[0]):
-        R = S[h].copy()
-        R[snap["comp_row"][h]] = 0
-        ic = (one / snap["col_smooth"][h]).astype(np.float32)
-        Rp = (R * ic[None, :]).astype(np.float32)
-        mx = np.abs(Rp).max(axis=1).astype(np.float32)
-        np.testing.assert_array_equal((mx / q127).astype(np.float32), snap["row_scale"][h])
-        with np.errstate(divide="ignore", invalid="ignore"):
-            inv = np.where(mx > 0, q127 / mx, np.float32(0)).astype(np.float32)
-        Q = np.where(mx[:, None] > 0, np.rint((Rp * inv[:, None]).astype(np.float32)), 0)
-        np.testing.assert_array_equal(np.clip(Q, -qm, qm).astype(np.int8), snap["codes"][h])
+def _golden_vals(name):
+    vals = {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                key, *rest = line.split()
+                vals[key] = [float(x) for x in rest]
+    return vals
+
+
+@pytest.mark.parametrize("name", ["quantizer_division_scale_case.txt",
+                                  "quantizer_division_smoothing_case.txt"])
+def test_quantizer_divides_in_fp32(name):
+    """Hand-worked cases (derivations in the fixtures) whose codes differ
+    between true FP32 quotients R / c and R' / sigma (the rule) and products
+    with a rounded inverse factor or scale: a half-way quotient is exact in
+    the first form and lands one FP32 step above the tie in the second."""
+    vals = _golden_vals(name)
+    dv, dk = (int(x) for x in vals["shape"])
+    S = np.array(vals["state"], np.float32).reshape(1, dv, dk)
+    s = oracle.quantize(S, int(vals["n_comp"][0]), smoothing=bool(vals["smoothing"][0]))
+    np.testing.assert_array_equal(s["col_smooth"][0], np.float32(vals["col_smooth"]))
+    np.testing.assert_array_equal(s["codes"][0].ravel(), np.int8(vals["codes"]))
+    np.testing.assert_allclose(s["row_scale"][0] * 127, vals["row_scale_times_127"], rtol=1e-6)
 
 
 # --------------------------------------------------------------------------
