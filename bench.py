@@ -112,6 +112,15 @@ def shard(rank: int, world: int, batch_per_rank: int):
     return range(b0, b0 + batch_per_rank)
 
 
+def shard_tokens(wl, rank: int, world: int, t0: int, t1: int, device):
+    """Inputs of tokens t0..t1-1 for this rank's shard, drawn by global
+    sequence index (the counter-based generator is keyed by it): the N ranks
+    together decode exactly the global batch one rank would."""
+    from linear_attention_recurrent_int8_b200 import synth
+    return synth.torch_tokens(wl.seed, list(shard(rank, world, wl.batch)), wl.heads, t0, t1,
+                              wl.d_k, wl.d_v, wl.gate, wl.io, device)
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -365,8 +374,7 @@ def run_lq(args, wl):
     n_slots = max(1, min(args.slots, args.steps + args.warmup))
     slots = []
     for sidx in range(n_slots):
-        tok = synth.torch_tokens(wl.seed + rank, wl.batch, wl.heads, sidx * W, (sidx + 1) * W,
-                                 wl.d_k, wl.d_v, wl.gate, wl.io, dev)
+        tok = shard_tokens(wl, rank, world, sidx * W, (sidx + 1) * W, dev)
         per_t = []
         for t in range(W):
             per_t.append([tok[k][:, t:t + 1].contiguous() for k in ("q", "k", "v", "alpha", "beta")])
@@ -511,9 +519,8 @@ def run_e2e(args, wl, st, cfg, dev, world, group):
     import linear_attention_recurrent_int8_b200 as lq
     from linear_attention_recurrent_int8_b200 import synth
     W = wl.window
-    rank, _, _ = _dist()
-    tok = synth.torch_tokens(wl.seed + rank, wl.batch, wl.heads, 0, W, wl.d_k, wl.d_v, wl.gate, wl.io,
-                             dev)
+    rank, world_, _ = _dist()
+    tok = shard_tokens(wl, rank, world_, 0, W, dev)
     # host layout [W][B, 1, H, ...]: each token's inputs are contiguous
     keys = ("q", "k", "v", "alpha", "beta")
     host = {k: tok[k].transpose(0, 1).unsqueeze(2).contiguous().cpu().pin_memory() for k in keys}

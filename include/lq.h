@@ -76,7 +76,7 @@ typedef enum { LQ_F32 = 0, LQ_BF16 = 1 } lq_dtype;
 
 typedef struct {
     int32_t batch;       /* B >= 1                                          */
-    int32_t heads;       /* H >= 1                                          */
+    int32_t heads;       /* H >= 1; B * H <= 2^24 (LQ_ERR_INVALID_ARGUMENT)  */
     int32_t d_k;         /* 64 or 128                                       */
     int32_t d_v;         /* 64 or 128                                       */
     int32_t window;      /* W in [1, 32]: tokens per quantization window    */
@@ -134,7 +134,15 @@ typedef struct {
  *   buf_k    float [B*H][W][d_k]      (16B) k~_t = beta_t k_t
  *   buf_u    float [B*H][W][d_v]      (16B) u_t = v_t - S_{t-1} b_t
  * `pos` counts the tokens buffered in the open window (the same for every
- * sequence of the batch).  `impl` is reserved (NULL). */
+ * sequence of the batch), or is LQ_POS_PER_SEQUENCE once lq_decode_ragged has
+ * run: the window positions then live on the device (its seq_pos array) and
+ * the calls that need every window closed (lq_decode_window,
+ * lq_window_commit, lq_prefill_chunk, lq_state_snapshot, lq_state_restore)
+ * return LQ_ERR_WINDOW_OPEN until lq_ragged_flush (or lq_state_init) returns
+ * pos to 0.  `impl` is reserved (NULL). */
+/* lq_state.pos after lq_decode_ragged: per-sequence window positions. */
+#define LQ_POS_PER_SEQUENCE (-1)
+
 typedef struct {
     lq_config cfg;
     lq_snapshot snap;
@@ -154,10 +162,15 @@ typedef struct {
 LQ_API int64_t lq_buffer_elems(const lq_config *cfg, int32_t which);
 
 /* Initialises `st` with configuration `cfg` and quantizes the FP32 state
- * S_init [B*H][d_v][d_k] (device, (16B)) into st->snap: compensator
- * selection, residual smoothing, per-row codes of lq_config.bits (the commit
- * quantizer).
- * S_init == NULL means the zero state.  Sets pos = 0. */
+ * S_init [B*H][d_v][d_k] (device, (16B)) into st->snap with the commit
+ * quantizer ("LeapQuant: ...", Abstract and Figure 4: the largest outliers
+ * become high-precision Compensator Tokens, the residual is smoothed across
+ * channels and quantized once): compensator selection, residual smoothing,
+ * per-row codes of lq_config.bits.  The residual's codes are taken with
+ * exact FP32 quotients (R / c_j, then R' / sigma_i), so they are a function
+ * of S_init alone.
+ * S_init == NULL means the zero state.  Sets pos = 0 (also from
+ * LQ_POS_PER_SEQUENCE). */
 LQ_API lq_status lq_state_init(lq_state *st, const lq_config *cfg, const float *S_init,
                         lq_stream_t stream);
 
@@ -166,7 +179,8 @@ LQ_API lq_status lq_state_init(lq_state *st, const lq_config *cfg, const float *
  * o_t = S_t q_t computed from the fixed quantized boundary state plus the buffered
  * FP32 records ("LeapQuant: ...", Figure 2), and the record (L_t, k~_t, u_t)
  * is appended.  All n_steps tokens run inside one launch.
- * Requires 0 <= n_steps and pos + n_steps <= W (else LQ_ERR_WINDOW_FULL);
+ * Requires 0 <= n_steps and pos + n_steps <= W (else LQ_ERR_WINDOW_FULL),
+ * and pos != LQ_POS_PER_SEQUENCE (else LQ_ERR_WINDOW_OPEN);
  * n_steps == 0 is a no-op.  When cfg.auto_commit is set and the window
  * becomes full, the call also commits it (lq_window_commit, a second launch
  * on the same stream) and pos returns to 0; otherwise pos += n_steps.  If the
@@ -188,10 +202,12 @@ LQ_API lq_status lq_decode_window(lq_state *st, const void *q, const void *k, co
  * (lq_window_commit's rule, on that sequence's heads only); then each active
  * seq_pos[b] advances to (seq_pos[b] + 1) mod W.  Three launches on `stream`
  * (decode, commit, position update).  Requires the batch-synchronous window
- * to be closed (pos == 0, else LQ_ERR_WINDOW_OPEN); st->pos is not used
- * afterwards.  A position >= W cannot be checked on the host: that sequence
- * is skipped (its position is left as it is) and the device error word
- * records it (lq_device_errors).
+ * to be closed (pos == 0 or LQ_POS_PER_SEQUENCE, else LQ_ERR_WINDOW_OPEN) and
+ * sets pos = LQ_POS_PER_SEQUENCE: windows may now be open on the device, so
+ * the calls that need them closed refuse until lq_ragged_flush.  A position
+ * >= W cannot be checked on the host: that sequence is skipped (its
+ * position is left as it is) and the device error word records it
+ * (LQ_DEVERR_BAD_POSITION).
  * If a later launch fails after an earlier one succeeded, LQ_ERR_CUDA is
  * returned with the earlier launches' effects in place. */
 LQ_API lq_status lq_decode_ragged(lq_state *st, int32_t *seq_pos, const void *q, const void *k,
@@ -203,8 +219,24 @@ LQ_API lq_status lq_decode_ragged(lq_state *st, int32_t *seq_pos, const void *q,
  * r largest-norm rows as Compensator Tokens, smooths the residual across key
  * channels and re-quantizes it (codes of lq_config.bits) into st->snap; pos
  * returns to 0.
- * A no-op when pos == 0. */
+ * A no-op when pos == 0; LQ_ERR_WINDOW_OPEN when pos == LQ_POS_PER_SEQUENCE
+ * (lq_ragged_flush commits per-sequence windows). */
 LQ_API lq_status lq_window_commit(lq_state *st, lq_stream_t stream);
+
+/* Closes every per-sequence window (the serving counterpart of
+ * lq_window_commit; "LeapQuant: ...", Figure 2 and Figure 4, applied to each
+ * sequence's own window): every sequence b with 1 <= seq_pos[b] < W commits
+ * its seq_pos[b] buffered records exactly as lq_window_commit would, then
+ * seq_pos[b] = 0.  Sequences at 0 or idle (negative) are untouched; a
+ * position >= W is left as it is and reported (LQ_DEVERR_BAD_POSITION).
+ * seq_pos: device int32 [B], 4-byte aligned, in/out (the array given to
+ * lq_decode_ragged).  Requires pos == 0 or LQ_POS_PER_SEQUENCE (else
+ * LQ_ERR_WINDOW_OPEN); sets pos = 0, after which snapshots, restores,
+ * prefill and synchronous decode are allowed again.  W launches on `stream`
+ * (one commit launch per buffered-record count 1 .. W-1 and the position
+ * reset); if one fails, LQ_ERR_CUDA is returned with the earlier ones'
+ * effects in place and pos unchanged. */
+LQ_API lq_status lq_ragged_flush(lq_state *st, int32_t *seq_pos, lq_stream_t stream);
 
 /* Prefill of T tokens from the FP32 state S_fp32 [B*H][d_v][d_k] (device,
  * (16B), in/out: the caller passes zeros for a fresh prompt; on return it
@@ -215,7 +247,8 @@ LQ_API lq_status lq_window_commit(lq_state *st, lq_stream_t stream);
  * tokens ("LeapQuant: ...", Figure 1(b)).  On return st->snap holds the
  * quantized state after T tokens, ready for decode.  The FP32 state is
  * carried across snapshots unquantized.
- * Requires pos == 0 (else LQ_ERR_WINDOW_OPEN), T >= 0, snapshot_every >= 1
+ * Requires pos == 0 (else LQ_ERR_WINDOW_OPEN; also LQ_POS_PER_SEQUENCE), T >= 0,
+ * snapshot_every >= 1
  * and, when snaps != NULL, T % snapshot_every == 0.  T == 0 is a no-op. */
 LQ_API lq_status lq_prefill_chunk(lq_state *st, float *S_fp32, const void *q, const void *k,
                            const void *v, const float *alpha, const float *beta,
@@ -223,11 +256,15 @@ LQ_API lq_status lq_prefill_chunk(lq_state *st, float *S_fp32, const void *q, co
                            void *o, lq_stream_t stream);
 
 /* Copies the committed boundary state into `dst` (device buffers of the same
- * sizes): a prefix-cache snapshot.  Requires pos == 0 (LQ_ERR_WINDOW_OPEN). */
+ * sizes): a prefix-cache snapshot, one quantized state kept per cached prefix
+ * ("LeapQuant: ...", Figure 1(b): one state per 1,024 cached tokens).
+ * Requires pos == 0 (else LQ_ERR_WINDOW_OPEN, also for LQ_POS_PER_SEQUENCE:
+ * an open window's buffered tokens are not part of the snapshot). */
 LQ_API lq_status lq_state_snapshot(const lq_state *st, const lq_snapshot *dst, lq_stream_t stream);
 
-/* Copies a snapshot back into st->snap and sets pos = 0 (resume from a
- * prefix-cache snapshot).  Requires pos == 0 (LQ_ERR_WINDOW_OPEN). */
+/* Copies a snapshot back into st->snap and sets pos = 0: resume from a
+ * prefix-cache snapshot ("LeapQuant: ...", Figure 1(b)).  Requires pos == 0
+ * (else LQ_ERR_WINDOW_OPEN, also for LQ_POS_PER_SEQUENCE). */
 LQ_API lq_status lq_state_restore(lq_state *st, const lq_snapshot *src, lq_stream_t stream);
 
 /* Comparator (not LeapQuant): n_steps of the recurrence on an FP32 state
@@ -245,9 +282,17 @@ LQ_API void lq_state_destroy(lq_state *st);
 /* Static string naming a status. */
 LQ_API const char *lq_status_string(lq_status s);
 
-/* Reads and clears the library's device error word (synchronizes the
- * device).  Bit 0: a kernel gave up waiting for its own asynchronous copies
- * (bounded wait expired); the affected outputs are not valid. */
+/* Bits of the device error word (lq_device_errors). */
+#define LQ_DEVERR_WAIT_TIMEOUT 1u  /* a kernel gave up waiting for its own
+                                      asynchronous copies (bounded wait
+                                      expired); the affected outputs are not
+                                      valid */
+#define LQ_DEVERR_BAD_POSITION 2u  /* lq_decode_ragged / lq_ragged_flush met a
+                                      per-sequence position >= W and skipped
+                                      that sequence */
+
+/* Reads and clears the library's device error word, an OR of LQ_DEVERR_*
+ * bits (synchronizes the device). */
 LQ_API lq_status lq_device_errors(uint32_t *flags);
 
 #ifdef __cplusplus

@@ -25,10 +25,12 @@ LQ_OK, LQ_ERR_INVALID_ARGUMENT, LQ_ERR_UNSUPPORTED, LQ_ERR_WINDOW_FULL, \
     LQ_ERR_WINDOW_OPEN, LQ_ERR_MISALIGNED, LQ_ERR_CUDA = range(7)
 LQ_GATE_SCALAR, LQ_GATE_DIAG = 0, 1
 LQ_F32, LQ_BF16 = 0, 1
+LQ_POS_PER_SEQUENCE = -1
+LQ_DEVERR_WAIT_TIMEOUT, LQ_DEVERR_BAD_POSITION = 1, 2
 
 # Every symbol include/lq.h declares.
 ABI_SYMBOLS = ("lq_buffer_elems", "lq_state_init", "lq_decode_window", "lq_decode_ragged",
-               "lq_window_commit",
+               "lq_ragged_flush", "lq_window_commit",
                "lq_prefill_chunk", "lq_state_snapshot", "lq_state_restore", "lq_fp32_step",
                "lq_state_destroy", "lq_status_string", "lq_device_errors")
 
@@ -78,6 +80,7 @@ def load_library(build: bool = True):
                 "lq_state_init": (I32, [ctypes.POINTER(LqState), ctypes.POINTER(LqConfig), P, P]),
                 "lq_decode_window": (I32, [ctypes.POINTER(LqState), P, P, P, P, P, I32, P, P]),
                 "lq_decode_ragged": (I32, [ctypes.POINTER(LqState), P, P, P, P, P, P, P, P]),
+                "lq_ragged_flush": (I32, [ctypes.POINTER(LqState), P, P]),
                 "lq_window_commit": (I32, [ctypes.POINTER(LqState), P]),
                 "lq_prefill_chunk": (I32, [ctypes.POINTER(LqState), P, P, P, P, P, P, I32, I32,
                                            ctypes.POINTER(LqSnapshot), P, P]),
@@ -113,6 +116,75 @@ def _stream(stream):
     import torch
     s = torch.cuda.current_stream() if stream is None else stream
     return ctypes.c_void_p(s.cuda_stream)
+
+
+# --------------------------------------------------------------------------
+# Argument checks (before any call into the library)
+# --------------------------------------------------------------------------
+#
+# The library checks pointers, sizes and alignment, but a pointer carries no
+# length: a tensor that is too small, of the wrong dtype or on another device
+# would be read past its end by the kernels' bulk copies.  Every wrapper
+# therefore checks each tensor against the configuration first -- dtype,
+# exact element count, contiguity, then that it lives on the state's CUDA
+# device -- and raises before the library is called.
+
+def _check_layout(t, name: str, dtype, numel: int, optional: bool = False) -> bool:
+    """dtype, element count and contiguity; False for an absent optional tensor."""
+    import torch
+    if t is None:
+        if optional:
+            return False
+        raise ValueError(f"{name}: a tensor is required")
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if t.numel() != numel:
+        raise ValueError(f"{name}: {t.numel()} elements, expected {numel} (shape {tuple(t.shape)})")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: not contiguous")
+    return True
+
+
+def _check_device(t, name: str, device):
+    import torch
+    dev = torch.device(device)
+    if t.device.type != "cuda" or dev.type != "cuda":
+        raise ValueError(f"{name}: on {t.device}, expected a CUDA tensor on {dev}")
+    if dev.index is not None and t.device.index != dev.index:
+        raise ValueError(f"{name}: on {t.device}, expected {dev}")
+
+
+def _check_tensors(device, *specs):
+    """specs: (tensor, name, dtype, numel[, optional]).  Every tensor's layout
+    is checked first, then every present tensor's device."""
+    present = [sp for sp in specs if _check_layout(*sp)]
+    for sp in present:
+        _check_device(sp[0], sp[1], device)
+
+
+def _token_specs(cfg: "Config", n: int, q, k, v, alpha, beta, o):
+    import torch
+    B, H = cfg.batch, cfg.heads
+    io = cfg.io_torch_dtype
+    return [(q, "q", io, B * n * H * cfg.d_k), (k, "k", io, B * n * H * cfg.d_k),
+            (v, "v", io, B * n * H * cfg.d_v),
+            (alpha, "alpha", torch.float32, B * n * H * cfg.gdim),
+            (beta, "beta", torch.float32, B * n * H), (o, "o", io, B * n * H * cfg.d_v)]
+
+
+def _snapshot_specs(cfg: "Config", snap: "Snapshot", name: str):
+    import torch
+    bh = cfg.batch * cfg.heads
+    t = snap.t
+    specs = [(t["codes"], f"{name}.codes", cfg.code_torch_dtype, bh * cfg.d_v * cfg.code_cols),
+             (t["row_scale"], f"{name}.row_scale", torch.float32, bh * cfg.d_v),
+             (t["col_smooth"], f"{name}.col_smooth", torch.float32, bh * cfg.d_k)]
+    if cfg.n_comp > 0:
+        specs += [(t["comp_row"], f"{name}.comp_row", torch.int32, bh * cfg.n_comp),
+                  (t["comp_val"], f"{name}.comp_val", torch.float32, bh * cfg.n_comp * cfg.d_k)]
+    return specs
 
 
 # --------------------------------------------------------------------------
@@ -232,12 +304,19 @@ def lq_buffer_elems(cfg: Config, which: int) -> int:
 
 
 def lq_state_init(st: State, S_init=None, stream=None) -> None:
+    import torch
+    cfg = st.cfg
+    _check_tensors(st.device, (S_init, "S_init", torch.float32,
+                               cfg.batch * cfg.heads * cfg.d_v * cfg.d_k, True),
+                   *_snapshot_specs(cfg, st.snap, "state.snap"))
     c = st.cfg.c()
     _check(load_library().lq_state_init(ctypes.byref(st.c), ctypes.byref(c), _ptr(S_init),
                                         _stream(stream)), "lq_state_init")
 
 
 def lq_decode_window(st: State, q, k, v, alpha, beta, n_steps: int, o, stream=None) -> None:
+    if int(n_steps) > 0:
+        _check_tensors(st.device, *_token_specs(st.cfg, int(n_steps), q, k, v, alpha, beta, o))
     _check(load_library().lq_decode_window(ctypes.byref(st.c), _ptr(q), _ptr(k), _ptr(v),
                                            _ptr(alpha), _ptr(beta), int(n_steps), _ptr(o),
                                            _stream(stream)), "lq_decode_window")
@@ -246,9 +325,21 @@ def lq_decode_window(st: State, q, k, v, alpha, beta, n_steps: int, o, stream=No
 def lq_decode_ragged(st: State, seq_pos, q, k, v, alpha, beta, o, stream=None) -> None:
     """One token per active sequence at its own window position (seq_pos:
     int32 device tensor [B], negative = idle slot; updated in place)."""
+    import torch
+    _check_tensors(st.device, (seq_pos, "seq_pos", torch.int32, st.cfg.batch),
+                   *_token_specs(st.cfg, 1, q, k, v, alpha, beta, o))
     _check(load_library().lq_decode_ragged(ctypes.byref(st.c), _ptr(seq_pos), _ptr(q), _ptr(k),
                                            _ptr(v), _ptr(alpha), _ptr(beta), _ptr(o),
                                            _stream(stream)), "lq_decode_ragged")
+
+
+def lq_ragged_flush(st: State, seq_pos, stream=None) -> None:
+    """Commits every sequence's open window (1 <= seq_pos[b] < W) and sets
+    those positions to 0; afterwards st.pos == 0."""
+    import torch
+    _check_tensors(st.device, (seq_pos, "seq_pos", torch.int32, st.cfg.batch))
+    _check(load_library().lq_ragged_flush(ctypes.byref(st.c), _ptr(seq_pos), _stream(stream)),
+           "lq_ragged_flush")
 
 
 def lq_window_commit(st: State, stream=None) -> None:
@@ -257,6 +348,19 @@ def lq_window_commit(st: State, stream=None) -> None:
 
 def lq_prefill_chunk(st: State, S_fp32, q, k, v, alpha, beta, T: int, snapshot_every: int,
                      snaps, o, stream=None) -> None:
+    import torch
+    cfg = st.cfg
+    if int(T) > 0:
+        specs = [(S_fp32, "S_fp32", torch.float32, cfg.batch * cfg.heads * cfg.d_v * cfg.d_k)]
+        specs += _token_specs(cfg, int(T), q, k, v, alpha, beta, o)
+        if snaps is not None:
+            if int(snapshot_every) < 1 or int(T) % int(snapshot_every) != 0 or \
+                    len(snaps) != int(T) // int(snapshot_every):
+                raise ValueError(f"snaps: {len(snaps)} snapshots for T = {T}, "
+                                 f"snapshot_every = {snapshot_every}")
+            for i, sn in enumerate(snaps):
+                specs += _snapshot_specs(cfg, sn, f"snaps[{i}]")
+        _check_tensors(st.device, *specs)
     arr = None
     if snaps is not None:
         arr = (LqSnapshot * len(snaps))(*[s.c() for s in snaps])
@@ -267,18 +371,25 @@ def lq_prefill_chunk(st: State, S_fp32, q, k, v, alpha, beta, T: int, snapshot_e
 
 
 def lq_state_snapshot(st: State, dst: Snapshot, stream=None) -> None:
+    _check_tensors(st.device, *_snapshot_specs(st.cfg, dst, "dst"))
     c = dst.c()
     _check(load_library().lq_state_snapshot(ctypes.byref(st.c), ctypes.byref(c), _stream(stream)),
            "lq_state_snapshot")
 
 
 def lq_state_restore(st: State, src: Snapshot, stream=None) -> None:
+    _check_tensors(st.device, *_snapshot_specs(st.cfg, src, "src"))
     c = src.c()
     _check(load_library().lq_state_restore(ctypes.byref(st.c), ctypes.byref(c), _stream(stream)),
            "lq_state_restore")
 
 
 def lq_fp32_step(cfg: Config, S, q, k, v, alpha, beta, n_steps: int, o, stream=None) -> None:
+    import torch
+    if int(n_steps) > 0:
+        dev = S.device if isinstance(S, torch.Tensor) else "cuda"
+        _check_tensors(dev, (S, "S", torch.float32, cfg.batch * cfg.heads * cfg.d_v * cfg.d_k),
+                       *_token_specs(cfg, int(n_steps), q, k, v, alpha, beta, o))
     c = cfg.c()
     _check(load_library().lq_fp32_step(ctypes.byref(c), _ptr(S), _ptr(q), _ptr(k), _ptr(v),
                                        _ptr(alpha), _ptr(beta), int(n_steps), _ptr(o),

@@ -17,7 +17,9 @@ bool aligned_to(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p
 lq_status check_config(const lq_config *c) {
     if (!c) return LQ_ERR_INVALID_ARGUMENT;
     if (c->batch < 1 || c->heads < 1) return LQ_ERR_INVALID_ARGUMENT;
-    if ((int64_t)c->batch * c->heads > 0x7fffffffLL) return LQ_ERR_INVALID_ARGUMENT;
+    // B * H bounded so that every grid (at most 16 CTAs per head) and every
+    // per-head int index stays far inside 2^31
+    if ((int64_t)c->batch * c->heads > (1LL << 24)) return LQ_ERR_INVALID_ARGUMENT;
     if (c->d_k < 1 || c->d_v < 1) return LQ_ERR_INVALID_ARGUMENT;
     if ((c->d_k != 64 && c->d_k != 128) || (c->d_v != 64 && c->d_v != 128))
         return LQ_ERR_UNSUPPORTED;
@@ -67,7 +69,8 @@ lq_status check_state(const lq_state *st) {
     if (!st->buf_gate || !st->buf_k || !st->buf_u) return LQ_ERR_INVALID_ARGUMENT;
     if (!aligned16(st->buf_gate) || !aligned16(st->buf_k) || !aligned16(st->buf_u))
         return LQ_ERR_MISALIGNED;
-    if (st->pos < 0 || st->pos > st->cfg.window) return LQ_ERR_INVALID_ARGUMENT;
+    if ((st->pos < 0 && st->pos != LQ_POS_PER_SEQUENCE) || st->pos > st->cfg.window)
+        return LQ_ERR_INVALID_ARGUMENT;
     return LQ_OK;
 }
 
@@ -184,6 +187,7 @@ lq_status lq_decode_window(lq_state *st, const void *q, const void *k, const voi
                            lq_stream_t stream) {
     lq_status e = check_state(st);
     if (e != LQ_OK) return e;
+    if (st->pos == LQ_POS_PER_SEQUENCE) return LQ_ERR_WINDOW_OPEN;
     if (n_steps < 0) return LQ_ERR_INVALID_ARGUMENT;
     if (n_steps == 0) return LQ_OK;
     if (st->pos + n_steps > st->cfg.window) return LQ_ERR_WINDOW_FULL;
@@ -210,7 +214,7 @@ lq_status lq_decode_ragged(lq_state *st, int32_t *seq_pos, const void *q, const 
                            lq_stream_t stream) {
     lq_status e = check_state(st);
     if (e != LQ_OK) return e;
-    if (st->pos != 0) return LQ_ERR_WINDOW_OPEN;
+    if (st->pos != 0 && st->pos != LQ_POS_PER_SEQUENCE) return LQ_ERR_WINDOW_OPEN;
     if (!seq_pos) return LQ_ERR_INVALID_ARGUMENT;
     if (!aligned_to(seq_pos, 4)) return LQ_ERR_MISALIGNED;
     e = check_tokens(&st->cfg, q, k, v, alpha, beta, o);
@@ -231,17 +235,45 @@ lq_status lq_decode_ragged(lq_state *st, int32_t *seq_pos, const void *q, const 
     e = cuda_status(lq::launch_decode(a, st->cfg.d_k, st->cfg.d_v, st->cfg.gate,
                                       st->cfg.io_dtype == LQ_BF16, s));
     if (e != LQ_OK) return e;
+    // from here on windows may be open on the device
+    st->pos = LQ_POS_PER_SEQUENCE;
     // the sequences whose window is now full (seq_pos == W - 1) commit W records
     a.pos = W;
     a.n_steps = 0;
+    a.commit_match = W - 1;
     e = cuda_status(lq::launch_commit(a, st->cfg.d_k, st->cfg.d_v, st->cfg.gate, s));
     if (e != LQ_OK) return e;
     return cuda_status(lq::launch_advance_positions(seq_pos, st->cfg.batch, W, s));
 }
 
+lq_status lq_ragged_flush(lq_state *st, int32_t *seq_pos, lq_stream_t stream) {
+    lq_status e = check_state(st);
+    if (e != LQ_OK) return e;
+    if (st->pos != 0 && st->pos != LQ_POS_PER_SEQUENCE) return LQ_ERR_WINDOW_OPEN;
+    if (!seq_pos) return LQ_ERR_INVALID_ARGUMENT;
+    if (!aligned_to(seq_pos, 4)) return LQ_ERR_MISALIGNED;
+    const int W = st->cfg.window;
+    cudaStream_t s = (cudaStream_t)stream;
+    lq::DecodeArgs a = decode_args(st);
+    a.seq_pos = seq_pos;
+    a.n_steps = 0;
+    // one commit launch per record count p: the sequences holding p records
+    for (int p = 1; p < W; ++p) {
+        a.pos = p;
+        a.commit_match = p;
+        e = cuda_status(lq::launch_commit(a, st->cfg.d_k, st->cfg.d_v, st->cfg.gate, s));
+        if (e != LQ_OK) return e;
+    }
+    e = cuda_status(lq::launch_reset_positions(seq_pos, st->cfg.batch, W, s));
+    if (e != LQ_OK) return e;
+    st->pos = 0;
+    return LQ_OK;
+}
+
 lq_status lq_window_commit(lq_state *st, lq_stream_t stream) {
     lq_status e = check_state(st);
     if (e != LQ_OK) return e;
+    if (st->pos == LQ_POS_PER_SEQUENCE) return LQ_ERR_WINDOW_OPEN;
     if (st->pos == 0) return LQ_OK;
     lq::DecodeArgs a = decode_args(st);
     a.n_steps = 0;

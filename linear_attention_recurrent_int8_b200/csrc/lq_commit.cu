@@ -155,13 +155,14 @@ __device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
 
 // The next head of this CTA's grid-stride walk at or after `bh` that commits
 // in this launch: every head with batch-synchronous positions; with
-// per-sequence positions the heads of sequences whose window has just
-// filled (seq_pos[b] == W - 1).  Every role walks the same sequence.
+// per-sequence positions the heads of sequences whose seq_pos equals
+// a.commit_match (W - 1: the window has just filled; p: a flush of the
+// windows holding p records).  Every role walks the same sequence.
 __device__ __forceinline__ int next_commit_head(const DecodeArgs &a, int bh) {
     const int BH = a.B * a.H;
     if (!a.seq_pos) return bh;
     for (; bh < BH; bh += gridDim.x)
-        if (a.seq_pos[bh / a.H] == a.W - 1) return bh;
+        if (a.seq_pos[bh / a.H] == a.commit_match) return bh;
     return BH;
 }
 
@@ -699,8 +700,24 @@ __global__ void advance_positions_kernel(int32_t *seq_pos, int B, int W) {
 }
 }  // namespace
 
+namespace {
+__global__ void reset_positions_kernel(int32_t *seq_pos, int B, int W) {
+    const int b = blockIdx.x * blockDim.x + threadIdx.x;
+    if (b < B) {
+        const int p = seq_pos[b];
+        if (p > 0 && p < W) seq_pos[b] = 0;
+        if (p >= W) atomicOr(&g_dev_error, kErrBadPosition);
+    }
+}
+}  // namespace
+
 cudaError_t launch_advance_positions(int32_t *seq_pos, int B, int W, cudaStream_t stream) {
     advance_positions_kernel<<<(B + 255) / 256, 256, 0, stream>>>(seq_pos, B, W);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_reset_positions(int32_t *seq_pos, int B, int W, cudaStream_t stream) {
+    reset_positions_kernel<<<(B + 255) / 256, 256, 0, stream>>>(seq_pos, B, W);
     return cudaGetLastError();
 }
 

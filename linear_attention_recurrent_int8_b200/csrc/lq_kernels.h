@@ -47,6 +47,10 @@ struct DecodeArgs {
     // seq_pos[b] < 0; the commit takes the sequences with seq_pos[b] == W - 1
     // (pos is then W).
     const int32_t *seq_pos;
+    // with seq_pos set, the commit takes the sequences whose seq_pos equals
+    // commit_match (W - 1 after a ragged decode; p, with pos = p, when the
+    // open windows of p records are flushed)
+    int commit_match;
 };
 
 // Arguments of the quantize-from-FP32 kernel (init, prefill snapshots).
@@ -86,6 +90,10 @@ cudaError_t launch_commit(const DecodeArgs &a, int d_k, int d_v, int gate, cudaS
 
 // seq_pos[b] <- (seq_pos[b] + 1) mod W for the sequences with 0 <= seq_pos[b] < W.
 cudaError_t launch_advance_positions(int32_t *seq_pos, int B, int W, cudaStream_t stream);
+
+// seq_pos[b] <- 0 for the sequences with 0 < seq_pos[b] < W (after their
+// windows were committed); a position >= W sets the device error word.
+cudaError_t launch_reset_positions(int32_t *seq_pos, int B, int W, cudaStream_t stream);
 
 // Reads the device error word and clears it (synchronizes the device).
 cudaError_t read_and_clear_dev_error(unsigned int *out);

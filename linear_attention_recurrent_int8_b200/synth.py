@@ -282,13 +282,16 @@ def torch_grid(seed: int, tid: int, bs, hs, cs, js, device):
     return torch.sqrt(-2.0 * torch.log(u1)) * torch.cos(2.0 * math.pi * u2)
 
 
-def torch_tokens(seed: int, batch: int, heads: int, t0: int, t1: int, d_k: int, d_v: int,
+def torch_tokens(seed: int, batch, heads: int, t0: int, t1: int, d_k: int, d_v: int,
                  gate: str, io: str, device):
-    """Device-side counterpart of :func:`tokens` for all sequences and heads.
+    """Device-side counterpart of :func:`tokens` for all heads of the sequences
+    ``batch`` (a count B, meaning sequences 0..B-1, or the sequences' global
+    indices, so that a shard draws exactly its slice of the global batch).
 
     Returns q, k, v in the io dtype and alpha, beta in float32, layout [B, T, H, d]."""
     import torch
-    bs, hs, ts = np.arange(batch), np.arange(heads), np.arange(t0, t1)
+    bs = np.arange(batch) if np.ndim(batch) == 0 else np.asarray(batch)
+    hs, ts = np.arange(heads), np.arange(t0, t1)
     jk, jv = np.arange(d_k), np.arange(d_v)
     q = torch_grid(seed, TID_Q, bs, hs, ts, jk, device)
     k = torch_grid(seed, TID_K, bs, hs, ts, jk, device)

@@ -233,3 +233,125 @@ def test_binding_structs_match_the_header_layout(tmp_path):
         assert got[(cname, "sizeof")] == ctypes.sizeof(py), cname
         for fname, _ in py._fields_:
             assert got[(cname, fname)] == getattr(py, fname).offset, (cname, fname)
+
+
+def test_per_sequence_mode_refuses_calls_that_need_closed_windows():
+    """After lq_decode_ragged the state's pos is LQ_POS_PER_SEQUENCE: windows
+    may be open on the device, so synchronous decode, commit, snapshot,
+    restore and prefill refuse (LQ_ERR_WINDOW_OPEN) until lq_ragged_flush."""
+    lib = lq.load_library()
+    cfg = lq.Config(batch=2, heads=3, window=4, n_comp=2)
+    per_seq = lambda: _fake_state(cfg, pos=lq.LQ_POS_PER_SEQUENCE)
+    assert _decode(per_seq(), 1) == lq.LQ_ERR_WINDOW_OPEN
+    assert lib.lq_window_commit(ctypes.byref(per_seq()), None) == lq.LQ_ERR_WINDOW_OPEN
+    dst = lq.LqSnapshot(0x30000000, 0x30100000, 0x30200000, 0x30300000, 0x30400000)
+    assert lib.lq_state_snapshot(ctypes.byref(per_seq()), ctypes.byref(dst), None) == \
+        lq.LQ_ERR_WINDOW_OPEN
+    assert lib.lq_state_restore(ctypes.byref(per_seq()), ctypes.byref(dst), None) == \
+        lq.LQ_ERR_WINDOW_OPEN
+    p = 0x40000000
+    args = [p, p + 0x100000, p + 0x200000, p + 0x300000, p + 0x400000, p + 0x500000]
+    assert lib.lq_prefill_chunk(ctypes.byref(per_seq()), *args, 128, 64, None, p + 0x600000,
+                                None) == lq.LQ_ERR_WINDOW_OPEN
+    # other negative positions stay invalid
+    assert _decode(_fake_state(cfg, pos=-2), 1) == lq.LQ_ERR_INVALID_ARGUMENT
+    # the flush: positions array required and aligned; an open synchronous window refuses
+    assert lib.lq_ragged_flush(ctypes.byref(per_seq()), None, None) == lq.LQ_ERR_INVALID_ARGUMENT
+    assert lib.lq_ragged_flush(ctypes.byref(per_seq()), p + 2, None) == lq.LQ_ERR_MISALIGNED
+    assert lib.lq_ragged_flush(ctypes.byref(_fake_state(cfg, pos=3)), p, None) == \
+        lq.LQ_ERR_WINDOW_OPEN
+    assert lib.lq_ragged_flush(None, p, None) == lq.LQ_ERR_INVALID_ARGUMENT
+
+
+def test_batch_times_heads_is_bounded():
+    """B * H <= 2^24 keeps every grid and per-head index inside 2^31."""
+    cfg = lq.Config(batch=1 << 12, heads=1 << 12, window=4, n_comp=2)
+    assert lq.lq_buffer_elems(cfg, 1) == (1 << 24) * 128
+    cfg.heads = (1 << 12) + 1
+    assert lq.lq_buffer_elems(cfg, 1) == -1
+    assert _decode(_fake_state(cfg), 1) == lq.LQ_ERR_INVALID_ARGUMENT
+
+
+def test_device_error_bits_match_the_header():
+    text = open(HEADER).read()
+    assert re.search(r"#define LQ_DEVERR_WAIT_TIMEOUT 1u", text)
+    assert re.search(r"#define LQ_DEVERR_BAD_POSITION 2u", text)
+    assert re.search(r"#define LQ_POS_PER_SEQUENCE \(-1\)", text)
+    assert (lq.LQ_DEVERR_WAIT_TIMEOUT, lq.LQ_DEVERR_BAD_POSITION, lq.LQ_POS_PER_SEQUENCE) == (1, 2, -1)
+
+
+# --------------------------------------------------------------------------
+# The Python binding checks every tensor before calling the library
+# --------------------------------------------------------------------------
+
+@pytest.fixture
+def no_library(monkeypatch):
+    """Any call that reaches the library fails the test."""
+    def _refuse(*a, **k):
+        raise AssertionError("the library was called")
+    monkeypatch.setattr(lq, "load_library", _refuse)
+
+
+def _cpu_tokens(cfg, n, io=None):
+    import torch
+    io = io or cfg.io_torch_dtype
+    B, H = cfg.batch, cfg.heads
+    return dict(q=torch.zeros((B, n, H, cfg.d_k), dtype=io), k=torch.zeros((B, n, H, cfg.d_k), dtype=io),
+                v=torch.zeros((B, n, H, cfg.d_v), dtype=io),
+                alpha=torch.ones((B, n, H, cfg.gdim) if cfg.gdim > 1 else (B, n, H)),
+                beta=torch.ones((B, n, H)), o=torch.zeros((B, n, H, cfg.d_v), dtype=io))
+
+
+def test_binding_rejects_bad_tensors_before_the_library(no_library):
+    import torch
+    cfg = lq.Config(batch=2, heads=3, d_k=64, d_v=128, window=4, n_comp=2, gate=lq.LQ_GATE_DIAG)
+    st = lq.State(cfg, "cpu")
+    t = _cpu_tokens(cfg, 2)
+    # wrong io dtype
+    bad = dict(t, q=t["q"].float())
+    with pytest.raises(TypeError, match="q: dtype"):
+        lq.lq_decode_window(st, bad["q"], bad["k"], bad["v"], bad["alpha"], bad["beta"], 2, bad["o"])
+    # one token short for n_steps = 2
+    bad = dict(t, v=t["v"][:, :1].contiguous())
+    with pytest.raises(ValueError, match="v: .* elements"):
+        lq.lq_decode_window(st, bad["q"], bad["k"], bad["v"], bad["alpha"], bad["beta"], 2, bad["o"])
+    # a scalar gate's alpha for a diagonal-gate configuration
+    bad = dict(t, alpha=torch.ones((2, 2, 3)))
+    with pytest.raises(ValueError, match="alpha"):
+        lq.lq_decode_window(st, bad["q"], bad["k"], bad["v"], bad["alpha"], bad["beta"], 2, bad["o"])
+    # non-contiguous
+    bad = dict(t, k=torch.zeros((2, 3, 2, 64), dtype=cfg.io_torch_dtype).transpose(1, 2))
+    with pytest.raises(ValueError, match="k: not contiguous"):
+        lq.lq_decode_window(st, bad["q"], bad["k"], bad["v"], bad["alpha"], bad["beta"], 2, bad["o"])
+    # right sizes, but host memory
+    with pytest.raises(ValueError, match="CUDA"):
+        lq.lq_decode_window(st, t["q"], t["k"], t["v"], t["alpha"], t["beta"], 2, t["o"])
+    # per-sequence positions: int32 [B]
+    t1 = _cpu_tokens(cfg, 1)
+    with pytest.raises(TypeError, match="seq_pos"):
+        lq.lq_decode_ragged(st, torch.zeros(2, dtype=torch.int64), *[t1[x] for x in
+                            ("q", "k", "v", "alpha", "beta", "o")])
+    with pytest.raises(ValueError, match="seq_pos"):
+        lq.lq_ragged_flush(st, torch.zeros(3, dtype=torch.int32))
+    # snapshots must match the configuration
+    other = lq.Snapshot(lq.Config(batch=2, heads=3, d_k=64, d_v=64, window=4, n_comp=2), "cpu")
+    with pytest.raises(ValueError, match="dst.codes"):
+        lq.lq_state_snapshot(st, other)
+    with pytest.raises(ValueError, match="src.codes"):
+        lq.lq_state_restore(st, other)
+    # init: the FP32 state's size
+    with pytest.raises(ValueError, match="S_init"):
+        lq.lq_state_init(st, torch.zeros((6, 128, 63)))
+    # prefill: state size, snapshot count
+    tp = _cpu_tokens(cfg, 128)
+    S = torch.zeros((6, 128, 64))
+    with pytest.raises(ValueError, match="S_fp32"):
+        lq.lq_prefill_chunk(st, S[:5], tp["q"], tp["k"], tp["v"], tp["alpha"], tp["beta"], 128, 64,
+                            None, tp["o"])
+    with pytest.raises(ValueError, match="snaps"):
+        lq.lq_prefill_chunk(st, S, tp["q"], tp["k"], tp["v"], tp["alpha"], tp["beta"], 128, 64,
+                            [lq.Snapshot(cfg, "cpu")], tp["o"])
+    # the FP32 comparator: bf16 state
+    with pytest.raises(TypeError, match="S: dtype"):
+        lq.lq_fp32_step(cfg, S.bfloat16(), t1["q"], t1["k"], t1["v"], t1["alpha"], t1["beta"], 1,
+                        t1["o"])

@@ -34,7 +34,7 @@ def _write_heads(st, snap, heads):
         st.snap.t[key][idx] = torch.from_numpy(src).to("cuda")
 
 
-def _run(dk, dv, gate, io, W, r, B, H, steps, start_of, bits=8):
+def _run(dk, dv, gate, io, W, r, B, H, steps, start_of, bits=8, flush=False):
     wl = synth.DecodeWorkload(f"ragged_{dk}_{dv}_{gate}", B, H, dk, dv, steps, W, r, gate, io, True,
                               max(1, dv // 100), max(1, dk // 100), 30.0)
     cfg = make_config(wl, auto_commit=0, bits=bits)
@@ -100,8 +100,54 @@ def _run(dk, dv, gate, io, W, r, B, H, steps, start_of, bits=8):
                 checked += 1
         want = [count[b] % W if s >= start_of[b] else -1 for b in range(B)]
         assert seq_pos.cpu().tolist() == want, "positions not advanced modulo W"
+    if flush:
+        checked += _flush_and_check(st, seq_pos, outs, count, anchor, start_of, steps, W, r, H, dk,
+                                    dv, gate, bits)
     assert lq.lq_device_errors() == 0
     return checked
+
+
+def _flush_and_check(st, seq_pos, outs, count, anchor, start_of, steps, W, r, H, dk, dv, gate,
+                     bits):
+    """lq_ragged_flush commits each sequence's open window (count % W
+    records) as the oracle's commit of those records would; sequences at a
+    window start and idle slots keep their snapshots; positions go to 0."""
+    B = len(count)
+    assert st.pos == lq.LQ_POS_PER_SEQUENCE
+    with pytest.raises(lq.LQError):  # windows may be open: the synchronous calls refuse
+        lq.lq_window_commit(st)
+    with pytest.raises(lq.LQError):
+        lq.lq_state_snapshot(st, lq.Snapshot(st.cfg, "cuda"))
+    before = download_snapshot(st)
+    lq.lq_ragged_flush(st, seq_pos)
+    torch.cuda.synchronize()
+    assert st.pos == 0
+    assert seq_pos.cpu().tolist() == [0 if steps > start_of[b] else -1 for b in range(B)]
+    after = download_snapshot(st)
+    flushed = 0
+    for b in range(B):
+        heads = np.arange(b * H, (b + 1) * H)
+        n = count[b] % W
+        if n == 0:
+            for key in before:
+                np.testing.assert_array_equal(after[key][heads], before[key][heads], err_msg=key)
+            continue
+        win = outs[b][-n:]
+        tok = {key: np.concatenate([t[key] for t, _ in win], axis=1) for key in win[0][0]}
+        d, kt, bb, vv, qq = oracle_tokens(tok, gate)
+        rec = oracle.empty_records(H, W, dk, dv, dk if gate == "diag" else 1)
+        oracle.window(anchor[b], rec, 0, d, kt, bb, vv, qq)
+        new, _ = oracle.commit(anchor[b], rec, n, r, True, bits)
+        compare_snapshots(_slice_snap(after, heads), new, new["row_norm"])
+        flushed += 1
+    # the state is closed again: a prefix-cache snapshot is allowed
+    dst = lq.Snapshot(st.cfg, "cuda")
+    lq.lq_state_snapshot(st, dst)
+    torch.cuda.synchronize()
+    for key in dst.t:
+        assert torch.equal(dst.t[key], st.snap.t[key]), key
+    assert flushed >= 1
+    return flushed
 
 
 @pytest.mark.parametrize("dk,dv,gate,io,W,r,B,H", [
@@ -147,3 +193,15 @@ def test_ragged_position_out_of_range_is_skipped_and_reported():
     assert np.all(oh[1] == SENTINEL) and np.all(oh[2] == SENTINEL)
     assert np.all(np.isfinite(oh[0])) and not np.all(oh[0] == SENTINEL)
     assert seq_pos.cpu().tolist() == [1, 4, -1]  # only valid positions advance
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+def test_ragged_flush_commits_every_open_window(bits):
+    """Staggered sequences left at positions 2, 1, 0, 3 and one idle slot:
+    the flush commits 2, 1, 0 and 3 records and closes the state."""
+    _run(128, 128, "scalar", "bf16", 4, 2, 5, 3, steps=6, start_of=[0, 1, 2, 3, 99], bits=bits,
+         flush=True)
+
+
+def test_ragged_flush_diagonal_gate_fp32():
+    _run(64, 128, "diag", "fp32", 5, 1, 4, 2, steps=7, start_of=[0, 2, 4, 99], flush=True)
