@@ -294,7 +294,7 @@ def test_errors_leave_state_unchanged():
     assert st.pos == 4
     before = {k: v.clone() for k, v in st.snap.t.items()}
     with pytest.raises(lq.LQError) as e:
-        lq.lq_decode_window(st, *[a[:, :1].contiguous() for a in args], 1, o)
+        lq.lq_decode_window(st, *[a[:, :1].contiguous() for a in args], 1, o[:, :1].contiguous())
     assert e.value.status == lq.LQ_ERR_WINDOW_FULL and st.pos == 4
     with pytest.raises(lq.LQError) as e:
         lq.lq_state_snapshot(st, lq.Snapshot(cfg, "cuda"))
