@@ -247,13 +247,31 @@ LQ_API lq_status lq_ragged_flush(lq_state *st, int32_t *seq_pos, lq_stream_t str
  * tokens ("LeapQuant: ...", Figure 1(b)).  On return st->snap holds the
  * quantized state after T tokens, ready for decode.  The FP32 state is
  * carried across snapshots unquantized.
+ *
+ * workspace (device, (16B), workspace_bytes long; may be NULL with 0 bytes):
+ * scratch of the chunked tensor-core prefill, used for the scalar gate with
+ * BF16 io and d_k = 128.  Tokens are taken in chunks of 64 within each
+ * snapshot interval, up to 16 chunks per pass of the workspace
+ * (lq_prefill_workspace_bytes gives the size for full passes; any size of at
+ * least one chunk, 32 KB per sequence and head, is used in shorter passes).
+ * Without a usable workspace, for other shapes, and for the last
+ * (snapshot_every mod 64) tokens of an interval, the recurrence runs token
+ * by token on the FP32 state (same arithmetic, CUDA cores).  The caller
+ * keeps the workspace alive until the call's work on `stream` has finished
+ * and does not share it between concurrent calls.
  * Requires pos == 0 (else LQ_ERR_WINDOW_OPEN; also LQ_POS_PER_SEQUENCE), T >= 0,
  * snapshot_every >= 1
  * and, when snaps != NULL, T % snapshot_every == 0.  T == 0 is a no-op. */
 LQ_API lq_status lq_prefill_chunk(lq_state *st, float *S_fp32, const void *q, const void *k,
                            const void *v, const float *alpha, const float *beta,
                            int32_t T, int32_t snapshot_every, const lq_snapshot *snaps,
-                           void *o, lq_stream_t stream);
+                           void *o, void *workspace, size_t workspace_bytes,
+                           lq_stream_t stream);
+
+/* Bytes of the workspace with which lq_prefill_chunk runs full passes of 16
+ * chunks of 64 tokens (16 x 64 x B x H x 32 KB); -1 for an invalid
+ * configuration, 0 when the configuration has no tensor-core prefill. */
+LQ_API int64_t lq_prefill_workspace_bytes(const lq_config *cfg);
 
 /* Copies the committed boundary state into `dst` (device buffers of the same
  * sizes): a prefix-cache snapshot, one quantized state kept per cached prefix

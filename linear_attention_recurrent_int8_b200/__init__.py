@@ -31,7 +31,7 @@ LQ_DEVERR_WAIT_TIMEOUT, LQ_DEVERR_BAD_POSITION = 1, 2
 # Every symbol include/lq.h declares.
 ABI_SYMBOLS = ("lq_buffer_elems", "lq_state_init", "lq_decode_window", "lq_decode_ragged",
                "lq_ragged_flush", "lq_window_commit",
-               "lq_prefill_chunk", "lq_state_snapshot", "lq_state_restore", "lq_fp32_step",
+               "lq_prefill_chunk", "lq_prefill_workspace_bytes", "lq_state_snapshot", "lq_state_restore", "lq_fp32_step",
                "lq_state_destroy", "lq_status_string", "lq_device_errors")
 
 
@@ -83,7 +83,8 @@ def load_library(build: bool = True):
                 "lq_ragged_flush": (I32, [ctypes.POINTER(LqState), P, P]),
                 "lq_window_commit": (I32, [ctypes.POINTER(LqState), P]),
                 "lq_prefill_chunk": (I32, [ctypes.POINTER(LqState), P, P, P, P, P, P, I32, I32,
-                                           ctypes.POINTER(LqSnapshot), P, P]),
+                                           ctypes.POINTER(LqSnapshot), P, P, ctypes.c_size_t, P]),
+                "lq_prefill_workspace_bytes": (ctypes.c_int64, [ctypes.POINTER(LqConfig)]),
                 "lq_state_snapshot": (I32, [ctypes.POINTER(LqState), ctypes.POINTER(LqSnapshot), P]),
                 "lq_state_restore": (I32, [ctypes.POINTER(LqState), ctypes.POINTER(LqSnapshot), P]),
                 "lq_fp32_step": (I32, [ctypes.POINTER(LqConfig), P, P, P, P, P, P, I32, P, P]),
@@ -346,8 +347,16 @@ def lq_window_commit(st: State, stream=None) -> None:
     _check(load_library().lq_window_commit(ctypes.byref(st.c), _stream(stream)), "lq_window_commit")
 
 
+def lq_prefill_workspace_bytes(cfg: Config) -> int:
+    c = cfg.c()
+    return load_library().lq_prefill_workspace_bytes(ctypes.byref(c))
+
+
 def lq_prefill_chunk(st: State, S_fp32, q, k, v, alpha, beta, T: int, snapshot_every: int,
-                     snaps, o, stream=None) -> None:
+                     snaps, o, stream=None, workspace="auto") -> None:
+    """workspace: "auto" allocates (torch) the size lq_prefill_workspace_bytes
+    gives for this call; a CUDA tensor is used as it is; None runs the
+    prefill token by token."""
     import torch
     cfg = st.cfg
     if int(T) > 0:
@@ -361,12 +370,27 @@ def lq_prefill_chunk(st: State, S_fp32, q, k, v, alpha, beta, T: int, snapshot_e
             for i, sn in enumerate(snaps):
                 specs += _snapshot_specs(cfg, sn, f"snaps[{i}]")
         _check_tensors(st.device, *specs)
+    ws, ws_bytes = None, 0
+    if isinstance(workspace, str):
+        if workspace != "auto":
+            raise ValueError(f"workspace: {workspace!r}")
+        n = lq_prefill_workspace_bytes(cfg) if int(T) > 0 else 0
+        if n > 0:
+            ws = torch.empty(n, dtype=torch.uint8, device=st.device)
+    elif workspace is not None:
+        if not isinstance(workspace, torch.Tensor) or not workspace.is_contiguous():
+            raise ValueError("workspace: expected a contiguous tensor")
+        _check_device(workspace, "workspace", st.device)
+        ws = workspace
+    if ws is not None:
+        ws_bytes = ws.numel() * ws.element_size()
     arr = None
     if snaps is not None:
         arr = (LqSnapshot * len(snaps))(*[s.c() for s in snaps])
     _check(load_library().lq_prefill_chunk(ctypes.byref(st.c), _ptr(S_fp32), _ptr(q), _ptr(k),
                                            _ptr(v), _ptr(alpha), _ptr(beta), int(T),
-                                           int(snapshot_every), arr, _ptr(o), _stream(stream)),
+                                           int(snapshot_every), arr, _ptr(o), _ptr(ws), ws_bytes,
+                                           _stream(stream)),
            "lq_prefill_chunk")
 
 

@@ -10,6 +10,9 @@
 
 namespace {
 
+constexpr int kChunkTokens = 64;  // tokens per chunk of the tensor-core prefill
+constexpr int kPassChunks = 16;   // chunks per pass of its workspace
+
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bool aligned_to(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -283,10 +286,16 @@ lq_status lq_window_commit(lq_state *st, lq_stream_t stream) {
     return LQ_OK;
 }
 
+int64_t lq_prefill_workspace_bytes(const lq_config *cfg) {
+    if (check_config(cfg) != LQ_OK) return -1;
+    if (!lq::chunk_path_supported(cfg->d_k, cfg->d_v, cfg->gate, cfg->io_dtype == LQ_BF16)) return 0;
+    return (int64_t)lq::chunk_workspace_bytes(cfg->batch * cfg->heads, kPassChunks);
+}
+
 lq_status lq_prefill_chunk(lq_state *st, float *S_fp32, const void *q, const void *k,
                            const void *v, const float *alpha, const float *beta, int32_t T,
                            int32_t snapshot_every, const lq_snapshot *snaps, void *o,
-                           lq_stream_t stream) {
+                           void *workspace, size_t workspace_bytes, lq_stream_t stream) {
     lq_status e = check_state(st);
     if (e != LQ_OK) return e;
     if (st->pos != 0) return LQ_ERR_WINDOW_OPEN;
@@ -295,6 +304,8 @@ lq_status lq_prefill_chunk(lq_state *st, float *S_fp32, const void *q, const voi
     if (snaps && T % snapshot_every != 0) return LQ_ERR_INVALID_ARGUMENT;
     if (!S_fp32) return LQ_ERR_INVALID_ARGUMENT;
     if (!aligned16(S_fp32)) return LQ_ERR_MISALIGNED;
+    if (!workspace != (workspace_bytes == 0)) return LQ_ERR_INVALID_ARGUMENT;
+    if (workspace && !aligned16(workspace)) return LQ_ERR_MISALIGNED;
     e = check_tokens(&st->cfg, q, k, v, alpha, beta, o);
     if (e != LQ_OK) return e;
     if (snaps) {
@@ -318,12 +329,45 @@ lq_status lq_prefill_chunk(lq_state *st, float *S_fp32, const void *q, const voi
     r.delta = c->delta;
     r.H = c->heads;
     r.T_total = T;
+    // chunks per pass of the tensor-core path (0: token by token)
+    const int BH = c->batch * c->heads;
+    int pass = 0;
+    if (workspace && lq::chunk_path_supported(c->d_k, c->d_v, c->gate, c->io_dtype == LQ_BF16)) {
+        const size_t per = lq::chunk_workspace_bytes(BH, 1);
+        pass = (int)(workspace_bytes / per < (size_t)kPassChunks ? workspace_bytes / per : kPassChunks);
+    }
+    lq::ChunkArgs ca{};
+    ca.S = S_fp32;
+    ca.alpha = alpha;
+    ca.beta = beta;
+    ca.o = o;
+    ca.ws = static_cast<float *>(workspace);
+    ca.B = c->batch;
+    ca.H = c->heads;
+    ca.DV = c->d_v;
+    ca.T_total = T;
+    ca.delta = c->delta;
     for (int t0 = 0, i = 0; t0 < T; t0 += snapshot_every, ++i) {
-        r.t0 = t0;
-        r.nt = T - t0 < snapshot_every ? T - t0 : snapshot_every;
-        e = cuda_status(lq::launch_recurrence(r, c->d_k, c->d_v, c->gate, c->io_dtype == LQ_BF16,
-                                              true, s));
-        if (e != LQ_OK) return e;
+        const int nt = T - t0 < snapshot_every ? T - t0 : snapshot_every;
+        int done = 0;
+        if (pass > 0) {
+            // whole chunks of this interval on the tensor cores, in passes
+            const int nch = nt / kChunkTokens;
+            for (int c0 = 0; c0 < nch; c0 += pass) {
+                ca.t0 = t0 + c0 * kChunkTokens;
+                ca.nc = nch - c0 < pass ? nch - c0 : pass;
+                e = cuda_status(lq::launch_prefill_chunks(ca, q, k, v, s));
+                if (e != LQ_OK) return e;
+            }
+            done = nch * kChunkTokens;
+        }
+        if (done < nt) {
+            r.t0 = t0 + done;
+            r.nt = nt - done;
+            e = cuda_status(lq::launch_recurrence(r, c->d_k, c->d_v, c->gate, c->io_dtype == LQ_BF16,
+                                                  true, s));
+            if (e != LQ_OK) return e;
+        }
         if (snaps) {
             e = cuda_status(lq::launch_quantize(quant_args(c, S_fp32, &snaps[i]), c->d_k, c->d_v, s));
             if (e != LQ_OK) return e;

@@ -80,6 +80,28 @@ struct RecurArgs {
     int t0, nt;   // tokens [t0, t0+nt) processed by this launch
 };
 
+// Arguments of the chunked prefill (lq_chunk.cu): one pass of nc chunks of
+// 64 tokens starting at token t0 of every sequence.
+struct ChunkArgs {
+    float *S;            // [BH][DV][128] FP32 state, in/out
+    const float *alpha;  // [B][T_total][H]
+    const float *beta;   // [B][T_total][H]
+    void *o;             // BF16 [B][T_total][H][DV]
+    float *ws;           // workspace [nc][BH][128][64] FP32 ([PT; T] of each chunk)
+    int B, H, DV, T_total, t0, nc, delta;
+};
+
+// Workspace bytes of a pass of `chunks` chunks over BH heads.
+size_t chunk_workspace_bytes(int BH, int chunks);
+
+// Whether the tensor-core chunked prefill covers this shape (scalar gate,
+// BF16 io, d_k = 128, d_v in {64, 128}).
+bool chunk_path_supported(int d_k, int d_v, int gate, bool bf16);
+
+// One pass: the [PT; T] preparation of every chunk, then the chunks in order.
+cudaError_t launch_prefill_chunks(const ChunkArgs &a, const void *q, const void *k, const void *v,
+                                  cudaStream_t stream);
+
 // Decodes a.n_steps >= 1 tokens (records a.pos .. a.pos + n_steps - 1).
 cudaError_t launch_decode(const DecodeArgs &a, int d_k, int d_v, int gate, bool bf16,
                           cudaStream_t stream);

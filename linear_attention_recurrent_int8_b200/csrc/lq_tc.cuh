@@ -124,6 +124,24 @@ __device__ __forceinline__ void tmem_load(uint32_t taddr, float (&v)[N]) {
     else tmem_load64(taddr, v);
 }
 
+// Instruction descriptor of kind::f16 with BF16 A and B, FP32 accumulator,
+// M x N tile; a_mn / b_mn select MN-major operands (else K-major).
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool b_mn) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// D (TMEM) = A B (+ D when `accumulate`), kind::f16 (BF16 operands), both
+// operands in shared memory; issued by one thread.
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, bool accumulate) {
+    asm volatile(
+        "{ .reg .pred p; setp.ne.b32 p, %4, 0; "
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"((uint32_t)accumulate)
+        : "memory");
+}
+
 // Warp maximum of |x| (identical in every lane).
 __device__ __forceinline__ float warp_max_abs(float x) {
     float r;

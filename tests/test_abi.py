@@ -158,18 +158,25 @@ def test_commit_snapshot_prefill_validation_without_launch():
     p = 0x40000000
     args = [p, p + 0x100000, p + 0x200000, p + 0x300000, p + 0x400000, p + 0x500000]
     st = _fake_state(cfg, pos=2)
-    assert lib.lq_prefill_chunk(ctypes.byref(st), *args, 128, 64, None, p + 0x600000, None) == \
+    assert lib.lq_prefill_chunk(ctypes.byref(st), *args, 128, 64, None, p + 0x600000, None, 0, None) == \
         lq.LQ_ERR_WINDOW_OPEN
     st = _fake_state(cfg)
-    assert lib.lq_prefill_chunk(ctypes.byref(st), *args, 0, 64, None, p + 0x600000, None) == lq.LQ_OK
-    assert lib.lq_prefill_chunk(ctypes.byref(st), *args, 128, 0, None, p + 0x600000, None) == \
+    assert lib.lq_prefill_chunk(ctypes.byref(st), *args, 0, 64, None, p + 0x600000, None, 0, None) == lq.LQ_OK
+    assert lib.lq_prefill_chunk(ctypes.byref(st), *args, 128, 0, None, p + 0x600000, None, 0, None) == \
         lq.LQ_ERR_INVALID_ARGUMENT
     snaps = (lq.LqSnapshot * 2)(dst, dst)
-    assert lib.lq_prefill_chunk(ctypes.byref(st), *args, 100, 64, snaps, p + 0x600000, None) == \
+    assert lib.lq_prefill_chunk(ctypes.byref(st), *args, 100, 64, snaps, p + 0x600000, None, 0, None) == \
         lq.LQ_ERR_INVALID_ARGUMENT
+    # workspace: pointer and size go together; 16-byte aligned
+    assert lib.lq_prefill_chunk(ctypes.byref(st), *args, 128, 64, None, p + 0x600000, None, 4096,
+                                None) == lq.LQ_ERR_INVALID_ARGUMENT
+    assert lib.lq_prefill_chunk(ctypes.byref(st), *args, 128, 64, None, p + 0x600000, p + 0x700000,
+                                0, None) == lq.LQ_ERR_INVALID_ARGUMENT
+    assert lib.lq_prefill_chunk(ctypes.byref(st), *args, 128, 64, None, p + 0x600000, p + 0x700008,
+                                4096, None) == lq.LQ_ERR_MISALIGNED
     bad = list(args)
     bad[0] += 4
-    assert lib.lq_prefill_chunk(ctypes.byref(st), *bad, 128, 64, None, p + 0x600000, None) == \
+    assert lib.lq_prefill_chunk(ctypes.byref(st), *bad, 128, 64, None, p + 0x600000, None, 0, None) == \
         lq.LQ_ERR_MISALIGNED
     # fp32 comparator: negative steps, null state
     c = cfg.c()
@@ -252,7 +259,7 @@ def test_per_sequence_mode_refuses_calls_that_need_closed_windows():
     p = 0x40000000
     args = [p, p + 0x100000, p + 0x200000, p + 0x300000, p + 0x400000, p + 0x500000]
     assert lib.lq_prefill_chunk(ctypes.byref(per_seq()), *args, 128, 64, None, p + 0x600000,
-                                None) == lq.LQ_ERR_WINDOW_OPEN
+                                None, 0, None) == lq.LQ_ERR_WINDOW_OPEN
     # other negative positions stay invalid
     assert _decode(_fake_state(cfg, pos=-2), 1) == lq.LQ_ERR_INVALID_ARGUMENT
     # the flush: positions array required and aligned; an open synchronous window refuses
@@ -355,3 +362,18 @@ def test_binding_rejects_bad_tensors_before_the_library(no_library):
     with pytest.raises(TypeError, match="S: dtype"):
         lq.lq_fp32_step(cfg, S.bfloat16(), t1["q"], t1["k"], t1["v"], t1["alpha"], t1["beta"], 1,
                         t1["o"])
+
+
+def test_prefill_workspace_bytes():
+    """16 chunks of 64 tokens per pass, 32 KB ([PT; T], 128 x 64 FP32) per
+    chunk and head; 0 where the tensor-core prefill does not apply."""
+    cfg = lq.Config(batch=2, heads=32, d_k=128, d_v=128, io_dtype=lq.LQ_BF16)
+    assert lq.lq_prefill_workspace_bytes(cfg) == 16 * 64 * 32768
+    cfg.d_v = 64
+    assert lq.lq_prefill_workspace_bytes(cfg) == 16 * 64 * 32768
+    for field, val in (("io_dtype", lq.LQ_F32), ("gate", lq.LQ_GATE_DIAG), ("d_k", 64)):
+        c2 = lq.Config(batch=2, heads=32, d_k=128, d_v=128, io_dtype=lq.LQ_BF16)
+        setattr(c2, field, val)
+        assert lq.lq_prefill_workspace_bytes(c2) == 0, field
+    cfg.window = 0
+    assert lq.lq_prefill_workspace_bytes(cfg) == -1

@@ -79,7 +79,7 @@ def test_per_token_without_smoothing():
 def test_prefill_65536_then_decode_sampled():
     """Chunked GDN prefill, batch 2 x 32 heads, T = 65536, a quantized
     snapshot every 1024 tokens; then 512 decode steps from the last snapshot
-    (W = 16, r = 4).  Two sampled heads follow the oracle over all tokens."""
+    (W = 16, r = 4).  Eight sampled heads follow the oracle over all tokens."""
     P = synth.PREFILL_WORKLOAD
     B, H, dk, dv, T, every, r = P["batch"], P["heads"], P["d_k"], P["d_v"], P["T"], \
         P["snapshot_every"], P["n_comp"]
@@ -88,7 +88,9 @@ def test_prefill_65536_then_decode_sampled():
                     gate=lq.LQ_GATE_SCALAR, io_dtype=lq.LQ_BF16, smoothing=1, auto_commit=1)
     st = lq.State(cfg, dev)
     lq.lq_state_init(st, None)
-    sample = [(0, 5), (1, 30)]
+    # eight sampled heads of both sequences (each head spans both value-row
+    # slices of the chunked scan)
+    sample = [(0, 0), (0, 5), (0, 17), (0, 31), (1, 2), (1, 13), (1, 24), (1, 30)]
     sb = np.array([s[0] for s in sample])
     sh = np.array([s[1] for s in sample])
     # device inputs for all heads, drawn in slices; sampled heads from numpy
