@@ -268,6 +268,30 @@ LQ_API lq_status lq_prefill_chunk(lq_state *st, float *S_fp32, const void *q, co
                            void *o, void *workspace, size_t workspace_bytes,
                            lq_stream_t stream);
 
+/* lq_prefill_chunk for callers that cannot supply device memory of their
+ * own -- for example a serving engine that reserved nearly all of HBM for its
+ * pool at start-up and hands kernels only their input and output tensors, or
+ * code that must not call cudaMalloc because it can synchronize the device.
+ * The paper has no counterpart to this call; it exists for such callers.
+ * Arguments and results are those of lq_prefill_chunk; the tensor-core
+ * prefill's scratch comes from a fixed 8 MiB array inside the library (held
+ * on every GPU that loads the library until the process exits) instead of a
+ * workspace argument, and the call allocates nothing.
+ *  - Limit: one chunk of scratch is 32 KB per sequence and head, so B * H
+ *    may be at most 256 when the tensor-core path applies (scalar gate, BF16
+ *    io, d_k = 128); above that the call returns LQ_ERR_UNSUPPORTED and does
+ *    nothing.  Passes hold min(16, 256 / (B * H)) chunks.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current); make that first call
+ *    before any stream capture.  A failed lookup returns LQ_ERR_CUDA.
+ *  - All calls share the one array, which keeps the last call's contents
+ *    (nothing in it needs to start at zero).  Calls whose work overlaps on
+ *    the GPU (other streams, other host threads) race on it: serialize them. */
+LQ_API lq_status lq_prefill_chunk_noalloc(lq_state *st, float *S_fp32, const void *q,
+                                          const void *k, const void *v, const float *alpha,
+                                          const float *beta, int32_t T, int32_t snapshot_every,
+                                          const lq_snapshot *snaps, void *o, lq_stream_t stream);
+
 /* Bytes of the workspace with which lq_prefill_chunk runs full passes of 16
  * chunks of 64 tokens (16 x 64 x B x H x 32 KB); -1 for an invalid
  * configuration, 0 when the configuration has no tensor-core prefill. */

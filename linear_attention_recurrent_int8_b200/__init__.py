@@ -31,7 +31,7 @@ LQ_DEVERR_WAIT_TIMEOUT, LQ_DEVERR_BAD_POSITION = 1, 2
 # Every symbol include/lq.h declares.
 ABI_SYMBOLS = ("lq_buffer_elems", "lq_state_init", "lq_decode_window", "lq_decode_ragged",
                "lq_ragged_flush", "lq_window_commit",
-               "lq_prefill_chunk", "lq_prefill_workspace_bytes", "lq_state_snapshot", "lq_state_restore", "lq_fp32_step",
+               "lq_prefill_chunk", "lq_prefill_chunk_noalloc", "lq_prefill_workspace_bytes", "lq_state_snapshot", "lq_state_restore", "lq_fp32_step",
                "lq_state_destroy", "lq_status_string", "lq_device_errors")
 
 
@@ -85,6 +85,8 @@ def load_library(build: bool = True):
                 "lq_prefill_chunk": (I32, [ctypes.POINTER(LqState), P, P, P, P, P, P, I32, I32,
                                            ctypes.POINTER(LqSnapshot), P, P, ctypes.c_size_t, P]),
                 "lq_prefill_workspace_bytes": (ctypes.c_int64, [ctypes.POINTER(LqConfig)]),
+                "lq_prefill_chunk_noalloc": (I32, [ctypes.POINTER(LqState), P, P, P, P, P, P, I32,
+                                                   I32, ctypes.POINTER(LqSnapshot), P, P]),
                 "lq_state_snapshot": (I32, [ctypes.POINTER(LqState), ctypes.POINTER(LqSnapshot), P]),
                 "lq_state_restore": (I32, [ctypes.POINTER(LqState), ctypes.POINTER(LqSnapshot), P]),
                 "lq_fp32_step": (I32, [ctypes.POINTER(LqConfig), P, P, P, P, P, P, I32, P, P]),
@@ -392,6 +394,33 @@ def lq_prefill_chunk(st: State, S_fp32, q, k, v, alpha, beta, T: int, snapshot_e
                                            int(snapshot_every), arr, _ptr(o), _ptr(ws), ws_bytes,
                                            _stream(stream)),
            "lq_prefill_chunk")
+
+
+def lq_prefill_chunk_noalloc(st: State, S_fp32, q, k, v, alpha, beta, T: int,
+                             snapshot_every: int, snaps, o, stream=None) -> None:
+    """lq_prefill_chunk with the library's fixed scratch array instead of a
+    workspace: for callers that cannot hand out more device memory.  Neither
+    this wrapper nor the library allocates anything."""
+    import torch
+    cfg = st.cfg
+    if int(T) > 0:
+        specs = [(S_fp32, "S_fp32", torch.float32, cfg.batch * cfg.heads * cfg.d_v * cfg.d_k)]
+        specs += _token_specs(cfg, int(T), q, k, v, alpha, beta, o)
+        if snaps is not None:
+            if int(snapshot_every) < 1 or int(T) % int(snapshot_every) != 0 or \
+                    len(snaps) != int(T) // int(snapshot_every):
+                raise ValueError(f"snaps: {len(snaps)} snapshots for T = {T}, "
+                                 f"snapshot_every = {snapshot_every}")
+            for i, sn in enumerate(snaps):
+                specs += _snapshot_specs(cfg, sn, f"snaps[{i}]")
+        _check_tensors(st.device, *specs)
+    arr = None
+    if snaps is not None:
+        arr = (LqSnapshot * len(snaps))(*[s.c() for s in snaps])
+    _check(load_library().lq_prefill_chunk_noalloc(ctypes.byref(st.c), _ptr(S_fp32), _ptr(q), _ptr(k),
+                                                   _ptr(v), _ptr(alpha), _ptr(beta), int(T),
+                                                   int(snapshot_every), arr, _ptr(o), _stream(stream)),
+           "lq_prefill_chunk_noalloc")
 
 
 def lq_state_snapshot(st: State, dst: Snapshot, stream=None) -> None:
