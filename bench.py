@@ -130,6 +130,19 @@ def measured_peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+def measured_bf16_tflops(sustained: bool):
+    """Dense BF16 tensor peak (TFLOP/s): the measured cuBLAS figure (burst, or
+    sustained under the power cap), else the pool's earlier measurement."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        key = "bf16_tflops_sustained" if sustained else "bf16_tflops"
+        if key in d:
+            return float(d[key]), "measured"
+    return (1400.0 if sustained else 1590.0), "fallback"
+
+
 # the sources of each kernel's translation unit (the .cu and the headers it includes)
 KERNEL_SOURCES = {
     "decode": ["lq_decode.cu", "lq_common.cuh", "lq_quant.cuh", "lq_kernels.h"],
@@ -586,9 +599,11 @@ def run_prefill(args):
     o = torch.empty((B, T, H, dv), dtype=torch.bfloat16, device=dev)
     snaps = [lq.Snapshot(cfg, dev) for _ in range(T // every)]
 
+    ws = torch.empty(max(1, lq.lq_prefill_workspace_bytes(cfg)), dtype=torch.uint8, device=dev)
+
     def one():
         S.zero_()
-        lq.lq_prefill_chunk(st, S, q, k, v, alpha, beta, T, every, snaps, o)
+        lq.lq_prefill_chunk(st, S, q, k, v, alpha, beta, T, every, snaps, o, workspace=ws)
 
     for _ in range(args.warmup):
         one()
@@ -601,21 +616,32 @@ def run_prefill(args):
     torch.cuda.synchronize()
     ms = a.elapsed_time(b) / args.steps
     nbytes = B * T * H * (2 * (2 * dk + dv) + 8 + 2 * dv)
-    flops = B * T * H * 3 * 2 * dk * dv
-    tflops = flops / (ms / 1e3) / 1e12
+    # the chunked algorithm's products per 64-token chunk and head (C = 64):
+    # [Q; K] K^T 2*2C*C*dk, X = [Q; K] S^T 2*2C*dk*dv, [PT; T] R 2*2C*C*dv,
+    # K^T U^ 2*dk*C*dv; the tensor pipe runs each S / R / U product on three
+    # BF16 parts (six for [PT; T] R), counted separately as executed work
+    C = 64
+    chunks = B * H * (T // C)
+    f_alg = 2 * 2 * C * C * dk + 2 * 2 * C * dk * dv + 2 * 2 * C * C * dv + 2 * dk * C * dv
+    f_exec = 2 * 2 * C * C * dk + 3 * 2 * 2 * C * dk * dv + 6 * 2 * 2 * C * C * dv + 3 * 2 * dk * C * dv
+    tflops = chunks * f_alg / (ms / 1e3) / 1e12
+    peak_t, peak_kind = measured_bf16_tflops(sustained=False)
     line = {"metric": "prefill tokens/s (state update + output, snapshots every 1024 tokens)",
             "value": B * T / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": f"gdn prefill batch {B} x {H} heads, d={dk}, T={T}, bf16, "
                                    f"snapshot every {every} (r={r})"},
-            # the token-sequential FP32 recurrence is bound by FP32 FMA issue:
-            # 3 x 2 d_k d_v FLOP per (token, head) against 148 SMs x 128 FP32
-            # lanes x 2 FLOP x 1.965 GHz
-            "roofline": {"bound": "alu", "achieved": tflops, "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s",
-                         "frac": tflops / FP32_ALU_TFLOPS, "traffic": None,
-                         "kernel": "recur_kernel (FP32 recurrence) + quantize_kernel (snapshots)"},
-            "detail": {"io_gbs": nbytes / (ms / 1e3) / 1e9, "snapshots": T // every}}
+            # the chunked prefill on the tensor core: the whole call (chunk
+            # preparation, the chunk scan, snapshot quantization) against the
+            # dense BF16 peak, algorithmic FLOPs of the chunked algorithm
+            "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak_t, "unit": "TFLOP/s",
+                         "frac": tflops / peak_t, "traffic": None, "peak_kind": peak_kind,
+                         "kernel": "chunk_prep_kernel + chunk_scan_kernel + quantize_kernel (whole call)"},
+            "detail": {"io_gbs": nbytes / (ms / 1e3) / 1e9, "snapshots": T // every,
+                       "executed_tensor_tflops": chunks * f_exec / (ms / 1e3) / 1e12,
+                       "us_per_chunk_per_head_chain": ms * 1e3 / (T // C),
+                       "fp32_recurrence_equiv_tflops": B * T * H * 3 * 2 * dk * dv / (ms / 1e3) / 1e12}}
     if not args.no_cpu:
         rate, dt, cores, sample = oracle_prefill_rate(P, args.cpu_seconds)
         line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",

@@ -253,7 +253,7 @@ LQ_API lq_status lq_ragged_flush(lq_state *st, int32_t *seq_pos, lq_stream_t str
  * BF16 io and d_k = 128.  Tokens are taken in chunks of 64 within each
  * snapshot interval, up to 16 chunks per pass of the workspace
  * (lq_prefill_workspace_bytes gives the size for full passes; any size of at
- * least one chunk, 32 KB per sequence and head, is used in shorter passes).
+ * least one chunk, 48 KB per sequence and head, is used in shorter passes).
  * Without a usable workspace, for other shapes, and for the last
  * (snapshot_every mod 64) tokens of an interval, the recurrence runs token
  * by token on the FP32 state (same arithmetic, CUDA cores).  The caller
@@ -277,10 +277,10 @@ LQ_API lq_status lq_prefill_chunk(lq_state *st, float *S_fp32, const void *q, co
  * prefill's scratch comes from a fixed 8 MiB array inside the library (held
  * on every GPU that loads the library until the process exits) instead of a
  * workspace argument, and the call allocates nothing.
- *  - Limit: one chunk of scratch is 32 KB per sequence and head, so B * H
- *    may be at most 256 when the tensor-core path applies (scalar gate, BF16
+ *  - Limit: one chunk of scratch is 48 KB per sequence and head, so B * H
+ *    may be at most 170 when the tensor-core path applies (scalar gate, BF16
  *    io, d_k = 128); above that the call returns LQ_ERR_UNSUPPORTED and does
- *    nothing.  Passes hold min(16, 256 / (B * H)) chunks.
+ *    nothing.  Passes hold min(16, floor(170 / (B * H))) chunks.
  *  - The first call on each device looks up the array's device address
  *    (cudaGetSymbolAddress, with that device current); make that first call
  *    before any stream capture.  A failed lookup returns LQ_ERR_CUDA.
@@ -293,7 +293,7 @@ LQ_API lq_status lq_prefill_chunk_noalloc(lq_state *st, float *S_fp32, const voi
                                           const lq_snapshot *snaps, void *o, lq_stream_t stream);
 
 /* Bytes of the workspace with which lq_prefill_chunk runs full passes of 16
- * chunks of 64 tokens (16 x 64 x B x H x 32 KB); -1 for an invalid
+ * chunks of 64 tokens (16 x B x H x 48 KB); -1 for an invalid
  * configuration, 0 when the configuration has no tensor-core prefill. */
 LQ_API int64_t lq_prefill_workspace_bytes(const lq_config *cfg);
 

@@ -24,7 +24,8 @@
 //  * chunk_prep_kernel (every chunk of every head in parallel): K K^T and
 //    Q K^T on the tensor core (BF16, exact products, FP32 sums), A and P on
 //    CUDA cores, then T and PT column by column (forward substitution, FP32),
-//    written to the caller's workspace as [PT; T] (128 x 64 FP32 per chunk);
+//    written to the caller's workspace as [PT; T] (128 x 64, three BF16 parts
+//    of each FP32 value, in the operand layout: 48 KB per chunk and head);
 //  * chunk_scan_kernel (one CTA per head and 64 value rows, the chunks of the
 //    pass in order): the three products that carry the state, FP32-faithful
 //    on the tensor core --
@@ -53,7 +54,11 @@ constexpr int kDVS = 64;         // value rows per scan CTA
 constexpr int kQKBytes = 2 * kC * kDK * 2;   // [Q; K] BF16 operand: 32 KB
 constexpr int kVBytes = kC * kDVS * 2;       // V slice: 8 KB
 constexpr int kTRows = 2 * kC;               // [PT; T]
-constexpr int kWsChunkFloats = kTRows * kC;  // 8192 floats = 32 KB per chunk and head
+// [PT; T] of one chunk and head in the workspace: three BF16 parts of the
+// K-major operand (element (r, m) of part p at byte p * 16384 +
+// (m / 8) * 2048 + 16 r + 2 (m % 8)), 48 KB
+constexpr int kTPartBytes = kTRows * kC * 2;
+constexpr int kWsChunkBytes = 3 * kTPartBytes;
 
 // ---------------------------------------------------------------------------
 // TMA (tiled bulk tensor copies, no multicast)
@@ -93,15 +98,18 @@ __device__ __forceinline__ uint64_t desc_kt_mn(const unsigned char *qk, int k16)
     return smem_desc(smem_u32(qk + 1024 + k16 * 256), 128, 2048);
 }
 
-// Three BF16 parts with x = p0 + p1 + p2 + O(2^-24 |x|): each part is the
-// nearest BF16 to the remainder (the remainders are exact FP32 differences).
-__device__ __forceinline__ void split_bf16x3(float x, __nv_bfloat16 &p0, __nv_bfloat16 &p1,
-                                             __nv_bfloat16 &p2) {
-    p0 = __float2bfloat16_rn(x);
-    const float r1 = x - __bfloat162float(p0);
-    p1 = __float2bfloat16_rn(r1);
-    const float r2 = r1 - __bfloat162float(p1);
-    p2 = __float2bfloat16_rn(r2);
+// Two values in three BF16 parts each, packed in pairs (x0 in the low half).
+__device__ __forceinline__ void split2_bf16x3(float x0, float x1, uint32_t &w0, uint32_t &w1,
+                                              uint32_t &w2) {
+    const __nv_bfloat162 p0 = __floats2bfloat162_rn(x0, x1);
+    const float2 b0 = __bfloat1622float2(p0);
+    const float r0 = x0 - b0.x, r1 = x1 - b0.y;
+    const __nv_bfloat162 p1 = __floats2bfloat162_rn(r0, r1);
+    const float2 b1 = __bfloat1622float2(p1);
+    const __nv_bfloat162 p2 = __floats2bfloat162_rn(r0 - b1.x, r1 - b1.y);
+    w0 = *reinterpret_cast<const uint32_t *>(&p0);
+    w1 = *reinterpret_cast<const uint32_t *>(&p1);
+    w2 = *reinterpret_cast<const uint32_t *>(&p2);
 }
 
 // The running log gate of a chunk, every lane: lane l holds L at tokens 2l
@@ -130,12 +138,14 @@ __device__ __forceinline__ float log_gate_at(float Le, float Lo, int t) {
 // ---------------------------------------------------------------------------
 
 constexpr int kPrepThreads = 128;
-constexpr int kAStride = 68;  // padded row stride (floats) of A and P in shared memory
+constexpr int kAStride = 68;  // padded row stride (floats) of A, P and the solved columns
 
 struct PrepSmem {
-    alignas(16) float A[kC][kAStride];
-    alignas(16) float P[kC][kAStride];
-    float alpha[kC], beta[kC];
+    alignas(16) float A[kC][kAStride];  // strictly lower (G .* beta_m K K^T)
+    alignas(16) float P[kC][kAStride];  // lower (G .* beta_m Q K^T)
+    alignas(16) float L2[kC];           // L_t log2(e)
+    alignas(16) float beta[kC];
+    float alpha[kC];
     uint64_t bar_in, bar_mma;
     uint32_t tmem;
 };
@@ -144,12 +154,57 @@ __host__ __device__ constexpr int prep_smem_bytes() {
     return kQKBytes + (int)sizeof(PrepSmem) + 128;
 }
 
+// Column m of T = (I + A)^{-1}: forward substitution in blocks of 8 rows, the
+// block's rows accumulated together against the solved rows above it (read
+// back from X[m], the column's row of the solved-column store).  Two lanes
+// (xor 1) share a column: each sums every other group of 4 solved rows, one
+// shuffle joins the halves, and both finish the block's own 8 x 8 triangle.
+__device__ __forceinline__ void solve_column(const PrepSmem &ps, float *Xm, int m, int half) {
+#pragma unroll 1
+    for (int blk = 0; blk < kC / 8; ++blk) {
+        const int r0 = 8 * blk;
+        float acc[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) acc[r] = 0.0f;
+#pragma unroll 1
+        for (int n = 4 * half; n < r0; n += 8) {
+            const float4 xv = *reinterpret_cast<const float4 *>(Xm + n);
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                const float4 av = *reinterpret_cast<const float4 *>(&ps.A[r0 + r][n]);
+                acc[r] = fmaf(av.x, xv.x, acc[r]);
+                acc[r] = fmaf(av.y, xv.y, acc[r]);
+                acc[r] = fmaf(av.z, xv.z, acc[r]);
+                acc[r] = fmaf(av.w, xv.w, acc[r]);
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < 8; ++r) acc[r] += __shfl_xor_sync(0xffffffffu, acc[r], 1);
+        float xb[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            float v = (r0 + r == m ? 1.0f : 0.0f) - acc[r];
+#pragma unroll
+            for (int n = 0; n < r; ++n) v = fmaf(-ps.A[r0 + r][r0 + n], xb[n], v);
+            xb[r] = v;
+        }
+        if (half == 0) {
+            *reinterpret_cast<float4 *>(Xm + r0) = make_float4(xb[0], xb[1], xb[2], xb[3]);
+            *reinterpret_cast<float4 *>(Xm + r0 + 4) = make_float4(xb[4], xb[5], xb[6], xb[7]);
+        }
+        __syncwarp();
+    }
+}
+
 __global__ void __launch_bounds__(kPrepThreads) chunk_prep_kernel(
     const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
     const ChunkArgs a) {
     extern __shared__ __align__(128) unsigned char smem[];
     unsigned char *qk = smem;
     PrepSmem &ps = *reinterpret_cast<PrepSmem *>(smem + kQKBytes);
+    // after the MMA the [Q; K] tile is dead: its space holds the solved
+    // columns, X[m][t] = T[t][m] (row stride kAStride)
+    float *X = reinterpret_cast<float *>(qk);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int c = blockIdx.x % a.nc, bh = blockIdx.x / a.nc;
     const int b = bh / a.H, h = bh % a.H;
@@ -175,38 +230,45 @@ __global__ void __launch_bounds__(kPrepThreads) chunk_prep_kernel(
         if (ok) {
             // D[128 x 64] = [Q; K] K^T: rows 0..63 Q K^T, rows 64..127 K K^T
             constexpr uint32_t idesc = idesc_bf16(128, kC, false, false);
-#pragma unroll 1
-            for (int k16 = 0; k16 < kDK / 16; ++k16) {
-                const uint64_t bd = smem_desc(smem_u32(qk + 1024 + k16 * 4096), 2048, 128);
-                mma_bf16(ps.tmem, desc_qk(qk, k16), bd, idesc, k16 > 0);
-            }
+            const uint64_t dA = desc_qk(qk, 0);
+            const uint64_t dB = smem_desc(smem_u32(qk + 1024), 2048, 128);
+#pragma unroll
+            for (int k16 = 0; k16 < kDK / 16; ++k16)
+                mma_bf16(ps.tmem, dA + ((k16 * 4096) >> 4), dB + ((k16 * 4096) >> 4), idesc, k16 > 0);
             mma_commit(&ps.bar_mma);
         }
     }
-    // every thread: L of the chunk (each warp computes it for itself)
-    float Le, Lo;
-    chunk_log_gate(ps.alpha, lane, Le, Lo);
-    const int r = tid, t = r & (kC - 1);
-    const bool qrow = r < kC;
-    const float Lt = log_gate_at(Le, Lo, t);
-    // thread 0's copies and MMAs went through, and the MMAs completed
+    if (warp == 1) {
+        // L_t log2(e) of the chunk
+        float Le, Lo;
+        chunk_log_gate(ps.alpha, lane, Le, Lo);
+        ps.L2[2 * lane] = Le * 1.4426950408889634f;
+        ps.L2[2 * lane + 1] = Lo * 1.4426950408889634f;
+    }
+    // thread 0's copies and MMAs went through (and L is in shared memory)
     bool good = !named_sync_or<1, kPrepThreads>(tid == 0 && !ok);
     if (good) good = mbar_wait_bounded(&ps.bar_mma, 0);
     if (good) {
+        // row r of the product: P (rows 0..63) or A (rows 64..127) with the
+        // gate ratio e^{L_t - L_m} = 2^{(L_t - L_m) log2 e} and beta_m
         tc_fence_after_sync();
+        const int r = tid, t = r & (kC - 1);
+        const bool qrow = r < kC;
         float x[64];
-        const uint32_t ta = ps.tmem + ((uint32_t)(32 * warp) << 16);
-        tmem_load<64>(ta, x);
+        tmem_load<64>(ps.tmem + ((uint32_t)(32 * warp) << 16), x);
+        const float Lt = ps.L2[t];
         float *row = qrow ? ps.P[t] : ps.A[t];
 #pragma unroll
         for (int m4 = 0; m4 < kC / 4; ++m4) {
+            const float4 l4 = *reinterpret_cast<const float4 *>(&ps.L2[4 * m4]);
+            const float4 b4 = *reinterpret_cast<const float4 *>(&ps.beta[4 * m4]);
+            const float lm[4] = {l4.x, l4.y, l4.z, l4.w}, bm[4] = {b4.x, b4.y, b4.z, b4.w};
             float v[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int m = 4 * m4 + e;
-                const float Lm = log_gate_at(Le, Lo, m);
                 const bool keep = qrow ? (m <= t) : (m < t && a.delta);
-                v[e] = keep ? ps.beta[m] * x[m] * expf(Lt - Lm) : 0.0f;
+                v[e] = keep ? bm[e] * x[m] * exp2f(Lt - lm[e]) : 0.0f;
             }
             *reinterpret_cast<float4 *>(row + 4 * m4) = make_float4(v[0], v[1], v[2], v[3]);
         }
@@ -219,43 +281,66 @@ __global__ void __launch_bounds__(kPrepThreads) chunk_prep_kernel(
     }
     if (bad) return;
 
-    // column m of T = (I + A)^{-1} (forward substitution) and of PT = P T
-    if (tid < kC) {
-        const int m = tid;
-        float xc[kC];
+    unsigned char *wsb = reinterpret_cast<unsigned char *>(a.ws) + ((size_t)c * a.B * a.H + bh) * kWsChunkBytes;
+    // T, column by column (two threads per column), into X
+    {
+        const int m = tid >> 1;
+        solve_column(ps, X + m * kAStride, m, tid & 1);
+    }
+    named_sync<1, kPrepThreads>();
+    // PT = P T: column m, rows in blocks of 8; thread (m, half) takes the
+    // blocks {0, 3, 4, 7} or {1, 2, 5, 6} (equal work: P is lower triangular)
+    {
+        const int m = tid & (kC - 1), half = tid >> 6;
+        const float *Xm = X + m * kAStride;
+#pragma unroll 1
+        for (int k = 0; k < 4; ++k) {
+            const int blk = half ? (k == 0 ? 1 : k == 1 ? 2 : k == 2 ? 5 : 6)
+                                 : (k == 0 ? 0 : k == 1 ? 3 : k == 2 ? 4 : 7);
+            const int r0 = 8 * blk;
+            float acc[8];
 #pragma unroll
-        for (int i = 0; i < kC; ++i) {
-            const float *Ar = ps.A[i];
-            float s0 = 0.0f, s1 = 0.0f, s2 = 0.0f, s3 = 0.0f;
+            for (int r = 0; r < 8; ++r) acc[r] = 0.0f;
+#pragma unroll 1
+            for (int n = 0; n < r0 + 8; n += 4) {
+                const float4 xv = *reinterpret_cast<const float4 *>(Xm + n);
 #pragma unroll
-            for (int n = 0; n + 4 <= i; n += 4) {
-                const float4 a4 = *reinterpret_cast<const float4 *>(Ar + n);
-                s0 = fmaf(a4.x, xc[n], s0);
-                s1 = fmaf(a4.y, xc[n + 1], s1);
-                s2 = fmaf(a4.z, xc[n + 2], s2);
-                s3 = fmaf(a4.w, xc[n + 3], s3);
+                for (int r = 0; r < 8; ++r) {
+                    const float4 pv = *reinterpret_cast<const float4 *>(&ps.P[r0 + r][n]);
+                    acc[r] = fmaf(pv.x, xv.x, acc[r]);
+                    acc[r] = fmaf(pv.y, xv.y, acc[r]);
+                    acc[r] = fmaf(pv.z, xv.z, acc[r]);
+                    acc[r] = fmaf(pv.w, xv.w, acc[r]);
+                }
             }
+            // PT rows into the (no longer needed) A buffer, row-major
 #pragma unroll
-            for (int n = i & ~3; n < i; ++n) s0 = fmaf(Ar[n], xc[n], s0);
-            xc[i] = (i == m ? 1.0f : 0.0f) - ((s0 + s1) + (s2 + s3));
+            for (int r = 0; r < 8; ++r) ps.A[r0 + r][m] = acc[r];
         }
-        float *wsb = a.ws + ((size_t)c * a.B * a.H + bh) * kWsChunkFloats;
+    }
+    named_sync<1, kPrepThreads>();
+    // row r of [PT; T] (PT row r, or T row r - 64 read down column X[.][r - 64])
+    // as three BF16 parts in the operand layout; a warp writes 512 contiguous
+    // bytes per 8-column group and part
+    {
+        const int r = tid;
+        float x[kC];
+        if (r < kC) {
 #pragma unroll
-        for (int i = 0; i < kC; ++i) {
-            const float *Pr = ps.P[i];
-            float s0 = 0.0f, s1 = 0.0f, s2 = 0.0f, s3 = 0.0f;
+            for (int m = 0; m < kC; ++m) x[m] = ps.A[r][m];
+        } else {
 #pragma unroll
-            for (int n = 0; n + 4 <= i + 1; n += 4) {
-                const float4 p4 = *reinterpret_cast<const float4 *>(Pr + n);
-                s0 = fmaf(p4.x, xc[n], s0);
-                s1 = fmaf(p4.y, xc[n + 1], s1);
-                s2 = fmaf(p4.z, xc[n + 2], s2);
-                s3 = fmaf(p4.w, xc[n + 3], s3);
-            }
+            for (int m = 0; m < kC; ++m) x[m] = X[m * kAStride + (r - kC)];
+        }
 #pragma unroll
-            for (int n = (i + 1) & ~3; n <= i; ++n) s0 = fmaf(Pr[n], xc[n], s0);
-            wsb[(size_t)i * kC + m] = (s0 + s1) + (s2 + s3);   // PT row i
-            wsb[(size_t)(kC + i) * kC + m] = xc[i];             // T row i
+        for (int g = 0; g < kC / 8; ++g) {
+            uint32_t p0[4], p1[4], p2[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) split2_bf16x3(x[8 * g + 2 * e], x[8 * g + 2 * e + 1], p0[e], p1[e], p2[e]);
+            unsigned char *d = wsb + g * 2048 + 16 * r;
+            *reinterpret_cast<uint4 *>(d) = make_uint4(p0[0], p0[1], p0[2], p0[3]);
+            *reinterpret_cast<uint4 *>(d + kTPartBytes) = make_uint4(p1[0], p1[1], p1[2], p1[3]);
+            *reinterpret_cast<uint4 *>(d + 2 * kTPartBytes) = make_uint4(p2[0], p2[1], p2[2], p2[3]);
         }
     }
 }
@@ -264,16 +349,21 @@ __global__ void __launch_bounds__(kPrepThreads) chunk_prep_kernel(
 // Phase 2: the chunks of the pass in order, the state carried on the tensor core
 // ---------------------------------------------------------------------------
 
-constexpr int kEpiWarps = 4, kMmaWarp = 4, kLoadWarp = 5, kTWarp0 = 6, kTWarps = 4;
-constexpr int kScanThreads = (kEpiWarps + 2 + kTWarps) * 32;
+// 8 epilogue warps: warp w serves TMEM lane quarter w % 4 and the 32
+// accumulator columns 32 (w / 4) .. 32 (w / 4) + 31 (value rows of the slice).
+// Warp 8 issues the MMAs, warp 9 loads the chunk inputs, lane 0 of warp 10
+// brings each chunk's [PT; T] operand in with bulk copies.
+constexpr int kEpiWarps = 8, kMmaWarp = 8, kLoadWarp = 9, kTWarp = 10;
+constexpr int kScanThreads = (kEpiWarps + 3) * 32;
+constexpr int kHalf = kDVS / 2;  // accumulator columns per epilogue thread
 
 // TMEM columns (256 allocated): the three accumulators
 constexpr uint32_t kColX = 0, kColOU = 64, kColS = 128;
 
 struct ScanBars {
-    uint64_t full[2], empty[2];      // input stages (TMA + cp.async)
-    uint64_t t_full, t_empty;        // [PT; T] operand in shared memory
-    uint64_t x_done, ou_done, s_done;  // MMA completions
+    uint64_t full[2], empty[2];          // input stages (TMA + cp.async)
+    uint64_t t_full, t_empty;            // [PT; T] operand in shared memory (bulk copies)
+    uint64_t x_done, ou_done, s_done;    // MMA completions
     uint64_t r_ready, u_ready, s_ready;  // operands written by the epilogue
     uint32_t tmem;
 };
@@ -286,7 +376,8 @@ __host__ __device__ constexpr ScanLayout scan_layout() {
     ScanLayout L{};
     L.bars = 0;
     L.qk = 1024;                          // [2][32 KB]
-    L.v = L.qk + 2 * kQKBytes;            // [2][8 KB] V slice, row-major [64 t][64 i]
+    L.v = L.qk + 2 * kQKBytes;            // [2][8 KB] V slice, [64 t][64 i], 128-byte swizzle
+                                          // (1024-byte aligned)
     L.ab = L.v + 2 * kVBytes;             // [2][alpha 64, beta 64]
     L.s3 = L.ab + 2 * 512;                // [3][16 KB] S^T split (MN-major B of the X product)
     L.ru = L.s3 + 3 * 16384;              // [3][8 KB] R, then U^ (MN-major B, BF16 parts)
@@ -295,10 +386,31 @@ __host__ __device__ constexpr ScanLayout scan_layout() {
     return L;
 }
 
+// Writes values x[8 g' .. 8 g' + 7] (g' = 0..N/8-1) as three BF16 parts: the
+// 16-byte word of each part at dst + part * part_bytes + (g0 + g') * stride.
+template <int N>
+__device__ __forceinline__ void store_parts(unsigned char *dst, const float (&x)[N], float scale,
+                                            int g0, int stride, int part_bytes) {
+#pragma unroll
+    for (int g = 0; g < N / 8; ++g) {
+        uint32_t a[4], b[4], c[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            split2_bf16x3(scale * x[8 * g + 2 * e], scale * x[8 * g + 2 * e + 1], a[e], b[e], c[e]);
+        unsigned char *d = dst + (g0 + g) * stride;
+        *reinterpret_cast<uint4 *>(d) = make_uint4(a[0], a[1], a[2], a[3]);
+        *reinterpret_cast<uint4 *>(d + part_bytes) = make_uint4(b[0], b[1], b[2], b[3]);
+        *reinterpret_cast<uint4 *>(d + 2 * part_bytes) = make_uint4(c[0], c[1], c[2], c[3]);
+    }
+}
+
 __global__ void __launch_bounds__(kScanThreads, 1) chunk_scan_kernel(
     const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
     const __grid_constant__ CUtensorMap vmap, const ChunkArgs a) {
-    extern __shared__ __align__(128) unsigned char smem[];
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    // the swizzled V tiles need 1024-byte aligned addresses: align the base
+    // (the launch reserves 1 KB for it)
+    unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     constexpr ScanLayout SL = scan_layout();
     ScanBars &sb = *reinterpret_cast<ScanBars *>(smem + SL.bars);
     unsigned char *qkbuf = smem + SL.qk;
@@ -316,16 +428,16 @@ __global__ void __launch_bounds__(kScanThreads, 1) chunk_scan_kernel(
 
     if (tid == 0) {
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&sb.full[s], 1);
+            mbar_init(&sb.full[s], 33);  // 32 loader lanes' gate copies + the TMA arrival
             mbar_init(&sb.empty[s], kEpiWarps);
         }
-        mbar_init(&sb.t_full, kTWarps);
+        mbar_init(&sb.t_full, 1);
         mbar_init(&sb.t_empty, 1);
         mbar_init(&sb.x_done, 1);
         mbar_init(&sb.ou_done, 1);
         mbar_init(&sb.s_done, 1);
-        mbar_init(&sb.r_ready, 2);
-        mbar_init(&sb.u_ready, 2);
+        mbar_init(&sb.r_ready, 4);
+        mbar_init(&sb.u_ready, 4);
         mbar_init(&sb.s_ready, kEpiWarps);
     }
     if (warp == kMmaWarp) tmem_alloc(&sb.tmem, 256);
@@ -336,127 +448,111 @@ __global__ void __launch_bounds__(kScanThreads, 1) chunk_scan_kernel(
 
     if (warp == kLoadWarp) {
         // ---------------------------------------------------------- loader
-        if (lane == 0) {
-            int c = 0;
-            for (; c < nc; ++c) {
-                const int s = c & 1;
-                if (c >= 2 && !mbar_wait_bounded(&sb.empty[s], ((c >> 1) - 1) & 1)) break;
-                const int tok0 = b * a.T_total + a.t0 + c * kC;
-                float *ab = abbuf + s * 128;
-                for (int t = 0; t < kC; ++t) {
-                    cp_async4(ab + t, a.alpha + ((size_t)tok0 + t) * a.H + h);
-                    cp_async4(ab + kC + t, a.beta + ((size_t)tok0 + t) * a.H + h);
-                }
-                cp_async_mbar_arrive(&sb.full[s]);
+        int c = 0;
+        for (; c < nc; ++c) {
+            const int s = c & 1;
+            if (c >= 2 && !mbar_wait_bounded(&sb.empty[s], ((c >> 1) - 1) & 1)) break;
+            const int tok0 = b * a.T_total + a.t0 + c * kC;
+            float *ab = abbuf + s * 128;
+            // gates: lane l copies tokens l and l + 32 of alpha and beta
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int t = lane + 32 * u;
+                cp_async4(ab + t, a.alpha + ((size_t)tok0 + t) * a.H + h);
+                cp_async4(ab + kC + t, a.beta + ((size_t)tok0 + t) * a.H + h);
+            }
+            asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(&sb.full[s]))
+                         : "memory");
+            if (lane == 0) {
                 mbar_arrive_expect_tx(&sb.full[s], kQKBytes + kVBytes);
                 load_qk(qkbuf + s * kQKBytes, &qmap, &kmap, h, tok0, &sb.full[s]);
                 tma_load_3d(vbuf + s * kVBytes, &vmap, i0, h, tok0, &sb.full[s]);
             }
-            // drain copies still in flight into this CTA (after an expired wait)
-            for (int j = c - 1; j >= 0 && j >= c - 2; --j) mbar_wait_bounded(&sb.full[j & 1], (j >> 1) & 1);
         }
+        // drain copies still in flight into this CTA (after an expired wait)
+        for (int j = c - 1; j >= 0 && j >= c - 2; --j) mbar_wait_bounded(&sb.full[j & 1], (j >> 1) & 1);
     } else if (warp == kMmaWarp) {
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0) {
             constexpr uint32_t idx = idesc_bf16(128, kDVS, false, true);
-            constexpr uint32_t idt = idesc_bf16(128, kDVS, false, true);
             constexpr uint32_t ids = idesc_bf16(128, kDVS, true, true);
+            // descriptors at offset 0; an operand offset of o bytes adds o >> 4
+            const uint64_t dS = smem_desc(smem_u32(s3), 128, 2048);     // S^T parts (MN-major B)
+            const uint64_t dT = smem_desc(smem_u32(tt), 2048, 128);     // [PT; T] parts (K-major A)
+            const uint64_t dR = smem_desc(smem_u32(ru), 128, 1024);     // R / U^ parts (MN-major B)
             for (int c = 0; c < nc; ++c) {
                 const int s = c & 1, ph = c & 1;
                 if (!mbar_wait_bounded(&sb.full[s], (c >> 1) & 1)) break;
                 if (!mbar_wait_bounded(&sb.s_ready, ph)) break;
                 tc_fence_after_sync();
-                const unsigned char *qk = qkbuf + s * kQKBytes;
+                const uint64_t dQK = smem_desc(smem_u32(qkbuf + s * kQKBytes), 2048, 128);
+                const uint64_t dKT = smem_desc(smem_u32(qkbuf + s * kQKBytes + 1024), 128, 2048);
                 // X = [Q; K] S^T, S = s0 + s1 + s2 (smallest part first)
-                bool acc = false;
+#pragma unroll
                 for (int k16 = 0; k16 < kDK / 16; ++k16)
-                    for (int p = 2; p >= 0; --p) {
-                        const uint64_t bd = smem_desc(smem_u32(s3 + p * 16384 + k16 * 256), 128, 2048);
-                        mma_bf16(tm + kColX, desc_qk(qk, k16), bd, idx, acc);
-                        acc = true;
-                    }
+#pragma unroll
+                    for (int p = 2; p >= 0; --p)
+                        mma_bf16(tm + kColX, dQK + ((k16 * 4096) >> 4), dS + ((p * 16384 + k16 * 256) >> 4),
+                                 idx, k16 > 0 || p < 2);
                 mma_commit(&sb.x_done);
                 if (!mbar_wait_bounded(&sb.r_ready, ph)) break;
                 if (!mbar_wait_bounded(&sb.t_full, ph)) break;
                 tc_fence_after_sync();
                 // [O_intra; U] = [PT; T] R: parts (p, q) with p + q <= 2, smallest first
-                acc = false;
+#pragma unroll
                 for (int k16 = 0; k16 < kC / 16; ++k16)
+#pragma unroll
                     for (int n = 0; n < 6; ++n) {
                         constexpr int kP[6] = {2, 1, 0, 1, 0, 0}, kQ[6] = {0, 1, 2, 0, 1, 0};
-                        const uint64_t ad = smem_desc(smem_u32(tt + kP[n] * 16384 + k16 * 4096), 2048, 128);
-                        const uint64_t bd = smem_desc(smem_u32(ru + kQ[n] * 8192 + k16 * 256), 128, 1024);
-                        mma_bf16(tm + kColOU, ad, bd, idt, acc);
-                        acc = true;
+                        mma_bf16(tm + kColOU, dT + ((kP[n] * 16384 + k16 * 4096) >> 4),
+                                 dR + ((kQ[n] * 8192 + k16 * 256) >> 4), idx, k16 > 0 || n > 0);
                     }
                 mma_commit(&sb.ou_done);
                 mma_commit(&sb.t_empty);
                 if (!mbar_wait_bounded(&sb.u_ready, ph)) break;
                 tc_fence_after_sync();
                 // D_S = K^T U^, U^ = u0 + u1 + u2
-                acc = false;
+#pragma unroll
                 for (int k16 = 0; k16 < kC / 16; ++k16)
-                    for (int p = 2; p >= 0; --p) {
-                        const uint64_t bd = smem_desc(smem_u32(ru + p * 8192 + k16 * 256), 128, 1024);
-                        mma_bf16(tm + kColS, desc_kt_mn(qk, k16), bd, ids, acc);
-                        acc = true;
-                    }
+#pragma unroll
+                    for (int p = 2; p >= 0; --p)
+                        mma_bf16(tm + kColS, dKT + ((k16 * 256) >> 4), dR + ((p * 8192 + k16 * 256) >> 4), ids,
+                                 k16 > 0 || p < 2);
                 mma_commit(&sb.s_done);
             }
         }
-    } else if (warp >= kTWarp0) {
+    } else if (warp == kTWarp) {
         // ---------------------------------------------------------- [PT; T] operand
-        // row r of [PT; T] as three BF16 parts, K-major (element (r, m) of a
-        // part at byte (m / 8) * 2048 + 16 r + 2 (m % 8))
-        const int r = tid - kTWarp0 * 32;
-        for (int c = 0; c < nc; ++c) {
-            const float *src = a.ws + ((size_t)c * a.B * a.H + bh) * kWsChunkFloats + (size_t)r * kC;
-            float x[kC];
-#pragma unroll
-            for (int q = 0; q < kC / 4; ++q) {
-                const float4 v = __ldcg(reinterpret_cast<const float4 *>(src) + q);
-                x[4 * q] = v.x, x[4 * q + 1] = v.y, x[4 * q + 2] = v.z, x[4 * q + 3] = v.w;
+        // the chunk's three BF16 parts, already in the operand layout in the
+        // workspace, by bulk copies once the previous chunk's MMAs read them
+        if (lane == 0) {
+            int c = 0;
+            for (; c < nc; ++c) {
+                if (c >= 1 && !mbar_wait_bounded(&sb.t_empty, (c - 1) & 1)) break;
+                const unsigned char *src =
+                    reinterpret_cast<const unsigned char *>(a.ws) + ((size_t)c * a.B * a.H + bh) * kWsChunkBytes;
+                mbar_arrive_expect_tx(&sb.t_full, kWsChunkBytes);
+                for (int p = 0; p < 3; ++p) bulk_g2s(tt + p * kTPartBytes, src + p * kTPartBytes, kTPartBytes, &sb.t_full);
             }
-            if (c >= 1 && !mbar_wait_bounded(&sb.t_empty, (c - 1) & 1)) break;
-#pragma unroll
-            for (int g = 0; g < kC / 8; ++g) {
-                __align__(16) __nv_bfloat16 p0[8], p1[8], p2[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) split_bf16x3(x[8 * g + e], p0[e], p1[e], p2[e]);
-                const int off = g * 2048 + 16 * r;
-                *reinterpret_cast<uint4 *>(tt + off) = *reinterpret_cast<const uint4 *>(p0);
-                *reinterpret_cast<uint4 *>(tt + 16384 + off) = *reinterpret_cast<const uint4 *>(p1);
-                *reinterpret_cast<uint4 *>(tt + 32768 + off) = *reinterpret_cast<const uint4 *>(p2);
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sb.t_full);
+            if (c > 0) mbar_wait_bounded(&sb.t_full, (c - 1) & 1);  // drain (after an expired wait)
         }
     } else {
-        // ---------------------------------------------------------- epilogue (warps 0..3)
-        const int r = tid;                 // TMEM lane
+        // ---------------------------------------------------------- epilogue (warps 0..7)
+        const int qtr = warp & 3, hf = warp >> 2;
+        const int r = 32 * qtr + lane;     // TMEM lane (row of the accumulators)
         const int t = r & (kC - 1);        // token of this row (rows 0..63 Q / O, 64..127 K / U)
-        const uint32_t ta = tm + ((uint32_t)(32 * warp) << 16);
-        float S[kDVS];                     // S[i0 + i][j = r], the state slice's column r
+        const int c0 = hf * kHalf;         // this thread's accumulator columns c0 .. c0 + 31
+        const uint32_t ta = tm + ((uint32_t)(32 * qtr) << 16) + c0;
+        float S[kHalf];                    // S[i0 + c0 + i][j = r], i = 0..31
         {
-            const float *Sg = a.S + ((size_t)bh * a.DV + i0) * kDK + r;
+            const float *Sg = a.S + ((size_t)bh * a.DV + i0 + c0) * kDK + r;
 #pragma unroll
-            for (int i = 0; i < kDVS; ++i) S[i] = Sg[(size_t)i * kDK];
+            for (int i = 0; i < kHalf; ++i) S[i] = Sg[(size_t)i * kDK];
         }
-        // write S^T (MN-major, N = value row i, K = key channel j = r) in three BF16 parts
+        // S^T (MN-major B: N = value row i, K = key channel j = r), three BF16 parts
         auto write_s3 = [&]() {
-#pragma unroll
-            for (int g = 0; g < kDVS / 8; ++g) {
-                __align__(16) __nv_bfloat16 p0[8], p1[8], p2[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) split_bf16x3(S[8 * g + e], p0[e], p1[e], p2[e]);
-                const int off = g * 2048 + 16 * r;
-                *reinterpret_cast<uint4 *>(s3 + off) = *reinterpret_cast<const uint4 *>(p0);
-                *reinterpret_cast<uint4 *>(s3 + 16384 + off) = *reinterpret_cast<const uint4 *>(p1);
-                *reinterpret_cast<uint4 *>(s3 + 32768 + off) = *reinterpret_cast<const uint4 *>(p2);
-            }
+            store_parts(s3 + 16 * r, S, 1.0f, c0 / 8, 2048, 16384);
             fence_proxy_async_smem();
-            tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sb.s_ready);
         };
@@ -475,31 +571,23 @@ __global__ void __launch_bounds__(kScanThreads, 1) chunk_scan_kernel(
             tc_fence_after_sync();
             if (r >= kC) {
                 // R_t = v_t - e^{L_t} (S_0 k_t) (or v_t when delta = 0), three BF16 parts
-                float xk[kDVS];
-                tmem_load<64>(ta + kColX, xk);
-                const __nv_bfloat16 *vr = reinterpret_cast<const __nv_bfloat16 *>(vbuf + s * kVBytes) + t * kDVS;
+                float xk[kHalf];
+                tmem_load<32>(ta + kColX, xk);
+                const unsigned char *vr = vbuf + s * kVBytes + t * 128;
 #pragma unroll
-                for (int q = 0; q < kDVS / 8; ++q) {
-                    // rotate the 16-byte reads so that a quarter-warp hits distinct banks
-                    const int qq = (q + t) & (kDVS / 8 - 1);
-                    const uint4 w = *reinterpret_cast<const uint4 *>(vr + 8 * qq);
-                    const __nv_bfloat16 *vv = reinterpret_cast<const __nv_bfloat16 *>(&w);
+                for (int q = 0; q < 4; ++q) {
+                    // the V tile is stored with the 128-byte swizzle: 16-byte
+                    // chunk k of row t sits at chunk k ^ (t % 8), so the eight
+                    // rows a quarter-warp reads hit distinct banks
+                    const uint4 w = *reinterpret_cast<const uint4 *>(vr + 16 * ((c0 / 8 + q) ^ (t & 7)));
+                    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        const float v = __bfloat162float(vv[e]);
-                        xk[8 * qq + e] = a.delta ? v - eLt * xk[8 * qq + e] : v;
+                        const float v = __uint_as_float((e & 1) ? (ww[e / 2] & 0xFFFF0000u) : (ww[e / 2] << 16));
+                        xk[8 * q + e] = a.delta ? fmaf(-eLt, xk[8 * q + e], v) : v;
                     }
                 }
-#pragma unroll
-                for (int g = 0; g < kDVS / 8; ++g) {
-                    __align__(16) __nv_bfloat16 p0[8], p1[8], p2[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) split_bf16x3(xk[8 * g + e], p0[e], p1[e], p2[e]);
-                    const int off = g * 1024 + 16 * t;
-                    *reinterpret_cast<uint4 *>(ru + off) = *reinterpret_cast<const uint4 *>(p0);
-                    *reinterpret_cast<uint4 *>(ru + 8192 + off) = *reinterpret_cast<const uint4 *>(p1);
-                    *reinterpret_cast<uint4 *>(ru + 16384 + off) = *reinterpret_cast<const uint4 *>(p2);
-                }
+                store_parts(ru + 16 * t, xk, 1.0f, c0 / 8, 1024, 8192);
                 fence_proxy_async_smem();
                 tc_fence_before_sync();
                 __syncwarp();
@@ -508,37 +596,28 @@ __global__ void __launch_bounds__(kScanThreads, 1) chunk_scan_kernel(
             if (!mbar_wait_bounded(&sb.ou_done, ph)) { ok = false; break; }
             tc_fence_after_sync();
             if (r < kC) {
-                // o_t = e^{L_t} (S_0 q_t) + O_intra_t, 32 value rows at a time
+                // o_t = e^{L_t} (S_0 q_t) + O_intra_t
+                float xq[kHalf], oi[kHalf];
+                tmem_load<32>(ta + kColX, xq);
+                tmem_load<32>(ta + kColOU, oi);
                 __nv_bfloat16 *og = static_cast<__nv_bfloat16 *>(a.o) +
-                                    (((size_t)b * a.T_total + a.t0 + c * kC + t) * a.H + h) * a.DV + i0;
+                                    (((size_t)b * a.T_total + a.t0 + c * kC + t) * a.H + h) * a.DV + i0 + c0;
 #pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    float xq[32], oi[32];
-                    tmem_load<32>(ta + kColX + 32 * hf, xq);
-                    tmem_load<32>(ta + kColOU + 32 * hf, oi);
+                for (int q = 0; q < kHalf / 8; ++q) {
+                    uint32_t w[4];
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        __align__(16) __nv_bfloat16 ob[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) ob[e] = __float2bfloat16_rn(fmaf(eLt, xq[8 * q + e], oi[8 * q + e]));
-                        *reinterpret_cast<uint4 *>(og + 32 * hf + 8 * q) = *reinterpret_cast<const uint4 *>(ob);
+                    for (int e = 0; e < 4; ++e) {
+                        const __nv_bfloat162 p = __floats2bfloat162_rn(fmaf(eLt, xq[8 * q + 2 * e], oi[8 * q + 2 * e]),
+                                                                       fmaf(eLt, xq[8 * q + 2 * e + 1], oi[8 * q + 2 * e + 1]));
+                        w[e] = *reinterpret_cast<const uint32_t *>(&p);
                     }
+                    *reinterpret_cast<uint4 *>(og + 8 * q) = make_uint4(w[0], w[1], w[2], w[3]);
                 }
             } else {
                 // U^_t = beta_t e^{L_C - L_t} u_t in three BF16 parts (MN-major B of K^T U^)
-                float u[kDVS];
-                tmem_load<64>(ta + kColOU, u);
-                const float gam = be[t] * expf(LC - Lt);
-#pragma unroll
-                for (int g = 0; g < kDVS / 8; ++g) {
-                    __align__(16) __nv_bfloat16 p0[8], p1[8], p2[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) split_bf16x3(gam * u[8 * g + e], p0[e], p1[e], p2[e]);
-                    const int off = g * 1024 + 16 * t;
-                    *reinterpret_cast<uint4 *>(ru + off) = *reinterpret_cast<const uint4 *>(p0);
-                    *reinterpret_cast<uint4 *>(ru + 8192 + off) = *reinterpret_cast<const uint4 *>(p1);
-                    *reinterpret_cast<uint4 *>(ru + 16384 + off) = *reinterpret_cast<const uint4 *>(p2);
-                }
+                float u[kHalf];
+                tmem_load<32>(ta + kColOU, u);
+                store_parts(ru + 16 * t, u, be[t] * expf(LC - Lt), c0 / 8, 1024, 8192);
                 fence_proxy_async_smem();
                 tc_fence_before_sync();
                 __syncwarp();
@@ -548,20 +627,21 @@ __global__ void __launch_bounds__(kScanThreads, 1) chunk_scan_kernel(
             tc_fence_after_sync();
             {
                 // S_C = e^{L_C} S_0 + (U^ ^T K)^T, column r of the slice
-                float ds[kDVS];
-                tmem_load<64>(ta + kColS, ds);
+                float ds[kHalf];
+                tmem_load<32>(ta + kColS, ds);
                 const float eLC = expf(LC);
 #pragma unroll
-                for (int i = 0; i < kDVS; ++i) S[i] = fmaf(eLC, S[i], ds[i]);
+                for (int i = 0; i < kHalf; ++i) S[i] = fmaf(eLC, S[i], ds[i]);
             }
+            tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sb.empty[s]);
             if (c + 1 < nc) write_s3();
         }
         if (ok) {
-            float *Sg = a.S + ((size_t)bh * a.DV + i0) * kDK + r;
+            float *Sg = a.S + ((size_t)bh * a.DV + i0 + c0) * kDK + r;
 #pragma unroll
-            for (int i = 0; i < kDVS; ++i) Sg[(size_t)i * kDK] = S[i];
+            for (int i = 0; i < kHalf; ++i) Sg[(size_t)i * kDK] = S[i];
         }
     }
     tc_fence_before_sync();
@@ -589,8 +669,10 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
 }
 
-// A 3-D map of a BF16 activation [B*T, H, D] (innermost D): box {box_d, 1, 64}.
-bool activation_map(CUtensorMap *m, const void *base, int D, int H, long long BT, int box_d) {
+// A 3-D map of a BF16 activation [B*T, H, D] (innermost D): box {box_d, 1, 64};
+// swizzle128 stores each 128-byte box row with the 128-byte swizzle.
+bool activation_map(CUtensorMap *m, const void *base, int D, int H, long long BT, int box_d,
+                    bool swizzle128 = false) {
     PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
     if (!enc) return false;
     const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)BT};
@@ -598,14 +680,15 @@ bool activation_map(CUtensorMap *m, const void *base, int D, int H, long long BT
     const cuuint32_t box[3] = {(cuuint32_t)box_d, 1, (cuuint32_t)kC};
     const cuuint32_t es[3] = {1, 1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_INTERLEAVE_NONE,
+               swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
 
 size_t chunk_workspace_bytes(int BH, int chunks) {
-    return (size_t)chunks * BH * kWsChunkFloats * sizeof(float);
+    return (size_t)chunks * BH * kWsChunkBytes;
 }
 
 bool chunk_path_supported(int d_k, int d_v, int gate, bool bf16) {
@@ -625,20 +708,20 @@ cudaError_t launch_prefill_chunks(const ChunkArgs &a, const void *q, const void 
                                  prep_smem_bytes());
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(chunk_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     scan_layout().bytes);
+                                     scan_layout().bytes + 1024);
         if (e != cudaSuccess) return e;
         configured.fetch_or(bit, std::memory_order_acq_rel);
     }
     const long long BT = (long long)a.B * a.T_total;
     CUtensorMap qm, km, vm;
     if (!activation_map(&qm, q, kDK, a.H, BT, 8) || !activation_map(&km, k, kDK, a.H, BT, 8) ||
-        !activation_map(&vm, v, a.DV, a.H, BT, kDVS))
+        !activation_map(&vm, v, a.DV, a.H, BT, kDVS, true))
         return cudaErrorInvalidValue;
     const int BH = a.B * a.H;
     chunk_prep_kernel<<<a.nc * BH, kPrepThreads, prep_smem_bytes(), stream>>>(qm, km, a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    chunk_scan_kernel<<<BH * (a.DV / kDVS), kScanThreads, scan_layout().bytes, stream>>>(qm, km, vm, a);
+    chunk_scan_kernel<<<BH * (a.DV / kDVS), kScanThreads, scan_layout().bytes + 1024, stream>>>(qm, km, vm, a);
     return cudaGetLastError();
 }
 

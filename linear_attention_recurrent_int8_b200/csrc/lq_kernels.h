@@ -87,7 +87,8 @@ struct ChunkArgs {
     const float *alpha;  // [B][T_total][H]
     const float *beta;   // [B][T_total][H]
     void *o;             // BF16 [B][T_total][H][DV]
-    float *ws;           // workspace [nc][BH][128][64] FP32 ([PT; T] of each chunk)
+    float *ws;           // workspace [nc][BH] blocks of 48 KB ([PT; T] of each chunk as
+                         // three BF16 parts in the tensor-core operand layout)
     int B, H, DV, T_total, t0, nc, delta;
 };
 

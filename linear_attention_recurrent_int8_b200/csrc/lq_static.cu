@@ -7,7 +7,7 @@
 // framework calls with input and output buffers and nothing else; code that
 // must not call cudaMalloc because a cudaMalloc can synchronize the device
 // and stall the other work on it.  For them this entry point takes the chunked
-// prefill's scratch ([PT; T] of every chunk of a pass, 32 KB per chunk and
+// prefill's scratch ([PT; T] of every chunk of a pass, 48 KB per chunk and
 // head) from g_prefill_scratch below, a file-scope array of
 // kStaticScratchBytes that every GPU which loads the library holds until the
 // process exits.  It allocates nothing: no cudaMalloc, no cudaFree, no

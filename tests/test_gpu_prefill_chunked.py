@@ -17,7 +17,7 @@ from lqtest import (compare_outputs, compare_snapshots, download_snapshot, heads
 
 pytestmark = pytest.mark.gpu
 
-CHUNK_BYTES = 128 * 64 * 4  # [PT; T] of one chunk and head
+CHUNK_BYTES = 3 * 128 * 64 * 2  # [PT; T] of one chunk and head, three BF16 parts
 
 
 def _run(B, H, dv, T, every, r, ws_chunks, delta=1, seed=0):

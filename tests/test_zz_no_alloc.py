@@ -56,9 +56,10 @@ def test_noalloc_prefill_matches_workspace_prefill_twice(B, H, dv, T, every):
 
 
 def test_noalloc_prefill_rejects_more_heads_than_its_array_holds():
-    cfg = lq.Config(batch=257, heads=1, d_k=128, d_v=64, window=16, n_comp=0, gate=lq.LQ_GATE_SCALAR,
+    """One chunk of scratch is 48 KB per sequence and head: 8 MiB holds 170."""
+    cfg = lq.Config(batch=171, heads=1, d_k=128, d_v=64, window=16, n_comp=0, gate=lq.LQ_GATE_SCALAR,
                     io_dtype=lq.LQ_BF16)
-    tok = synth.tokens(0, np.arange(257), np.arange(1), 0, 64, 128, 64, "scalar", "bf16")
+    tok = synth.tokens(0, np.arange(171), np.arange(1), 0, 64, 128, 64, "scalar", "bf16")
     with pytest.raises(lq.LQError) as e:
         _prefill(lq.lq_prefill_chunk_noalloc, cfg, tok, 64, 64)
     assert e.value.status == lq.LQ_ERR_UNSUPPORTED
