@@ -324,12 +324,12 @@ def synth_workload(name):
 def workload_config(wl, args):
     return {
         "workload": (f"{wl.name}: {'KDA per-channel' if wl.gate == 'diag' else 'GDN scalar'}-gate "
-                     f"decode, batch {wl.batch} x {wl.heads} heads, d_k={wl.d_k}, d_v={wl.d_v}, "
+                     f"{'' if wl.delta else 'b = 0 (no delta rule) '}decode, batch {wl.batch} x {wl.heads} heads, d_k={wl.d_k}, d_v={wl.d_v}, "
                      f"window W={wl.window}, r={wl.n_comp} compensators, {wl.io} q/k/v/o, "
                      f"{state_words(args.bits)} state with per-row scales"),
         "batch_per_gpu": wl.batch, "heads": wl.heads, "d_k": wl.d_k, "d_v": wl.d_v,
         "window": wl.window, "n_comp": wl.n_comp, "gate": wl.gate, "io": wl.io,
-        "smoothing": bool(wl.smoothing), "bits": args.bits,
+        "smoothing": bool(wl.smoothing), "bits": args.bits, "delta": wl.delta,
         "state": f"{state_words(args.bits)} + fp32 row scales",
         "step": f"one window: {wl.window} decode launches and the window commit",
         "tokens_per_step_per_gpu": wl.batch * wl.window,
@@ -373,7 +373,7 @@ def run_lq(args, wl):
     cfg = lq.Config(batch=wl.batch, heads=wl.heads, d_k=wl.d_k, d_v=wl.d_v, window=wl.window,
                     n_comp=wl.n_comp, gate=lq.LQ_GATE_DIAG if wl.gate == "diag" else lq.LQ_GATE_SCALAR,
                     io_dtype=lq.LQ_BF16 if wl.io == "bf16" else lq.LQ_F32,
-                    smoothing=int(wl.smoothing), auto_commit=0, bits=args.bits)
+                    smoothing=int(wl.smoothing), auto_commit=0, delta=wl.delta, bits=args.bits)
     W = wl.window
     e = 2 if wl.io == "bf16" else 4
     st = lq.State(cfg, dev)
@@ -908,6 +908,8 @@ def main(argv=None):
     ap.add_argument("--window", type=int, default=None, help="override W (comparators / sweep)")
     ap.add_argument("--n-comp", type=int, default=None, help="override r")
     ap.add_argument("--no-smoothing", action="store_true")
+    ap.add_argument("--delta", type=int, choices=[0, 1], default=None,
+                    help="0: the b = 0 rows of equation 1 (linear attention / Mamba2 / GLA)")
     ap.add_argument("--bits", type=int, choices=[8, 6, 4, 16], default=8,
                     help="code width of the state (8; 6 and 4 are the narrow variants; 16 = BF16)")
     ap.add_argument("--slots", type=int, default=8, help="distinct input windows (graphs)")
@@ -931,6 +933,8 @@ def main(argv=None):
         over["n_comp"] = args.n_comp
     if args.no_smoothing:
         over["smoothing"] = False
+    if args.delta is not None:
+        over["delta"] = args.delta
     if over:
         wl = dataclasses.replace(wl, **over)
 

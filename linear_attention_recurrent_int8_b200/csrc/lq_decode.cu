@@ -37,7 +37,8 @@
 //    forms S^_0 x for its rows (dp4a of the codes with the limbs, FP32
 //    combine, transposing warp reduction), then u_t and o_t for the same rows
 //    from the coefficients and its own buffered u.  No CTA barrier is needed
-//    per head; the consumers release the stage through "empty".
+//    per head; the consumers release the stage through "empty".  With b = 0
+//    (delta = 0) the x_k side is neither split nor multiplied.
 // The window commit is a separate kernel (lq_commit.cu).
 // Every wait is bounded (lq_common.cuh); a wait that expires sets the device
 // error word and the waiting warp stops.
@@ -336,7 +337,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a,
                         store_vec<CPL>(xs + DK + j0, xq);
                         if (lane == 0) lscale[0] = lscale[1] = 1.0f;
                     } else {
-                        split_limbs<CPL, 3>(xk, limb, DK, lscale, j0);
+                        // b = 0 rows: the consumers skip x_k, so it is not split
+                        if (a.delta) split_limbs<CPL, 3>(xk, limb, DK, lscale, j0);
                         split_limbs<CPL, 3>(xq, limb + 3 * DK, DK, lscale + 1, j0);
                     }
                     kq = group_sum<32>(kq);
@@ -436,6 +438,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a,
     const int src_k = (rloc % RPI16) * LPR16 + transposed_owner<2 * NRM, LPR16>(rloc / RPI16);
     const int src_q = (rloc % RPI16) * LPR16 + transposed_owner<2 * NRM, LPR16>(NRM + rloc / RPI16);
 
+    const bool delta = a.delta != 0;  // b = 0 rows (delta = 0): no S^_0 x_k products
     int i = 0;
     for (int bh = next_decode_head<RAGGED>(a, blockIdx.x); bh < BH; bh = next_decode_head<RAGGED>(a, bh + gridDim.x), ++i) {
         const int s = i % S;
@@ -495,8 +498,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a,
                         // element 2i in the low half of word i, 2i+1 in the high half
                         const float lo = __uint_as_float(ww[i] << 16);
                         const float hi = __uint_as_float(ww[i] & 0xFFFF0000u);
-                        ak = fmaf(lo, xk[2 * i], ak);
-                        ak = fmaf(hi, xk[2 * i + 1], ak);
+                        if (delta) {
+                            ak = fmaf(lo, xk[2 * i], ak);
+                            ak = fmaf(hi, xk[2 * i + 1], ak);
+                        }
                         aq = fmaf(lo, xq[2 * i], aq);
                         aq = fmaf(hi, xq[2 * i + 1], aq);
                     }
@@ -509,7 +514,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a,
                 uint4 lw[6];
 #pragma unroll
                 for (int v = 0; v < 6; ++v)
-                    lw[v] = *reinterpret_cast<const uint4 *>(limb + v * DK + 16 * cc);
+                    lw[v] = (v < 3 && !delta) ? make_uint4(0u, 0u, 0u, 0u)
+                                              : *reinterpret_cast<const uint4 *>(limb + v * DK + 16 * cc);
                 float vals[2 * NRM];
 #pragma unroll
                 for (int n = 0; n < NRM; ++n) {
@@ -527,6 +533,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a,
                     int acc[6];
 #pragma unroll
                     for (int v = 0; v < 6; ++v) {
+                        if (v < 3 && !delta) {  // warp-uniform: the b-side sums are 0
+                            acc[v] = 0;
+                            continue;
+                        }
                         int x = __dp4a((int)w.x, (int)lw[v].x, 0);
                         x = __dp4a((int)w.y, (int)lw[v].y, x);
                         x = __dp4a((int)w.z, (int)lw[v].z, x);
@@ -544,7 +554,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a,
                 const float sg = sig_s[row];
                 // 2^-18 (4-bit codes enter as 16 Q), 2^-14, or 1 (FP32 sums of a BF16 residual)
                 constexpr float kUnit = PACK4 ? 3.814697265625e-06f : BF16S ? 1.0f : 6.103515625e-05f;
-                const float yk = __shfl_sync(0xffffffffu, y, src_k) * (sg * (lscale[0] * kUnit));
+                const float yk = delta ? __shfl_sync(0xffffffffu, y, src_k) * (sg * (lscale[0] * kUnit)) : 0.0f;
                 const float yq = __shfl_sync(0xffffffffu, y, src_q) * (sg * (lscale[1] * kUnit));
                 float hb = part == 0 ? yk : 0.0f, p = part == 0 ? yq : 0.0f;
                 for (int m = part; m < nrec; m += LPRD) {
