@@ -91,13 +91,6 @@ __device__ __forceinline__ uint64_t desc_qk(const unsigned char *qk, int k16) {
     return smem_desc(smem_u32(qk + k16 * 4096), 2048, 128);
 }
 
-// The chunk's K rows read as an MN-major operand K^T (M = key channel j,
-// K = token t): element (j, t) at 1024 + (j / 8) * 2048 + (t / 8) * 128 +
-// 16 (t % 8) + 2 (j % 8), i.e. LBO (K groups) = 128, SBO (MN groups) = 2048.
-__device__ __forceinline__ uint64_t desc_kt_mn(const unsigned char *qk, int k16) {
-    return smem_desc(smem_u32(qk + 1024 + k16 * 256), 128, 2048);
-}
-
 // Two values in three BF16 parts each, packed in pairs (x0 in the low half).
 __device__ __forceinline__ void split2_bf16x3(float x0, float x1, uint32_t &w0, uint32_t &w1,
                                               uint32_t &w2) {
@@ -655,19 +648,6 @@ __global__ void __launch_bounds__(kScanThreads, 1) chunk_scan_kernel(
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
-
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-    static std::atomic<void *> fn{nullptr};
-    void *f = fn.load(std::memory_order_acquire);
-    if (!f) {
-        cudaDriverEntryPointQueryResult q{};
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
-            q != cudaDriverEntryPointSuccess)
-            return nullptr;
-        fn.store(f, std::memory_order_release);
-    }
-    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-}
 
 // A 3-D map of a BF16 activation [B*T, H, D] (innermost D): box {box_d, 1, 64};
 // swizzle128 stores each 128-byte box row with the 128-byte swizzle.

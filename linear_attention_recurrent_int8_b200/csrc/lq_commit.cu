@@ -149,9 +149,6 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
     return r;
 }
 
-__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
 
 // The next head of this CTA's grid-stride walk at or after `bh` that commits
 // in this launch: every head with batch-synchronous positions; with

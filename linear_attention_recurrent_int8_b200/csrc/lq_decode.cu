@@ -48,6 +48,7 @@
 
 #include "lq_kernels.h"
 #include "lq_quant.cuh"
+#include "lq_tc.cuh"
 
 namespace lq {
 
@@ -69,14 +70,17 @@ struct PrepLayout {
     int limb, lscale, coefA, coefG, bytes;
 };
 
-__host__ __device__ inline PrepLayout prep_layout(int DK, int fmt) {
+__host__ __device__ inline PrepLayout prep_layout(int DK, int fmt, bool tc = false) {
     PrepLayout P{};
     int o = 0;
     P.limb = o;                            // int8 [6][DK]: x_k limbs 0..2, x_q limbs 0..2,
-    o += fmt == kCodesBF16 ? 8 * DK : 6 * DK;  // or (BF16 residual) float [2][DK]: x_k, x_q
+                                           // or (BF16 residual) float [2][DK]: x_k, x_q;
+                                           // none with the tensor-core matvec (the limbs
+                                           // are the stage's B operand)
+    o += tc ? 0 : fmt == kCodesBF16 ? 8 * DK : 6 * DK;
     P.lscale = o; o += 16;                 // float [2]: scales of x_k, x_q
-    P.coefA = o;  o += 4 * kCoef;          // records, compensators
-    P.coefG = o;  o += 4 * kCoef;          // records, compensators, own token (k~.q)
+    P.coefA = o;  o += align16(4 * kCoef);  // records, compensators (16-byte aligned)
+    P.coefG = o;  o += align16(4 * kCoef);  // records, compensators, own token (k~.q)
     P.bytes = align16(o);
     return P;
 }
@@ -85,14 +89,24 @@ __host__ __device__ inline PrepLayout prep_layout(int DK, int fmt) {
 // of record slots the stage holds (records read plus records written), `n`
 // the number of tokens of the call; `fmt` the residual's storage.
 struct StageLayout {
-    int codes, sig, cs, compv, compr, recK, recU, recL, q, k, v, al, scal, prep, bytes;
+    int codes, bop, sig, cs, compv, compr, recK, recU, recL, q, k, v, al, scal, prep, bytes;
 };
 
+// Rows of the tensor-core matvec's B operand for n tokens: 8 per token (x_k
+// limbs 0..2, x_q limbs 0..2, two unused), N = 8 for one token, else a
+// multiple of 16 (the kind::i8 shapes with M = 128).
+__host__ __device__ constexpr int tc_rows(int n) { return n == 1 ? 8 : 16 * ((n + 1) / 2); }
+
+// With tc (tensor-core matvec) the codes and the B operand are not part of
+// the stage (they live in a separate 1024-byte aligned array, tc_tile_bytes
+// per stage) and codes = bop = -1.
 __host__ __device__ inline StageLayout stage_layout(int DK, int DV, int gate, int R, int nrec,
-                                                   int n, int e, int fmt) {
+                                                   int n, int e, int fmt, bool tc = false) {
     StageLayout L{};
     int o = 0;
-    L.codes = o; o += align16(DV * code_row_bytes(fmt, DK));
+    L.codes = tc ? -1 : o;
+    o += tc ? 0 : align16(DV * code_row_bytes(fmt, DK));
+    L.bop = -1;
     L.sig = o;   o += align16(4 * DV);
     L.cs = o;    o += align16(4 * DK);
     L.compv = o; o += align16(4 * R * DK);
@@ -105,20 +119,26 @@ __host__ __device__ inline StageLayout stage_layout(int DK, int DV, int gate, in
     L.v = o;     o += align16(e * DV);
     L.al = o;    o += gate == 1 ? align16(4 * DK) : 0;
     L.scal = o;  o += 16;                  // float: alpha (scalar gate), beta of token 0
-    L.prep = o;  o += n * prep_layout(DK, fmt).bytes;
+    L.prep = o;  o += n * prep_layout(DK, fmt, tc).bytes;
     L.bytes = align16(o);
     return L;
 }
+
+// Bytes of one stage's tensor-core tile: the 128 x 128 codes (128-byte
+// swizzle) and the B operand of n tokens; a multiple of 1024.
+__host__ __device__ constexpr int tc_tile_bytes(int n) { return 128 * 128 + 128 * tc_rows(n); }
 
 __host__ __device__ constexpr int header_bytes() { return 3 * kMaxStages * 8; }
 
 // Splits the d_k-vector x (lane l holds x_j for the CPL channels
 // j = j0 .. j0+CPL-1) into NL int8 limbs with one scale s = max_j |x_j| / 127:
 // x ~= s (X0 + X1/2^7 [+ X2/2^14]), |error| <= s / 2^(7 NL - 6) (plus FP32
-// rounding).  Writes limb[0..NL-1][j] and *lscale.
-template <int CPL, int NL>
+// rounding).  Writes limb l as row row0 + l of `limb` -- plain rows of DK
+// bytes, or (SW128, d_k = 128) the rows of a K-major operand with the
+// 128-byte swizzle -- and *lscale.
+template <int CPL, int NL, bool SW128 = false>
 __device__ __forceinline__ void split_limbs(const float (&x)[CPL], int8_t *limb, int DK,
-                                            float *lscale, int j0) {
+                                            float *lscale, int j0, int row0) {
     float m = 0.0f;
 #pragma unroll
     for (int e = 0; e < CPL; ++e) m = fmaxf(m, fabsf(x[e]));
@@ -139,22 +159,30 @@ __device__ __forceinline__ void split_limbs(const float (&x)[CPL], int8_t *limb,
     }
 #pragma unroll
     for (int l = 0; l < NL; ++l) {
-        if constexpr (CPL == 4) *reinterpret_cast<uint32_t *>(limb + l * DK + j0) = w[l];
-        else *reinterpret_cast<uint16_t *>(limb + l * DK + j0) = (uint16_t)w[l];
+        const int r = row0 + l;
+        if constexpr (SW128) {
+            static_assert(CPL == 4, "the swizzled operand has d_k = 128");
+            const int off = (r >> 3) * 1024 + (r & 7) * 128 + ((((j0 >> 4) ^ r) & 7) << 4) + (j0 & 15);
+            *reinterpret_cast<uint32_t *>(limb + off) = w[l];
+        } else if constexpr (CPL == 4) {
+            *reinterpret_cast<uint32_t *>(limb + r * DK + j0) = w[l];
+        } else {
+            *reinterpret_cast<uint16_t *>(limb + r * DK + j0) = (uint16_t)w[l];
+        }
     }
     if (threadIdx.x % 32 == 0) *lscale = m * (1.0f / 127.0f);
 }
 
-// The next head (sequence-major index) of this CTA's grid-stride walk at or
+// The next head (sequence-major index) of a walk with stride `stride` at or
 // after `bh` that decodes in this launch: every head with batch-synchronous
 // positions; with per-sequence positions the heads of sequences whose
 // position is in [0, W) (a position >= W is recorded as an error and skipped).
-// Every role of the CTA walks the same sequence.
+// Every role of a pipeline walks the same sequence.
 template <bool RAGGED>
-__device__ __forceinline__ int next_decode_head(const DecodeArgs &a, int bh) {
+__device__ __forceinline__ int next_decode_head(const DecodeArgs &a, int bh, int stride) {
     if constexpr (RAGGED) {
         const int BH = a.B * a.H;
-        for (; bh < BH; bh += gridDim.x) {
+        for (; bh < BH; bh += stride) {
             const int p = a.seq_pos[bh / a.H];
             if (p >= 0 && p < a.W) return bh;
             if (p >= a.W) atomicOr(&g_dev_error, kErrBadPosition);
@@ -162,6 +190,212 @@ __device__ __forceinline__ int next_decode_head(const DecodeArgs &a, int bh) {
         return BH;
     } else {
         return bh;
+    }
+}
+
+// The prep warps of a head (one role per warp): prep A (isA) the limbs of
+// x_k = c e^L k and x_q = c e^L q and k~_t . q_t (one warp, or with NA = 2
+// warp `arole` 0 x_k and warp 1 x_q and k~_t . q_t); prep-B warp `bpart` of
+// NPB the new records (L_t, k~_t) and its share of the coefficient passes.
+// Every token of the call is prepared before "prepared" is signalled.  With
+// TC the limbs are written as the rows of the tensor-core matvec's B operand.
+template <int DK, int DV, int GATE, bool BF16, bool RAGGED, int FMT, bool TC, int NA, int NPB>
+__device__ __forceinline__ void prep_role(const DecodeArgs &a, const StageLayout &SL,
+                                          const PrepLayout &PL, unsigned char *stages,
+                                          uint64_t *full, uint64_t *prepared, uint64_t *empty,
+                                          int S, bool isA, int arole, int bpart, int lane,
+                                          int vblock, int vgrid, unsigned char *tiles = nullptr) {
+    constexpr bool BF16S = FMT == kCodesBF16;
+    const int BH = a.B * a.H, R = a.R, W = a.W, nsteps = a.n_steps;
+    constexpr int CPL = DK / 32;          // contiguous key channels per lane
+    const int j0 = CPL * lane;
+    int i = 0;
+    for (int bh = next_decode_head<RAGGED>(a, vblock, vgrid); bh < BH; bh = next_decode_head<RAGGED>(a, bh + vgrid, vgrid), ++i) {
+        const int s = i % S;
+        const int pos = RAGGED ? a.seq_pos[bh / a.H] : a.pos;  // records buffered
+        if (!mbar_wait_bounded(&full[s], (i / S) & 1)) break;
+        unsigned char *st = stages + (size_t)s * SL.bytes;
+        const float *cs_s = reinterpret_cast<const float *>(st + SL.cs);
+        const float *compv_s = reinterpret_cast<const float *>(st + SL.compv);
+        const float *scal = reinterpret_cast<const float *>(st + SL.scal);
+        float *recK_s = reinterpret_cast<float *>(st + SL.recK);
+        float *recL_s = reinterpret_cast<float *>(st + SL.recL);
+        const int b = bh / a.H, h = bh % a.H;
+        float Ls = (GATE == 0 && pos > 0) ? recL_s[pos - 1] : 0.0f;  // scalar gate chain
+        float Lc[CPL];                                             // diagonal, own channels
+        if (GATE == 1 && pos > 0) {
+            load_vec<CPL>(Lc, recL_s + (pos - 1) * DK + j0);
+        } else {
+#pragma unroll
+            for (int e = 0; e < CPL; ++e) Lc[e] = 0.0f;
+        }
+        for (int sidx = 0; sidx < nsteps; ++sidx) {
+            const int t = pos + sidx + 1, nrec = t - 1;
+            const size_t tok = ((size_t)b * nsteps + sidx) * a.H + h;
+            const float beta = sidx == 0 ? scal[1] : a.beta[tok];
+            unsigned char *slot = st + SL.prep + sidx * PL.bytes;
+            float *coefA = reinterpret_cast<float *>(slot + PL.coefA);
+            float *coefG = reinterpret_cast<float *>(slot + PL.coefG);
+            float g_s = 0.0f;
+            if (GATE == 0) {
+                Ls = Ls + logf(sidx == 0 ? scal[0] : a.alpha[tok]);
+                g_s = expf(Ls);
+            }
+            float kj[CPL], qj[CPL], gj[CPL];
+            if (sidx == 0) {
+                load_io_vec<BF16, CPL>(qj, st + SL.q, j0);
+                load_io_vec<BF16, CPL>(kj, st + SL.k, j0);
+            } else {
+                load_io_vec<BF16, CPL>(qj, a.q, tok * DK + j0);
+                load_io_vec<BF16, CPL>(kj, a.k, tok * DK + j0);
+            }
+            if (GATE == 1) {
+                float al[CPL];
+                if (sidx == 0) load_vec<CPL>(al, reinterpret_cast<const float *>(st + SL.al) + j0);
+                else load_vec<CPL>(al, a.alpha + tok * DK + j0);
+#pragma unroll
+                for (int e = 0; e < CPL; ++e) {
+                    Lc[e] = Lc[e] + logf(al[e]);
+                    gj[e] = expf(Lc[e]);
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < CPL; ++e) gj[e] = g_s;
+            }
+            if (isA) {
+                // limbs of x_k = c e^L k and x_q = c e^L q; own-token k~ . q
+                int8_t *limb = reinterpret_cast<int8_t *>(slot + PL.limb);
+                float *lscale = reinterpret_cast<float *>(slot + PL.lscale);
+                float cj[CPL], xk[CPL], xq[CPL], kq = 0.0f;
+                load_vec<CPL>(cj, cs_s + j0);
+#pragma unroll
+                for (int e = 0; e < CPL; ++e) {
+                    xk[e] = a.delta ? cj[e] * (gj[e] * kj[e]) : 0.0f;  // b = 0 rows: no S b term
+                    xq[e] = cj[e] * (gj[e] * qj[e]);
+                    kq = fmaf(beta * kj[e], qj[e], kq);
+                }
+                // with NA = 2 prep-A warps, warp arole 0 takes x_k, warp 1 x_q and k~ . q
+                const bool doK = NA == 1 || arole == 0, doQ = NA == 1 || arole == 1;
+                if constexpr (BF16S) {
+                    // the FP32 vectors themselves, unit scales
+                    float *xs = reinterpret_cast<float *>(limb);
+                    store_vec<CPL>(xs + j0, xk);
+                    store_vec<CPL>(xs + DK + j0, xq);
+                    if (lane == 0) lscale[0] = lscale[1] = 1.0f;
+                } else {
+                    // b = 0 rows: the consumers skip x_k, so it is not split
+                    if constexpr (TC) {
+                        // rows 8 sidx + 0..2 (x_k) and + 3..5 (x_q) of the B operand
+                        int8_t *bop = reinterpret_cast<int8_t *>(tiles + (size_t)s * tc_tile_bytes(nsteps) + DV * DK);
+                        if (doK && a.delta) split_limbs<CPL, 3, true>(xk, bop, DK, lscale, j0, 8 * sidx);
+                        if (doQ) split_limbs<CPL, 3, true>(xq, bop, DK, lscale + 1, j0, 8 * sidx + 3);
+                    } else {
+                        if (a.delta) split_limbs<CPL, 3>(xk, limb, DK, lscale, j0, 0);
+                        split_limbs<CPL, 3>(xq, limb, DK, lscale + 1, j0, 3);
+                    }
+                }
+                if (doQ) {
+                    kq = group_sum<32>(kq);
+                    if (lane == 0) coefG[nrec + R] = kq;
+                }
+            } else {
+                // records of this token: L_t and k~_t.  When a later token of
+                // the call follows, every prep-B warp writes the same values
+                // to shared memory (it reads them back there); warp 0 of them
+                // also writes global memory.
+                float ktj[CPL];
+#pragma unroll
+                for (int e = 0; e < CPL; ++e) ktj[e] = beta * kj[e];
+                if (sidx + 1 < nsteps) {
+                    store_vec<CPL>(recK_s + nrec * DK + j0, ktj);
+                    if (GATE == 1) store_vec<CPL>(recL_s + nrec * DK + j0, Lc);
+                    if (GATE == 0 && lane == 0) recL_s[nrec] = Ls;
+                }
+                if (bpart == 0) {
+                    store_vec<CPL>(a.buf_k + ((size_t)bh * W + nrec) * DK + j0, ktj);
+                    if (GATE == 1)
+                        store_vec<CPL>(a.buf_gate + ((size_t)bh * W + nrec) * DK + j0, Lc);
+                    if (GATE == 0 && lane == 0) a.buf_gate[(size_t)bh * W + nrec] = Ls;
+                }
+                __syncwarp();
+                // coefficients of records 0..nrec-1 and compensators, P = 8
+                // items per pass, passes shared round-robin by the prep-B
+                // warps; the 2P partial dot products of a pass are reduced
+                // together with a transposing reduction
+                const int nitems = nrec + R;
+                float kb[CPL];  // the b-side channels: k, or 0 for the b = 0 rows
+#pragma unroll
+                for (int e = 0; e < CPL; ++e) kb[e] = a.delta ? kj[e] : 0.0f;
+                auto coef_pass = [&](auto PC, int base) {
+                    constexpr int P = decltype(PC)::value;
+                    float part[2 * P];
+#pragma unroll
+                    for (int q8 = 0; q8 < P; ++q8) {
+                        const int it = base + q8;
+                        float da = 0.0f, dq = 0.0f;
+                        if constexpr (GATE == 0) {
+                            // scalar gate: raw dot products of the item's row
+                            // (record it, or compensator it - nrec) with k and
+                            // q; the gate factor is applied after the
+                            // reduction.  Items past the end read the last
+                            // record or compensator row and are not stored.
+                            const bool isrec = it < nrec || R == 0;
+                            const int ri = isrec ? min(it, nrec - 1) : min(it - nrec, R - 1);
+                            const float *row = (isrec ? recK_s : compv_s) + ri * DK;
+                            float w[CPL];
+                            load_vec<CPL>(w, row + j0);
+#pragma unroll
+                            for (int e = 0; e < CPL; ++e) {
+                                da = fmaf(w[e], kb[e], da);
+                                dq = fmaf(w[e], qj[e], dq);
+                            }
+                        } else if (it < nitems) {
+                            float w[CPL];
+                            if (it < nrec) {
+                                load_vec<CPL>(w, recK_s + it * DK + j0);
+                                float Lm[CPL];
+                                load_vec<CPL>(Lm, recL_s + it * DK + j0);
+#pragma unroll
+                                for (int e = 0; e < CPL; ++e) w[e] *= expf(Lc[e] - Lm[e]);
+#pragma unroll
+                                for (int e = 0; e < CPL; ++e) {
+                                    da = fmaf(w[e], kb[e], da);
+                                    dq = fmaf(w[e], qj[e], dq);
+                                }
+                            } else {
+                                load_vec<CPL>(w, compv_s + (it - nrec) * DK + j0);
+#pragma unroll
+                                for (int e = 0; e < CPL; ++e) {
+                                    da = fmaf(w[e], gj[e] * kb[e], da);
+                                    dq = fmaf(w[e], gj[e] * qj[e], dq);
+                                }
+                            }
+                        }
+                        part[q8] = da;
+                        part[P + q8] = dq;
+                    }
+                    transposed_sum<2 * P, 32>(part, lane);
+                    const int idx = transposed_index<2 * P, 32>(lane);
+                    const int it = base + (idx % P);
+                    if (it < nitems && lane == transposed_owner<2 * P, 32>(idx)) {
+                        float v = part[0];
+                        // scalar gate: e^{L_t - L_m} for a record, e^{L_t} for a compensator
+                        if (GATE == 0) v *= it < nrec ? expf(Ls - recL_s[it]) : g_s;
+                        if (idx < P) coefA[it] = v;
+                        else coefG[it] = v;
+                    }
+                };
+                for (int base = 8 * bpart; base < nitems; base += 8 * NPB)
+                    coef_pass(std::integral_constant<int, 8>{}, base);
+            }
+            __syncwarp();
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            mbar_arrive(&prepared[s]);
+            mbar_arrive(&empty[s]);
+        }
     }
 }
 
@@ -186,6 +420,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a,
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int BH = a.B * a.H;
     const int R = a.R, W = a.W;
+    const int vblock = blockIdx.x, vgrid = gridDim.x;  // this CTA's walk over the heads
 
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
@@ -201,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a,
         if (lane != 0) return;
         int i = 0;
         bool ok = true;
-        for (int bh = next_decode_head<RAGGED>(a, blockIdx.x); bh < BH; bh = next_decode_head<RAGGED>(a, bh + gridDim.x), ++i) {
+        for (int bh = next_decode_head<RAGGED>(a, vblock, vgrid); bh < BH; bh = next_decode_head<RAGGED>(a, bh + vgrid, vgrid), ++i) {
             const int s = i % S, use = i / S;
             const int pos = RAGGED ? a.seq_pos[bh / a.H] : a.pos;  // records buffered
             if (use > 0 && !mbar_wait_bounded(&empty[s], (use - 1) & 1)) {
@@ -261,170 +496,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a,
 
     // ------------------------------------------------------------ prep warps
     if (warp >= kPrepAWarp) {
-        const bool isA = warp == kPrepAWarp;
-        const int bpart = warp - kPrepBWarp;  // prep B: this warp's share of coefficient passes
-        constexpr int CPL = DK / 32;          // contiguous key channels per lane
-        const int j0 = CPL * lane;
-        int i = 0;
-        for (int bh = next_decode_head<RAGGED>(a, blockIdx.x); bh < BH; bh = next_decode_head<RAGGED>(a, bh + gridDim.x), ++i) {
-            const int s = i % S;
-            const int pos = RAGGED ? a.seq_pos[bh / a.H] : a.pos;  // records buffered
-            if (!mbar_wait_bounded(&full[s], (i / S) & 1)) break;
-            unsigned char *st = stages + (size_t)s * SL.bytes;
-            const float *cs_s = reinterpret_cast<const float *>(st + SL.cs);
-            const float *compv_s = reinterpret_cast<const float *>(st + SL.compv);
-            const float *scal = reinterpret_cast<const float *>(st + SL.scal);
-            float *recK_s = reinterpret_cast<float *>(st + SL.recK);
-            float *recL_s = reinterpret_cast<float *>(st + SL.recL);
-            const int b = bh / a.H, h = bh % a.H;
-            float Ls = (GATE == 0 && pos > 0) ? recL_s[pos - 1] : 0.0f;  // scalar gate chain
-            float Lc[CPL];                                             // diagonal, own channels
-            if (GATE == 1 && pos > 0) {
-                load_vec<CPL>(Lc, recL_s + (pos - 1) * DK + j0);
-            } else {
-#pragma unroll
-                for (int e = 0; e < CPL; ++e) Lc[e] = 0.0f;
-            }
-            for (int sidx = 0; sidx < nsteps; ++sidx) {
-                const int t = pos + sidx + 1, nrec = t - 1;
-                const size_t tok = ((size_t)b * nsteps + sidx) * a.H + h;
-                const float beta = sidx == 0 ? scal[1] : a.beta[tok];
-                unsigned char *slot = st + SL.prep + sidx * PL.bytes;
-                float *coefA = reinterpret_cast<float *>(slot + PL.coefA);
-                float *coefG = reinterpret_cast<float *>(slot + PL.coefG);
-                float g_s = 0.0f;
-                if (GATE == 0) {
-                    Ls = Ls + logf(sidx == 0 ? scal[0] : a.alpha[tok]);
-                    g_s = expf(Ls);
-                }
-                float kj[CPL], qj[CPL], gj[CPL];
-                if (sidx == 0) {
-                    load_io_vec<BF16, CPL>(qj, st + SL.q, j0);
-                    load_io_vec<BF16, CPL>(kj, st + SL.k, j0);
-                } else {
-                    load_io_vec<BF16, CPL>(qj, a.q, tok * DK + j0);
-                    load_io_vec<BF16, CPL>(kj, a.k, tok * DK + j0);
-                }
-                if (GATE == 1) {
-                    float al[CPL];
-                    if (sidx == 0) load_vec<CPL>(al, reinterpret_cast<const float *>(st + SL.al) + j0);
-                    else load_vec<CPL>(al, a.alpha + tok * DK + j0);
-#pragma unroll
-                    for (int e = 0; e < CPL; ++e) {
-                        Lc[e] = Lc[e] + logf(al[e]);
-                        gj[e] = expf(Lc[e]);
-                    }
-                } else {
-#pragma unroll
-                    for (int e = 0; e < CPL; ++e) gj[e] = g_s;
-                }
-                if (isA) {
-                    // limbs of x_k = c e^L k and x_q = c e^L q; own-token k~ . q
-                    int8_t *limb = reinterpret_cast<int8_t *>(slot + PL.limb);
-                    float *lscale = reinterpret_cast<float *>(slot + PL.lscale);
-                    float cj[CPL], xk[CPL], xq[CPL], kq = 0.0f;
-                    load_vec<CPL>(cj, cs_s + j0);
-#pragma unroll
-                    for (int e = 0; e < CPL; ++e) {
-                        xk[e] = a.delta ? cj[e] * (gj[e] * kj[e]) : 0.0f;  // b = 0 rows: no S b term
-                        xq[e] = cj[e] * (gj[e] * qj[e]);
-                        kq = fmaf(beta * kj[e], qj[e], kq);
-                    }
-                    if constexpr (BF16S) {
-                        // the FP32 vectors themselves, unit scales
-                        float *xs = reinterpret_cast<float *>(limb);
-                        store_vec<CPL>(xs + j0, xk);
-                        store_vec<CPL>(xs + DK + j0, xq);
-                        if (lane == 0) lscale[0] = lscale[1] = 1.0f;
-                    } else {
-                        // b = 0 rows: the consumers skip x_k, so it is not split
-                        if (a.delta) split_limbs<CPL, 3>(xk, limb, DK, lscale, j0);
-                        split_limbs<CPL, 3>(xq, limb + 3 * DK, DK, lscale + 1, j0);
-                    }
-                    kq = group_sum<32>(kq);
-                    if (lane == 0) coefG[nrec + R] = kq;
-                } else {
-                    // records of this token: L_t and k~_t.  Every prep-B warp
-                    // writes the same values to shared memory (it reads them
-                    // back for later tokens of the call); warp 0 of them also
-                    // writes global memory.
-                    float ktj[CPL];
-#pragma unroll
-                    for (int e = 0; e < CPL; ++e) ktj[e] = beta * kj[e];
-                    store_vec<CPL>(recK_s + nrec * DK + j0, ktj);
-                    if (GATE == 1) store_vec<CPL>(recL_s + nrec * DK + j0, Lc);
-                    if (GATE == 0 && lane == 0) recL_s[nrec] = Ls;
-                    if (bpart == 0) {
-                        store_vec<CPL>(a.buf_k + ((size_t)bh * W + nrec) * DK + j0, ktj);
-                        if (GATE == 1)
-                            store_vec<CPL>(a.buf_gate + ((size_t)bh * W + nrec) * DK + j0, Lc);
-                        if (GATE == 0 && lane == 0) a.buf_gate[(size_t)bh * W + nrec] = Ls;
-                    }
-                    __syncwarp();
-                    // coefficients of records 0..nrec-1 and compensators, P = 8
-                    // items per pass, passes shared round-robin by the prep-B
-                    // warps; the 2P partial dot products of a pass are reduced
-                    // together with a transposing reduction
-                    const int nitems = nrec + R;
-                    float kb[CPL];  // the b-side channels: k, or 0 for the b = 0 rows
-#pragma unroll
-                    for (int e = 0; e < CPL; ++e) kb[e] = a.delta ? kj[e] : 0.0f;
-                    auto coef_pass = [&](auto PC, int base) {
-                        constexpr int P = decltype(PC)::value;
-                        float part[2 * P];
-#pragma unroll
-                        for (int q8 = 0; q8 < P; ++q8) {
-                            const int it = base + q8;
-                            float da = 0.0f, dq = 0.0f;
-                            if (it < nitems) {
-                                float w[CPL];
-                                if (it < nrec) {
-                                    load_vec<CPL>(w, recK_s + it * DK + j0);
-                                    if (GATE == 1) {
-                                        float Lm[CPL];
-                                        load_vec<CPL>(Lm, recL_s + it * DK + j0);
-#pragma unroll
-                                        for (int e = 0; e < CPL; ++e) w[e] *= expf(Lc[e] - Lm[e]);
-                                    }
-#pragma unroll
-                                    for (int e = 0; e < CPL; ++e) {
-                                        da = fmaf(w[e], kb[e], da);
-                                        dq = fmaf(w[e], qj[e], dq);
-                                    }
-                                } else {
-                                    load_vec<CPL>(w, compv_s + (it - nrec) * DK + j0);
-#pragma unroll
-                                    for (int e = 0; e < CPL; ++e) {
-                                        da = fmaf(w[e], gj[e] * kb[e], da);
-                                        dq = fmaf(w[e], gj[e] * qj[e], dq);
-                                    }
-                                }
-                            }
-                            part[q8] = da;
-                            part[P + q8] = dq;
-                        }
-                        transposed_sum<2 * P, 32>(part, lane);
-                        const int idx = transposed_index<2 * P, 32>(lane);
-                        const int it = base + (idx % P);
-                        if (it < nitems && lane == transposed_owner<2 * P, 32>(idx)) {
-                            float v = part[0];
-                            if (GATE == 0 && it < nrec) v *= expf(Ls - recL_s[it]);
-                            if (idx < P) coefA[it] = v;
-                            else coefG[it] = v;
-                        }
-                    };
-                    for (int base = 8 * bpart; base < nitems; base += 8 * kPrepBWarps)
-                        coef_pass(std::integral_constant<int, 8>{}, base);
-                }
-                __syncwarp();
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&prepared[s]);
-                mbar_arrive(&empty[s]);
-            }
-        }
+        prep_role<DK, DV, GATE, BF16, RAGGED, FMT, false, 1, kPrepBWarps>(
+            a, SL, PL, stages, full, prepared, empty, S, warp == kPrepAWarp, 0, warp - kPrepBWarp, lane,
+            blockIdx.x, gridDim.x);
         return;
     }
 
@@ -440,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a,
 
     const bool delta = a.delta != 0;  // b = 0 rows (delta = 0): no S^_0 x_k products
     int i = 0;
-    for (int bh = next_decode_head<RAGGED>(a, blockIdx.x); bh < BH; bh = next_decode_head<RAGGED>(a, bh + gridDim.x), ++i) {
+    for (int bh = next_decode_head<RAGGED>(a, vblock, vgrid); bh < BH; bh = next_decode_head<RAGGED>(a, bh + vgrid, vgrid), ++i) {
         const int s = i % S;
         const int pos = RAGGED ? a.seq_pos[bh / a.H] : a.pos;  // records buffered
         if (!mbar_wait_bounded(&prepared[s], (i / S) & 1)) break;
@@ -592,6 +666,323 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a,
     }
 }
 
+// ---------------------------------------------------------------------------
+// Tensor-core matvec variant (d_k = d_v = 128, one int8 code per byte)
+// ---------------------------------------------------------------------------
+//
+// The boundary matvec of D2 is a product of the 128 x 128 code matrix with
+// the six limb vectors of a token (x_k limbs 0..2, x_q limbs 0..2): the
+// kind::i8 tensor-core MMA computes it exactly in int32, the same sums the
+// dp4a chain forms.  A kernel that allocates TMEM runs one CTA per SM, so
+// the CTA holds npipe (1 or 2) independent pipelines of 12 warps, each with
+// its own stage ring, barriers and TMEM columns, walking its own share of
+// the heads (pipeline p of CTA c: heads c npipe + p, stride gridDim npipe);
+// at most 80 registers a thread.  Roles of a pipeline (warp index mod 12):
+//  * producer (warp 4, one lane): the codes by one tiled TMA box (128 rows x
+//    128 bytes, 128-byte swizzle, no multicast) and the other operands by
+//    bulk copies, as in decode_kernel -> "full";
+//  * MMA (warp 5, one lane): 4 MMAs of 128 x N x 32 (N = 8 per token) into the
+//    stage's TMEM accumulator, completion by tcgen05.commit -> "mma_done";
+//  * prep A (warps 6, 7: x_k, and x_q with k~ . q) and prep B (warps 8-11,
+//    records and coefficient passes): as in decode_kernel; prep A writes the
+//    limbs as the rows of the MMA's K-major B operand -> "prepared";
+//  * epilogue (warps 0-3): warp w reads TMEM lanes 32w..32w+31 = value rows,
+//    one row per lane, so y_k and y_q arrive without any cross-lane
+//    reduction; then D3-D6 for that row as in decode_kernel -> "empty".
+constexpr int kTcEpiWarps = 4;
+constexpr int kTcProducerWarp = 4, kTcMmaWarp = 5, kTcPrepAWarp = 6, kTcPrepAWarps = 2;
+constexpr int kTcPrepBWarp = 8, kTcPrepBWarps = 4;
+constexpr int kTcPrepWarps = kTcPrepAWarps + kTcPrepBWarps;
+constexpr int kTcPipeWarps = 12, kTcMaxPipes = 2;
+constexpr int kTcThreads = kTcMaxPipes * kTcPipeWarps * 32;
+constexpr int kTcHeader = 1024;  // barriers + TMEM slot; the stages follow 1024-aligned
+
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int c0, int c1,
+                                            uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+        "l"(map), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// S stages per pipeline; npipe pipelines (blockDim = npipe x 12 warps);
+// tcols TMEM columns allocated (S x N per pipeline).
+template <int GATE, bool BF16, bool RAGGED>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    decode_tc_kernel(const DecodeArgs a, const int S, const int npipe, const int tcols,
+                     const __grid_constant__ CUtensorMap codes_map) {
+    constexpr int DK = 128, DV = 128, FMT = kCodesI8;
+    constexpr int E = BF16 ? 2 : 4;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    // the swizzled operands need 1024-byte aligned addresses: align the base
+    unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    constexpr int NBAR = kTcMaxPipes * kMaxStages;
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int pipe = (tid >> 5) / kTcPipeWarps, warp = (tid >> 5) % kTcPipeWarps;  // role in the pipeline
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem) + pipe * kMaxStages;
+    uint64_t *prepared = full + NBAR;
+    uint64_t *mma_done = prepared + NBAR;
+    uint64_t *empty = mma_done + NBAR;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(reinterpret_cast<uint64_t *>(smem) + 4 * NBAR);
+    const int nsteps = a.n_steps;
+    const StageLayout SL = stage_layout(DK, DV, GATE, a.R, a.pos + nsteps, nsteps, E, FMT, true);
+    const PrepLayout PL = prep_layout(DK, FMT, true);
+    const int TB = tc_tile_bytes(nsteps);
+    // this pipeline's tiles (codes + B operand, 1024-aligned) and stages
+    unsigned char *tiles = smem + kTcHeader + (size_t)pipe * S * TB;
+    unsigned char *stages = smem + kTcHeader + (size_t)npipe * S * TB + (size_t)pipe * S * SL.bytes;
+    const int NB = tc_rows(nsteps);  // accumulator columns per stage
+    const int BH = a.B * a.H, R = a.R, W = a.W;
+    const int vblock = blockIdx.x * npipe + pipe, vgrid = gridDim.x * npipe;  // this pipeline's walk
+
+    if (tid < 32) tmem_alloc(tmem_slot, tcols);
+    if (tid == 0) {
+        uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
+        for (int q = 0; q < npipe; ++q)
+            for (int s = 0; s < S; ++s) {
+                mbar_init(&bars[q * kMaxStages + s], 1);                                // full
+                mbar_init(&bars[NBAR + q * kMaxStages + s], kTcPrepWarps);             // prepared
+                mbar_init(&bars[2 * NBAR + q * kMaxStages + s], 1);                    // mma_done
+                mbar_init(&bars[3 * NBAR + q * kMaxStages + s], kTcEpiWarps + kTcPrepWarps);  // empty
+            }
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot + (uint32_t)(pipe * S * NB);  // this pipeline's columns
+
+    if (warp == kTcProducerWarp) {
+        // ---------------------------------------------------------- producer
+        if (lane == 0) {
+            int i = 0;
+            bool ok = true;
+            for (int bh = next_decode_head<RAGGED>(a, vblock, vgrid); bh < BH;
+                 bh = next_decode_head<RAGGED>(a, bh + vgrid, vgrid), ++i) {
+                const int s = i % S, use = i / S;
+                const int pos = RAGGED ? a.seq_pos[bh / a.H] : a.pos;  // records buffered
+                if (use > 0 && !mbar_wait_bounded(&empty[s], (use - 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                unsigned char *st = stages + (size_t)s * SL.bytes;
+                const int b = bh / a.H, h = bh % a.H;
+                const size_t tok = (size_t)b * nsteps * a.H + h;  // token 0 of this call
+                const uint32_t in_bytes = (uint32_t)(E * (2 * DK + DV) + (GATE == 1 ? 4 * DK : 0));
+                const uint32_t bytes = DV * DK + 4 * DV + 4 * DK + 4 * R * DK + 4 * pos * (DK + DV) +
+                                       (GATE == 1 ? 4 * pos * DK : 0) + in_bytes;
+                float *scal = reinterpret_cast<float *>(st + SL.scal);
+                if (GATE == 0) cp_async4(scal, a.alpha + tok);
+                cp_async4(scal + 1, a.beta + tok);
+                if (GATE == 0)
+                    for (int m = 0; m < pos; ++m)
+                        cp_async4(st + SL.recL + 4 * m, a.buf_gate + (size_t)bh * W + m);
+                for (int c = 0; c < R; ++c)
+                    cp_async4(st + SL.compr + 4 * c, a.comp_row + (size_t)bh * R + c);
+                cp_async_mbar_arrive(&full[s]);
+                mbar_arrive_expect_tx(&full[s], bytes);
+                tma_load_2d(tiles + (size_t)s * TB, &codes_map, 0, bh * DV, &full[s]);
+                bulk_g2s(st + SL.sig, a.row_scale + (size_t)bh * DV, 4 * DV, &full[s]);
+                bulk_g2s(st + SL.cs, a.col_smooth + (size_t)bh * DK, 4 * DK, &full[s]);
+                if (R > 0) bulk_g2s(st + SL.compv, a.comp_val + (size_t)bh * R * DK, 4 * R * DK, &full[s]);
+                if (pos > 0) {
+                    bulk_g2s(st + SL.recK, a.buf_k + (size_t)bh * W * DK, 4 * pos * DK, &full[s]);
+                    bulk_g2s(st + SL.recU, a.buf_u + (size_t)bh * W * DV, 4 * pos * DV, &full[s]);
+                    if (GATE == 1)
+                        bulk_g2s(st + SL.recL, a.buf_gate + (size_t)bh * W * DK, 4 * pos * DK, &full[s]);
+                }
+                const unsigned char *qg = static_cast<const unsigned char *>(a.q);
+                const unsigned char *kg = static_cast<const unsigned char *>(a.k);
+                const unsigned char *vg = static_cast<const unsigned char *>(a.v);
+                bulk_g2s(st + SL.q, qg + tok * DK * E, E * DK, &full[s]);
+                bulk_g2s(st + SL.k, kg + tok * DK * E, E * DK, &full[s]);
+                bulk_g2s(st + SL.v, vg + tok * DV * E, E * DV, &full[s]);
+                if (GATE == 1) bulk_g2s(st + SL.al, a.alpha + tok * DK, 4 * DK, &full[s]);
+            }
+            if (!ok) {
+                // drain the copies still in flight into this CTA's shared memory
+                for (int j = i - 1; j >= 0 && j >= i - S; --j) mbar_wait_bounded(&full[j % S], (j / S) & 1);
+            }
+        }
+    } else if (warp >= kTcPrepAWarp) {
+        // ---------------------------------------------------------- prep
+        prep_role<DK, DV, GATE, BF16, RAGGED, FMT, true, kTcPrepAWarps, kTcPrepBWarps>(
+            a, SL, PL, stages, full, prepared, empty, S, warp < kTcPrepBWarp, warp - kTcPrepAWarp,
+            warp - kTcPrepBWarp, lane, vblock, vgrid, tiles);
+    } else if (warp == kTcMmaWarp) {
+        // ---------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = idesc_i8(DV, NB);
+            int i = 0, last = -1;
+            for (int bh = next_decode_head<RAGGED>(a, vblock, vgrid); bh < BH;
+                 bh = next_decode_head<RAGGED>(a, bh + vgrid, vgrid), ++i) {
+                const int s = i % S;
+                if (!mbar_wait_bounded(&full[s], (i / S) & 1)) break;
+                if (!mbar_wait_bounded(&prepared[s], (i / S) & 1)) break;
+                tc_fence_after_sync();
+                const uint32_t a0 = smem_u32(tiles + (size_t)s * TB), b0 = a0 + DV * DK;
+#pragma unroll
+                for (int k = 0; k < DK / 32; ++k)
+                    mma_i8(tmem + (uint32_t)(s * NB), smem_desc_sw128(a0 + 32 * k),
+                           smem_desc_sw128(b0 + 32 * k), idesc, k > 0);
+                mma_commit(&mma_done[s]);
+                last = i;
+            }
+            // every MMA issued has completed before TMEM is released
+            if (last >= 0) mbar_wait_bounded(&mma_done[last % S], (last / S) & 1);
+        }
+    } else {
+        // ---------------------------------------------------------- epilogue
+        const int row = warp * 32 + lane;  // TMEM lane = value row
+        const uint32_t tlane = (uint32_t)(warp * 32) << 16;
+        const bool delta = a.delta != 0;
+        int i = 0;
+        for (int bh = next_decode_head<RAGGED>(a, vblock, vgrid); bh < BH;
+             bh = next_decode_head<RAGGED>(a, bh + vgrid, vgrid), ++i) {
+            const int s = i % S;
+            const int pos = RAGGED ? a.seq_pos[bh / a.H] : a.pos;  // records buffered
+            if (!mbar_wait_bounded(&mma_done[s], (i / S) & 1)) break;
+            if (!mbar_wait_bounded(&prepared[s], (i / S) & 1)) break;
+            tc_fence_after_sync();
+            unsigned char *st = stages + (size_t)s * SL.bytes;
+            const float *sig_s = reinterpret_cast<const float *>(st + SL.sig);
+            const int *compr_s = reinterpret_cast<const int *>(st + SL.compr);
+            float *recU_s = reinterpret_cast<float *>(st + SL.recU);
+            const int b = bh / a.H, h = bh % a.H;
+            float *bufU = a.buf_u + (size_t)bh * W * DV;
+            const float sg = sig_s[row];
+            for (int sidx = 0; sidx < nsteps; ++sidx) {
+                const int t = pos + sidx + 1, nrec = t - 1;
+                const size_t tok = ((size_t)b * nsteps + sidx) * a.H + h;
+                const unsigned char *slot = st + SL.prep + sidx * PL.bytes;
+                const float *lscale = reinterpret_cast<const float *>(slot + PL.lscale);
+                const float *coefA = reinterpret_cast<const float *>(slot + PL.coefA);
+                const float *coefG = reinterpret_cast<const float *>(slot + PL.coefG);
+                // D2: the six exact int32 limb sums of this row; (A0 2^7 + A1)
+                // 2^7 + A2 in units of 2^-14 of the vector's scale
+                int acc[8];
+                tmem_load8_i32(tmem + tlane + (uint32_t)(s * NB + 8 * sidx), acc);
+                const float vk = fmaf(__int2float_rn(acc[0] * 128 + acc[1]), 128.0f, small_int_to_f32(acc[2]));
+                const float vq = fmaf(__int2float_rn(acc[3] * 128 + acc[4]), 128.0f, small_int_to_f32(acc[5]));
+                constexpr float kUnit = 6.103515625e-05f;  // 2^-14
+                // D3-D6 for this row
+                float hb = delta ? vk * (sg * (lscale[0] * kUnit)) : 0.0f;
+                float p = vq * (sg * (lscale[1] * kUnit));
+                int m = 0;
+                for (; m + 4 <= nrec; m += 4) {  // coefficients are 16-byte aligned
+                    const float4 ca = *reinterpret_cast<const float4 *>(coefA + m);
+                    const float4 cg = *reinterpret_cast<const float4 *>(coefG + m);
+                    const float u0 = recU_s[m * DV + row], u1 = recU_s[(m + 1) * DV + row];
+                    const float u2 = recU_s[(m + 2) * DV + row], u3 = recU_s[(m + 3) * DV + row];
+                    hb = fmaf(ca.x, u0, hb);
+                    p = fmaf(cg.x, u0, p);
+                    hb = fmaf(ca.y, u1, hb);
+                    p = fmaf(cg.y, u1, p);
+                    hb = fmaf(ca.z, u2, hb);
+                    p = fmaf(cg.z, u2, p);
+                    hb = fmaf(ca.w, u3, hb);
+                    p = fmaf(cg.w, u3, p);
+                }
+                for (; m < nrec; ++m) {
+                    const float um = recU_s[m * DV + row];
+                    hb = fmaf(coefA[m], um, hb);
+                    p = fmaf(coefG[m], um, p);
+                }
+                for (int c = 0; c < R; ++c)
+                    if (compr_s[c] == row) {
+                        hb += coefA[nrec + c];
+                        p += coefG[nrec + c];
+                    }
+                const float vi = sidx == 0 ? load_io<BF16>(st + SL.v, row) : load_io<BF16>(a.v, tok * DV + row);
+                const float u = vi - hb;
+                const float o = fmaf(coefG[nrec + R], u, p);
+                store_io<BF16>(a.o, tok * DV + row, o);
+                recU_s[nrec * DV + row] = u;
+                bufU[(size_t)nrec * DV + row] = u;
+            }
+            // this head's TMEM reads are complete: release the stage (and its
+            // accumulator) to the producer
+            tc_fence_before_sync();
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+        }
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    if (tid < 32) {
+        tc_fence_after_sync();
+        tmem_dealloc(*tmem_slot, tcols);
+    }
+}
+
+// The 2-D map of all codes [B*H*128 rows][128 bytes]: one box = one head's
+// 128 x 128 codes, stored with the 128-byte swizzle.
+bool codes_tensor_map(CUtensorMap *m, const int8_t *codes, long long rows) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {128, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {128};
+    const cuuint32_t box[2] = {128, 128};
+    const cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t *>(codes), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int GATE, bool BF16, bool RAGGED>
+cudaError_t launch_tc(const DecodeArgs &a, cudaStream_t stream) {
+    constexpr int E = BF16 ? 2 : 4;
+    static std::atomic<uint64_t> configured{0};  // devices already set up
+    static int sm_count[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    auto kern = decode_tc_kernel<GATE, BF16, RAGGED>;
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(configured.load(std::memory_order_acquire) & bit)) {
+        int optin = 0, sms = 0;
+        e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        sm_count[dev & 63] = sms;
+        configured.fetch_or(bit, std::memory_order_acq_rel);
+    }
+    const StageLayout SL = stage_layout(128, 128, GATE, a.R, a.pos + a.n_steps, a.n_steps, E, kCodesI8, true);
+    const int fixed = 1024 + kTcHeader;  // alignment slack + header
+    const int NB = tc_rows(a.n_steps);
+    const int per_stage = SL.bytes + tc_tile_bytes(a.n_steps);
+    auto cols_for = [NB](int cols) {
+        int c = 32;
+        while (c < cols) c <<= 1;
+        return c;
+    };
+    // one CTA per SM; two pipelines when each gets at least two stages,
+    // else one pipeline with as many stages as fit (shared memory and the
+    // 512 TMEM columns)
+    const int per_sm = 227 * 1024;  // the one CTA of the SM takes all of it
+    int npipe = 2, S = (per_sm - fixed) / (2 * per_stage);
+    if (S > kMaxStages) S = kMaxStages;
+    while (S >= 2 && cols_for(2 * S * NB) > 512) --S;
+    if (S < 2) {
+        npipe = 1;
+        S = (per_sm - fixed) / per_stage;
+        if (S > kMaxStages) S = kMaxStages;
+        while (S >= 1 && cols_for(S * NB) > 512) --S;
+    }
+    if (S < 1) return cudaErrorInvalidConfiguration;
+    const int smem = fixed + npipe * S * per_stage;
+    CUtensorMap map;
+    if (!codes_tensor_map(&map, a.codes, (long long)a.B * a.H * 128)) return cudaErrorInvalidValue;
+    const int BH = a.B * a.H;
+    int grid = sm_count[dev & 63];
+    if (grid * npipe > BH) grid = (BH + npipe - 1) / npipe;
+    kern<<<grid, npipe * kTcPipeWarps * 32, smem, stream>>>(a, S, npipe, cols_for(npipe * S * NB), map);
+    return cudaGetLastError();
+}
+
 template <int DK, int DV, int GATE, bool BF16, bool RAGGED, int FMT>
 cudaError_t launch_d(const DecodeArgs &a, cudaStream_t stream) {
     constexpr int E = BF16 ? 2 : 4;
@@ -643,6 +1034,10 @@ cudaError_t launch_d(const DecodeArgs &a, cudaStream_t stream) {
 template <int DK, int DV, int GATE, bool BF16>
 cudaError_t launch_dr(const DecodeArgs &a, cudaStream_t stream) {
     const int fmt = code_format(a.bits);
+    if constexpr (DK == 128 && DV == 128) {
+        if (fmt == kCodesI8)  // the tensor-core matvec
+            return a.seq_pos ? launch_tc<GATE, BF16, true>(a, stream) : launch_tc<GATE, BF16, false>(a, stream);
+    }
     if (fmt == kCodesI4)
         return a.seq_pos ? launch_d<DK, DV, GATE, BF16, true, kCodesI4>(a, stream)
                          : launch_d<DK, DV, GATE, BF16, false, kCodesI4>(a, stream);

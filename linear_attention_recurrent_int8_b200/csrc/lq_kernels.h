@@ -2,8 +2,12 @@
 // the kernel launchers.  Not installed; not part of the ABI.
 #pragma once
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+
+#include <atomic>
 
 namespace lq {
 
@@ -16,6 +20,21 @@ __host__ __device__ constexpr int code_format(int bits) {
 // Bytes of one value row of the residual with d_k key channels.
 __host__ __device__ constexpr int code_row_bytes(int fmt, int dk) {
     return fmt == kCodesI4 ? dk / 2 : fmt == kCodesBF16 ? 2 * dk : dk;
+}
+
+// cuTensorMapEncodeTiled of the driver, looked up once (nullptr when the
+// driver does not provide it).
+inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static std::atomic<void *> fn{nullptr};
+    void *f = fn.load(std::memory_order_acquire);
+    if (!f) {
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        fn.store(f, std::memory_order_release);
+    }
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
 }
 
 // Arguments of the decode and commit kernels.

@@ -1,6 +1,7 @@
 // lq_tc.cuh -- 5th-generation tensor core (tcgen05) helpers for sm_100a:
 // tensor-memory (TMEM) allocation, shared-memory matrix descriptors, the
-// kind::tf32 MMA with its completion signalled on an mbarrier, TMEM loads.
+// kind::tf32, kind::f16 (BF16) and kind::i8 MMAs with their completion
+// signalled on an mbarrier, TMEM loads and stores.
 //
 // Operand layout used here (no swizzle, both operands K-major): a matrix of
 // R rows and K 32-bit elements is stored as K/4 slabs of R rows x 16 bytes;
@@ -139,6 +140,46 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64
         "{ .reg .pred p; setp.ne.b32 p, %4, 0; "
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }" ::"r"(d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"((uint32_t)accumulate)
+        : "memory");
+}
+
+// Shared-memory descriptor of a K-major operand stored with the 128-byte
+// swizzle: rows of 128 bytes, 8-row atoms of 1024 bytes (the stride byte
+// offset), atoms 1024-byte aligned; inside an atom the 16-byte chunk c of row
+// r sits at chunk c ^ (r % 8).  A K step inside the 128-byte row advances the
+// start address by the step's bytes.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | (1ull << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor of kind::i8: signed 8-bit A and B, both K-major,
+// signed 32-bit accumulator, no saturation, M x N tile.
+__host__ __device__ constexpr uint32_t idesc_i8(int M, int N) {
+    return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
+           ((uint32_t)(M >> 4) << 24);
+}
+
+// D (TMEM, int32) = A B^T (+ D when `accumulate`), kind::i8, both operands in
+// shared memory; issued by one thread.
+__device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, bool accumulate) {
+    asm volatile(
+        "{ .reg .pred p; setp.ne.b32 p, %4, 0; "
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p; }" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"((uint32_t)accumulate)
+        : "memory");
+}
+
+// 8 consecutive 32-bit TMEM columns of the warp's 32 lanes (32x32b.x8), as
+// int32; the wait is part of the statement.
+__device__ __forceinline__ void tmem_load8_i32(uint32_t taddr, int (&v)[8]) {
+    asm volatile(
+        "{ tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n\t"
+        "tcgen05.wait::ld.sync.aligned; }"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+          "=r"(v[7])
+        : "r"(taddr)
         : "memory");
 }
 
