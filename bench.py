@@ -51,31 +51,32 @@ FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # Algorithmic bytes (per (sequence, head) and launch)
 # --------------------------------------------------------------------------
 
-def snapshot_bytes(dk, dv, r, bits=8):
+def snapshot_bytes(dk, dv, r, bits=8, svd=False):
     """Codes (one byte per code, half a byte at 4 bits, two bytes per BF16
-    value at 16), row scales, smoothing factors and compensators of one head."""
+    value at 16), row scales, smoothing factors and compensators of one head
+    (row indices and k~_c rows; with the SVD rule also the u_c vectors)."""
     codes = dv * dk // 2 if bits == 4 else 2 * dv * dk if bits == 16 else dv * dk
-    return codes + 4 * dv + 4 * dk + r * (4 + 4 * dk)
+    return codes + 4 * dv + 4 * dk + r * (4 + 4 * dk) + (4 * r * dv if svd else 0)
 
 
 def record_bytes(dk, dv, gate):
     return 4 * ((dk if gate == "diag" else 1) + dk + dv)
 
 
-def decode_launch_bytes(dk, dv, r, gate, e, t, bits=8):
+def decode_launch_bytes(dk, dv, r, gate, e, t, bits=8, svd=False):
     """Bytes one decode launch at window position t must move per head:
     read the snapshot and the t-1 buffered records, read q, k, v, alpha,
     beta, write o and record t."""
     G = dk if gate == "diag" else 1
     rec = record_bytes(dk, dv, gate)
-    return (snapshot_bytes(dk, dv, r, bits) + (t - 1) * rec + e * (2 * dk + dv) + 4 * G + 4 + e * dv
-            + rec)
+    return (snapshot_bytes(dk, dv, r, bits, svd) + (t - 1) * rec + e * (2 * dk + dv) + 4 * G + 4
+            + e * dv + rec)
 
 
-def commit_launch_bytes(dk, dv, r, gate, n, bits=8):
+def commit_launch_bytes(dk, dv, r, gate, n, bits=8, svd=False):
     """Bytes the commit of a window of n records must move per head: read the
     snapshot and the n records, write the new snapshot."""
-    return 2 * snapshot_bytes(dk, dv, r, bits) + n * record_bytes(dk, dv, gate)
+    return 2 * snapshot_bytes(dk, dv, r, bits, svd) + n * record_bytes(dk, dv, gate)
 
 
 # --------------------------------------------------------------------------
@@ -145,7 +146,7 @@ def measured_bf16_tflops(sustained: bool):
 
 # the sources of each kernel's translation unit (the .cu and the headers it includes)
 KERNEL_SOURCES = {
-    "decode": ["lq_decode.cu", "lq_common.cuh", "lq_quant.cuh", "lq_kernels.h"],
+    "decode": ["lq_decode.cu", "lq_common.cuh", "lq_quant.cuh", "lq_tc.cuh", "lq_kernels.h"],
     "commit": ["lq_commit.cu", "lq_common.cuh", "lq_quant.cuh", "lq_tc.cuh", "lq_kernels.h"],
 }
 
@@ -313,7 +314,16 @@ def profile_key(kernel, wl, args):
     if (wl.window, wl.n_comp, bool(wl.smoothing)) != (base.window, base.n_comp, bool(base.smoothing)) \
             or args.bits != 8:
         key += f"_W{wl.window}_r{wl.n_comp}_s{int(bool(wl.smoothing))}_b{args.bits}"
+    if getattr(args, "comp_rule", "rows") == "svd":
+        key += "_svd"
     return key
+
+
+def decode_kernel_name(wl, args):
+    """The decode kernel the library launches for this workload: the
+    tensor-core matvec for d_k = d_v = 128 with one code per byte, else the
+    dp4a / FP32 kernel."""
+    return "decode_tc_kernel" if wl.d_k == 128 and wl.d_v == 128 and args.bits in (8, 6) else "decode_kernel"
 
 
 def synth_workload(name):
@@ -330,6 +340,7 @@ def workload_config(wl, args):
         "batch_per_gpu": wl.batch, "heads": wl.heads, "d_k": wl.d_k, "d_v": wl.d_v,
         "window": wl.window, "n_comp": wl.n_comp, "gate": wl.gate, "io": wl.io,
         "smoothing": bool(wl.smoothing), "bits": args.bits, "delta": wl.delta,
+        "comp_rule": args.comp_rule,
         "state": f"{state_words(args.bits)} + fp32 row scales",
         "step": f"one window: {wl.window} decode launches and the window commit",
         "tokens_per_step_per_gpu": wl.batch * wl.window,
@@ -373,7 +384,9 @@ def run_lq(args, wl):
     cfg = lq.Config(batch=wl.batch, heads=wl.heads, d_k=wl.d_k, d_v=wl.d_v, window=wl.window,
                     n_comp=wl.n_comp, gate=lq.LQ_GATE_DIAG if wl.gate == "diag" else lq.LQ_GATE_SCALAR,
                     io_dtype=lq.LQ_BF16 if wl.io == "bf16" else lq.LQ_F32,
-                    smoothing=int(wl.smoothing), auto_commit=0, delta=wl.delta, bits=args.bits)
+                    smoothing=int(wl.smoothing), auto_commit=0, delta=wl.delta, bits=args.bits,
+                    comp_rule=lq.LQ_COMP_SVD if args.comp_rule == "svd" else lq.LQ_COMP_ROWS)
+    svd = args.comp_rule == "svd" and wl.n_comp > 0
     W = wl.window
     e = 2 if wl.io == "bf16" else 4
     st = lq.State(cfg, dev)
@@ -465,7 +478,8 @@ def run_lq(args, wl):
         evs = graphs[gi][1]
         for t in range(W):
             dec_ms.append(evs[t].elapsed_time(evs[t + 1]))
-            dec_bytes += nh * decode_launch_bytes(wl.d_k, wl.d_v, wl.n_comp, wl.gate, e, t + 1, args.bits)
+            dec_bytes += nh * decode_launch_bytes(wl.d_k, wl.d_v, wl.n_comp, wl.gate, e, t + 1, args.bits,
+                                                  svd)
         com_ms.append(evs[W].elapsed_time(evs[W + 1]))
     peak, peak_kind = measured_peaks()
     dec_avg_ms = sum(dec_ms) / len(dec_ms)
@@ -473,7 +487,7 @@ def run_lq(args, wl):
     traffic = profiled_traffic(profile_key("decode", wl, args))
     roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
             "frac": achieved / peak, "traffic": traffic,
-            "kernel": "decode_kernel (window positions 1..W)",
+            "kernel": f"{decode_kernel_name(wl, args)} (window positions 1..W)",
             "bytes_per_launch": dec_bytes / len(dec_ms), "avg_launch_us": dec_avg_ms * 1e3,
             "peak_source": f"{peak_kind} hbm_gbs (copy)"}
     extra = {}
@@ -484,7 +498,7 @@ def run_lq(args, wl):
         pos_us.append(round(1e3 * sum(vals) / len(vals), 1))
     extra["launch_us_by_position"] = pos_us
     c_avg = sum(com_ms) / len(com_ms)
-    c_bytes = nh * commit_launch_bytes(wl.d_k, wl.d_v, wl.n_comp, wl.gate, W, args.bits)
+    c_bytes = nh * commit_launch_bytes(wl.d_k, wl.d_v, wl.n_comp, wl.gate, W, args.bits, svd)
     extra["commit"] = {"kernel": "commit_kernel", "avg_launch_us": c_avg * 1e3,
                        "bytes_per_launch": c_bytes, "achieved_gbs": c_bytes / (c_avg / 1e3) / 1e9,
                        "frac": c_bytes / (c_avg / 1e3) / 1e9 / peak,
@@ -689,7 +703,7 @@ def run_ragged(args, wl):
     cfg = lq.Config(batch=wl.batch, heads=wl.heads, d_k=wl.d_k, d_v=wl.d_v, window=W, n_comp=wl.n_comp,
                     gate=lq.LQ_GATE_DIAG if wl.gate == "diag" else lq.LQ_GATE_SCALAR,
                     io_dtype=lq.LQ_BF16 if wl.io == "bf16" else lq.LQ_F32, smoothing=int(wl.smoothing),
-                    bits=args.bits)
+                    bits=args.bits, comp_rule=lq.LQ_COMP_SVD if args.comp_rule == "svd" else lq.LQ_COMP_ROWS)
     st = lq.State(cfg, dev)
     S0 = synth.torch_initial_state(wl.seed, range(wl.batch), range(wl.heads), wl.d_k, wl.d_v,
                                    wl.outlier_rows, wl.outlier_cols, wl.outlier_scale, dev)
@@ -836,16 +850,17 @@ def run_mse(args, wl):
     S0 = S0.reshape(wl.nh, wl.d_v, wl.d_k).contiguous()
     sm0 = int(wl.smoothing)
     variants = {"per_window": (wl.window, wl.n_comp, sm0, 8),
+                "per_window_svd": (wl.window, wl.n_comp, sm0, 8, lq.LQ_COMP_SVD),
                 "per_token": (1, 0, sm0, 8), "per_token_plain": (1, 0, 0, 8),
                 "per_window_6bit": (wl.window, wl.n_comp, sm0, 6), "per_token_6bit": (1, 0, sm0, 6),
                 "per_window_4bit": (wl.window, wl.n_comp, sm0, 4), "per_token_4bit": (1, 0, sm0, 4),
                 "per_window_bf16": (wl.window, 0, 0, 16), "per_token_bf16": (1, 0, 0, 16)}
     states, cfgs = {}, {}
-    for name, (W, r, sm, bits) in variants.items():
+    for name, (W, r, sm, bits, *rule) in variants.items():
         cfg = lq.Config(batch=wl.batch, heads=wl.heads, d_k=wl.d_k, d_v=wl.d_v, window=W, n_comp=r,
                         gate=lq.LQ_GATE_DIAG if wl.gate == "diag" else lq.LQ_GATE_SCALAR,
                         io_dtype=lq.LQ_BF16 if wl.io == "bf16" else lq.LQ_F32, smoothing=sm,
-                        auto_commit=1, bits=bits)
+                        auto_commit=1, bits=bits, comp_rule=rule[0] if rule else lq.LQ_COMP_ROWS)
         st = lq.State(cfg, dev)
         lq.lq_state_init(st, S0)
         states[name], cfgs[name] = st, cfg
@@ -867,7 +882,9 @@ def run_mse(args, wl):
     def dequant(st):
         t = st.snap.t
         Sh = (t["row_scale"][:, :, None] * codes_float(st) * t["col_smooth"][:, None, :])
-        if t["comp_row"].numel():
+        if "comp_u" in t:  # SVD rule: rank-one compensators
+            Sh += torch.einsum("hcv,hck->hvk", t["comp_u"], t["comp_val"])
+        elif t["comp_row"].numel():
             Sh.scatter_add_(1, t["comp_row"].long()[:, :, None].expand(-1, -1, wl.d_k), t["comp_val"])
         return Sh
 
@@ -888,7 +905,8 @@ def run_mse(args, wl):
     return {"report": "state MSE relative to the mean square of the FP32 state, at window ends",
             "workload": wl.name, "batch": wl.batch, "heads": wl.heads, "steps": steps,
             "window": W, "n_comp": wl.n_comp, "results": out,
-            "variants": {n: {"window": v[0], "n_comp": v[1], "smoothing": bool(v[2]), "bits": v[3]}
+            "variants": {n: {"window": v[0], "n_comp": v[1], "smoothing": bool(v[2]), "bits": v[3],
+                             "comp_rule": "svd" if v[4:] == (lq.LQ_COMP_SVD,) else "rows"}
                          for n, v in variants.items()}}
 
 
@@ -910,6 +928,8 @@ def main(argv=None):
     ap.add_argument("--no-smoothing", action="store_true")
     ap.add_argument("--delta", type=int, choices=[0, 1], default=None,
                     help="0: the b = 0 rows of equation 1 (linear attention / Mamba2 / GLA)")
+    ap.add_argument("--comp-rule", choices=["rows", "svd"], default="rows",
+                    help="compensator rule: top-r rows (default) or top-r singular triplets")
     ap.add_argument("--bits", type=int, choices=[8, 6, 4, 16], default=8,
                     help="code width of the state (8; 6 and 4 are the narrow variants; 16 = BF16)")
     ap.add_argument("--slots", type=int, default=8, help="distinct input windows (graphs)")

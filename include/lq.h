@@ -74,6 +74,20 @@ typedef enum {
 typedef enum { LQ_GATE_SCALAR = 0, LQ_GATE_DIAG = 1 } lq_gate;
 typedef enum { LQ_F32 = 0, LQ_BF16 = 1 } lq_dtype;
 
+/* How the r Compensator Tokens of a snapshot are chosen ("LeapQuant: ...",
+ * Abstract and Figure 4 keep the state's largest outliers in high precision
+ * and flatten the residual's row norms, without fixing the rule):
+ *   LQ_COMP_ROWS  the r value rows of largest l2 norm, stored exactly
+ *                 (comp_row, comp_val);
+ *   LQ_COMP_SVD   the r largest singular triplets of the FP32 state, as
+ *                 rank-one terms u_c k~_c^T with u_c = s_c U_c (comp_u) and
+ *                 k~_c = V_c (comp_val), the largest-magnitude entry of k~_c
+ *                 positive; the residual S - sum_c u_c k~_c^T is smoothed
+ *                 and quantized as with LQ_COMP_ROWS.  This library's variant:
+ *                 the pages fix no rule, and the singular triplets are
+ *                 computed by subspace iteration (see lq_state_init). */
+typedef enum { LQ_COMP_ROWS = 0, LQ_COMP_SVD = 1 } lq_comp_rule;
+
 typedef struct {
     int32_t batch;       /* B >= 1                                          */
     int32_t heads;       /* H >= 1; B * H <= 2^24 (LQ_ERR_INVALID_ARGUMENT)  */
@@ -101,6 +115,7 @@ typedef struct {
                             ablation: compensators as above, the residual
                             stored as BF16 values (round to nearest even),
                             no smoothing, row_scale = col_smooth = 1.      */
+    int32_t comp_rule;   /* lq_comp_rule (0 = LQ_COMP_ROWS)                  */
 } lq_config;
 
 /* The quantized boundary state of every (b, h), all device memory:
@@ -118,14 +133,17 @@ typedef struct {
  *   comp_row   int32   [B*H][r]                row index of each compensator,
  *                                              largest l2 norm first
  *   comp_val   float   [B*H][r][d_k]    (16B)  the compensator rows (FP32)
- * S^_0 = Diag(row_scale) codes Diag(col_smooth) + sum_c e_{comp_row[c]} comp_val[c]^T.
- * comp_row and comp_val may be NULL when r == 0. */
+ *   comp_u     float   [B*H][r][d_v]    (16B)  LQ_COMP_SVD: u_c = s_c U_c
+ * S^_0 = Diag(row_scale) codes Diag(col_smooth) + sum_c e_{comp_row[c]} comp_val[c]^T
+ * (LQ_COMP_ROWS), or + sum_c comp_u[c] comp_val[c]^T (LQ_COMP_SVD; comp_row
+ * then holds zeros).  comp_row, comp_val and comp_u may be NULL when r == 0. */
 typedef struct {
     int8_t *codes;
     float *row_scale;
     float *col_smooth;
     int32_t *comp_row;
     float *comp_val;
+    float *comp_u;   /* LQ_COMP_SVD only (else ignored, may be NULL)      */
 } lq_snapshot;
 
 /* A decode state.  The caller fills `snap` and the three window buffers with
@@ -158,7 +176,7 @@ typedef struct {
  * int8, uint8 at bits = 4, bf16 at bits = 16); -1 for an invalid
  * configuration.
  * which: 0 codes, 1 row_scale, 2 col_smooth, 3 comp_row, 4 comp_val,
- *        5 buf_gate, 6 buf_k, 7 buf_u. */
+ *        5 buf_gate, 6 buf_k, 7 buf_u, 8 comp_u (0 with LQ_COMP_ROWS). */
 LQ_API int64_t lq_buffer_elems(const lq_config *cfg, int32_t which);
 
 /* Initialises `st` with configuration `cfg` and quantizes the FP32 state
@@ -169,6 +187,17 @@ LQ_API int64_t lq_buffer_elems(const lq_config *cfg, int32_t which);
  * per-row codes of lq_config.bits.  The residual's codes are taken with
  * exact FP32 quotients (R / c_j, then R' / sigma_i), so they are a function
  * of S_init alone.
+ * With cfg.comp_rule = LQ_COMP_SVD the compensators are the r largest
+ * singular triplets of each head's FP32 state, computed on the device by
+ * subspace iteration: the Gram matrix S^T S, r + 8 basis vectors (at most
+ * d_k; deterministic start vectors, or at a window commit the previous
+ * compensators' k~_c in the first r), 16 iterations each orthonormalised by
+ * an FP64 Cholesky factorisation, then a Rayleigh-Ritz step (FP64 Jacobi
+ * eigensolver) on the basis.  Singular values and well-separated singular
+ * vectors match an exact SVD to FP32 accuracy; vectors of nearly equal
+ * singular values are a valid basis of their (ill-defined) subspace, not a
+ * particular one.  It is much slower than LQ_COMP_ROWS (one CTA of 512
+ * threads per head at init, prefill snapshots and every window commit).
  * S_init == NULL means the zero state.  Sets pos = 0 (also from
  * LQ_POS_PER_SEQUENCE). */
 LQ_API lq_status lq_state_init(lq_state *st, const lq_config *cfg, const float *S_init,

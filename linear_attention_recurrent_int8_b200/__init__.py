@@ -25,6 +25,7 @@ LQ_OK, LQ_ERR_INVALID_ARGUMENT, LQ_ERR_UNSUPPORTED, LQ_ERR_WINDOW_FULL, \
     LQ_ERR_WINDOW_OPEN, LQ_ERR_MISALIGNED, LQ_ERR_CUDA = range(7)
 LQ_GATE_SCALAR, LQ_GATE_DIAG = 0, 1
 LQ_F32, LQ_BF16 = 0, 1
+LQ_COMP_ROWS, LQ_COMP_SVD = 0, 1
 LQ_POS_PER_SEQUENCE = -1
 LQ_DEVERR_WAIT_TIMEOUT, LQ_DEVERR_BAD_POSITION = 1, 2
 
@@ -44,13 +45,13 @@ class LQError(RuntimeError):
 class LqConfig(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("batch", "heads", "d_k", "d_v", "window", "n_comp",
                                               "gate", "io_dtype", "smoothing", "auto_commit", "delta",
-                                              "bits")]
+                                              "bits", "comp_rule")]
 
 
 class LqSnapshot(ctypes.Structure):
     _fields_ = [("codes", ctypes.c_void_p), ("row_scale", ctypes.c_void_p),
                 ("col_smooth", ctypes.c_void_p), ("comp_row", ctypes.c_void_p),
-                ("comp_val", ctypes.c_void_p)]
+                ("comp_val", ctypes.c_void_p), ("comp_u", ctypes.c_void_p)]
 
 
 class LqState(ctypes.Structure):
@@ -187,6 +188,8 @@ def _snapshot_specs(cfg: "Config", snap: "Snapshot", name: str):
     if cfg.n_comp > 0:
         specs += [(t["comp_row"], f"{name}.comp_row", torch.int32, bh * cfg.n_comp),
                   (t["comp_val"], f"{name}.comp_val", torch.float32, bh * cfg.n_comp * cfg.d_k)]
+    if cfg.svd:
+        specs += [(t["comp_u"], f"{name}.comp_u", torch.float32, bh * cfg.n_comp * cfg.d_v)]
     return specs
 
 
@@ -208,11 +211,17 @@ class Config:
     auto_commit: int = 1
     delta: int = 1
     bits: int = 8  # code width: 8, 6 (one code per byte), 4 (two per byte), 16 (BF16 residual)
+    comp_rule: int = LQ_COMP_ROWS  # LQ_COMP_ROWS (top-r rows) or LQ_COMP_SVD (top-r singular triplets)
 
     def c(self) -> LqConfig:
         return LqConfig(self.batch, self.heads, self.d_k, self.d_v, self.window, self.n_comp,
                         self.gate, self.io_dtype, self.smoothing, self.auto_commit, self.delta,
-                        self.bits)
+                        self.bits, self.comp_rule)
+
+    @property
+    def svd(self) -> bool:
+        """The SVD compensator rule is in effect (with r = 0 the rules coincide)."""
+        return self.comp_rule == LQ_COMP_SVD and self.n_comp > 0
 
     @property
     def code_cols(self) -> int:
@@ -249,6 +258,9 @@ class Snapshot:
                 comp_row=torch.zeros((bh, cfg.n_comp), dtype=torch.int32, device=device),
                 comp_val=torch.zeros((bh, cfg.n_comp, cfg.d_k), dtype=torch.float32, device=device),
             )
+            if cfg.svd:
+                tensors["comp_u"] = torch.zeros((bh, cfg.n_comp, cfg.d_v), dtype=torch.float32,
+                                                device=device)
         self.t = tensors
 
     def __getitem__(self, key):
@@ -257,10 +269,12 @@ class Snapshot:
     def c(self) -> LqSnapshot:
         t = self.t
         has = t["comp_row"].numel() > 0
+        cu = t.get("comp_u")
         return LqSnapshot(t["codes"].data_ptr(), t["row_scale"].data_ptr(),
                           t["col_smooth"].data_ptr(),
                           t["comp_row"].data_ptr() if has else None,
-                          t["comp_val"].data_ptr() if has else None)
+                          t["comp_val"].data_ptr() if has else None,
+                          cu.data_ptr() if cu is not None and cu.numel() > 0 else None)
 
     def cpu(self) -> dict:
         return {k: v.cpu().numpy() for k, v in self.t.items()}

@@ -35,8 +35,13 @@ lq_status check_config(const lq_config *c) {
         return LQ_ERR_INVALID_ARGUMENT;
     if (c->bits != 0 && c->bits != 8 && c->bits != 6 && c->bits != 4 && c->bits != 16)
         return LQ_ERR_INVALID_ARGUMENT;
+    if (c->comp_rule != LQ_COMP_ROWS && c->comp_rule != LQ_COMP_SVD) return LQ_ERR_INVALID_ARGUMENT;
+    if (c->comp_rule == LQ_COMP_SVD && c->n_comp > c->d_k) return LQ_ERR_INVALID_ARGUMENT;
     return LQ_OK;
 }
+
+// The SVD compensator rule is in effect (with r = 0 both rules are the same).
+bool svd_rule(const lq_config *c) { return c->comp_rule == LQ_COMP_SVD && c->n_comp > 0; }
 
 // Code width of a valid configuration (0 means 8).
 int code_bits(const lq_config *c) { return c->bits == 0 ? 8 : c->bits; }
@@ -60,6 +65,8 @@ lq_status check_snapshot(const lq_config *c, const lq_snapshot *s) {
         return LQ_ERR_MISALIGNED;
     if (c->n_comp > 0 && (!aligned16(s->comp_val) || !aligned_to(s->comp_row, 4)))
         return LQ_ERR_MISALIGNED;
+    if (svd_rule(c) && !s->comp_u) return LQ_ERR_INVALID_ARGUMENT;
+    if (svd_rule(c) && !aligned16(s->comp_u)) return LQ_ERR_MISALIGNED;
     return LQ_OK;
 }
 
@@ -96,6 +103,7 @@ lq::DecodeArgs decode_args(const lq_state *st) {
     a.col_smooth = st->snap.col_smooth;
     a.comp_row = st->cfg.n_comp > 0 ? st->snap.comp_row : nullptr;
     a.comp_val = st->cfg.n_comp > 0 ? st->snap.comp_val : nullptr;
+    a.comp_u = svd_rule(&st->cfg) ? st->snap.comp_u : nullptr;
     a.buf_gate = st->buf_gate;
     a.buf_k = st->buf_k;
     a.buf_u = st->buf_u;
@@ -118,6 +126,7 @@ lq::QuantArgs quant_args(const lq_config *c, const float *S, const lq_snapshot *
     a.col_smooth = s->col_smooth;
     a.comp_row = c->n_comp > 0 ? s->comp_row : nullptr;
     a.comp_val = c->n_comp > 0 ? s->comp_val : nullptr;
+    a.comp_u = svd_rule(c) ? s->comp_u : nullptr;
     a.BH = c->batch * c->heads;
     a.R = c->n_comp;
     a.smoothing = c->smoothing;
@@ -141,6 +150,8 @@ lq_status copy_snapshot(const lq_config *c, const lq_snapshot *dst, const lq_sna
     if (e == cudaSuccess && c->n_comp > 0)
         e = cudaMemcpyAsync(dst->comp_val, src->comp_val, bh * c->n_comp * c->d_k * 4, kind,
                             stream);
+    if (e == cudaSuccess && svd_rule(c))
+        e = cudaMemcpyAsync(dst->comp_u, src->comp_u, bh * c->n_comp * c->d_v * 4, kind, stream);
     return cuda_status(e);
 }
 
@@ -161,6 +172,7 @@ int64_t lq_buffer_elems(const lq_config *cfg, int32_t which) {
         case 5: return bh * cfg->window * G;
         case 6: return bh * cfg->window * cfg->d_k;
         case 7: return bh * cfg->window * cfg->d_v;
+        case 8: return cfg->comp_rule == LQ_COMP_SVD ? bh * cfg->n_comp * cfg->d_v : 0;
         default: return -1;
     }
 }

@@ -721,6 +721,7 @@ cudaError_t launch_reset_positions(int32_t *seq_pos, int B, int W, cudaStream_t 
 cudaError_t launch_commit(const DecodeArgs &a, int d_k, int d_v, int gate, cudaStream_t stream) {
     if (a.pos < 1 || a.pos > 32 || a.R < 0 || a.R > kMaxComp) return cudaErrorInvalidValue;
     if (a.bits != 8 && a.bits != 6 && a.bits != 4 && a.bits != 16) return cudaErrorInvalidValue;
+    if (a.comp_u && a.R > 0) return launch_svd_commit(a, d_k, d_v, gate, stream);
     if (d_k == 128 && d_v == 128) return launch_c_d<128, 128>(a, gate, stream);
     if (d_k == 128 && d_v == 64) return launch_c_d<128, 64>(a, gate, stream);
     if (d_k == 64 && d_v == 128) return launch_c_d<64, 128>(a, gate, stream);

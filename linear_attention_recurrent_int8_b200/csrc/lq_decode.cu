@@ -14,7 +14,8 @@
 // (D_{1..t-1} b_t = e^{L_{t-1}} alpha_t k_t = e^{L_t} k_t for both gate kinds;
 // e^{x} is per key channel for the diagonal gate.)  Compensator Tokens are
 // pseudo-records at window position 0 (Figure 4; they share the update path
-// of real tokens), so they enter with decay e^{L_t}.
+// of real tokens), so they enter with decay e^{L_t}: record (e_row, comp_val)
+// under the row rule, (u_c, k~_c) under the SVD rule (lq_svd.cu).
 //
 // The boundary state's residual is stored as 8-bit (or 6-bit) codes one per
 // byte, 4-bit codes two per byte (layout in lq_quant.cuh), or BF16 values
@@ -89,7 +90,7 @@ __host__ __device__ inline PrepLayout prep_layout(int DK, int fmt, bool tc = fal
 // of record slots the stage holds (records read plus records written), `n`
 // the number of tokens of the call; `fmt` the residual's storage.
 struct StageLayout {
-    int codes, bop, sig, cs, compv, compr, recK, recU, recL, q, k, v, al, scal, prep, bytes;
+    int codes, bop, sig, cs, compv, compr, compu, recK, recU, recL, q, k, v, al, scal, prep, bytes;
 };
 
 // Rows of the tensor-core matvec's B operand for n tokens: 8 per token (x_k
@@ -100,8 +101,10 @@ __host__ __device__ constexpr int tc_rows(int n) { return n == 1 ? 8 : 16 * ((n 
 // With tc (tensor-core matvec) the codes and the B operand are not part of
 // the stage (they live in a separate 1024-byte aligned array, tc_tile_bytes
 // per stage) and codes = bop = -1.
+// ru: rows of rank-one compensator vectors u_c (R with the SVD rule, else 0).
 __host__ __device__ inline StageLayout stage_layout(int DK, int DV, int gate, int R, int nrec,
-                                                   int n, int e, int fmt, bool tc = false) {
+                                                   int n, int e, int fmt, bool tc = false,
+                                                   int ru = 0) {
     StageLayout L{};
     int o = 0;
     L.codes = tc ? -1 : o;
@@ -111,6 +114,7 @@ __host__ __device__ inline StageLayout stage_layout(int DK, int DV, int gate, in
     L.cs = o;    o += align16(4 * DK);
     L.compv = o; o += align16(4 * R * DK);
     L.compr = o; o += align16(4 * kMaxComp);
+    L.compu = o; o += align16(4 * ru * DV);
     L.recK = o;  o += align16(4 * nrec * DK);
     L.recU = o;  o += align16(4 * nrec * DV);
     L.recL = o;  o += align16(4 * nrec * (gate == 1 ? DK : 1));
@@ -318,7 +322,7 @@ __device__ __forceinline__ void prep_role(const DecodeArgs &a, const StageLayout
                     if (GATE == 0 && lane == 0) a.buf_gate[(size_t)bh * W + nrec] = Ls;
                 }
                 __syncwarp();
-                // coefficients of records 0..nrec-1 and compensators, P = 8
+                // coefficients of records 0..nrec-1 and compensators, P
                 // items per pass, passes shared round-robin by the prep-B
                 // warps; the 2P partial dot products of a pass are reduced
                 // together with a transposing reduction
@@ -385,12 +389,19 @@ __device__ __forceinline__ void prep_role(const DecodeArgs &a, const StageLayout
                         else coefG[it] = v;
                     }
                 };
-                for (int base = 8 * bpart; base < nitems; base += 8 * NPB)
-                    coef_pass(std::integral_constant<int, 8>{}, base);
+                // passes of 4 items over four prep-B warps (tensor-core decode),
+                // of 8 items over two (dp4a decode)
+                constexpr int PI = NPB >= 4 ? 4 : 8;
+                for (int base = PI * bpart; base < nitems; base += PI * NPB)
+                    coef_pass(std::integral_constant<int, PI>{}, base);
             }
             __syncwarp();
         }
-        fence_proxy_async_smem();
+        // generic-proxy writes that a later asynchronous copy into this stage
+        // (or the tensor-core MMA) reads or overwrites: the limbs of the MMA's
+        // B operand, and the records of a multi-token call.  The coefficients
+        // live in the prep slot, which no copy writes.
+        if ((isA && TC) || nsteps > 1) fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
             mbar_arrive(&prepared[s]);
@@ -413,7 +424,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a,
     uint64_t *prepared = full + kMaxStages;
     uint64_t *empty = prepared + kMaxStages;
     const int nsteps = a.n_steps;
-    const StageLayout SL = stage_layout(DK, DV, GATE, a.R, a.pos + nsteps, nsteps, E, FMT);
+    const StageLayout SL = stage_layout(DK, DV, GATE, a.R, a.pos + nsteps, nsteps, E, FMT, false, a.comp_u ? a.R : 0);
     const PrepLayout PL = prep_layout(DK, FMT);
     unsigned char *stages = smem + header_bytes();
 
@@ -449,7 +460,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a,
             const uint32_t in_bytes =
                 nsteps > 0 ? (uint32_t)(E * (2 * DK + DV) + (GATE == 1 ? 4 * DK : 0)) : 0u;
             const uint32_t bytes = DV * CRB + 4 * DV + 4 * DK + 4 * R * DK + 4 * pos * (DK + DV) +
-                                   (GATE == 1 ? 4 * pos * DK : 0) + in_bytes;
+                                   (GATE == 1 ? 4 * pos * DK : 0) + in_bytes + (a.comp_u ? 4 * R * DV : 0);
             // small operands by 4-byte copies, tracked by the same barrier:
             // alpha and beta of token 0, the scalar-gate records, the
             // compensator rows
@@ -469,6 +480,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a,
             bulk_g2s(st + SL.sig, a.row_scale + (size_t)bh * DV, 4 * DV, &full[s]);
             bulk_g2s(st + SL.cs, a.col_smooth + (size_t)bh * DK, 4 * DK, &full[s]);
             if (R > 0) bulk_g2s(st + SL.compv, a.comp_val + (size_t)bh * R * DK, 4 * R * DK, &full[s]);
+            if (a.comp_u) bulk_g2s(st + SL.compu, a.comp_u + (size_t)bh * R * DV, 4 * R * DV, &full[s]);
             if (pos > 0) {
                 bulk_g2s(st + SL.recK, a.buf_k + (size_t)bh * W * DK, 4 * pos * DK, &full[s]);
                 bulk_g2s(st + SL.recU, a.buf_u + (size_t)bh * W * DV, 4 * pos * DV, &full[s]);
@@ -642,11 +654,21 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a,
                     p += __shfl_xor_sync(0xffffffffu, p, o);
                 }
                 if (part == 0) {
-                    for (int c = 0; c < R; ++c)
-                        if (compr_s[c] == row) {
-                            hb += coefA[nrec + c];
-                            p += coefG[nrec + c];
+                    if (a.comp_u) {
+                        // rank-one compensators (SVD rule): u_c[row] times the coefficient
+                        const float *compu_s = reinterpret_cast<const float *>(st + SL.compu);
+                        for (int c = 0; c < R; ++c) {
+                            const float uc = compu_s[c * DV + row];
+                            hb = fmaf(coefA[nrec + c], uc, hb);
+                            p = fmaf(coefG[nrec + c], uc, p);
                         }
+                    } else {
+                        for (int c = 0; c < R; ++c)
+                            if (compr_s[c] == row) {
+                                hb += coefA[nrec + c];
+                                p += coefG[nrec + c];
+                            }
+                    }
                     const float vi = sidx == 0 ? load_io<BF16>(st + SL.v, row)
                                                : load_io<BF16>(a.v, tok * DV + row);
                     const float u = vi - hb;
@@ -726,7 +748,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint64_t *empty = mma_done + NBAR;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(reinterpret_cast<uint64_t *>(smem) + 4 * NBAR);
     const int nsteps = a.n_steps;
-    const StageLayout SL = stage_layout(DK, DV, GATE, a.R, a.pos + nsteps, nsteps, E, FMT, true);
+    const StageLayout SL = stage_layout(DK, DV, GATE, a.R, a.pos + nsteps, nsteps, E, FMT, true, a.comp_u ? a.R : 0);
     const PrepLayout PL = prep_layout(DK, FMT, true);
     const int TB = tc_tile_bytes(nsteps);
     // this pipeline's tiles (codes + B operand, 1024-aligned) and stages
@@ -770,7 +792,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 const size_t tok = (size_t)b * nsteps * a.H + h;  // token 0 of this call
                 const uint32_t in_bytes = (uint32_t)(E * (2 * DK + DV) + (GATE == 1 ? 4 * DK : 0));
                 const uint32_t bytes = DV * DK + 4 * DV + 4 * DK + 4 * R * DK + 4 * pos * (DK + DV) +
-                                       (GATE == 1 ? 4 * pos * DK : 0) + in_bytes;
+                                       (GATE == 1 ? 4 * pos * DK : 0) + in_bytes + (a.comp_u ? 4 * R * DV : 0);
                 float *scal = reinterpret_cast<float *>(st + SL.scal);
                 if (GATE == 0) cp_async4(scal, a.alpha + tok);
                 cp_async4(scal + 1, a.beta + tok);
@@ -785,6 +807,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 bulk_g2s(st + SL.sig, a.row_scale + (size_t)bh * DV, 4 * DV, &full[s]);
                 bulk_g2s(st + SL.cs, a.col_smooth + (size_t)bh * DK, 4 * DK, &full[s]);
                 if (R > 0) bulk_g2s(st + SL.compv, a.comp_val + (size_t)bh * R * DK, 4 * R * DK, &full[s]);
+                if (a.comp_u) bulk_g2s(st + SL.compu, a.comp_u + (size_t)bh * R * DV, 4 * R * DV, &full[s]);
                 if (pos > 0) {
                     bulk_g2s(st + SL.recK, a.buf_k + (size_t)bh * W * DK, 4 * pos * DK, &full[s]);
                     bulk_g2s(st + SL.recU, a.buf_u + (size_t)bh * W * DV, 4 * pos * DV, &full[s]);
@@ -888,11 +911,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     hb = fmaf(coefA[m], um, hb);
                     p = fmaf(coefG[m], um, p);
                 }
-                for (int c = 0; c < R; ++c)
-                    if (compr_s[c] == row) {
-                        hb += coefA[nrec + c];
-                        p += coefG[nrec + c];
+                if (a.comp_u) {
+                    // rank-one compensators (SVD rule): u_c[row] times the coefficient
+                    const float *compu_s = reinterpret_cast<const float *>(st + SL.compu);
+                    for (int c = 0; c < R; ++c) {
+                        const float uc = compu_s[c * DV + row];
+                        hb = fmaf(coefA[nrec + c], uc, hb);
+                        p = fmaf(coefG[nrec + c], uc, p);
                     }
+                } else {
+                    for (int c = 0; c < R; ++c)
+                        if (compr_s[c] == row) {
+                            hb += coefA[nrec + c];
+                            p += coefG[nrec + c];
+                        }
+                }
                 const float vi = sidx == 0 ? load_io<BF16>(st + SL.v, row) : load_io<BF16>(a.v, tok * DV + row);
                 const float u = vi - hb;
                 const float o = fmaf(coefG[nrec + R], u, p);
@@ -950,7 +983,8 @@ cudaError_t launch_tc(const DecodeArgs &a, cudaStream_t stream) {
         sm_count[dev & 63] = sms;
         configured.fetch_or(bit, std::memory_order_acq_rel);
     }
-    const StageLayout SL = stage_layout(128, 128, GATE, a.R, a.pos + a.n_steps, a.n_steps, E, kCodesI8, true);
+    const StageLayout SL = stage_layout(128, 128, GATE, a.R, a.pos + a.n_steps, a.n_steps, E, kCodesI8, true,
+                                        a.comp_u ? a.R : 0);
     const int fixed = 1024 + kTcHeader;  // alignment slack + header
     const int NB = tc_rows(a.n_steps);
     const int per_stage = SL.bytes + tc_tile_bytes(a.n_steps);
@@ -1004,7 +1038,8 @@ cudaError_t launch_d(const DecodeArgs &a, cudaStream_t stream) {
         configured.fetch_or(bit, std::memory_order_acq_rel);
     }
     // a stage holds the records this launch reads and writes (pos + n_steps)
-    const StageLayout SL = stage_layout(DK, DV, GATE, a.R, a.pos + a.n_steps, a.n_steps, E, FMT);
+    const StageLayout SL = stage_layout(DK, DV, GATE, a.R, a.pos + a.n_steps, a.n_steps, E, FMT, false,
+                                        a.comp_u ? a.R : 0);
     const int fixed = header_bytes();
     // two CTAs per SM when registers allow it and each can hold at least
     // two stages, else one CTA per SM with as many stages as fit

@@ -44,6 +44,7 @@ struct DecodeArgs {
     float *col_smooth;
     int32_t *comp_row;
     float *comp_val;
+    float *comp_u;  // SVD compensator rule: u_c [BH][R][DV]; nullptr for the row rule
     float *buf_gate;
     float *buf_k;
     float *buf_u;
@@ -80,6 +81,7 @@ struct QuantArgs {
     float *col_smooth;
     int32_t *comp_row;
     float *comp_val;
+    float *comp_u;  // SVD compensator rule: u_c [BH][R][DV]; nullptr for the row rule
     int BH, R, smoothing;
     int bits;  // code width: 8 or 6 (one code per byte), 4 (two per byte), 16 (BF16)
 };
@@ -140,7 +142,15 @@ cudaError_t launch_reset_positions(int32_t *seq_pos, int B, int W, cudaStream_t 
 // Reads the device error word and clears it (synchronizes the device).
 cudaError_t read_and_clear_dev_error(unsigned int *out);
 
+// Quantizes FP32 states (a.S) into snapshots; with a.comp_u set, by the SVD
+// compensator rule (lq_svd.cu).
 cudaError_t launch_quantize(const QuantArgs &a, int d_k, int d_v, cudaStream_t stream);
+
+// The SVD compensator rule (lq_svd.cu): snapshots of FP32 states (a.S), and
+// the window commit of a.pos >= 1 records (rebuild from the snapshot and the
+// records, then the rule), written over the snapshot.
+cudaError_t launch_svd_quantize(const QuantArgs &a, int d_k, int d_v, cudaStream_t stream);
+cudaError_t launch_svd_commit(const DecodeArgs &a, int d_k, int d_v, int gate, cudaStream_t stream);
 
 // rows_per_cta selects the parallelisation: the full head (one CTA per head,
 // for a few tokens) or a slice of rows (many CTAs per head, for long runs).

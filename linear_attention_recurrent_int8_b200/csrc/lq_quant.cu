@@ -47,6 +47,14 @@ cudaError_t launch_q(const QuantArgs &a, cudaStream_t stream) {
 }  // namespace
 
 cudaError_t launch_quantize(const QuantArgs &a, int d_k, int d_v, cudaStream_t stream) {
+    if (a.comp_u && a.R > 0) {
+        if (a.S) return launch_svd_quantize(a, d_k, d_v, stream);
+        // the zero state under the SVD rule: every u_c = 0, and the row
+        // rule's kernel writes the zero residual (codes, sigma = 0, c = 1)
+        // and zero k~_c
+        const cudaError_t e = cudaMemsetAsync(a.comp_u, 0, (size_t)a.BH * a.R * d_v * sizeof(float), stream);
+        if (e != cudaSuccess) return e;
+    }
     if (d_k == 128 && d_v == 128) return launch_q<128, 128>(a, stream);
     if (d_k == 128 && d_v == 64) return launch_q<128, 64>(a, stream);
     if (d_k == 64 && d_v == 128) return launch_q<64, 128>(a, stream);

@@ -46,7 +46,13 @@ def test_buffer_elems():
     want = [bh * 64 * 128, bh * 64, bh * 128, bh * 4, bh * 4 * 128, bh * 16 * 128,
             bh * 16 * 128, bh * 16 * 64]
     assert [lq.lq_buffer_elems(cfg, w) for w in range(8)] == want
-    assert lq.lq_buffer_elems(cfg, 8) == -1
+    assert lq.lq_buffer_elems(cfg, 8) == 0  # comp_u: only with the SVD rule
+    assert lq.lq_buffer_elems(cfg, 9) == -1
+    cfg.comp_rule = lq.LQ_COMP_SVD
+    assert lq.lq_buffer_elems(cfg, 8) == bh * 4 * 64
+    cfg.comp_rule = 2
+    assert lq.lq_buffer_elems(cfg, 8) == -1  # not a rule
+    cfg.comp_rule = lq.LQ_COMP_ROWS
     cfg.gate = lq.LQ_GATE_SCALAR
     assert lq.lq_buffer_elems(cfg, 5) == bh * 16
     # code bytes: one per code at 8 and 6 bits (0 means 8), half a byte at 4

@@ -58,6 +58,15 @@ def test_profile_key_names_overrides():
     A.bits = 8
     w8 = dataclasses.replace(wl, window=8)
     assert bench.profile_key("commit", w8, A) == "commit:gdn_256x32_d128_bf16_W8_r4_s1_b8"
+    A.comp_rule = "svd"
+    assert bench.profile_key("decode", wl, A) == "decode:gdn_256x32_d128_bf16_svd"
+
+
+def test_svd_rule_byte_model():
+    """The SVD rule adds the r u_c vectors (4 d_v bytes each) to a snapshot."""
+    assert bench.snapshot_bytes(128, 128, 4, 8, svd=True) == 19472 + 4 * 4 * 128
+    assert bench.decode_launch_bytes(128, 128, 4, "scalar", 2, 1, 8, True) == \
+        bench.decode_launch_bytes(128, 128, 4, "scalar", 2, 1, 8) + 4 * 4 * 128
 
 
 def test_narrow_code_byte_models():
