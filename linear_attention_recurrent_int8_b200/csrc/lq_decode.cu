@@ -139,10 +139,11 @@ __host__ __device__ constexpr int header_bytes() { return 3 * kMaxStages * 8; }
 // x ~= s (X0 + X1/2^7 [+ X2/2^14]), |error| <= s / 2^(7 NL - 6) (plus FP32
 // rounding).  Writes limb l as row row0 + l of `limb` -- plain rows of DK
 // bytes, or (SW128, d_k = 128) the rows of a K-major operand with the
-// 128-byte swizzle -- and *lscale.
+// 128-byte swizzle -- and *lscale = s * post (post: a factor of the vector
+// that was left out of x, such as a scalar gate).
 template <int CPL, int NL, bool SW128 = false>
 __device__ __forceinline__ void split_limbs(const float (&x)[CPL], int8_t *limb, int DK,
-                                            float *lscale, int j0, int row0) {
+                                            float *lscale, int j0, int row0, float post = 1.0f) {
     float m = 0.0f;
 #pragma unroll
     for (int e = 0; e < CPL; ++e) m = fmaxf(m, fabsf(x[e]));
@@ -174,7 +175,7 @@ __device__ __forceinline__ void split_limbs(const float (&x)[CPL], int8_t *limb,
             *reinterpret_cast<uint16_t *>(limb + r * DK + j0) = (uint16_t)w[l];
         }
     }
-    if (threadIdx.x % 32 == 0) *lscale = m * (1.0f / 127.0f);
+    if (threadIdx.x % 32 == 0) *lscale = (m * (1.0f / 127.0f)) * post;
 }
 
 // The next head (sequence-major index) of a walk with stride `stride` at or
@@ -272,12 +273,17 @@ __device__ __forceinline__ void prep_role(const DecodeArgs &a, const StageLayout
                 float *lscale = reinterpret_cast<float *>(slot + PL.lscale);
                 float cj[CPL], xk[CPL], xq[CPL], kq = 0.0f;
                 load_vec<CPL>(cj, cs_s + j0);
+                // scalar gate with integer limbs: e^{L_t} goes into the limb
+                // scales (after the split), off the split's dependency chain
+                constexpr bool GPOST = GATE == 0 && !BF16S;
 #pragma unroll
                 for (int e = 0; e < CPL; ++e) {
-                    xk[e] = a.delta ? cj[e] * (gj[e] * kj[e]) : 0.0f;  // b = 0 rows: no S b term
-                    xq[e] = cj[e] * (gj[e] * qj[e]);
+                    const float g = GPOST ? 1.0f : gj[e];
+                    xk[e] = a.delta ? cj[e] * (g * kj[e]) : 0.0f;  // b = 0 rows: no S b term
+                    xq[e] = cj[e] * (g * qj[e]);
                     kq = fmaf(beta * kj[e], qj[e], kq);
                 }
+                const float gpost = GPOST ? g_s : 1.0f;
                 // with NA = 2 prep-A warps, warp arole 0 takes x_k, warp 1 x_q and k~ . q
                 const bool doK = NA == 1 || arole == 0, doQ = NA == 1 || arole == 1;
                 if constexpr (BF16S) {
@@ -291,11 +297,11 @@ __device__ __forceinline__ void prep_role(const DecodeArgs &a, const StageLayout
                     if constexpr (TC) {
                         // rows 8 sidx + 0..2 (x_k) and + 3..5 (x_q) of the B operand
                         int8_t *bop = reinterpret_cast<int8_t *>(tiles + (size_t)s * tc_tile_bytes(nsteps) + DV * DK);
-                        if (doK && a.delta) split_limbs<CPL, 3, true>(xk, bop, DK, lscale, j0, 8 * sidx);
-                        if (doQ) split_limbs<CPL, 3, true>(xq, bop, DK, lscale + 1, j0, 8 * sidx + 3);
+                        if (doK && a.delta) split_limbs<CPL, 3, true>(xk, bop, DK, lscale, j0, 8 * sidx, gpost);
+                        if (doQ) split_limbs<CPL, 3, true>(xq, bop, DK, lscale + 1, j0, 8 * sidx + 3, gpost);
                     } else {
-                        if (a.delta) split_limbs<CPL, 3>(xk, limb, DK, lscale, j0, 0);
-                        split_limbs<CPL, 3>(xq, limb, DK, lscale + 1, j0, 3);
+                        if (a.delta) split_limbs<CPL, 3>(xk, limb, DK, lscale, j0, 0, gpost);
+                        split_limbs<CPL, 3>(xq, limb, DK, lscale + 1, j0, 3, gpost);
                     }
                 }
                 if (doQ) {

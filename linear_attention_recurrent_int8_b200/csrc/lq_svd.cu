@@ -20,10 +20,12 @@
 //  3. subspace iteration on G with P = r + 8 basis vectors (rounded up to 4,
 //     at most d_k): deterministic start vectors, or at a commit the old
 //     compensators' k~_c in the first r columns; 16 steps V <- orth(G V),
-//     each orthonormalised by classical Gram-Schmidt applied twice (FP32);
+//     each orthonormalised by classical Gram-Schmidt applied twice (FP32,
+//     four CTA barriers per column);
 //  4. Rayleigh-Ritz: H = V^T G V (FP64), its eigenvectors by a cyclic Jacobi
 //     method with the round-robin pair ordering (P/2 rotations per round,
-//     FP64), the r largest; k~_c = V z_c, u_c = S k~_c;
+//     FP64; sweeps until the off-diagonal part is at round-off, at most 8),
+//     the r largest; k~_c = V z_c, u_c = S k~_c;
 //  5. the residual S - sum_c u_c k~_c^T into the register tile and C3-C4.
 // The convergence rate of step 3 is (s_{P+1} / s_r)^2 per step.  A commit's
 // rebuilt state is dominated by the W buffered rank-one records, so P > W
@@ -57,6 +59,7 @@ struct SvdSmem {
     double H[kMaxP * kMaxP];           // Rayleigh quotient, rotated in place
     double Z[kMaxP * kMaxP];           // its eigenvectors (columns)
     double rc[kMaxP / 2], rs[kMaxP / 2];
+    int jacobi_done;                   // the off-diagonal part has vanished
     float dot[kMaxP];
     alignas(16) float uc[kMaxComp * DV];
     alignas(16) float vc[kMaxComp * DK];
@@ -83,49 +86,75 @@ __device__ __forceinline__ float start_entry(int j, int c, int DK) {
 
 // Classical Gram-Schmidt applied twice to the columns of X (DK x P, pitch
 // kMaxP), written to V: column c loses its components along V's columns
-// 0..c-1 (twice), then is normalised.  A column that vanishes is replaced by
-// a start vector and orthogonalised again (once; a second loss leaves it 0).
+// 0..c-1 (twice), then is normalised.  Four CTA barriers per column: warp 0
+// normalises column c-1 (and takes its dot product with column c) while the
+// other warps form column c's first projections.  A column that vanishes
+// exactly becomes 0.
 template <int DK>
 __device__ void orthonormalise(float *V, float *X, float *dot, int P) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    for (int c = 0; c < P; ++c) {
-        bool retried = false;
-        for (int pass = 0; pass < 3; ++pass) {
-            // pass 0, 1: projections; pass 2: the norm
-            const int nd = pass < 2 ? c : 1;
-            for (int k = warp; k < nd; k += kSWarps) {
-                float d = 0.0f;
-                for (int j = lane; j < DK; j += 32)
-                    d = fmaf(pass < 2 ? V[j * kMaxP + k] : X[j * kMaxP + c], X[j * kMaxP + c], d);
+    constexpr int RPL = DK / 32;  // rows per lane in a one-warp column pass
+    // warp 0: V[:, c] = X[:, c] / |X[:, c]|, then dot[c] = X[:, c + 1] . V[:, c]
+    auto finalise = [&](int c, bool with_next) {
+        float x[RPL], n2 = 0.0f;
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
-                if (lane == 0) dot[k] = d;
-            }
+        for (int t = 0; t < RPL; ++t) {
+            x[t] = X[(lane + 32 * t) * kMaxP + c];
+            n2 = fmaf(x[t], x[t], n2);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) n2 += __shfl_xor_sync(0xffffffffu, n2, o);
+        const float inv = n2 > 1e-30f ? rsqrtf(n2) : 0.0f;
+        float d = 0.0f;
+#pragma unroll
+        for (int t = 0; t < RPL; ++t) {
+            const int j = lane + 32 * t;
+            const float v = x[t] * inv;
+            V[j * kMaxP + c] = v;
+            if (with_next) d = fmaf(v, X[j * kMaxP + c + 1], d);
+        }
+        if (with_next) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+            if (lane == 0) dot[c] = d;
+        }
+    };
+    // dot[k] = X[:, c] . V[:, k] for k in [0, kend), warps from `first` on
+    auto dots = [&](int c, int kend, int first) {
+        for (int k = warp - first; k < kend; k += kSWarps - first) {
+            if (k < 0) continue;
+            float d = 0.0f;
+            for (int j = lane; j < DK; j += 32) d = fmaf(V[j * kMaxP + k], X[j * kMaxP + c], d);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+            if (lane == 0) dot[k] = d;
+        }
+    };
+    auto update = [&](int c) {
+        for (int j = tid; j < DK; j += kSThreads) {
+            float x = X[j * kMaxP + c];
+            for (int k = 0; k < c; ++k) x = fmaf(-dot[k], V[j * kMaxP + k], x);
+            X[j * kMaxP + c] = x;
+        }
+    };
+    for (int c = 0; c < P; ++c) {
+        // first pass: column c-1 is finalised by warp 0, which also takes
+        // the projection on it; the other warps take columns 0..c-2
+        if (c > 0) {
+            if (warp == 0) finalise(c - 1, true);
+            else dots(c, c - 1, 1);
             cta_sync();
-            if (pass < 2) {
-                if (c > 0)
-                    for (int j = tid; j < DK; j += kSThreads) {
-                        float x = X[j * kMaxP + c];
-                        for (int k = 0; k < c; ++k) x = fmaf(-dot[k], V[j * kMaxP + k], x);
-                        X[j * kMaxP + c] = x;
-                    }
-            } else {
-                const float n2 = dot[0];
-                const bool dead = !(n2 > 1e-30f);
-                for (int j = tid; j < DK; j += kSThreads)
-                    V[j * kMaxP + c] = dead ? 0.0f : X[j * kMaxP + c] * rsqrtf(n2);
-                if (dead && !retried) {
-                    // replace the column and redo it
-                    retried = true;
-                    for (int j = tid; j < DK; j += kSThreads) X[j * kMaxP + c] = start_entry(j, c + 97, DK);
-                    cta_sync();
-                    pass = -1;
-                    continue;
-                }
-            }
+            update(c);
+            cta_sync();
+            // second pass
+            dots(c, c, 0);
+            cta_sync();
+            update(c);
             cta_sync();
         }
     }
+    if (warp == 0) finalise(P - 1, false);
+    cta_sync();
 }
 
 // Arguments: FP32 states (S != nullptr), or a rebuild from the snapshot and
@@ -186,7 +215,10 @@ __global__ void __launch_bounds__(kSThreads, 1) svd_kernel(const SvdArgs A) {
         // start: the old compensators' k~_c, then start vectors
         for (int idx = tid; idx < DK * P; idx += kSThreads) {
             const int j = idx / P, c = idx % P;
-            sm.X[j * kMaxP + c] = c < R ? a.comp_val[((size_t)bh * R + c) * DK + j] : start_entry(j, c, DK);
+            // the old k~_c plus a small start-vector part, so that a zero
+            // compensator (after the zero state) still gives a basis vector
+            sm.X[j * kMaxP + c] = c < R ? fmaf(1e-3f, start_entry(j, c, DK), a.comp_val[((size_t)bh * R + c) * DK + j])
+                                        : start_entry(j, c, DK);
         }
         cta_sync();
         // S_ij = sigma_i Q_ij c_j e^{L_n,j} + sum_m U[m][i] K^[m][j]
@@ -308,6 +340,24 @@ __global__ void __launch_bounds__(kSThreads, 1) svd_kernel(const SvdArgs A) {
     // players p(k) and p(P-1-k) of the circle (player 0 fixed, the others
     // rotated by t); the P/2 pairs of a round are disjoint
     for (int sweep = 0; sweep < kSweeps; ++sweep) {
+        // stop once the off-diagonal part is at FP64 round-off of the diagonal
+        if (warp == 0) {
+            double off = 0.0, dia = 0.0;
+            for (int idx = lane; idx < P * P; idx += 32) {
+                const int x = idx / P, y = idx % P;
+                const double h = sm.H[x * kMaxP + y];
+                if (x == y) dia = fma(h, h, dia);
+                else off = fma(h, h, off);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                off += __shfl_xor_sync(0xffffffffu, off, o);
+                dia += __shfl_xor_sync(0xffffffffu, dia, o);
+            }
+            if (lane == 0) sm.jacobi_done = off <= 1e-30 * dia;
+        }
+        cta_sync();
+        if (sm.jacobi_done) break;
         for (int t = 0; t < P - 1; ++t) {
             auto player = [&](int k) { return k == 0 ? 0 : 1 + (k - 1 + t) % (P - 1); };
             if (tid < P / 2) {
