@@ -280,14 +280,24 @@ LQ_API lq_status lq_ragged_flush(lq_state *st, int32_t *seq_pos, lq_stream_t str
  * workspace (device, (16B), workspace_bytes long; may be NULL with 0 bytes):
  * scratch of the chunked tensor-core prefill, used for the scalar gate with
  * BF16 io and d_k = 128.  Tokens are taken in chunks of 64 within each
- * snapshot interval, up to 16 chunks per pass of the workspace
- * (lq_prefill_workspace_bytes gives the size for full passes; any size of at
- * least one chunk, 48 KB per sequence and head, is used in shorter passes).
+ * snapshot interval, up to 16 chunks per pass of the workspace.  A
+ * workspace of two full passes (lq_prefill_workspace_bytes) is used as two
+ * halves: the next pass's chunk preparation runs while the current pass is
+ * scanned; any smaller size of at least one chunk, 48 KB per sequence and
+ * head, is used for one pass at a time of up to 16 chunks.
  * Without a usable workspace, for other shapes, and for the last
  * (snapshot_every mod 64) tokens of an interval, the recurrence runs token
  * by token on the FP32 state (same arithmetic, CUDA cores).  The caller
  * keeps the workspace alive until the call's work on `stream` has finished
  * and does not share it between concurrent calls.
+ * The call runs its kernels on three internal streams of the current device
+ * (the scans at the highest stream priority, the chunk preparation at the
+ * lowest, snapshot quantization beside the next pass's preparation), forked
+ * from `stream` by an event at the start and joined back into it at the end:
+ * to the caller the work is ordered on `stream` like a single launch.  The
+ * first call on each device creates those streams and events (held until the
+ * process exits): make that first call before any stream capture.  Calls from
+ * several host threads are serialized while they enqueue.
  * Requires pos == 0 (else LQ_ERR_WINDOW_OPEN; also LQ_POS_PER_SEQUENCE), T >= 0,
  * snapshot_every >= 1
  * and, when snaps != NULL, T % snapshot_every == 0.  T == 0 is a no-op. */
@@ -311,8 +321,10 @@ LQ_API lq_status lq_prefill_chunk(lq_state *st, float *S_fp32, const void *q, co
  *    io, d_k = 128); above that the call returns LQ_ERR_UNSUPPORTED and does
  *    nothing.  Passes hold min(16, floor(170 / (B * H))) chunks.
  *  - The first call on each device looks up the array's device address
- *    (cudaGetSymbolAddress, with that device current); make that first call
- *    before any stream capture.  A failed lookup returns LQ_ERR_CUDA.
+ *    (cudaGetSymbolAddress, with that device current) and creates
+ *    lq_prefill_chunk's internal streams and events (no device memory is
+ *    allocated); make that first call before any stream capture.  A failed
+ *    lookup returns LQ_ERR_CUDA.
  *  - All calls share the one array, which keeps the last call's contents
  *    (nothing in it needs to start at zero).  Calls whose work overlaps on
  *    the GPU (other streams, other host threads) race on it: serialize them. */
@@ -322,8 +334,9 @@ LQ_API lq_status lq_prefill_chunk_noalloc(lq_state *st, float *S_fp32, const voi
                                           const lq_snapshot *snaps, void *o, lq_stream_t stream);
 
 /* Bytes of the workspace with which lq_prefill_chunk runs full passes of 16
- * chunks of 64 tokens (16 x B x H x 48 KB); -1 for an invalid
- * configuration, 0 when the configuration has no tensor-core prefill. */
+ * chunks of 64 tokens, two passes in flight (2 x 16 x B x H x 48 KB); -1 for
+ * an invalid configuration, 0 when the configuration has no tensor-core
+ * prefill. */
 LQ_API int64_t lq_prefill_workspace_bytes(const lq_config *cfg);
 
 /* Copies the committed boundary state into `dst` (device buffers of the same

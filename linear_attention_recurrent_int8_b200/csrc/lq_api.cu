@@ -4,6 +4,7 @@
 // error has no side effect.  No exception crosses the ABI.
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/lq.h"
 #include "lq_kernels.h"
@@ -135,6 +136,59 @@ lq::QuantArgs quant_args(const lq_config *c, const float *S, const lq_snapshot *
 }
 
 lq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? LQ_OK : LQ_ERR_CUDA; }
+
+// Internal streams and events of the prefill, one set per device, created on
+// first use and kept until the process exits.  The scans (the sequential
+// chain) run on `chain` at the highest stream priority; the chunk preparation
+// of the next pass runs on `prep` at the lowest, into the other half of a
+// double workspace, on the SMs the scan leaves free; snapshot quantization
+// runs on `snap` while the next pass is prepared.  Each call forks them from
+// the caller's stream and joins them back, so the call keeps stream order
+// (and works inside a stream capture once the set exists).
+struct PrefillStreams {
+    cudaStream_t chain, prep, snap;
+    cudaEvent_t fork, join, prep_done[2], scan_done[2], snap_in, snap_done;
+};
+
+std::mutex g_prefill_mutex;  // guards the sets and each call's enqueue sequence
+
+// The current device's set (nullptr for device ordinals past 63, which then
+// run everything on the caller's stream).  Called with g_prefill_mutex held.
+cudaError_t prefill_streams(PrefillStreams **out) {
+    static PrefillStreams sets[64];
+    static bool ready[64];
+    *out = nullptr;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaSuccess;
+    PrefillStreams &p = sets[dev];
+    if (!ready[dev]) {
+        int least = 0, greatest = 0;
+        e = cudaDeviceGetStreamPriorityRange(&least, &greatest);
+        cudaStream_t *streams[3] = {&p.chain, &p.prep, &p.snap};
+        const int prio[3] = {greatest, least, greatest};
+        cudaEvent_t *events[8] = {&p.fork, &p.join, &p.prep_done[0], &p.prep_done[1],
+                                  &p.scan_done[0], &p.scan_done[1], &p.snap_in, &p.snap_done};
+        int ns = 0, nev = 0;  // created so far
+        while (e == cudaSuccess && ns < 3) {
+            e = cudaStreamCreateWithPriority(streams[ns], cudaStreamNonBlocking, prio[ns]);
+            if (e == cudaSuccess) ++ns;
+        }
+        while (e == cudaSuccess && nev < 8) {
+            e = cudaEventCreateWithFlags(events[nev], cudaEventDisableTiming);
+            if (e == cudaSuccess) ++nev;
+        }
+        if (e != cudaSuccess) {
+            for (int i = 0; i < nev; ++i) cudaEventDestroy(*events[i]);
+            for (int i = 0; i < ns; ++i) cudaStreamDestroy(*streams[i]);
+            return e;
+        }
+        ready[dev] = true;
+    }
+    *out = &p;
+    return cudaSuccess;
+}
 
 lq_status copy_snapshot(const lq_config *c, const lq_snapshot *dst, const lq_snapshot *src,
                         cudaStream_t stream) {
@@ -301,7 +355,8 @@ lq_status lq_window_commit(lq_state *st, lq_stream_t stream) {
 int64_t lq_prefill_workspace_bytes(const lq_config *cfg) {
     if (check_config(cfg) != LQ_OK) return -1;
     if (!lq::chunk_path_supported(cfg->d_k, cfg->d_v, cfg->gate, cfg->io_dtype == LQ_BF16)) return 0;
-    return (int64_t)lq::chunk_workspace_bytes(cfg->batch * cfg->heads, kPassChunks);
+    // two full passes: one prepared while the other is scanned
+    return (int64_t)lq::chunk_workspace_bytes(cfg->batch * cfg->heads, 2 * kPassChunks);
 }
 
 lq_status lq_prefill_chunk(lq_state *st, float *S_fp32, const void *q, const void *k,
@@ -341,51 +396,113 @@ lq_status lq_prefill_chunk(lq_state *st, float *S_fp32, const void *q, const voi
     r.delta = c->delta;
     r.H = c->heads;
     r.T_total = T;
-    // chunks per pass of the tensor-core path (0: token by token)
-    const int BH = c->batch * c->heads;
-    int pass = 0;
-    if (workspace && lq::chunk_path_supported(c->d_k, c->d_v, c->gate, c->io_dtype == LQ_BF16)) {
-        const size_t per = lq::chunk_workspace_bytes(BH, 1);
-        pass = (int)(workspace_bytes / per < (size_t)kPassChunks ? workspace_bytes / per : kPassChunks);
-    }
     lq::ChunkArgs ca{};
     ca.S = S_fp32;
     ca.alpha = alpha;
     ca.beta = beta;
     ca.o = o;
-    ca.ws = static_cast<float *>(workspace);
     ca.B = c->batch;
     ca.H = c->heads;
     ca.DV = c->d_v;
     ca.T_total = T;
     ca.delta = c->delta;
-    for (int t0 = 0, i = 0; t0 < T; t0 += snapshot_every, ++i) {
+
+    std::lock_guard<std::mutex> lock(g_prefill_mutex);
+    PrefillStreams *ps = nullptr;
+    e = cuda_status(prefill_streams(&ps));
+    if (e != LQ_OK) return e;
+    // chunks per pass of the tensor-core path (0: token by token); two
+    // workspace halves (the next pass prepared while this one is scanned)
+    // when the workspace holds two full passes
+    const int BH = c->batch * c->heads;
+    int pass = 0, nbuf = 1;
+    size_t per = 0;
+    if (workspace && lq::chunk_path_supported(c->d_k, c->d_v, c->gate, c->io_dtype == LQ_BF16)) {
+        per = lq::chunk_workspace_bytes(BH, 1);
+        const size_t chunks = workspace_bytes / per;
+        if (ps && chunks >= 2 * (size_t)kPassChunks) nbuf = 2;
+        pass = (int)(chunks < (size_t)kPassChunks ? chunks : kPassChunks);
+    }
+    cudaStream_t chain = s, prep = s, snap = s;
+    cudaError_t ce = cudaSuccess;
+    if (ps) {
+        chain = ps->chain;
+        prep = nbuf == 2 ? ps->prep : ps->chain;
+        snap = ps->snap;
+        ce = cudaEventRecord(ps->fork, s);
+        if (ce == cudaSuccess) ce = cudaStreamWaitEvent(ps->chain, ps->fork, 0);
+        if (ce == cudaSuccess) ce = cudaStreamWaitEvent(ps->prep, ps->fork, 0);
+        if (ce == cudaSuccess) ce = cudaStreamWaitEvent(ps->snap, ps->fork, 0);
+        if (ce != cudaSuccess) return cuda_status(ce);
+    }
+    // a snapshot quantization on `snap` reads the state: the chain waits for
+    // it before it writes the state again
+    bool snap_pending = false;
+    auto wait_snap = [&]() -> cudaError_t {
+        if (!snap_pending) return cudaSuccess;
+        snap_pending = false;
+        return cudaStreamWaitEvent(chain, ps->snap_done, 0);
+    };
+    unsigned char *wsb = static_cast<unsigned char *>(workspace);
+    int g = 0;  // passes so far
+    for (int t0 = 0, i = 0; ce == cudaSuccess && t0 < T; t0 += snapshot_every, ++i) {
         const int nt = T - t0 < snapshot_every ? T - t0 : snapshot_every;
         int done = 0;
         if (pass > 0) {
             // whole chunks of this interval on the tensor cores, in passes
             const int nch = nt / kChunkTokens;
-            for (int c0 = 0; c0 < nch; c0 += pass) {
+            for (int c0 = 0; ce == cudaSuccess && c0 < nch; c0 += pass, ++g) {
+                const int buf = g % nbuf;
                 ca.t0 = t0 + c0 * kChunkTokens;
                 ca.nc = nch - c0 < pass ? nch - c0 : pass;
-                e = cuda_status(lq::launch_prefill_chunks(ca, q, k, v, s));
-                if (e != LQ_OK) return e;
+                ca.ws = reinterpret_cast<float *>(wsb + (size_t)buf * pass * per);
+                if (nbuf == 2) {
+                    // the half's previous reader, the scan of pass g - 2, is done
+                    if (g >= 2) ce = cudaStreamWaitEvent(prep, ps->scan_done[buf], 0);
+                    if (ce == cudaSuccess) ce = lq::launch_chunk_prep(ca, q, k, prep);
+                    if (ce == cudaSuccess) ce = cudaEventRecord(ps->prep_done[buf], prep);
+                    if (ce == cudaSuccess) ce = cudaStreamWaitEvent(chain, ps->prep_done[buf], 0);
+                } else {
+                    ce = lq::launch_chunk_prep(ca, q, k, chain);
+                }
+                if (ce == cudaSuccess) ce = wait_snap();
+                if (ce == cudaSuccess) ce = lq::launch_chunk_scan(ca, q, k, v, chain);
+                if (ce == cudaSuccess && nbuf == 2) ce = cudaEventRecord(ps->scan_done[buf], chain);
             }
             done = nch * kChunkTokens;
         }
-        if (done < nt) {
+        if (ce == cudaSuccess && done < nt) {
             r.t0 = t0 + done;
             r.nt = nt - done;
-            e = cuda_status(lq::launch_recurrence(r, c->d_k, c->d_v, c->gate, c->io_dtype == LQ_BF16,
-                                                  true, s));
-            if (e != LQ_OK) return e;
+            ce = wait_snap();
+            if (ce == cudaSuccess)
+                ce = lq::launch_recurrence(r, c->d_k, c->d_v, c->gate, c->io_dtype == LQ_BF16, true, chain);
         }
-        if (snaps) {
-            e = cuda_status(lq::launch_quantize(quant_args(c, S_fp32, &snaps[i]), c->d_k, c->d_v, s));
-            if (e != LQ_OK) return e;
+        if (ce == cudaSuccess && snaps) {
+            if (ps) {
+                ce = cudaEventRecord(ps->snap_in, chain);
+                if (ce == cudaSuccess) ce = cudaStreamWaitEvent(snap, ps->snap_in, 0);
+                if (ce == cudaSuccess)
+                    ce = lq::launch_quantize(quant_args(c, S_fp32, &snaps[i]), c->d_k, c->d_v, snap);
+                if (ce == cudaSuccess) ce = cudaEventRecord(ps->snap_done, snap);
+                snap_pending = ce == cudaSuccess;
+            } else {
+                ce = lq::launch_quantize(quant_args(c, S_fp32, &snaps[i]), c->d_k, c->d_v, chain);
+            }
         }
     }
-    return cuda_status(lq::launch_quantize(quant_args(c, S_fp32, &st->snap), c->d_k, c->d_v, s));
+    if (ce == cudaSuccess) ce = wait_snap();
+    if (ce == cudaSuccess) ce = lq::launch_quantize(quant_args(c, S_fp32, &st->snap), c->d_k, c->d_v, chain);
+    if (ps) {
+        // join every internal stream back into the caller's stream (also
+        // after a failed launch, so that later work on it stays ordered)
+        for (cudaStream_t x : {ps->prep, ps->snap, ps->chain}) {
+            cudaError_t je = cudaEventRecord(ps->join, x);
+            if (je == cudaSuccess) je = cudaStreamWaitEvent(s, ps->join, 0);
+            if (ce == cudaSuccess) ce = je;
+        }
+    }
+    return cuda_status(ce);
 }
 
 lq_status lq_state_snapshot(const lq_state *st, const lq_snapshot *dst, lq_stream_t stream) {

@@ -675,9 +675,9 @@ bool chunk_path_supported(int d_k, int d_v, int gate, bool bf16) {
     return bf16 && gate == 0 && d_k == kDK && (d_v == 64 || d_v == 128);
 }
 
-cudaError_t launch_prefill_chunks(const ChunkArgs &a, const void *q, const void *k, const void *v,
-                                  cudaStream_t stream) {
-    if (a.nc < 1 || a.DV % kDVS != 0) return cudaErrorInvalidValue;
+namespace {
+// Sets the kernels' shared-memory limits once per device.
+cudaError_t configure_chunk_kernels() {
     static std::atomic<uint64_t> configured{0};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -692,15 +692,33 @@ cudaError_t launch_prefill_chunks(const ChunkArgs &a, const void *q, const void 
         if (e != cudaSuccess) return e;
         configured.fetch_or(bit, std::memory_order_acq_rel);
     }
+    return cudaSuccess;
+}
+}  // namespace
+
+cudaError_t launch_chunk_prep(const ChunkArgs &a, const void *q, const void *k, cudaStream_t stream) {
+    if (a.nc < 1 || a.DV % kDVS != 0) return cudaErrorInvalidValue;
+    cudaError_t e = configure_chunk_kernels();
+    if (e != cudaSuccess) return e;
+    const long long BT = (long long)a.B * a.T_total;
+    CUtensorMap qm, km;
+    if (!activation_map(&qm, q, kDK, a.H, BT, 8) || !activation_map(&km, k, kDK, a.H, BT, 8))
+        return cudaErrorInvalidValue;
+    chunk_prep_kernel<<<a.nc * a.B * a.H, kPrepThreads, prep_smem_bytes(), stream>>>(qm, km, a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_chunk_scan(const ChunkArgs &a, const void *q, const void *k, const void *v,
+                              cudaStream_t stream) {
+    if (a.nc < 1 || a.DV % kDVS != 0) return cudaErrorInvalidValue;
+    cudaError_t e = configure_chunk_kernels();
+    if (e != cudaSuccess) return e;
     const long long BT = (long long)a.B * a.T_total;
     CUtensorMap qm, km, vm;
     if (!activation_map(&qm, q, kDK, a.H, BT, 8) || !activation_map(&km, k, kDK, a.H, BT, 8) ||
         !activation_map(&vm, v, a.DV, a.H, BT, kDVS, true))
         return cudaErrorInvalidValue;
     const int BH = a.B * a.H;
-    chunk_prep_kernel<<<a.nc * BH, kPrepThreads, prep_smem_bytes(), stream>>>(qm, km, a);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
     chunk_scan_kernel<<<BH * (a.DV / kDVS), kScanThreads, scan_layout().bytes + 1024, stream>>>(qm, km, vm, a);
     return cudaGetLastError();
 }

@@ -120,9 +120,12 @@ size_t chunk_workspace_bytes(int BH, int chunks);
 // BF16 io, d_k = 128, d_v in {64, 128}).
 bool chunk_path_supported(int d_k, int d_v, int gate, bool bf16);
 
-// One pass: the [PT; T] preparation of every chunk, then the chunks in order.
-cudaError_t launch_prefill_chunks(const ChunkArgs &a, const void *q, const void *k, const void *v,
-                                  cudaStream_t stream);
+// One pass in two launches: the [PT; T] preparation of every chunk into
+// a.ws (reads q, k, alpha, beta), then the chunks in order (reads a.ws, q, k,
+// v, alpha, beta and the state; writes the outputs and the state).
+cudaError_t launch_chunk_prep(const ChunkArgs &a, const void *q, const void *k, cudaStream_t stream);
+cudaError_t launch_chunk_scan(const ChunkArgs &a, const void *q, const void *k, const void *v,
+                              cudaStream_t stream);
 
 // Decodes a.n_steps >= 1 tokens (records a.pos .. a.pos + n_steps - 1).
 cudaError_t launch_decode(const DecodeArgs &a, int d_k, int d_v, int gate, bool bf16,

@@ -63,10 +63,10 @@ lq_status lq_prefill_chunk_noalloc(lq_state *st, float *S_fp32, const void *q, c
                                    int32_t T, int32_t snapshot_every, const lq_snapshot *snaps,
                                    void *o, lq_stream_t stream) {
     if (!st) return LQ_ERR_INVALID_ARGUMENT;
-    // bytes of a 16-chunk pass (0: this shape has no chunked path, so no scratch)
-    const int64_t full_pass = lq_prefill_workspace_bytes(&st->cfg);
-    if (full_pass < 0) return LQ_ERR_INVALID_ARGUMENT;
-    const int64_t one_chunk = full_pass / 16;
+    // bytes of two 16-chunk passes (0: this shape has no chunked path, so no scratch)
+    const int64_t two_passes = lq_prefill_workspace_bytes(&st->cfg);
+    if (two_passes < 0) return LQ_ERR_INVALID_ARGUMENT;
+    const int64_t one_chunk = two_passes / 32;
     if (one_chunk > (int64_t)kStaticScratchBytes) return LQ_ERR_UNSUPPORTED;
     void *ws = nullptr;
     size_t ws_bytes = 0;

@@ -371,13 +371,13 @@ def test_binding_rejects_bad_tensors_before_the_library(no_library):
 
 
 def test_prefill_workspace_bytes():
-    """16 chunks of 64 tokens per pass, 48 KB ([PT; T], 128 x 64 values in
-    three BF16 parts) per chunk and head; 0 where the tensor-core prefill does
-    not apply."""
+    """Two passes (one prepared while the other is scanned) of 16 chunks of
+    64 tokens, 48 KB ([PT; T], 128 x 64 values in three BF16 parts) per chunk
+    and head; 0 where the tensor-core prefill does not apply."""
     cfg = lq.Config(batch=2, heads=32, d_k=128, d_v=128, io_dtype=lq.LQ_BF16)
-    assert lq.lq_prefill_workspace_bytes(cfg) == 16 * 64 * 49152
+    assert lq.lq_prefill_workspace_bytes(cfg) == 2 * 16 * 64 * 49152
     cfg.d_v = 64
-    assert lq.lq_prefill_workspace_bytes(cfg) == 16 * 64 * 49152
+    assert lq.lq_prefill_workspace_bytes(cfg) == 2 * 16 * 64 * 49152
     for field, val in (("io_dtype", lq.LQ_F32), ("gate", lq.LQ_GATE_DIAG), ("d_k", 64)):
         c2 = lq.Config(batch=2, heads=32, d_k=128, d_v=128, io_dtype=lq.LQ_BF16)
         setattr(c2, field, val)

@@ -1,7 +1,9 @@
 """The chunked tensor-core prefill (scalar gate, BF16 io, d_k = 128) against
 the oracle's token recurrence: outputs, the carried FP32 state and every
 snapshot, for several pass sizes of the workspace (one chunk up to sixteen
-per pass), intervals that end in a ragged tail of fewer than 64 tokens, both
+per pass, and two workspace halves where the next pass is prepared while the
+current one is scanned), intervals that end in a ragged tail of fewer than
+64 tokens, both
 value-row splits (d_v = 128: two CTAs per head; d_v = 64: one), and the b = 0
 instance.  The same call without a workspace (token by token) agrees too."""
 import numpy as np
@@ -58,6 +60,9 @@ def _run(B, H, dv, T, every, r, ws_chunks, delta=1, seed=0):
     (1, 2, 128, 320, 320, 1, 1),       # passes of one chunk
     (2, 2, 128, 200, 100, 3, 16),      # intervals of 64 + a 36-token tail on the token path
     (1, 3, 128, 2176, 2176, 4, 16),    # 34 chunks: passes of 16, 16, 2
+    (1, 3, 128, 2176, 2176, 4, 32),    # the same in two workspace halves (next pass prepared during the scan)
+    (2, 2, 128, 4096, 1024, 4, 32),    # two halves, four snapshot intervals of one pass each
+    (2, 2, 64, 2112, 704, 2, 40),      # two halves with spare bytes; 11-chunk intervals, d_v = 64
 ])
 def test_chunked_prefill_matches_oracle(B, H, dv, T, every, r, ws_chunks):
     _run(B, H, dv, T, every, r, ws_chunks)
