@@ -22,8 +22,9 @@
 //
 // Two kernels per pass of up to kMaxPassChunks chunks:
 //  * chunk_prep_kernel (every chunk of every head in parallel): K K^T and
-//    Q K^T on the tensor core (BF16, exact products, FP32 sums), A and P on
-//    CUDA cores, then T and PT column by column (forward substitution, FP32),
+//    Q K^T with warp-level tensor-core MMAs (BF16, exact products, FP32
+//    sums; several CTAs share an SM), A and P on CUDA cores, then T and PT
+//    column by column (forward substitution, FP32),
 //    written to the caller's workspace as [PT; T] (128 x 64, three BF16 parts
 //    of each FP32 value, in the operand layout: 48 KB per chunk and head);
 //  * chunk_scan_kernel (one CTA per head and 64 value rows, the chunks of the
@@ -86,11 +87,6 @@ __device__ __forceinline__ void load_qk(unsigned char *qk, const CUtensorMap *qm
     }
 }
 
-// Descriptor of the K-major [Q; K] operand at K-step k16 (16 channels).
-__device__ __forceinline__ uint64_t desc_qk(const unsigned char *qk, int k16) {
-    return smem_desc(smem_u32(qk + k16 * 4096), 2048, 128);
-}
-
 // Two values in three BF16 parts each, packed in pairs (x0 in the low half).
 __device__ __forceinline__ void split2_bf16x3(float x0, float x1, uint32_t &w0, uint32_t &w1,
                                               uint32_t &w2) {
@@ -139,9 +135,25 @@ struct PrepSmem {
     alignas(16) float L2[kC];           // L_t log2(e)
     alignas(16) float beta[kC];
     float alpha[kC];
-    uint64_t bar_in, bar_mma;
-    uint32_t tmem;
+    uint64_t bar_in;
 };
+
+// Four 8 x 8 BF16 matrices of the [Q; K] tile into the fragment registers of
+// a warp-level MMA; lane i addresses row i % 8 of matrix i / 8.
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], const unsigned char *p) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(smem_u32(p)));
+}
+
+// D += A B for one 16 x 8 tile, K = 16: BF16 inputs, FP32 accumulation.
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
 
 __host__ __device__ constexpr int prep_smem_bytes() {
     return kQKBytes + (int)sizeof(PrepSmem) + 128;
@@ -203,33 +215,15 @@ __global__ void __launch_bounds__(kPrepThreads) chunk_prep_kernel(
     const int b = bh / a.H, h = bh % a.H;
     const int tok0 = b * a.T_total + a.t0 + c * kC;  // flattened (sequence, token) row
 
-    if (tid == 0) {
-        mbar_init(&ps.bar_in, 1);
-        mbar_init(&ps.bar_mma, 1);
-    }
-    if (warp == 0) tmem_alloc(&ps.tmem, 64);
+    if (tid == 0) mbar_init(&ps.bar_in, 1);
     // gates of the chunk
     if (tid < kC) ps.alpha[tid] = a.alpha[((size_t)tok0 + tid) * a.H + h];
     else ps.beta[tid - kC] = a.beta[((size_t)tok0 + tid - kC) * a.H + h];
-    tc_fence_before_sync();
     __syncthreads();
-    tc_fence_after_sync();
 
-    bool ok = true;
     if (tid == 0) {
         mbar_arrive_expect_tx(&ps.bar_in, kQKBytes);
         load_qk(qk, &qmap, &kmap, h, tok0, &ps.bar_in);
-        ok = mbar_wait_bounded(&ps.bar_in, 0);
-        if (ok) {
-            // D[128 x 64] = [Q; K] K^T: rows 0..63 Q K^T, rows 64..127 K K^T
-            constexpr uint32_t idesc = idesc_bf16(128, kC, false, false);
-            const uint64_t dA = desc_qk(qk, 0);
-            const uint64_t dB = smem_desc(smem_u32(qk + 1024), 2048, 128);
-#pragma unroll
-            for (int k16 = 0; k16 < kDK / 16; ++k16)
-                mma_bf16(ps.tmem, dA + ((k16 * 4096) >> 4), dB + ((k16 * 4096) >> 4), idesc, k16 > 0);
-            mma_commit(&ps.bar_mma);
-        }
     }
     if (warp == 1) {
         // L_t log2(e) of the chunk
@@ -238,40 +232,74 @@ __global__ void __launch_bounds__(kPrepThreads) chunk_prep_kernel(
         ps.L2[2 * lane] = Le * 1.4426950408889634f;
         ps.L2[2 * lane + 1] = Lo * 1.4426950408889634f;
     }
-    // thread 0's copies and MMAs went through (and L is in shared memory)
-    bool good = !named_sync_or<1, kPrepThreads>(tid == 0 && !ok);
-    if (good) good = mbar_wait_bounded(&ps.bar_mma, 0);
+    // every thread observes the copies' completion (the tile is read through
+    // the generic proxy), and L is in shared memory after the barrier
+    const bool ok = mbar_wait_bounded(&ps.bar_in, 0);
+    const bool good = !named_sync_or<1, kPrepThreads>(!ok);
     if (good) {
-        // row r of the product: P (rows 0..63) or A (rows 64..127) with the
-        // gate ratio e^{L_t - L_m} = 2^{(L_t - L_m) log2 e} and beta_m
-        tc_fence_after_sync();
-        const int r = tid, t = r & (kC - 1);
-        const bool qrow = r < kC;
-        float x[64];
-        tmem_load<64>(ps.tmem + ((uint32_t)(32 * warp) << 16), x);
-        const float Lt = ps.L2[t];
-        float *row = qrow ? ps.P[t] : ps.A[t];
+        // D[128 x 64] = [Q; K] K^T with warp-level MMAs (exact BF16 products,
+        // FP32 sums): warp w takes rows 32w..32w+31 -- Q K^T for warps 0-1,
+        // K K^T for warps 2-3 -- as two 16-row tiles by eight 8-column tiles.
+        // (A tcgen05 product here would hold the kernel to one CTA per SM;
+        // its time is the CUDA-core phases below, which want several.)
+        float d[2][8][4];
 #pragma unroll
-        for (int m4 = 0; m4 < kC / 4; ++m4) {
-            const float4 l4 = *reinterpret_cast<const float4 *>(&ps.L2[4 * m4]);
-            const float4 b4 = *reinterpret_cast<const float4 *>(&ps.beta[4 * m4]);
-            const float lm[4] = {l4.x, l4.y, l4.z, l4.w}, bm[4] = {b4.x, b4.y, b4.z, b4.w};
-            float v[4];
+        for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int m = 4 * m4 + e;
-                const bool keep = qrow ? (m <= t) : (m < t && a.delta);
-                v[e] = keep ? bm[e] * x[m] * exp2f(Lt - lm[e]) : 0.0f;
+            for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) d[mt][nt][e] = 0.0f;
+        const int mi = lane >> 3, ri = lane & 7;  // this lane's matrix and row in ldmatrix
+#pragma unroll 2
+        for (int k16 = 0; k16 < kDK / 16; ++k16) {
+            // A tiles: matrices (rows +0 / +8) x (channels +0 / +8)
+            uint32_t af[2][4];
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt) {
+                const int row = 32 * warp + 16 * mt + 8 * (mi & 1) + ri;
+                ldmatrix_x4(af[mt], qk + (2 * k16 + (mi >> 1)) * 2048 + 16 * row);
             }
-            *reinterpret_cast<float4 *>(row + 4 * m4) = make_float4(v[0], v[1], v[2], v[3]);
+            // B = K^T: token n's row of K, channels +0 / +8, two 8-token tiles
+#pragma unroll
+            for (int np = 0; np < 4; ++np) {
+                uint32_t bf[4];
+                const int n = 16 * np + 8 * (mi >> 1) + ri;
+                ldmatrix_x4(bf, qk + (2 * k16 + (mi & 1)) * 2048 + 1024 + 16 * n);
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt) {
+                    mma_bf16_16816(d[mt][2 * np], af[mt], bf[0], bf[1]);
+                    mma_bf16_16816(d[mt][2 * np + 1], af[mt], bf[2], bf[3]);
+                }
+            }
         }
+        // element (row, m) of the product: P (rows 0..63) or A (rows
+        // 64..127) with the gate ratio e^{L_t - L_m} = 2^{(L_t - L_m) log2 e}
+        // and beta_m; a thread holds rows g, g + 8 of each 16-row tile and
+        // columns 2c, 2c + 1 of each 8-column tile
+        const int g = lane >> 2, c2 = 2 * (lane & 3);
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+                const int r = 32 * warp + 16 * mt + 8 * hr + g, t = r & (kC - 1);
+                const bool qrow = r < kC;
+                const float Lt = ps.L2[t];
+                float *rowp = qrow ? ps.P[t] : ps.A[t];
+#pragma unroll
+                for (int nt = 0; nt < 8; ++nt) {
+                    const int m = 8 * nt + c2;
+                    const float2 lm = *reinterpret_cast<const float2 *>(&ps.L2[m]);
+                    const float2 bm = *reinterpret_cast<const float2 *>(&ps.beta[m]);
+                    const bool k0 = qrow ? (m <= t) : (m < t && a.delta);
+                    const bool k1 = qrow ? (m + 1 <= t) : (m + 1 < t && a.delta);
+                    const float v0 = k0 ? bm.x * d[mt][nt][2 * hr] * exp2f(Lt - lm.x) : 0.0f;
+                    const float v1 = k1 ? bm.y * d[mt][nt][2 * hr + 1] * exp2f(Lt - lm.y) : 0.0f;
+                    *reinterpret_cast<float2 *>(rowp + m) = make_float2(v0, v1);
+                }
+            }
     }
-    tc_fence_before_sync();
+    // every warp's reads of the [Q; K] tile are done before it holds X
     const bool bad = named_sync_or<1, kPrepThreads>(!good);
-    if (warp == 0) {
-        tc_fence_after_sync();
-        tmem_dealloc(ps.tmem, 64);
-    }
     if (bad) return;
 
     unsigned char *wsb = reinterpret_cast<unsigned char *>(a.ws) + ((size_t)c * a.B * a.H + bh) * kWsChunkBytes;
