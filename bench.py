@@ -347,6 +347,9 @@ def workload_config(wl, args):
         "l2": l2_note(wl.batch * wl.heads * decode_launch_bytes(
             wl.d_k, wl.d_v, wl.n_comp, wl.gate, 2 if wl.io == "bf16" else 4, 1, args.bits)),
         "graph": not args.no_graph,
+        "launch_timing": ("per-launch CUDA events only in the last `slots` windows of the timed "
+                          "region (the roofline's launch durations); the other windows run "
+                          "without event nodes"),
     }
 
 
@@ -424,27 +427,38 @@ def run_lq(args, wl):
     run_window(slots[0])
     torch.cuda.synchronize()
 
+    # Each slot has a graph without event nodes and one with an event node
+    # around every launch.  An event node adds about 5 us to a window (18 per
+    # window), so the timed region replays the plain graphs except in its
+    # last len(graphs) windows, whose per-launch events give the launch
+    # durations of the roofline; one warm-up round replays the instrumented
+    # graphs once before the timing.
     graphs = []
     if not args.no_graph:
         s = torch.cuda.Stream(device=dev)
         for slot in slots:
+            g_plain = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_plain, stream=s):
+                run_window(slot)
             # external events become event-record nodes of the graph
             evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(W + 2)]
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=s):
+            g_inst = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_inst, stream=s):
                 run_window(slot, evs)
-            graphs.append((g, evs))
+            graphs.append((g_plain, g_inst, evs))
         assert st.pos == 0
     else:
         for slot in slots:
-            graphs.append((None, [torch.cuda.Event(enable_timing=True) for _ in range(W + 2)]))
+            graphs.append((None, None, [torch.cuda.Event(enable_timing=True) for _ in range(W + 2)]))
+    n_g = len(graphs)
 
-    def step(i):
-        g, evs = graphs[i % len(graphs)]
-        if g is not None:
-            g.replay()
+    def step(i, timed=None):
+        g_plain, g_inst, evs = graphs[i % n_g]
+        inst = timed >= args.steps - n_g if timed is not None else n_g <= i < 2 * n_g
+        if g_plain is not None:
+            (g_inst if inst else g_plain).replay()
         else:
-            run_window(slots[i % len(slots)], evs)
+            run_window(slots[i % len(slots)], evs if inst else None)
 
     sampler = ClockSampler(local) if not args.no_clocks else None
     t_warm0 = time.monotonic()
@@ -459,7 +473,7 @@ def run_lq(args, wl):
     t0 = time.monotonic()
     start.record(cur)
     for i in range(args.steps):
-        step(args.warmup + i)
+        step(args.warmup + i, i)
     end.record(cur)
     torch.cuda.synchronize()
     t1 = time.monotonic()
@@ -470,12 +484,13 @@ def run_lq(args, wl):
     elapsed = start.elapsed_time(end)
     elapsed_max, value = aggregate(elapsed, wl.batch * W * args.steps, world, group)
 
-    # per-launch times from the event nodes of the last replay of each graph
+    # per-launch times from the event nodes of the instrumented windows (the
+    # last n_g of the timed region, one per slot)
     dec_ms, com_ms, dec_bytes = [], [], 0.0
     nh = wl.nh
-    used = range(min(len(graphs), args.steps + args.warmup))
+    used = sorted({(args.warmup + j) % n_g for j in range(max(0, args.steps - n_g), args.steps)})
     for gi in used:
-        evs = graphs[gi][1]
+        evs = graphs[gi][2]
         for t in range(W):
             dec_ms.append(evs[t].elapsed_time(evs[t + 1]))
             dec_bytes += nh * decode_launch_bytes(wl.d_k, wl.d_v, wl.n_comp, wl.gate, e, t + 1, args.bits,
@@ -494,7 +509,7 @@ def run_lq(args, wl):
     # average duration of the launch at each window position (us), then the commit
     pos_us = []
     for t in range(W):
-        vals = [graphs[gi][1][t].elapsed_time(graphs[gi][1][t + 1]) for gi in used]
+        vals = [graphs[gi][2][t].elapsed_time(graphs[gi][2][t + 1]) for gi in used]
         pos_us.append(round(1e3 * sum(vals) / len(vals), 1))
     extra["launch_us_by_position"] = pos_us
     c_avg = sum(com_ms) / len(com_ms)
