@@ -1076,10 +1076,8 @@ template <int DK, int DV, int GATE, bool BF16>
 cudaError_t launch_dr(const DecodeArgs &a, cudaStream_t stream) {
     const int fmt = code_format(a.bits);
     if constexpr (DK == 128 && DV == 128) {
-        // the tensor-core matvec for batch-synchronous positions; with
-        // per-sequence positions every launch sizes its stages for W - 1
-        // records, where the dp4a kernel is the faster of the two
-        if (fmt == kCodesI8 && !a.seq_pos) return launch_tc<GATE, BF16, false>(a, stream);
+        if (fmt == kCodesI8)  // the tensor-core matvec
+            return a.seq_pos ? launch_tc<GATE, BF16, true>(a, stream) : launch_tc<GATE, BF16, false>(a, stream);
     }
     if (fmt == kCodesI4)
         return a.seq_pos ? launch_d<DK, DV, GATE, BF16, true, kCodesI4>(a, stream)
