@@ -663,6 +663,53 @@ def run_e2e(args, wl, st, cfg, dev, world, group):
             "steps": n, "copies": "chunks of 4 tokens on an upload and a download stream, overlapping the decode"}
 
 
+DEFAULT_WORKLOAD = "gdn_256x32_d128_bf16"
+
+# Secondary workloads of the default run: (name, mode, workload, steps, warmup,
+# the equivalent command's flags).
+SECONDARY = (
+    ("kda_128x32_d128_bf16", "decode", "kda_128x32_d128_bf16", 40, 20,
+     "--workload kda_128x32_d128_bf16 --steps 40 --warmup 20"),
+    ("prefill_2x32_T65536", "prefill", DEFAULT_WORKLOAD, 3, 3, "--mode prefill --steps 3 --warmup 3"),
+    ("ragged_gdn_256x32_d128_bf16", "ragged", DEFAULT_WORKLOAD, 20, 5, "--mode ragged --steps 20 --warmup 5"),
+)
+
+
+def run_secondary(args):
+    """The default decode run also times, after the headline's timed region,
+    short runs of the secondary workloads (KDA decode, the 65,536-token
+    prefill, per-sequence window positions), each exactly as its own mode
+    would (no CPU baseline, no e2e, no clock sampling), so that one run
+    records them; a failure is reported in its entry, not raised."""
+    import copy
+
+    from linear_attention_recurrent_int8_b200 import synth
+    out = {}
+    for name, mode, workload, steps, warmup, flags in SECONDARY:
+        a = copy.copy(args)
+        a.mode, a.workload, a.steps, a.warmup = mode, workload, steps, warmup
+        a.no_cpu = a.no_e2e = a.no_clocks = a.no_secondary = True
+        try:
+            wl = synth.WORKLOADS[workload]
+            if mode == "prefill":
+                l = run_prefill(a)
+            elif mode == "ragged":
+                l = run_ragged(a, wl)
+            else:
+                l = run_lq(a, wl)
+            e = {k: l[k] for k in ("metric", "value", "unit", "ms_per_step", "steps", "warmup")}
+            e["command"] = f"python bench.py {flags} --no-cpu --no-e2e --no-clocks"
+            if "roofline" in l:
+                e["roofline"] = {k: l["roofline"][k] for k in ("bound", "achieved", "peak", "unit", "frac",
+                                                               "traffic", "avg_launch_us") if k in l["roofline"]}
+            if "commit" in l.get("detail", {}):
+                e["commit_avg_launch_us"] = l["detail"]["commit"]["avg_launch_us"]
+            out[name] = e
+        except Exception as exc:  # recorded, so that the headline line still prints
+            out[name] = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+    return out
+
+
 def run_prefill(args):
     """Prefill throughput: batch 2 x 32 heads, T tokens, bf16, a snapshot every
     1024 tokens (prompt tokens/s)."""
@@ -993,7 +1040,7 @@ def run_mse(args, wl):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["lq", "reference"], default="lq")
     ap.add_argument("--mode", choices=["decode", "prefill", "fp32step", "mse", "init", "ragged"],
@@ -1020,6 +1067,8 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-seconds", type=float, default=5.0)
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the secondary workloads that the default decode run also times")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)
 
@@ -1052,6 +1101,9 @@ def main(argv=None):
         line = run_ragged(args, wl)
     else:
         line = run_lq(args, wl)
+        if line is not None and not over and _dist()[1] == 1 and not args.no_secondary and \
+                args.workload == DEFAULT_WORKLOAD and args.bits == 8 and args.comp_rule == "rows":
+            line["detail"]["secondary"] = run_secondary(args)
     if line is not None:
         print(json.dumps(line), flush=True)
 

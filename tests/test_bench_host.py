@@ -108,3 +108,14 @@ def test_reference_arm_line_on_cpu(bits):
 def test_l2_note_says_which():
     assert bench.l2_note(160e6).startswith("inputs larger than L2")
     assert "L2-resident" in bench.l2_note(28e6)
+
+
+def test_secondary_workloads_are_known():
+    """The default run's secondary entries name existing workloads and modes."""
+    from linear_attention_recurrent_int8_b200 import synth
+    assert bench.DEFAULT_WORKLOAD in synth.WORKLOADS
+    for name, mode, workload, steps, warmup, flags in bench.SECONDARY:
+        assert workload in synth.WORKLOADS, name
+        assert mode in ("decode", "prefill", "ragged"), name
+        assert steps >= 1 and warmup >= 3, name
+        assert f"--steps {steps}" in flags and f"--warmup {warmup}" in flags, name
